@@ -1,0 +1,137 @@
+"""Float64 CPU oracle for the RWKV-7 (x070) state recurrence -- TEST INFRASTRUCTURE.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The CUDA library never calls it, and it
+imports nothing from the CUDA library: the two share only the seeded input
+generator ``wkv7_inputs``.
+
+The arithmetic lives in ``wkv7_oracle.c`` (token-by-token definition, see its
+header for the passages it follows).  This module compiles it with gcc
+(``-O2 -ffp-contract=off``, no fast-math) and wraps it with ctypes.
+
+Pins: every function here is checked by ``tests/test_oracle_pins.py`` against
+closed forms, a matrix-product restatement evaluated with numpy, a hand-worked
+example, invariances and a long-double build of the same source.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+from typing import Optional, Tuple
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "wkv7_oracle.c")
+_BUILD = os.path.join(_HERE, "_build")
+_LIBS = {"double": "liboracle_wkv7.so", "long double": "liboracle_wkv7_ld.so"}
+_lock = threading.Lock()
+_loaded = {}
+
+
+def build(force: bool = False) -> None:
+    """Compile both precisions of the oracle library (idempotent)."""
+    os.makedirs(_BUILD, exist_ok=True)
+    for real, name in _LIBS.items():
+        out = os.path.join(_BUILD, name)
+        if not force and os.path.exists(out) and os.path.getmtime(out) >= os.path.getmtime(_SRC):
+            continue
+        tmp = out + ".tmp%d" % os.getpid()
+        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread", "-ffp-contract=off",
+               "-fno-fast-math", f"-DORACLE_REAL={real}", _SRC, "-o", tmp]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, out)
+
+
+def _lib(real: str = "double") -> ctypes.CDLL:
+    with _lock:
+        if real not in _loaded:
+            build()
+            lib = ctypes.CDLL(os.path.join(_BUILD, _LIBS[real]))
+            dp = ctypes.POINTER(ctypes.c_double)
+            fp = ctypes.POINTER(ctypes.c_float)
+            ci = ctypes.c_int
+            lib.wkv7_oracle_f64.argtypes = [ci, ci, ci, ci] + [dp] * 6 + [dp, dp, dp, ci]
+            lib.wkv7_oracle_f64.restype = ci
+            lib.wkv7_oracle_f32in.argtypes = [ci, ci, ci, ci] + [fp] * 6 + [dp, dp, dp, ci]
+            lib.wkv7_oracle_f32in.restype = ci
+            lib.wkv7_oracle_real_bytes.restype = ci
+            _loaded[real] = lib
+        return _loaded[real]
+
+
+def _as_np(x, dt) -> np.ndarray:
+    if hasattr(x, "detach"):  # torch tensor on the CPU
+        x = x.detach()
+        import torch
+
+        x = x.to(torch.float64 if dt == np.float64 else torch.float32).contiguous().numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=dt))
+
+
+def default_threads() -> int:
+    return max(1, len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count() or 1)
+
+
+def wkv7(r, w, k, v, a, b, s_in=None, *, nthreads: Optional[int] = None, precision: str = "auto",
+         real: str = "double") -> Tuple[np.ndarray, np.ndarray]:
+    """Run the recurrence over ``[B, T, H, N]`` operands.
+
+    ``precision``: ``"f32in"`` passes the operands as float32 (exact for fp32 and
+    bf16 data), ``"f64"`` as float64; ``"auto"`` keeps float64 arrays as float64
+    and everything else as float32.  ``s_in`` is ``[B, H, N, N]`` or None (zero).
+    Returns ``(y [B, T, H, N], s_out [B, H, N, N])`` as float64 numpy arrays.
+    """
+    shp = tuple(r.shape)
+    if len(shp) != 4:
+        raise ValueError("operands must be [B, T, H, N]")
+    B, T, H, N = shp
+    for x in (w, k, v, a, b):
+        if tuple(x.shape) != shp:
+            raise ValueError("operand shapes differ")
+    if precision == "auto":
+        is64 = getattr(r, "dtype", None) in (np.float64,) or str(getattr(r, "dtype", "")) == "torch.float64"
+        precision = "f64" if is64 else "f32in"
+    dt = np.float64 if precision == "f64" else np.float32
+    ops = [_as_np(x, dt) for x in (r, w, k, v, a, b)]
+    sin = None if s_in is None else _as_np(s_in, np.float64)
+    if sin is not None and sin.shape != (B, H, N, N):
+        raise ValueError("s_in must be [B, H, N, N]")
+    y = np.zeros((B, T, H, N), dtype=np.float64)
+    s_out = np.zeros((B, H, N, N), dtype=np.float64)
+    lib = _lib(real)
+    cptr = ctypes.POINTER(ctypes.c_double if dt == np.float64 else ctypes.c_float)
+    dp = ctypes.POINTER(ctypes.c_double)
+    fn = lib.wkv7_oracle_f64 if dt == np.float64 else lib.wkv7_oracle_f32in
+    rc = fn(B, T, H, N, *[o.ctypes.data_as(cptr) for o in ops],
+            None if sin is None else sin.ctypes.data_as(dp), y.ctypes.data_as(dp),
+            s_out.ctypes.data_as(dp), int(nthreads or default_threads()))
+    if rc != 0:
+        raise RuntimeError(f"oracle failed with code {rc}")
+    return y, s_out
+
+
+def wkv7_varlen(r, w, k, v, a, b, cu_seqlens, s_in=None, *, nthreads: Optional[int] = None):
+    """Ragged batch in packed layout: operands ``[total_T, H, N]``, rows split by
+    ``cu_seqlens`` (``B + 1`` offsets).  Each row is an independent sequence.
+    Returns ``(y [total_T, H, N], s_out [B, H, N, N])``."""
+    cu = [int(x) for x in (cu_seqlens.tolist() if hasattr(cu_seqlens, "tolist") else cu_seqlens)]
+    Bn = len(cu) - 1
+    total, H, N = tuple(r.shape)
+    y = np.zeros((total, H, N), dtype=np.float64)
+    s_out = np.zeros((Bn, H, N, N), dtype=np.float64)
+    for bi in range(Bn):
+        lo, hi = cu[bi], cu[bi + 1]
+        sl = [x[lo:hi][None] for x in (r, w, k, v, a, b)]
+        si = None if s_in is None else s_in[bi:bi + 1]
+        yb, sb = wkv7(*sl, si, nthreads=nthreads)
+        y[lo:hi] = yb[0]
+        s_out[bi] = sb[0]
+    return y, s_out
+
+
+def real_bytes(real: str = "double") -> int:
+    return int(_lib(real).wkv7_oracle_real_bytes())

@@ -1,0 +1,153 @@
+/*
+ * rwkv7.h -- C ABI of the RWKV-7 (x070) state-recurrence library for NVIDIA
+ * B200 (sm_100a).
+ *
+ * The operation (RWKV-7 G0 7.2B walkthrough, lshu.cn/news/198401, section 7.1,
+ * "the two core operators of x070"): for every batch row b and head h an
+ * N x N float32 state S (N = 64; row i = value channel, column j = key
+ * channel) is updated token by token as
+ *
+ *     sa   = S a_t                                   (state before the update)
+ *     S    = S diag(w_t) + sa b_t^T + v_t k_t^T
+ *     y_t  = S r_t                                   (state after the update)
+ *
+ * "Prefill" runs this over a whole sequence at once (the pages' GPT mode,
+ * kernel wkv7); "decode" runs one token and updates the state in place (the
+ * pages' RNN mode, kernel wkv7s).  The RWKV-LM README copy (oa0.com/c/1004164)
+ * notes that the state and w must be kept in fp32 because w can be very close
+ * to 1: the state is float32 everywhere here and all accumulation is float32.
+ *
+ * Layouts (row-major, contiguous, no padding):
+ *   prefill operands r, w, k, v, a, b and output y : [B, T, H, N]
+ *   varlen operands and y (packed tokens)          : [total_T, H, N]
+ *   decode operands and y                          : [B, H, N]
+ *   states s_in, s_out, s_inout                    : [B, H, N, N] float32,
+ *                                                    element (b,h,i,j) at ((b*H+h)*N+i)*N+j
+ *   "_bf16" entry points take the operands and write y as bfloat16 bit
+ *   patterns (uint16_t); the others use float32.
+ *
+ * Ownership and execution:
+ *   - Every pointer is a device pointer owned by the caller; the library
+ *     allocates nothing per call and keeps no pointer after returning.
+ *   - Calls only enqueue work on `stream` (NULL = the legacy default stream)
+ *     and return; they never synchronise, so they can be captured into a CUDA
+ *     graph.  Results are ready once the stream reaches that point.
+ *   - s_in may be NULL (zero initial state) and may equal s_out (in place).
+ *     y must not overlap any other argument.
+ *   - Every pointer must be 16-byte aligned.
+ *
+ * Errors: a call returns RWKV7_OK once its kernels are enqueued.  Arguments are
+ * checked on the host first and nothing is launched when one is wrong:
+ *   N != 64                                  -> RWKV7_ERR_UNSUPPORTED
+ *   B, H <= 0, T < 0, a NULL required pointer -> RWKV7_ERR_INVALID
+ *   a pointer that is not 16-byte aligned     -> RWKV7_ERR_ALIGN
+ *   a failed launch                           -> RWKV7_ERR_CUDA
+ * Kernels that wait on an mbarrier give up after a bounded number of polls,
+ * record the fact in a device error word and return; rwkv7_get_last_error()
+ * reads and clears that word (it synchronises the current device).
+ * No C++ exception crosses this interface.
+ */
+#ifndef RWKV7_H
+#define RWKV7_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define RWKV7_API __attribute__((visibility("default")))
+#else
+#define RWKV7_API
+#endif
+
+/* Same type as cudaStream_t, declared without the CUDA headers. */
+struct CUstream_st;
+typedef struct CUstream_st *rwkv7_stream_t;
+
+typedef enum rwkv7_status {
+  RWKV7_OK = 0,
+  RWKV7_ERR_INVALID = 1,
+  RWKV7_ERR_ALIGN = 2,
+  RWKV7_ERR_CUDA = 3,
+  RWKV7_ERR_TIMEOUT = 4,
+  RWKV7_ERR_UNSUPPORTED = 5
+} rwkv7_status;
+
+/* Prefill kernels: AUTO picks by T and dtype; SCAN is the sequential kernel
+ * (state in registers); CHUNK is the chunked tensor-core kernel (bf16 only). */
+typedef enum rwkv7_prefill_path {
+  RWKV7_PATH_AUTO = 0,
+  RWKV7_PATH_SCAN = 1,
+  RWKV7_PATH_CHUNK = 2
+} rwkv7_prefill_path;
+
+/* ---- prefill ("GPT mode", wkv7) ------------------------------------------
+ * Runs T tokens of every (b, h) from s_in (NULL = zero) and writes y for
+ * every token and the final state to s_out.  T == 0 copies s_in (or zeros)
+ * to s_out and writes no y.  Float32 operands; uses the sequential kernel. */
+RWKV7_API rwkv7_status rwkv7_wkv_prefill(int B, int T, int H, int N, const float *r, const float *w,
+                               const float *k, const float *v, const float *a, const float *b,
+                               const float *s_in, float *y, float *s_out, rwkv7_stream_t stream);
+
+/* Same, bfloat16 operands and y (bit patterns), float32 state. */
+RWKV7_API rwkv7_status rwkv7_wkv_prefill_bf16(int B, int T, int H, int N, const uint16_t *r,
+                                    const uint16_t *w, const uint16_t *k, const uint16_t *v,
+                                    const uint16_t *a, const uint16_t *b, const float *s_in,
+                                    uint16_t *y, float *s_out, rwkv7_stream_t stream);
+
+/* bfloat16 prefill with an explicit kernel choice (for cross-checks and
+ * timing).  `path` is an rwkv7_prefill_path value; an unknown value returns
+ * RWKV7_ERR_INVALID. */
+RWKV7_API rwkv7_status rwkv7_wkv_prefill_bf16_path(int path, int B, int T, int H, int N, const uint16_t *r,
+                                         const uint16_t *w, const uint16_t *k, const uint16_t *v,
+                                         const uint16_t *a, const uint16_t *b, const float *s_in,
+                                         uint16_t *y, float *s_out, rwkv7_stream_t stream);
+
+/* Ragged batch in packed layout: B sequences, row b owns the tokens
+ * cu_seqlens[b] .. cu_seqlens[b+1]-1 of the [total_T, H, N] operands.
+ * cu_seqlens is a DEVICE array of B+1 non-decreasing int32 offsets with
+ * cu_seqlens[0] = 0 and cu_seqlens[B] = total_T (not checked on the host,
+ * since it lives on the device; rows whose offsets fall outside
+ * [0, total_T] are skipped and leave their y and s_out untouched).
+ * `max_T` is an upper bound on the longest row (used for scheduling; rows
+ * longer than it are still processed completely).  s_in / s_out are
+ * [B, H, N, N]. */
+RWKV7_API rwkv7_status rwkv7_wkv_prefill_varlen_bf16(int path, int B, int total_T, int max_T, int H, int N,
+                                           const int32_t *cu_seqlens, const uint16_t *r,
+                                           const uint16_t *w, const uint16_t *k,
+                                           const uint16_t *v, const uint16_t *a,
+                                           const uint16_t *b, const float *s_in, uint16_t *y,
+                                           float *s_out, rwkv7_stream_t stream);
+
+/* ---- decode ("RNN mode", wkv7s) ------------------------------------------
+ * One token for every (b, h): operands [B, H, N], state [B, H, N, N] updated
+ * in place, y [B, H, N]. */
+RWKV7_API rwkv7_status rwkv7_wkv_decode(int B, int H, int N, const float *r, const float *w, const float *k,
+                              const float *v, const float *a, const float *b, float *s_inout,
+                              float *y, rwkv7_stream_t stream);
+
+RWKV7_API rwkv7_status rwkv7_wkv_decode_bf16(int B, int H, int N, const uint16_t *r, const uint16_t *w,
+                                   const uint16_t *k, const uint16_t *v, const uint16_t *a,
+                                   const uint16_t *b, float *s_inout, uint16_t *y,
+                                   rwkv7_stream_t stream);
+
+/* ---- status ---------------------------------------------------------------- */
+
+/* Static English description of a status code (never NULL). */
+RWKV7_API const char *rwkv7_status_string(rwkv7_status status);
+
+/* Reads and clears the device error word of the current device (RWKV7_OK or
+ * RWKV7_ERR_TIMEOUT), and reports a pending CUDA error as RWKV7_ERR_CUDA.
+ * Synchronises the current device. */
+RWKV7_API rwkv7_status rwkv7_get_last_error(void);
+
+/* Library version as major*10000 + minor*100 + patch. */
+RWKV7_API int rwkv7_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RWKV7_H */

@@ -1,0 +1,218 @@
+"""Python binding of the RWKV-7 (x070) state-recurrence library ``librwkv7.so``.
+
+Argument marshalling only: every function here checks tensor shapes, dtypes
+and devices, passes raw device pointers and the current CUDA stream to the
+``extern "C"`` entry point of the same name (declared in ``include/rwkv7.h``)
+and raises on a non-OK status.  All computation happens in the CUDA kernels.
+There is no CPU fallback: if the library is missing, importing the entry
+points raises.
+
+The recurrence (RWKV-7 G0 7.2B walkthrough, lshu.cn/news/198401, section 7.1),
+per batch row b and head h, with a float32 64 x 64 state S:
+
+    sa = S a_t;   S = S diag(w_t) + sa b_t^T + v_t k_t^T;   y_t = S r_t
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+__all__ = [
+    "RWKV7_PATH_AUTO", "RWKV7_PATH_SCAN", "RWKV7_PATH_CHUNK", "Rwkv7Error", "library_path", "load_library",
+    "rwkv7_wkv_prefill", "rwkv7_wkv_prefill_bf16", "rwkv7_wkv_prefill_bf16_path", "rwkv7_wkv_prefill_varlen_bf16",
+    "rwkv7_wkv_decode", "rwkv7_wkv_decode_bf16", "rwkv7_status_string", "rwkv7_get_last_error", "rwkv7_version",
+    "prefill", "decode_", "EXPORTED_SYMBOLS",
+]
+
+RWKV7_PATH_AUTO, RWKV7_PATH_SCAN, RWKV7_PATH_CHUNK = 0, 1, 2
+N_HEAD = 64
+
+EXPORTED_SYMBOLS = (
+    "rwkv7_wkv_prefill", "rwkv7_wkv_prefill_bf16", "rwkv7_wkv_prefill_bf16_path", "rwkv7_wkv_prefill_varlen_bf16",
+    "rwkv7_wkv_decode", "rwkv7_wkv_decode_bf16", "rwkv7_status_string", "rwkv7_get_last_error", "rwkv7_version",
+)
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_lib: Optional[ctypes.CDLL] = None
+
+
+class Rwkv7Error(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn}: {rwkv7_status_string(status)} (status {status})")
+        self.status = status
+
+
+def library_path() -> str:
+    return os.path.join(_HERE, "librwkv7.so")
+
+
+def load_library() -> ctypes.CDLL:
+    """Load ``librwkv7.so`` (built in-tree by ``rwkv_delta_rule_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = library_path()
+    if not os.path.exists(path):
+        raise RuntimeError(f"librwkv7.so not built ({path}); run `python -m rwkv_delta_rule_b200.build`")
+    lib = ctypes.CDLL(path)
+    vp, ci = ctypes.c_void_p, ctypes.c_int
+    pre = [ci, ci, ci, ci] + [vp] * 6 + [vp, vp, vp, vp]
+    for name, args in (
+        ("rwkv7_wkv_prefill", pre),
+        ("rwkv7_wkv_prefill_bf16", pre),
+        ("rwkv7_wkv_prefill_bf16_path", [ci] + pre),
+        ("rwkv7_wkv_prefill_varlen_bf16", [ci, ci, ci, ci, ci, ci, vp] + [vp] * 6 + [vp, vp, vp, vp]),
+        ("rwkv7_wkv_decode", [ci, ci, ci] + [vp] * 6 + [vp, vp, vp]),
+        ("rwkv7_wkv_decode_bf16", [ci, ci, ci] + [vp] * 6 + [vp, vp, vp]),
+    ):
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = ci
+    lib.rwkv7_status_string.argtypes = [ci]
+    lib.rwkv7_status_string.restype = ctypes.c_char_p
+    lib.rwkv7_get_last_error.argtypes = []
+    lib.rwkv7_get_last_error.restype = ci
+    lib.rwkv7_version.argtypes = []
+    lib.rwkv7_version.restype = ci
+    _lib = lib
+    return lib
+
+
+# ---- marshalling helpers ------------------------------------------------------------------------
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _check(t: Optional[torch.Tensor], name: str, dtype: torch.dtype, shape=None, allow_none=False):
+    if t is None:
+        if allow_none:
+            return
+        raise ValueError(f"{name} is required")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _call(name: str, *args) -> None:
+    st = getattr(load_library(), name)(*args)
+    if st != 0:
+        raise Rwkv7Error(name, st)
+
+
+def _prefill_common(name, dtype, r, w, k, v, a, b, s_in, y, s_out, stream, path=None):
+    B, T, H, N = r.shape
+    for nm, t in (("r", r), ("w", w), ("k", k), ("v", v), ("a", a), ("b", b), ("y", y)):
+        _check(t, nm, dtype, (B, T, H, N))
+    _check(s_in, "s_in", torch.float32, (B, H, N, N), allow_none=True)
+    _check(s_out, "s_out", torch.float32, (B, H, N, N))
+    args = [B, T, H, N] + [_ptr(t) for t in (r, w, k, v, a, b, s_in, y, s_out)] + [_stream(stream)]
+    if path is not None:
+        args = [int(path)] + args
+    _call(name, *args)
+
+
+# ---- entry points (same names as the C ABI) --------------------------------------------------------
+
+def rwkv7_wkv_prefill(r, w, k, v, a, b, s_in, y, s_out, stream=None) -> None:
+    """float32 prefill: operands / y ``[B,T,H,64]``, states ``[B,H,64,64]`` (s_in may be None)."""
+    _prefill_common("rwkv7_wkv_prefill", torch.float32, r, w, k, v, a, b, s_in, y, s_out, stream)
+
+
+def rwkv7_wkv_prefill_bf16(r, w, k, v, a, b, s_in, y, s_out, stream=None) -> None:
+    """bfloat16 prefill (kernel chosen by the library), float32 states."""
+    _prefill_common("rwkv7_wkv_prefill_bf16", torch.bfloat16, r, w, k, v, a, b, s_in, y, s_out, stream)
+
+
+def rwkv7_wkv_prefill_bf16_path(path, r, w, k, v, a, b, s_in, y, s_out, stream=None) -> None:
+    """bfloat16 prefill with an explicit kernel (RWKV7_PATH_SCAN or RWKV7_PATH_CHUNK)."""
+    _prefill_common("rwkv7_wkv_prefill_bf16_path", torch.bfloat16, r, w, k, v, a, b, s_in, y, s_out, stream,
+                    path=path)
+
+
+def rwkv7_wkv_prefill_varlen_bf16(path, cu_seqlens, max_T, r, w, k, v, a, b, s_in, y, s_out, stream=None) -> None:
+    """Ragged bfloat16 prefill: operands / y ``[total_T,H,64]`` packed, ``cu_seqlens`` int32 ``[B+1]`` on the
+    device, states ``[B,H,64,64]``."""
+    total, H, N = r.shape
+    Bn = cu_seqlens.numel() - 1
+    _check(cu_seqlens, "cu_seqlens", torch.int32, (Bn + 1,))
+    for nm, t in (("r", r), ("w", w), ("k", k), ("v", v), ("a", a), ("b", b), ("y", y)):
+        _check(t, nm, torch.bfloat16, (total, H, N))
+    _check(s_in, "s_in", torch.float32, (Bn, H, N, N), allow_none=True)
+    _check(s_out, "s_out", torch.float32, (Bn, H, N, N))
+    _call("rwkv7_wkv_prefill_varlen_bf16", int(path), Bn, total, int(max_T), H, N, _ptr(cu_seqlens),
+          *[_ptr(t) for t in (r, w, k, v, a, b, s_in, y, s_out)], _stream(stream))
+
+
+def _decode_common(name, dtype, r, w, k, v, a, b, s_inout, y, stream):
+    B, H, N = r.shape
+    for nm, t in (("r", r), ("w", w), ("k", k), ("v", v), ("a", a), ("b", b), ("y", y)):
+        _check(t, nm, dtype, (B, H, N))
+    _check(s_inout, "s_inout", torch.float32, (B, H, N, N))
+    _call(name, B, H, N, *[_ptr(t) for t in (r, w, k, v, a, b, s_inout, y)], _stream(stream))
+
+
+def rwkv7_wkv_decode(r, w, k, v, a, b, s_inout, y, stream=None) -> None:
+    """float32 one-token step: operands / y ``[B,H,64]``, state ``[B,H,64,64]`` updated in place."""
+    _decode_common("rwkv7_wkv_decode", torch.float32, r, w, k, v, a, b, s_inout, y, stream)
+
+
+def rwkv7_wkv_decode_bf16(r, w, k, v, a, b, s_inout, y, stream=None) -> None:
+    """bfloat16 one-token step, float32 state updated in place."""
+    _decode_common("rwkv7_wkv_decode_bf16", torch.bfloat16, r, w, k, v, a, b, s_inout, y, stream)
+
+
+def rwkv7_status_string(status: int) -> str:
+    return load_library().rwkv7_status_string(int(status)).decode()
+
+
+def rwkv7_get_last_error() -> int:
+    return int(load_library().rwkv7_get_last_error())
+
+
+def rwkv7_version() -> int:
+    return int(load_library().rwkv7_version())
+
+
+# ---- conveniences: allocate outputs with torch, then call the entry points ------------------------
+
+def prefill(r, w, k, v, a, b, s_in=None, *, path: int = RWKV7_PATH_AUTO, stream=None):
+    """Allocate ``y`` and ``s_out`` and run prefill; returns ``(y, s_out)``."""
+    B, T, H, N = r.shape
+    y = torch.empty_like(r)
+    s_out = torch.empty((B, H, N, N), dtype=torch.float32, device=r.device)
+    if r.dtype == torch.float32:
+        if path not in (RWKV7_PATH_AUTO, RWKV7_PATH_SCAN):
+            raise ValueError("float32 prefill runs on the scan kernel only")
+        rwkv7_wkv_prefill(r, w, k, v, a, b, s_in, y, s_out, stream)
+    else:
+        rwkv7_wkv_prefill_bf16_path(path, r, w, k, v, a, b, s_in, y, s_out, stream)
+    return y, s_out
+
+
+def decode_(r, w, k, v, a, b, state, y=None, *, stream=None):
+    """One decode step updating ``state`` in place; returns ``y``."""
+    if y is None:
+        y = torch.empty_like(r)
+    if r.dtype == torch.float32:
+        rwkv7_wkv_decode(r, w, k, v, a, b, state, y, stream)
+    else:
+        rwkv7_wkv_decode_bf16(r, w, k, v, a, b, state, y, stream)
+    return y

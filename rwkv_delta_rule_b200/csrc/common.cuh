@@ -1,0 +1,92 @@
+// common.cuh -- small device helpers shared by the kernels of this library.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace rwkv7 {
+
+constexpr int kN = 64;  // head size; the pages fix it at 64 (compile-time -D_N_=64)
+
+// Device error word: kernels that give up on a bounded wait store a nonzero
+// code through the pointer they are given (the library's word, defined in
+// rwkv7_api.cu); the host reads and clears it in rwkv7_get_last_error().
+enum DeviceError : int { kDevErrNone = 0, kDevErrTimeout = 1 };
+
+__device__ __forceinline__ void report_device_error(int *word, int code) {
+  if (word != nullptr) atomicCAS(word, 0, code);
+}
+
+// ---- element conversions ---------------------------------------------------
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
+  return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+__device__ __forceinline__ uint16_t float_to_bf16_bits(float f) {
+  __nv_bfloat16 h = __float2bfloat16_rn(f);
+  return *reinterpret_cast<uint16_t *>(&h);
+}
+
+// Storage-type traits: float32 or bfloat16 bit patterns.
+template <typename T> struct Elem;
+template <> struct Elem<float> {
+  static __device__ __forceinline__ float load(const float *p) { return *p; }
+  static __device__ __forceinline__ void store(float *p, float v) { *p = v; }
+  // four consecutive elements (16-byte aligned for float)
+  static __device__ __forceinline__ void load4(const float *p, float out[4]) {
+    float4 v = *reinterpret_cast<const float4 *>(p);
+    out[0] = v.x; out[1] = v.y; out[2] = v.z; out[3] = v.w;
+  }
+};
+template <> struct Elem<uint16_t> {
+  static __device__ __forceinline__ float load(const uint16_t *p) { return bf16_bits_to_float(*p); }
+  static __device__ __forceinline__ void store(uint16_t *p, float v) { *p = float_to_bf16_bits(v); }
+  // four consecutive elements (8-byte aligned)
+  static __device__ __forceinline__ void load4(const uint16_t *p, float out[4]) {
+    uint2 v = *reinterpret_cast<const uint2 *>(p);
+    out[0] = __uint_as_float(v.x << 16);
+    out[1] = __uint_as_float(v.x & 0xffff0000u);
+    out[2] = __uint_as_float(v.y << 16);
+    out[3] = __uint_as_float(v.y & 0xffff0000u);
+  }
+};
+
+// ---- cp.async (16-byte, L2-only) ---------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_u32(smem_dst)), "l"(gmem_src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N> __device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+
+// Sequence bounds for row b: fixed-length batches use start = b*T, len = T;
+// ragged batches read them from the device offsets.  A row whose offsets are
+// out of range gets len = -1 and is skipped by the caller.
+struct SeqBounds {
+  long long start;
+  int len;
+};
+__device__ __forceinline__ SeqBounds seq_bounds(const int32_t *cu_seqlens, int b, int T, long long total_T) {
+  SeqBounds sb;
+  if (cu_seqlens == nullptr) {
+    sb.start = static_cast<long long>(b) * T;
+    sb.len = T;
+  } else {
+    const long long lo = cu_seqlens[b], hi = cu_seqlens[b + 1];
+    if (lo < 0 || hi < lo || hi > total_T) {
+      sb.start = 0;
+      sb.len = -1;
+    } else {
+      sb.start = lo;
+      sb.len = static_cast<int>(hi - lo);
+    }
+  }
+  return sb;
+}
+
+}  // namespace rwkv7

@@ -1,0 +1,22 @@
+// launch.h -- internal launchers behind the C ABI (not exported).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace rwkv7 {
+
+// Sequential scan over [B,T,H,64] (cu_seqlens == nullptr) or a packed ragged
+// batch (cu_seqlens = device offsets, total_T tokens).  TIn: float or
+// uint16_t (bfloat16 bits).
+template <typename TIn>
+cudaError_t launch_scan(const TIn *r, const TIn *w, const TIn *k, const TIn *v, const TIn *a, const TIn *b,
+                        const float *s_in, TIn *y, float *s_out, const int32_t *cu_seqlens, int B, int T,
+                        long long total_T, int H, cudaStream_t stream);
+
+// One decode step over [B,H,64], state updated in place.
+template <typename TIn>
+cudaError_t launch_decode(const TIn *r, const TIn *w, const TIn *k, const TIn *v, const TIn *a, const TIn *b,
+                          float *s, TIn *y, int B, int H, cudaStream_t stream);
+
+}  // namespace rwkv7

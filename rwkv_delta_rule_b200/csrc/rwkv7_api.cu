@@ -1,0 +1,133 @@
+// rwkv7_api.cu -- the extern "C" entry points declared in include/rwkv7.h:
+// host-side argument checks, kernel choice and launches.  Nothing here
+// allocates, synchronises or touches the data; every step of the computation
+// runs in the kernels.
+#include "../../include/rwkv7.h"
+#include "common.cuh"
+#include "launch.h"
+
+namespace rwkv7 {
+
+__device__ int g_error_word = 0;
+
+namespace {
+
+constexpr int kVersion = 100;  // 0.1.0
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+template <typename... P> bool all_aligned(const P *...ps) { return (aligned16(ps) && ...); }
+template <typename... P> bool none_null(const P *...ps) { return ((ps != nullptr) && ...); }
+
+rwkv7_status from_cuda(cudaError_t e) { return e == cudaSuccess ? RWKV7_OK : RWKV7_ERR_CUDA; }
+
+// Checks shared by every prefill entry point.  `need_ops` is false when no
+// token is processed (T == 0), in which case operand pointers may be NULL.
+template <typename TIn>
+rwkv7_status check_prefill(int B, long long tokens, int H, int N, const TIn *r, const TIn *w, const TIn *k,
+                           const TIn *v, const TIn *a, const TIn *b, const float *s_in, const TIn *y,
+                           const float *s_out) {
+  if (N != kN) return RWKV7_ERR_UNSUPPORTED;
+  if (B <= 0 || H <= 0 || tokens < 0) return RWKV7_ERR_INVALID;
+  if (s_out == nullptr) return RWKV7_ERR_INVALID;
+  const bool need_ops = tokens > 0;
+  if (need_ops && !none_null(r, w, k, v, a, b, y)) return RWKV7_ERR_INVALID;
+  if (!all_aligned(r, w, k, v, a, b, y, s_in, s_out)) return RWKV7_ERR_ALIGN;
+  if (static_cast<long long>(B) > 65535) return RWKV7_ERR_INVALID;  // grid.y limit of the launches
+  return RWKV7_OK;
+}
+
+}  // namespace
+}  // namespace rwkv7
+
+using namespace rwkv7;
+
+extern "C" {
+
+const char *rwkv7_status_string(rwkv7_status status) {
+  switch (status) {
+    case RWKV7_OK: return "ok";
+    case RWKV7_ERR_INVALID: return "invalid argument";
+    case RWKV7_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case RWKV7_ERR_CUDA: return "CUDA error";
+    case RWKV7_ERR_TIMEOUT: return "device wait timed out";
+    case RWKV7_ERR_UNSUPPORTED: return "unsupported size (head size must be 64)";
+  }
+  return "unknown status";
+}
+
+int rwkv7_version(void) { return kVersion; }
+
+rwkv7_status rwkv7_get_last_error(void) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return RWKV7_ERR_CUDA;
+  int word = 0;
+  const int zero = 0;
+  if (cudaMemcpyFromSymbol(&word, g_error_word, sizeof(int)) != cudaSuccess) return RWKV7_ERR_CUDA;
+  if (word != 0 && cudaMemcpyToSymbol(g_error_word, &zero, sizeof(int)) != cudaSuccess) return RWKV7_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return RWKV7_ERR_CUDA;
+  return word == kDevErrNone ? RWKV7_OK : RWKV7_ERR_TIMEOUT;
+}
+
+rwkv7_status rwkv7_wkv_prefill(int B, int T, int H, int N, const float *r, const float *w, const float *k,
+                               const float *v, const float *a, const float *b, const float *s_in, float *y,
+                               float *s_out, rwkv7_stream_t stream) {
+  const rwkv7_status st = check_prefill(B, T, H, N, r, w, k, v, a, b, s_in, y, s_out);
+  if (st != RWKV7_OK) return st;
+  return from_cuda(launch_scan<float>(r, w, k, v, a, b, s_in, y, s_out, nullptr, B, T,
+                                      static_cast<long long>(B) * T, H, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+rwkv7_status rwkv7_wkv_prefill_bf16_path(int path, int B, int T, int H, int N, const uint16_t *r, const uint16_t *w,
+                                         const uint16_t *k, const uint16_t *v, const uint16_t *a, const uint16_t *b,
+                                         const float *s_in, uint16_t *y, float *s_out, rwkv7_stream_t stream) {
+  if (path != RWKV7_PATH_AUTO && path != RWKV7_PATH_SCAN && path != RWKV7_PATH_CHUNK) return RWKV7_ERR_INVALID;
+  const rwkv7_status st = check_prefill(B, T, H, N, r, w, k, v, a, b, s_in, y, s_out);
+  if (st != RWKV7_OK) return st;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if (path == RWKV7_PATH_CHUNK) return RWKV7_ERR_UNSUPPORTED;  // chunked kernel not built yet
+  return from_cuda(launch_scan<uint16_t>(r, w, k, v, a, b, s_in, y, s_out, nullptr, B, T,
+                                         static_cast<long long>(B) * T, H, cs));
+}
+
+rwkv7_status rwkv7_wkv_prefill_bf16(int B, int T, int H, int N, const uint16_t *r, const uint16_t *w,
+                                    const uint16_t *k, const uint16_t *v, const uint16_t *a, const uint16_t *b,
+                                    const float *s_in, uint16_t *y, float *s_out, rwkv7_stream_t stream) {
+  return rwkv7_wkv_prefill_bf16_path(RWKV7_PATH_AUTO, B, T, H, N, r, w, k, v, a, b, s_in, y, s_out, stream);
+}
+
+rwkv7_status rwkv7_wkv_prefill_varlen_bf16(int path, int B, int total_T, int max_T, int H, int N,
+                                           const int32_t *cu_seqlens, const uint16_t *r, const uint16_t *w,
+                                           const uint16_t *k, const uint16_t *v, const uint16_t *a,
+                                           const uint16_t *b, const float *s_in, uint16_t *y, float *s_out,
+                                           rwkv7_stream_t stream) {
+  if (path != RWKV7_PATH_AUTO && path != RWKV7_PATH_SCAN && path != RWKV7_PATH_CHUNK) return RWKV7_ERR_INVALID;
+  if (max_T < 0 || cu_seqlens == nullptr || !aligned16(cu_seqlens)) {
+    if (cu_seqlens != nullptr && !aligned16(cu_seqlens) && max_T >= 0) return RWKV7_ERR_ALIGN;
+    return RWKV7_ERR_INVALID;
+  }
+  const rwkv7_status st = check_prefill(B, total_T, H, N, r, w, k, v, a, b, s_in, y, s_out);
+  if (st != RWKV7_OK) return st;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if (path == RWKV7_PATH_CHUNK) return RWKV7_ERR_UNSUPPORTED;  // chunked kernel not built yet
+  return from_cuda(launch_scan<uint16_t>(r, w, k, v, a, b, s_in, y, s_out, cu_seqlens, B, 0, total_T, H, cs));
+}
+
+rwkv7_status rwkv7_wkv_decode(int B, int H, int N, const float *r, const float *w, const float *k, const float *v,
+                              const float *a, const float *b, float *s_inout, float *y, rwkv7_stream_t stream) {
+  if (N != kN) return RWKV7_ERR_UNSUPPORTED;
+  if (B <= 0 || H <= 0 || !none_null(r, w, k, v, a, b, s_inout, y)) return RWKV7_ERR_INVALID;
+  if (!all_aligned(r, w, k, v, a, b, s_inout, y)) return RWKV7_ERR_ALIGN;
+  return from_cuda(launch_decode<float>(r, w, k, v, a, b, s_inout, y, B, H, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+rwkv7_status rwkv7_wkv_decode_bf16(int B, int H, int N, const uint16_t *r, const uint16_t *w, const uint16_t *k,
+                                   const uint16_t *v, const uint16_t *a, const uint16_t *b, float *s_inout,
+                                   uint16_t *y, rwkv7_stream_t stream) {
+  if (N != kN) return RWKV7_ERR_UNSUPPORTED;
+  if (B <= 0 || H <= 0 || !none_null(r, w, k, v, a, b, s_inout, y)) return RWKV7_ERR_INVALID;
+  if (!all_aligned(r, w, k, v, a, b, s_inout, y)) return RWKV7_ERR_ALIGN;
+  return from_cuda(
+      launch_decode<uint16_t>(r, w, k, v, a, b, s_inout, y, B, H, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

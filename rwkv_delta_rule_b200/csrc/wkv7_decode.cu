@@ -1,0 +1,107 @@
+// wkv7_decode.cu -- one-token step of the x070 recurrence ("RNN mode"),
+// updating the float32 state in place.
+//
+// Operation (RWKV-7 G0 7.2B walkthrough, lshu.cn/news/198401, sections 3.2
+// and 7.1: wkv7s is the single-step form of the same update):
+//   sa = S a;  S = S diag(w) + sa b^T + v k^T;  y = S r.
+//
+// The step is bound by HBM: every (b, h) reads and writes its 16 KiB state
+// once and touches only 7 vectors of 64 elements besides.  One CTA of 256
+// threads owns one (b, h).  Thread t holds columns 4*(t%16) .. +3 of rows
+// t/16 + 16*m (m = 0..3): four 16-byte loads per thread, issued together,
+// and a warp covers two whole 256-byte rows per load.  The row sums S a and
+// S r are finished with four xor-shuffles inside each 16-lane half-warp.
+#include "common.cuh"
+#include "launch.h"
+
+namespace rwkv7 {
+
+template <typename TIn> struct DecodeArgs {
+  const TIn *r, *w, *k, *v, *a, *b;
+  float *s;
+  TIn *y;
+};
+
+__device__ __forceinline__ float4 ld_state(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+__device__ __forceinline__ void st_state(float *p, float4 x) { *reinterpret_cast<float4 *>(p) = x; }
+
+template <typename TIn>
+__global__ void __launch_bounds__(256) wkv7_decode_kernel(DecodeArgs<TIn> A) {
+  const long long pair = blockIdx.x;  // b * H + h
+  const int tid = threadIdx.x;
+  const int c4 = tid & 15;   // column chunk: columns 4*c4 .. 4*c4+3
+  const int rg = tid >> 4;   // rows rg + 16*m
+  float *S = A.s + pair * (kN * kN);
+
+  float4 st[4];
+#pragma unroll
+  for (int m = 0; m < 4; ++m) st[m] = ld_state(S + (rg + 16 * m) * kN + 4 * c4);
+
+  const long long vb = pair * kN;
+  float ww[4], kk[4], aa[4], bb[4], rr[4], vv[4];
+  Elem<TIn>::load4(A.w + vb + 4 * c4, ww);
+  Elem<TIn>::load4(A.k + vb + 4 * c4, kk);
+  Elem<TIn>::load4(A.a + vb + 4 * c4, aa);
+  Elem<TIn>::load4(A.b + vb + 4 * c4, bb);
+  Elem<TIn>::load4(A.r + vb + 4 * c4, rr);
+#pragma unroll
+  for (int m = 0; m < 4; ++m) vv[m] = Elem<TIn>::load(A.v + vb + rg + 16 * m);
+
+  float sa[4];
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    float p = st[m].x * aa[0];
+    p = fmaf(st[m].y, aa[1], p);
+    p = fmaf(st[m].z, aa[2], p);
+    p = fmaf(st[m].w, aa[3], p);
+    sa[m] = p;
+  }
+#pragma unroll
+  for (int off = 8; off >= 1; off >>= 1)
+#pragma unroll
+    for (int m = 0; m < 4; ++m) sa[m] += __shfl_xor_sync(0xffffffffu, sa[m], off);
+
+  float yv[4];
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    float4 x = st[m];
+    x.x = fmaf(x.x, ww[0], fmaf(sa[m], bb[0], vv[m] * kk[0]));
+    x.y = fmaf(x.y, ww[1], fmaf(sa[m], bb[1], vv[m] * kk[1]));
+    x.z = fmaf(x.z, ww[2], fmaf(sa[m], bb[2], vv[m] * kk[2]));
+    x.w = fmaf(x.w, ww[3], fmaf(sa[m], bb[3], vv[m] * kk[3]));
+    st[m] = x;
+    float p = x.x * rr[0];
+    p = fmaf(x.y, rr[1], p);
+    p = fmaf(x.z, rr[2], p);
+    p = fmaf(x.w, rr[3], p);
+    yv[m] = p;
+  }
+#pragma unroll
+  for (int m = 0; m < 4; ++m) st_state(S + (rg + 16 * m) * kN + 4 * c4, st[m]);
+#pragma unroll
+  for (int off = 8; off >= 1; off >>= 1)
+#pragma unroll
+    for (int m = 0; m < 4; ++m) yv[m] += __shfl_xor_sync(0xffffffffu, yv[m], off);
+  if (c4 == 0) {
+#pragma unroll
+    for (int m = 0; m < 4; ++m) Elem<TIn>::store(A.y + vb + rg + 16 * m, yv[m]);
+  }
+}
+
+template <typename TIn>
+cudaError_t launch_decode(const TIn *r, const TIn *w, const TIn *k, const TIn *v, const TIn *a, const TIn *b,
+                          float *s, TIn *y, int B, int H, cudaStream_t stream) {
+  DecodeArgs<TIn> A{r, w, k, v, a, b, s, y};
+  const long long pairs = static_cast<long long>(B) * H;
+  if (pairs > 0x7fffffffLL) return cudaErrorInvalidValue;
+  wkv7_decode_kernel<TIn><<<static_cast<unsigned>(pairs), 256, 0, stream>>>(A);
+  return cudaGetLastError();
+}
+
+template cudaError_t launch_decode<float>(const float *, const float *, const float *, const float *, const float *,
+                                          const float *, float *, float *, int, int, cudaStream_t);
+template cudaError_t launch_decode<uint16_t>(const uint16_t *, const uint16_t *, const uint16_t *, const uint16_t *,
+                                             const uint16_t *, const uint16_t *, float *, uint16_t *, int, int,
+                                             cudaStream_t);
+
+}  // namespace rwkv7

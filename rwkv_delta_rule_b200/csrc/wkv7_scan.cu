@@ -1,0 +1,207 @@
+// wkv7_scan.cu -- sequential-scan prefill: the x070 recurrence token by token
+// with the float32 state held in registers.
+//
+// Operation (RWKV-7 G0 7.2B walkthrough, lshu.cn/news/198401, section 7.1):
+//   sa = S a_t;  S = S diag(w_t) + sa b_t^T + v_t k_t^T;  y_t = S r_t.
+//
+// Rows of S are independent of each other: row i needs only its own values,
+// v_t[i] and the shared vectors r, w, k, a, b.  So a (b, h) pair is split
+// into 64 / ROWS row groups, one CTA each, and every row is spread over a quad
+// of 4 lanes that hold 16 columns each.  The two per-token dot products (S a
+// and S r) are finished with two xor-shuffles inside the quad.
+//
+// Column ownership inside a quad: lane q holds the 4-column chunks starting
+// at 16*m + 4*q (m = 0..3), so one vector read by a quad touches 4 adjacent
+// chunks of shared memory and 8 quads read the same addresses (broadcast).
+//
+// Per-token operands are staged into shared memory in tiles of TT tokens
+// with cp.async, double-buffered, and y is staged per tile and written back
+// as contiguous runs of ROWS elements.
+#include "common.cuh"
+#include "launch.h"
+
+namespace rwkv7 {
+
+template <typename TIn, int ROWS> struct ScanCfg {
+  static constexpr int kThreads = ROWS * 4;
+  static constexpr int kTT = sizeof(TIn) == 2 ? 32 : 16;  // tokens per tile (24+ KB per buffer)
+  static constexpr int kVecElems = 5 * kN;                 // r, w, k, a, b
+  static constexpr int kTokElems = kVecElems + ROWS;       // + this CTA's slice of v
+  static constexpr int kBufElems = kTT * kTokElems;
+  static constexpr int kEPC = 16 / static_cast<int>(sizeof(TIn));  // elements per 16-byte chunk
+  static constexpr int kChunksVec = kN / kEPC;
+  static constexpr int kChunksV = ROWS / kEPC;
+  static constexpr int kChunksTok = 5 * kChunksVec + kChunksV;
+  static constexpr size_t kSmemBytes = 2 * kBufElems * sizeof(TIn) + kTT * ROWS * sizeof(float);
+  static_assert((kTokElems * sizeof(TIn)) % 16 == 0, "token stride must keep 16-byte alignment");
+  static_assert(ROWS % kEPC == 0, "row slice must be whole 16-byte chunks");
+};
+
+template <typename TIn> struct ScanArgs {
+  const TIn *r, *w, *k, *v, *a, *b;
+  const float *s_in;
+  TIn *y;
+  float *s_out;
+  const int32_t *cu_seqlens;  // nullptr: fixed length T
+  int T;
+  long long total_T;
+  int H;
+};
+
+template <typename TIn, int ROWS>
+__device__ __forceinline__ void scan_load_tile(const ScanArgs<TIn> &A, TIn *buf, long long tok0, int ntok, int h,
+                                               int row0) {
+  using C = ScanCfg<TIn, ROWS>;
+  const int total = ntok * C::kChunksTok;
+  for (int c = threadIdx.x; c < total; c += C::kThreads) {
+    const int tt = c / C::kChunksTok, cc = c - tt * C::kChunksTok;
+    const long long base = ((tok0 + tt) * A.H + h) * kN;
+    TIn *dst = buf + tt * C::kTokElems;
+    if (cc < 5 * C::kChunksVec) {
+      const int vid = cc / C::kChunksVec, part = cc - vid * C::kChunksVec;
+      const TIn *src = vid == 0 ? A.r : vid == 1 ? A.w : vid == 2 ? A.k : vid == 3 ? A.a : A.b;
+      cp_async16(dst + vid * kN + part * C::kEPC, src + base + part * C::kEPC);
+    } else {
+      const int part = cc - 5 * C::kChunksVec;
+      cp_async16(dst + C::kVecElems + part * C::kEPC, A.v + base + row0 + part * C::kEPC);
+    }
+  }
+}
+
+template <typename TIn, int ROWS>
+__global__ void __launch_bounds__(ScanCfg<TIn, ROWS>::kThreads) wkv7_scan_kernel(ScanArgs<TIn> A) {
+  using C = ScanCfg<TIn, ROWS>;
+  constexpr int kSplits = kN / ROWS;
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  TIn *bufs = reinterpret_cast<TIn *>(smem_raw);
+  float *ys = reinterpret_cast<float *>(smem_raw + 2 * C::kBufElems * sizeof(TIn));
+
+  const int h = blockIdx.x / kSplits;
+  const int row0 = (blockIdx.x - h * kSplits) * ROWS;
+  const int bidx = blockIdx.y;
+  const SeqBounds sb = seq_bounds(A.cu_seqlens, bidx, A.T, A.total_T);
+  if (sb.len < 0) return;
+
+  const int tid = threadIdx.x;
+  const int rloc = tid >> 2, q = tid & 3;
+  const int row = row0 + rloc;
+  const long long sbase = (static_cast<long long>(bidx) * A.H + h) * (kN * kN) + static_cast<long long>(row) * kN;
+
+  float s[16];
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (A.s_in != nullptr) x = *reinterpret_cast<const float4 *>(A.s_in + sbase + 16 * m + 4 * q);
+    s[4 * m + 0] = x.x; s[4 * m + 1] = x.y; s[4 * m + 2] = x.z; s[4 * m + 3] = x.w;
+  }
+
+  const int ntiles = (sb.len + C::kTT - 1) / C::kTT;
+  if (ntiles > 0) {
+    scan_load_tile<TIn, ROWS>(A, bufs, sb.start, min(C::kTT, sb.len), h, row0);
+    cp_async_commit();
+  }
+  for (int tile = 0; tile < ntiles; ++tile) {
+    const int t0 = tile * C::kTT;
+    const int ntok = min(C::kTT, sb.len - t0);
+    if (tile + 1 < ntiles) {
+      const int t1 = t0 + C::kTT;
+      scan_load_tile<TIn, ROWS>(A, bufs + ((tile + 1) & 1) * C::kBufElems, sb.start + t1, min(C::kTT, sb.len - t1),
+                                h, row0);
+      cp_async_commit();
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+
+    const TIn *buf = bufs + (tile & 1) * C::kBufElems;
+#pragma unroll 2
+    for (int tt = 0; tt < ntok; ++tt) {
+      const TIn *tok = buf + tt * C::kTokElems;
+      float rr[16], ww[16], kk[16], aa[16], bb[16];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int col = 16 * m + 4 * q;
+        Elem<TIn>::load4(tok + 0 * kN + col, rr + 4 * m);
+        Elem<TIn>::load4(tok + 1 * kN + col, ww + 4 * m);
+        Elem<TIn>::load4(tok + 2 * kN + col, kk + 4 * m);
+        Elem<TIn>::load4(tok + 3 * kN + col, aa + 4 * m);
+        Elem<TIn>::load4(tok + 4 * kN + col, bb + 4 * m);
+      }
+      const float vi = Elem<TIn>::load(tok + C::kVecElems + rloc);
+
+      // sa = S a (state before this token), four partial sums then the quad
+      float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
+#pragma unroll
+      for (int c = 0; c < 16; c += 4) {
+        p0 = fmaf(s[c + 0], aa[c + 0], p0);
+        p1 = fmaf(s[c + 1], aa[c + 1], p1);
+        p2 = fmaf(s[c + 2], aa[c + 2], p2);
+        p3 = fmaf(s[c + 3], aa[c + 3], p3);
+      }
+      float sa = (p0 + p1) + (p2 + p3);
+      sa += __shfl_xor_sync(0xffffffffu, sa, 1);
+      sa += __shfl_xor_sync(0xffffffffu, sa, 2);
+
+      // S = S diag(w) + sa b^T + v k^T
+#pragma unroll
+      for (int c = 0; c < 16; ++c) s[c] = fmaf(s[c], ww[c], fmaf(sa, bb[c], vi * kk[c]));
+
+      // y = S r (updated state)
+      p0 = p1 = p2 = p3 = 0.f;
+#pragma unroll
+      for (int c = 0; c < 16; c += 4) {
+        p0 = fmaf(s[c + 0], rr[c + 0], p0);
+        p1 = fmaf(s[c + 1], rr[c + 1], p1);
+        p2 = fmaf(s[c + 2], rr[c + 2], p2);
+        p3 = fmaf(s[c + 3], rr[c + 3], p3);
+      }
+      float y = (p0 + p1) + (p2 + p3);
+      y += __shfl_xor_sync(0xffffffffu, y, 1);
+      y += __shfl_xor_sync(0xffffffffu, y, 2);
+      if (q == 0) ys[tt * ROWS + rloc] = y;
+    }
+    __syncthreads();
+    for (int e = tid; e < ntok * ROWS; e += C::kThreads) {
+      const int tt = e / ROWS, rr_ = e - tt * ROWS;
+      const long long yi = ((sb.start + t0 + tt) * A.H + h) * kN + row0 + rr_;
+      Elem<TIn>::store(A.y + yi, ys[e]);
+    }
+    // the next iteration's first __syncthreads orders these reads of ys
+    // before the next tile's writes to it
+  }
+
+#pragma unroll
+  for (int m = 0; m < 4; ++m)
+    *reinterpret_cast<float4 *>(A.s_out + sbase + 16 * m + 4 * q) =
+        make_float4(s[4 * m + 0], s[4 * m + 1], s[4 * m + 2], s[4 * m + 3]);
+}
+
+template <typename TIn, int ROWS>
+static cudaError_t launch_scan_rows(const ScanArgs<TIn> &A, int B, cudaStream_t stream) {
+  using C = ScanCfg<TIn, ROWS>;
+  auto kern = wkv7_scan_kernel<TIn, ROWS>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(C::kSmemBytes));
+  if (e != cudaSuccess) return e;
+  dim3 grid(A.H * (kN / ROWS), B);
+  kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(A);
+  return cudaGetLastError();
+}
+
+template <typename TIn>
+cudaError_t launch_scan(const TIn *r, const TIn *w, const TIn *k, const TIn *v, const TIn *a, const TIn *b,
+                        const float *s_in, TIn *y, float *s_out, const int32_t *cu_seqlens, int B, int T,
+                        long long total_T, int H, cudaStream_t stream) {
+  ScanArgs<TIn> A{r, w, k, v, a, b, s_in, y, s_out, cu_seqlens, T, total_T, H};
+  return launch_scan_rows<TIn, 16>(A, B, stream);
+}
+
+template cudaError_t launch_scan<float>(const float *, const float *, const float *, const float *, const float *,
+                                        const float *, const float *, float *, float *, const int32_t *, int, int,
+                                        long long, int, cudaStream_t);
+template cudaError_t launch_scan<uint16_t>(const uint16_t *, const uint16_t *, const uint16_t *, const uint16_t *,
+                                           const uint16_t *, const uint16_t *, const float *, uint16_t *, float *,
+                                           const int32_t *, int, int, long long, int, cudaStream_t);
+
+}  // namespace rwkv7

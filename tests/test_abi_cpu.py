@@ -1,0 +1,107 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every entry point that include/rwkv7.h declares, and rejects bad arguments
+before launching anything (these calls return before any CUDA call)."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import rwkv_delta_rule_b200 as lib7
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "rwkv7.h")
+
+
+@pytest.fixture(scope="module")
+def cdll():
+    from rwkv_delta_rule_b200 import build
+
+    build.build()
+    return lib7.load_library()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"RWKV7_API\s+[\w\s\*]+?\b(rwkv7_\w+)\s*\(", text)))
+
+
+def test_header_declares_binding_names():
+    assert declared_symbols() == sorted(lib7.EXPORTED_SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol(cdll):
+    out = subprocess.run(["nm", "-D", "--defined-only", lib7.library_path()], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r" T (rwkv7_\w+)", out))
+    for sym in declared_symbols():
+        assert sym in exported, sym
+        assert hasattr(cdll, sym)
+    # nothing else leaks out (the CUDA runtime is linked statically and hidden)
+    assert all(s.startswith("rwkv7_") for s in re.findall(r" T (\w+)", out))
+
+
+def test_library_needs_no_shared_cuda_runtime():
+    out = subprocess.run(["ldd", lib7.library_path()], capture_output=True, text=True).stdout
+    assert "libcudart" not in out
+
+
+def test_status_strings(cdll):
+    assert lib7.rwkv7_status_string(0) == "ok"
+    assert "64" in lib7.rwkv7_status_string(5)
+    assert lib7.rwkv7_status_string(99) == "unknown status"
+    assert lib7.rwkv7_version() >= 100
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: every call below fails validation first
+MIS = 0x10008   # 8-byte aligned only
+
+
+def prefill_bf16(cdll, B=1, T=4, H=1, N=64, ptr=FAKE, s_out=FAKE, path=None):
+    args = [B, T, H, N] + [ptr] * 6 + [None, ptr, s_out, None]
+    if path is None:
+        return cdll.rwkv7_wkv_prefill_bf16(*args)
+    return cdll.rwkv7_wkv_prefill_bf16_path(path, *args)
+
+
+def test_rejects_head_size(cdll):
+    assert prefill_bf16(cdll, N=32) == 5
+    assert cdll.rwkv7_wkv_prefill(1, 4, 1, 128, *([FAKE] * 6), None, FAKE, FAKE, None) == 5
+    assert cdll.rwkv7_wkv_decode_bf16(1, 1, 63, *([FAKE] * 6), FAKE, FAKE, None) == 5
+
+
+def test_rejects_bad_sizes_and_nulls(cdll):
+    assert prefill_bf16(cdll, B=0) == 1
+    assert prefill_bf16(cdll, H=-1) == 1
+    assert prefill_bf16(cdll, T=-1) == 1
+    assert prefill_bf16(cdll, ptr=None) == 1
+    assert prefill_bf16(cdll, s_out=None) == 1
+    assert prefill_bf16(cdll, path=7) == 1
+    assert cdll.rwkv7_wkv_decode(0, 1, 64, *([FAKE] * 6), FAKE, FAKE, None) == 1
+    assert cdll.rwkv7_wkv_decode(1, 1, 64, *([FAKE] * 5), None, FAKE, FAKE, None) == 1
+
+
+def test_rejects_misaligned(cdll):
+    assert prefill_bf16(cdll, ptr=MIS) == 2
+    assert prefill_bf16(cdll, s_out=MIS) == 2
+    assert cdll.rwkv7_wkv_decode_bf16(1, 1, 64, *([FAKE] * 5), MIS, FAKE, FAKE, None) == 2
+
+
+def test_varlen_rejects(cdll):
+    base = [FAKE] * 6 + [None, FAKE, FAKE, None]
+    assert cdll.rwkv7_wkv_prefill_varlen_bf16(0, 2, 10, 8, 1, 64, None, *base) == 1  # no offsets
+    assert cdll.rwkv7_wkv_prefill_varlen_bf16(0, 2, 10, 8, 1, 64, MIS, *base) == 2
+    assert cdll.rwkv7_wkv_prefill_varlen_bf16(0, 2, 10, -1, 1, 64, FAKE, *base) == 1
+    assert cdll.rwkv7_wkv_prefill_varlen_bf16(9, 2, 10, 8, 1, 64, FAKE, *base) == 1
+    assert cdll.rwkv7_wkv_prefill_varlen_bf16(0, 2, 10, 8, 1, 32, FAKE, *base) == 5
+
+
+def test_binding_rejects_cpu_tensors():
+    import torch
+
+    x = torch.zeros(1, 2, 1, 64, dtype=torch.bfloat16)
+    s = torch.zeros(1, 1, 64, 64)
+    with pytest.raises(ValueError):
+        lib7.rwkv7_wkv_prefill_bf16(x, x, x, x, x, x, None, x, s)

@@ -333,37 +333,41 @@ def run_ours(args):
     tokens_per_step = B * T * world
     value = tokens_per_step * args.steps / (ms_total / 1e3)
 
-    # end to end through the C ABI with host buffers
-    host = {n: d[n].pin_memory() for n in OPS}
-    host_s0 = d["s0"].pin_memory()
-    host_y = torch.empty(y.shape, dtype=y.dtype).pin_memory()
-    host_s = torch.empty(s_out.shape, dtype=torch.float32).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in host.values()) + host_s0.numel() * 4
-    d2h = host_y.numel() * host_y.element_size() + host_s.numel() * 4
+    e2e = None
+    if not args.no_e2e:
+        # end to end through the C ABI with host buffers
+        host = {n: d[n].pin_memory() for n in OPS}
+        host_s0 = d["s0"].pin_memory()
+        host_y = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+        host_s = torch.empty(s_out.shape, dtype=torch.float32).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host.values()) + host_s0.numel() * 4
+        d2h = host_y.numel() * host_y.element_size() + host_s.numel() * 4
 
-    def e2e_step():
-        for n in OPS:
-            dd[n].copy_(host[n], non_blocking=True)
-        s0.copy_(host_s0, non_blocking=True)
-        step()
-        host_y.copy_(y, non_blocking=True)
-        host_s.copy_(s_out, non_blocking=True)
+        def e2e_step():
+            for n in OPS:
+                dd[n].copy_(host[n], non_blocking=True)
+            s0.copy_(host_s0, non_blocking=True)
+            step()
+            host_y.copy_(y, non_blocking=True)
+            host_s.copy_(s_out, non_blocking=True)
 
-    for _ in range(2):
-        e2e_step()
-    torch.cuda.synchronize()
-    k_e2e = max(3, min(args.steps, 20))
-    barrier(world)
-    torch.cuda.synchronize()
-    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a0.record(stream)
-    for _ in range(k_e2e):
-        e2e_step()
-    a1.record(stream)
-    torch.cuda.synchronize()
-    barrier(world)
-    e2e_ms = max_over_ranks(a0.elapsed_time(a1), world)
-    e2e_value = tokens_per_step * k_e2e / (e2e_ms / 1e3)
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        k_e2e = max(3, min(args.steps, 20))
+        barrier(world)
+        torch.cuda.synchronize()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(k_e2e):
+            e2e_step()
+        a1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        e2e_ms = max_over_ranks(a0.elapsed_time(a1), world)
+        e2e_value = tokens_per_step * k_e2e / (e2e_ms / 1e3)
+        e2e = {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "steps": k_e2e}
 
     peaks, peak_kind = load_peaks()
     algo = prefill_bytes(B, T, H)
@@ -374,7 +378,7 @@ def run_ours(args):
 
     decode = None
     if not args.no_decode:
-        decode = bench_decode(lib7, dev)
+        decode = bench_decode(lib7, dev, steps_target=args.decode_steps, layers=args.decode_layers)
         decode["frac"] = decode["achieved_gbs"] / peaks["hbm_gbs"]
         assert lib7.rwkv7_get_last_error() == 0
 
@@ -395,8 +399,7 @@ def run_ours(args):
                    "parallelism": f"replicas x{world} (batch-sharded, no exchange)",
                    "l2": "operands larger than L2 (355 MB per step vs 126 MB); no flush",
                    "path": args.path, "state": "float32 in/out"},
-        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "steps": k_e2e},
+        "e2e": e2e,
         "roofline": roofline,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks.summary(),
@@ -422,6 +425,9 @@ def main():
     ap.add_argument("--batch", type=int, default=0, help="override B (profiling runs only)")
     ap.add_argument("--seqlen", type=int, default=0, help="override T (profiling runs only)")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--decode-steps", type=int, default=1024)
+    ap.add_argument("--decode-layers", type=int, default=24, help="distinct decode states rotated over")
+    ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--ref-tokens", type=int, default=4096)

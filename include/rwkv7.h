@@ -75,8 +75,11 @@ typedef enum rwkv7_status {
   RWKV7_ERR_UNSUPPORTED = 5
 } rwkv7_status;
 
-/* Prefill kernels: AUTO picks by T and dtype; SCAN is the sequential kernel
- * (state in registers); CHUNK is the chunked tensor-core kernel (bf16 only). */
+/* Prefill kernels: AUTO picks by T and dtype (bf16 with T >= 128 -> CHUNK,
+ * otherwise SCAN); SCAN is the sequential kernel (state in registers); CHUNK
+ * is the chunked tensor-core kernel (bf16 only).  CHUNK requires every decay
+ * w >= 0.27 (it divides by products of up to 64 decays in float32); the
+ * model's decay exp(-e^-0.5 sigmoid(x)) always lies in [0.5452, 1). */
 typedef enum rwkv7_prefill_path {
   RWKV7_PATH_AUTO = 0,
   RWKV7_PATH_SCAN = 1,

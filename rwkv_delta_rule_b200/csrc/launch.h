@@ -19,4 +19,11 @@ template <typename TIn>
 cudaError_t launch_decode(const TIn *r, const TIn *w, const TIn *k, const TIn *v, const TIn *a, const TIn *b,
                           float *s, TIn *y, int B, int H, cudaStream_t stream);
 
+// Chunked tensor-core prefill (bfloat16 operands), same layouts as
+// launch_scan.  err_word: device word that bounded waits report into.
+cudaError_t launch_chunk(const uint16_t *r, const uint16_t *w, const uint16_t *k, const uint16_t *v,
+                         const uint16_t *a, const uint16_t *b, const float *s_in, uint16_t *y, float *s_out,
+                         const int32_t *cu_seqlens, int B, int T, long long total_T, int H, int *err_word,
+                         cudaStream_t stream);
+
 }  // namespace rwkv7

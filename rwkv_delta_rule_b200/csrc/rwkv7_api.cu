@@ -21,6 +21,26 @@ template <typename... P> bool none_null(const P *...ps) { return ((ps != nullptr
 
 rwkv7_status from_cuda(cudaError_t e) { return e == cudaSuccess ? RWKV7_OK : RWKV7_ERR_CUDA; }
 
+// Device address of the error word on the current device (looked up once per device).
+int *error_word_ptr() {
+  static int *cache[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+  if (dev >= 0 && dev < 64 && cache[dev] != nullptr) return cache[dev];
+  void *p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess) return nullptr;
+  if (dev >= 0 && dev < 64) cache[dev] = static_cast<int *>(p);
+  return static_cast<int *>(p);
+}
+
+// Kernel choice for bf16 prefill.  AUTO takes the chunked tensor-core kernel
+// once a sequence spans two chunks; shorter ones are latency-bound either way
+// and the sequential scan has no set-up cost.
+constexpr long long kChunkMinT = 128;
+bool use_chunk(int path, long long max_T) {
+  return path == RWKV7_PATH_CHUNK || (path == RWKV7_PATH_AUTO && max_T >= kChunkMinT);
+}
+
 // Checks shared by every prefill entry point.  `need_ops` is false when no
 // token is processed (T == 0), in which case operand pointers may be NULL.
 template <typename TIn>
@@ -84,9 +104,10 @@ rwkv7_status rwkv7_wkv_prefill_bf16_path(int path, int B, int T, int H, int N, c
   const rwkv7_status st = check_prefill(B, T, H, N, r, w, k, v, a, b, s_in, y, s_out);
   if (st != RWKV7_OK) return st;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  if (path == RWKV7_PATH_CHUNK) return RWKV7_ERR_UNSUPPORTED;  // chunked kernel not built yet
-  return from_cuda(launch_scan<uint16_t>(r, w, k, v, a, b, s_in, y, s_out, nullptr, B, T,
-                                         static_cast<long long>(B) * T, H, cs));
+  const long long total = static_cast<long long>(B) * T;
+  if (use_chunk(path, T))
+    return from_cuda(launch_chunk(r, w, k, v, a, b, s_in, y, s_out, nullptr, B, T, total, H, error_word_ptr(), cs));
+  return from_cuda(launch_scan<uint16_t>(r, w, k, v, a, b, s_in, y, s_out, nullptr, B, T, total, H, cs));
 }
 
 rwkv7_status rwkv7_wkv_prefill_bf16(int B, int T, int H, int N, const uint16_t *r, const uint16_t *w,
@@ -108,7 +129,9 @@ rwkv7_status rwkv7_wkv_prefill_varlen_bf16(int path, int B, int total_T, int max
   const rwkv7_status st = check_prefill(B, total_T, H, N, r, w, k, v, a, b, s_in, y, s_out);
   if (st != RWKV7_OK) return st;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  if (path == RWKV7_PATH_CHUNK) return RWKV7_ERR_UNSUPPORTED;  // chunked kernel not built yet
+  if (use_chunk(path, max_T))
+    return from_cuda(
+        launch_chunk(r, w, k, v, a, b, s_in, y, s_out, cu_seqlens, B, 0, total_T, H, error_word_ptr(), cs));
   return from_cuda(launch_scan<uint16_t>(r, w, k, v, a, b, s_in, y, s_out, cu_seqlens, B, 0, total_T, H, cs));
 }
 

@@ -15,7 +15,7 @@ import torch
 import oracle
 import rwkv_delta_rule_b200 as rk
 import wkv7_inputs as wi
-from helpers import OPS, TOL_BF16, TOL_F32, need_cuda, oracle_ops, rel_err, to_dev
+from helpers import OPS, TOL_BF16, TOL_BF16_PAIR, TOL_F32, need_cuda, oracle_ops, rel_err, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -44,14 +44,40 @@ def test_scan_f32_prefill_b1_t64_h2():
     assert rel_err(s, so) <= TOL_F32
 
 
-@pytest.mark.parametrize("T", [1, 2, 31, 32, 33, 63, 64, 65, 100, 257])
-def test_scan_bf16_ragged_tails(T):
+PATHS = [pytest.param(rk.RWKV7_PATH_SCAN, id="scan"), pytest.param(rk.RWKV7_PATH_CHUNK, id="chunk")]
+
+
+@pytest.mark.parametrize("path", PATHS)
+@pytest.mark.parametrize("T", [1, 2, 31, 32, 33, 63, 64, 65, 100, 127, 128, 129, 257])
+def test_bf16_ragged_tails(T, path):
     d = wi.draw(2, T, 3, seed=100 + T, dtype="bf16", s0_std=0.1)
     yo, so = oracle.wkv7(*oracle_ops(d), d["s0"])
     dd = to_dev(d)
-    y, s = gpu_prefill(dd, dd["s0"], rk.RWKV7_PATH_SCAN)
+    y, s = gpu_prefill(dd, dd["s0"], path)
     assert rel_err(y, yo) <= TOL_BF16
     assert rel_err(s, so) <= TOL_BF16
+
+
+@pytest.mark.parametrize("path", PATHS)
+@pytest.mark.parametrize("z_mean", [-3.0, 1.0, 3.0])
+def test_bf16_decay_regimes(z_mean, path):
+    """Slow (w ~ 0.97), fast (w ~ 0.65) and fastest (w ~ 0.56) decay."""
+    d = wi.draw(2, 700, 2, seed=int(20 + z_mean), dtype="bf16", z_mean=z_mean, s0_std=0.1)
+    yo, so = oracle.wkv7(*oracle_ops(d), d["s0"])
+    dd = to_dev(d)
+    y, s = gpu_prefill(dd, dd["s0"], path)
+    assert rel_err(y, yo) <= TOL_BF16
+    assert rel_err(s, so) <= TOL_BF16
+
+
+def test_chunk_matches_scan_elementwise():
+    """The two kernels agree with each other on every element (both fp32-state)."""
+    d = wi.draw(3, 640, 4, seed=33, dtype="bf16", s0_std=0.1)
+    dd = to_dev(d)
+    yc, sc = gpu_prefill(dd, dd["s0"], rk.RWKV7_PATH_CHUNK)
+    ys, ss = gpu_prefill(dd, dd["s0"], rk.RWKV7_PATH_SCAN)
+    assert rel_err(yc, ys.float().cpu().numpy()) <= TOL_BF16_PAIR
+    assert rel_err(sc, ss.cpu().numpy()) <= 1e-3
 
 
 def test_scan_f32_longer_with_state():
@@ -63,46 +89,39 @@ def test_scan_f32_longer_with_state():
     assert rel_err(s, so) <= TOL_F32
 
 
-def test_slow_decay_bf16():
-    """z ~ N(-3, 1): w ~ 0.97, long memory."""
-    d = wi.draw(2, 700, 2, seed=8, dtype="bf16", z_mean=-3.0, s0_std=0.1)
-    yo, so = oracle.wkv7(*oracle_ops(d), d["s0"])
-    dd = to_dev(d)
-    y, s = gpu_prefill(dd, dd["s0"], rk.RWKV7_PATH_SCAN)
-    assert rel_err(y, yo) <= TOL_BF16
-    assert rel_err(s, so) <= TOL_BF16
-
-
-def test_t_zero_copies_state():
+@pytest.mark.parametrize("path", PATHS)
+def test_t_zero_copies_state(path):
     d = wi.draw(2, 0, 3, seed=9, dtype="bf16", s0_std=0.1)
     dd = to_dev(d)
-    y, s = gpu_prefill(dd, dd["s0"])
+    y, s = gpu_prefill(dd, dd["s0"], path)
     assert torch.equal(s, dd["s0"])
-    y, s = gpu_prefill(dd, None)
+    y, s = gpu_prefill(dd, None, path)
     assert torch.count_nonzero(s) == 0
 
 
-def test_in_place_state():
-    d = wi.draw(1, 45, 2, seed=10, dtype="bf16", s0_std=0.1)
+@pytest.mark.parametrize("path", PATHS)
+def test_in_place_state(path):
+    d = wi.draw(1, 145, 2, seed=10, dtype="bf16", s0_std=0.1)
     yo, so = oracle.wkv7(*oracle_ops(d), d["s0"])
     dd = to_dev(d)
     st = dd["s0"].clone()
     y = torch.empty_like(dd["r"])
-    rk.rwkv7_wkv_prefill_bf16(*[dd[n] for n in OPS], st, y, st)
+    rk.rwkv7_wkv_prefill_bf16_path(path, *[dd[n] for n in OPS], st, y, st)
     torch.cuda.synchronize()
     assert rel_err(y, yo) <= TOL_BF16
     assert rel_err(st, so) <= TOL_BF16
 
 
-def test_chained_calls_equal_one_call():
-    d = wi.draw(2, 130, 2, seed=11, dtype="bf16", s0_std=0.1)
+@pytest.mark.parametrize("path", PATHS)
+def test_chained_calls_equal_one_call(path):
+    d = wi.draw(2, 230, 2, seed=11, dtype="bf16", s0_std=0.1)
     yo, so = oracle.wkv7(*oracle_ops(d), d["s0"])
     dd = to_dev(d)
     s = dd["s0"]
     ys = []
-    for lo, hi in ((0, 1), (1, 64), (64, 65), (65, 130)):
+    for lo, hi in ((0, 1), (1, 64), (64, 65), (65, 130), (130, 230)):
         part = {n: dd[n][:, lo:hi].contiguous() for n in OPS}
-        yp, s = gpu_prefill(part, s)
+        yp, s = gpu_prefill(part, s, path)
         ys.append(yp)
     assert rel_err(torch.cat(ys, 1), yo) <= TOL_BF16
     assert rel_err(s, so) <= TOL_BF16
@@ -124,15 +143,16 @@ def test_decode_steps_equal_oracle(dtype):
     assert rel_err(st, so) <= tol
 
 
-def test_varlen_small():
-    lens = torch.tensor([1, 0, 33, 64, 65, 7])
+@pytest.mark.parametrize("path", PATHS)
+def test_varlen_small(path):
+    lens = torch.tensor([1, 0, 33, 64, 65, 7, 200])
     d = wi.draw_packed(lens, 3, seed=13, s0_std=0.1)
     cu = d["cu_seqlens"]
     yo, so = oracle.wkv7_varlen(*oracle_ops(d), cu, d["s0"])
     dd = to_dev(d)
     y = torch.empty_like(dd["r"])
     s = torch.empty_like(dd["s0"])
-    rk.rwkv7_wkv_prefill_varlen_bf16(rk.RWKV7_PATH_AUTO, cu.cuda(), int(lens.max()), *[dd[n] for n in OPS],
+    rk.rwkv7_wkv_prefill_varlen_bf16(path, cu.cuda(), int(lens.max()), *[dd[n] for n in OPS],
                                      dd["s0"], y, s)
     torch.cuda.synchronize()
     assert rel_err(y, yo) <= TOL_BF16
@@ -163,10 +183,10 @@ def test_full_prefill_d768_b8_t4096():
     case = wi.CASES["prefill_d768_b8_t4096"]
     d = wi.draw_case(case)
     dd = to_dev(d)
-    y, s = gpu_prefill(dd, dd["s0"])
+    y, s = gpu_prefill(dd, dd["s0"], rk.RWKV7_PATH_CHUNK)
     check_pairs(d, d["s0"], y.cpu(), s.cpu(), sampled_pairs(case.B, case.H, 6, 1), TOL_BF16)
     ys, ss = gpu_prefill(dd, dd["s0"], rk.RWKV7_PATH_SCAN)
-    assert rel_err(y, ys.float().cpu().numpy()) <= TOL_BF16
+    assert rel_err(y, ys.float().cpu().numpy()) <= TOL_BF16_PAIR
     assert rel_err(s, ss.cpu().numpy()) <= TOL_BF16
 
 
@@ -197,11 +217,16 @@ def test_full_decode_l24_d1024_equals_prefill():
         rk.rwkv7_wkv_decode_bf16(*[steps[n][t] for n in OPS], st, y[t])
     torch.cuda.synchronize()
     y = y.transpose(0, 1)
-    yp, sp = gpu_prefill(dd, None, rk.RWKV7_PATH_SCAN)
-    # decode == prefill on every element (both float32-state GPU paths)
-    assert rel_err(y, yp.float().cpu().numpy()) <= TOL_BF16
-    assert rel_err(st, sp.cpu().numpy()) <= 1e-4
-    check_pairs(d, None, y.cpu(), st.cpu(), sampled_pairs(case.B, case.H, 4, 3), TOL_BF16)
+    pairs = sampled_pairs(case.B, case.H, 4, 3)
+    check_pairs(d, None, y.cpu(), st.cpu(), pairs, TOL_BF16)
+    # decode == prefill on every element, for both prefill kernels; each
+    # prefill also against the oracle on the sampled pairs
+    for path, tol_s in ((rk.RWKV7_PATH_SCAN, 1e-4), (rk.RWKV7_PATH_CHUNK, 2e-3)):
+        yp, sp = gpu_prefill(dd, None, path)
+        assert rel_err(y, yp.float().cpu().numpy()) <= TOL_BF16_PAIR
+        assert rel_err(st, sp.cpu().numpy()) <= tol_s
+        check_pairs(d, None, yp.cpu(), sp.cpu(), pairs, TOL_BF16)
+        del yp, sp
 
 
 @pytest.mark.slow

@@ -156,13 +156,9 @@ def dist_setup():
 
 
 def max_over_ranks(x: float, world: int) -> float:
-    if world == 1:
-        return x
-    import torch.distributed as dist
+    from rwkv_delta_rule_b200.dist import max_over_ranks as _max
 
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    return x if world == 1 else _max(x)
 
 
 def barrier(world: int):
@@ -294,7 +290,9 @@ def run_ours(args):
     B = args.batch or case.B
     T = args.seqlen or case.T
     H = case.H
-    d = wi.draw(B, T, H, seed=case.seed + 7919 * rank, dtype="bf16", s0_std=case.s0_std)
+    from rwkv_delta_rule_b200.dist import rank_seed
+
+    d = wi.draw(B, T, H, seed=rank_seed(case.seed, rank), dtype="bf16", s0_std=case.s0_std)
     dd = {n: d[n].to(dev) for n in OPS}
     s0 = d["s0"].to(dev)
     y = torch.empty_like(dd["r"])

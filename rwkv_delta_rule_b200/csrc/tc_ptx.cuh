@@ -184,3 +184,60 @@ __device__ __forceinline__ uint32_t to_tf32(float x) {
 
 }  // namespace tc
 }  // namespace rwkv7
+
+namespace rwkv7 {
+namespace tc {
+
+// Approximate reciprocal (one MUFU op, about 1 ulp; denormals flushed).
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;\n" : "=f"(r) : "f"(x));
+  return r;
+}
+
+// Warp-level tf32 MMA (m16n8k8, row.col), accumulating into d.
+__device__ __forceinline__ void mma_m16n8k8_tf32(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// acc (16x16, two 16x8 n-tiles in mma C layout) += A (16x16 row-major at ap,
+// row stride lda) * B (16x16 row-major at bp, row stride ldb); float32 in
+// shared memory, rounded to tf32 on load.
+__device__ __forceinline__ void block16_mma(float (&acc)[2][4], const float *ap, int lda, const float *bp, int ldb,
+                                            int lane) {
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int kt = 0; kt < 2; ++kt) {
+    uint32_t a[4];
+    a[0] = to_tf32(ap[g * lda + 8 * kt + t]);
+    a[1] = to_tf32(ap[(g + 8) * lda + 8 * kt + t]);
+    a[2] = to_tf32(ap[g * lda + 8 * kt + t + 4]);
+    a[3] = to_tf32(ap[(g + 8) * lda + 8 * kt + t + 4]);
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      uint32_t b[2];
+      b[0] = to_tf32(bp[(8 * kt + t) * ldb + 8 * nt + g]);
+      b[1] = to_tf32(bp[(8 * kt + t + 4) * ldb + 8 * nt + g]);
+      mma_m16n8k8_tf32(acc[nt], a, b);
+    }
+  }
+}
+
+// Stores a 16x16 mma-layout accumulator to a row-major float32 block.
+__device__ __forceinline__ void block16_store(float *dst, int ld, const float (&acc)[2][4], int lane) {
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt) {
+    dst[g * ld + 8 * nt + 2 * t] = acc[nt][0];
+    dst[g * ld + 8 * nt + 2 * t + 1] = acc[nt][1];
+    dst[(g + 8) * ld + 8 * nt + 2 * t] = acc[nt][2];
+    dst[(g + 8) * ld + 8 * nt + 2 * t + 1] = acc[nt][3];
+  }
+}
+
+}  // namespace tc
+}  // namespace rwkv7

@@ -53,23 +53,28 @@ constexpr uint32_t TM_D4 = 320;  // 64 cols: Y (lanes 0-63), X (lanes 64-127)
 constexpr uint32_t TM_A2 = 384;  // 64 cols: Mrb (lanes 0-63), B-^T (lanes 64-127)
 
 // shared memory map (bytes from a 1024-aligned base)
-constexpr uint32_t kTile = C * kN * 2;           // one bf16 64x64 tile
-constexpr uint32_t OFF_RAW = 0;                  // r w k a b v tiles, row-major [token][channel]
-constexpr uint32_t OFF_A1 = OFF_RAW + 6 * kTile; // tf32 K-major 128x64 (32 KB); later B3 + Lab
-constexpr uint32_t OFF_B1 = OFF_A1 + 32768;      // tf32 K-major 128x64 (32 KB); later Tinv, then B2
-constexpr uint32_t OFF_A3 = OFF_B1 + 32768;      // bf16 MN-major M=128 x K=64 (16 KB)
-constexpr uint32_t OFF_B4 = OFF_A3 + 16384;      // tf32 K-major N=64 (value i) x K=128 (key j | token m) (32 KB)
-constexpr uint32_t OFF_MISC = OFF_B4 + 32768;
-constexpr uint32_t OFF_B3 = OFF_A1;              // bf16 K-major 64x64 (8 KB)
-constexpr uint32_t OFF_LS = OFF_A1 + 8192;       // float [64][65]  (Lab, strictly lower)
-constexpr uint32_t OFF_TS = OFF_B1;              // float [64][65]  (Tinv in float32)
-constexpr uint32_t OFF_ZS = OFF_B1 + 64 * 65 * 4;  // float [3][16][17]
-constexpr uint32_t OFF_B2 = OFF_B1;              // tf32 K-major 128x64 (32 KB)
-constexpr uint32_t kSmemBytes = OFF_MISC + 2048 + 1024;  // + misc + alignment slack
-constexpr int LDS = 65;                          // padded row stride of Ls / Ts
+constexpr uint32_t kTile = C * kN * 2;            // one bf16 64x64 tile
+constexpr uint32_t OFF_RAW = 0;                   // r w k a b v tiles, row-major [token][channel]
+constexpr uint32_t OFF_A1 = OFF_RAW + 6 * kTile;  // tf32 K-major [R~; A~] 128x64 (32 KB)
+constexpr uint32_t OFF_B1 = OFF_A1 + 32768;       // tf32 K-major [B^; K^] 128x64 (32 KB)
+constexpr uint32_t OFF_A3 = OFF_B1 + 32768;       // bf16 MN-major [A~^T; Lak^T], M=128 x K=64 (16 KB)
+constexpr uint32_t OFF_B4S = OFF_A3 + 16384;      // tf32 K-major S0^T part of the chain B: row i, K = j (16 KB)
+constexpr uint32_t OFF_B4V = OFF_B4S + 16384;     // tf32 K-major V part of the chain B: row i, K = m (16 KB)
+constexpr uint32_t OFF_MISC = OFF_B4V + 16384;
+// regions reused once MMA1 has consumed A1 / B1
+constexpr int LDL = 68;                           // row stride (floats) of Lab: conflict-free as an mma A operand
+constexpr int LDT = 72;                           // row stride (floats) of Tinv: conflict-free as an mma B operand
+constexpr uint32_t OFF_LS = OFF_A1;               // float [64][LDL]
+constexpr uint32_t OFF_ZS = OFF_A1 + 64 * LDL * 4;  // float [3 warps][16][24]
+constexpr uint32_t OFF_B2 = OFF_A1;               // tf32 K-major [W~ U~]^T 128x64 (after the inverse)
+constexpr uint32_t OFF_TS = OFF_B1;               // float [64][LDT]
+constexpr uint32_t OFF_B3 = OFF_B1 + 19456;       // bf16 K-major Tinv 64x64 (8 KB), 1024-aligned
+constexpr uint32_t MISC_GC = 256;                 // float [64]   Gamma at the chunk end
+constexpr uint32_t MISC_TOT = 512;                // float [16][64] per-token-group decay products
+constexpr uint32_t kSmemBytes = OFF_MISC + MISC_TOT + 16 * 64 * 4 + 1024;
 
-static_assert(OFF_LS + 64 * LDS * 4 <= OFF_B1, "Lab scratch overflows its region");
-static_assert(OFF_ZS + 3 * 16 * 17 * 4 <= OFF_A3, "Tinv scratch overflows its region");
+static_assert(OFF_ZS + 3 * 16 * 24 * 4 <= OFF_B1, "inverse scratch overflows A1");
+static_assert(OFF_TS + 64 * LDT * 4 <= OFF_B3 && OFF_B3 + 8192 <= OFF_A3, "inverse scratch overflows B1");
 
 struct Maps {
   CUtensorMap m[6];  // r, w, k, a, b, v: dims {64, H, tokens}, box {64, 1, 64}
@@ -88,53 +93,55 @@ struct Args {
 
 enum { RAW_R = 0, RAW_W = 1, RAW_K = 2, RAW_A = 3, RAW_B = 4, RAW_V = 5 };
 
-// address helpers (byte offsets inside a region)
+// byte offset of element (row, k) in a K-major tf32 operand with `rows` rows
 __device__ __forceinline__ uint32_t kmaj_tf32(uint32_t rows, uint32_t row, uint32_t k) {
   return (k >> 5) * (rows * 128u) + tc::sw128(row, (k & 31u) >> 2) + (k & 3u) * 4u;
 }
+// byte offset of element (k, mn) in an MN-major bf16 operand with `krows` K rows
 __device__ __forceinline__ uint32_t mnmaj_bf16(uint32_t krows, uint32_t k, uint32_t mn) {
   return (mn >> 6) * (krows * 128u) + tc::sw128(k, (mn & 63u) >> 3) + (mn & 7u) * 2u;
 }
 
-__device__ __forceinline__ float raw_at(const uint16_t *raw, int tile, int t, int j) {
-  return bf16_bits_to_float(raw[tile * (C * kN) + t * kN + j]);
+// four consecutive bf16 channels of one token row of a raw tile
+__device__ __forceinline__ void raw4(const uint8_t *smem, int tile, int t, int j0, float (&o)[4]) {
+  const uint2 u = *reinterpret_cast<const uint2 *>(smem + OFF_RAW + tile * kTile + (t * kN + j0) * 2);
+  o[0] = __uint_as_float(u.x << 16);
+  o[1] = __uint_as_float(u.x & 0xffff0000u);
+  o[2] = __uint_as_float(u.y << 16);
+  o[3] = __uint_as_float(u.y & 0xffff0000u);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return static_cast<uint32_t>(float_to_bf16_bits(lo)) | (static_cast<uint32_t>(float_to_bf16_bits(hi)) << 16);
 }
 
+__device__ __forceinline__ void st_tf32x4(uint8_t *p, float a, float b, float c, float d) {
+  *reinterpret_cast<uint4 *>(p) = make_uint4(tc::to_tf32(a), tc::to_tf32(b), tc::to_tf32(c), tc::to_tf32(d));
+}
+
 // Writes 32 consecutive float32 values as tf32 into one 128-byte swizzled row.
 __device__ __forceinline__ void store_row_tf32(uint8_t *region_row_block, uint32_t row, const float (&v)[32]) {
 #pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    uint4 q;
-    q.x = tc::to_tf32(v[4 * c + 0]);
-    q.y = tc::to_tf32(v[4 * c + 1]);
-    q.z = tc::to_tf32(v[4 * c + 2]);
-    q.w = tc::to_tf32(v[4 * c + 3]);
-    *reinterpret_cast<uint4 *>(region_row_block + tc::sw128(row, c)) = q;
-  }
+  for (int c = 0; c < 8; ++c)
+    st_tf32x4(region_row_block + tc::sw128(row, c), v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
 }
 
-// B4 holds [S0^T; V] as the K-major B operand of the chain product: row n is
-// the value channel i, K runs over key channels j (0..63) then tokens m
-// (64..127).  A channel thread owns S^T[j][32*ch + x] = S[32*ch + x][j], i.e.
-// column K = j of rows 32*ch .. 32*ch+31.
-__device__ __forceinline__ void store_state_tf32(uint8_t *sB4, int j, int ch, const float (&st)[32]) {
+// B4S holds S0^T as the K-major B operand of the chain product: row = value
+// channel i, K = key channel j.  A state thread owns S^T[j][32*ch + x].
+__device__ __forceinline__ void store_state_tf32(uint8_t *sB4S, int j, int ch, const float (&st)[32]) {
 #pragma unroll
   for (int x = 0; x < 32; ++x)
-    *reinterpret_cast<uint32_t *>(sB4 + kmaj_tf32(64, 32 * ch + x, j)) = tc::to_tf32(st[x]);
+    *reinterpret_cast<uint32_t *>(sB4S + kmaj_tf32(64, 32 * ch + x, j)) = tc::to_tf32(st[x]);
 }
 
 __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_constant__ Maps maps, const Args A) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const uint16_t *raw = reinterpret_cast<const uint16_t *>(smem + OFF_RAW);
   uint8_t *sA1 = smem + OFF_A1;
   uint8_t *sB1 = smem + OFF_B1;
   uint8_t *sA3 = smem + OFF_A3;
-  uint8_t *sB4 = smem + OFF_B4;
+  uint8_t *sB4S = smem + OFF_B4S;
+  uint8_t *sB4V = smem + OFF_B4V;
   uint8_t *sB3 = smem + OFF_B3;
   uint8_t *sB2 = smem + OFF_B2;
   float *Ls = reinterpret_cast<float *>(smem + OFF_LS);
@@ -144,20 +151,24 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
   uint64_t *bar_mma = bar_tma + 1;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_MISC + 16);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 20);
-  float *gtot = reinterpret_cast<float *>(smem + OFF_MISC + 64);  // [2][64]
+  float *GCs = reinterpret_cast<float *>(smem + OFF_MISC + MISC_GC);
+  float *tot = reinterpret_cast<float *>(smem + OFF_MISC + MISC_TOT);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int q = warp & 3;    // TMEM lane quadrant of this warp
-  const int ch = warp >> 2;  // which half of the columns this warp handles
+  const int ch = warp >> 2;  // which half of a 64-column block this warp handles
   const int h = blockIdx.x;
   const int bidx = blockIdx.y;
   const SeqBounds sb = seq_bounds(A.cu_seqlens, bidx, A.T, A.total_T);
   if (sb.len < 0) return;
   const int nchunks = (sb.len + C - 1) / C;
-  const bool chan_thread = q >= 2;          // channel-major role (owns TMEM lanes 64..127)
-  const int j = tid & 63;                   // channel of a channel-major thread
+  const bool hi_lanes = q >= 2;  // owns TMEM lanes 64..127
+  const int j = tid & 63;        // for hi-lane threads: the key channel of its lane
   const long long pair = static_cast<long long>(bidx) * A.H + h;
+  // operand-construction layout: 4 channels x 4 tokens per thread
+  const int cq = 8 * (warp & 1) + (lane & 7), tg = 4 * (warp >> 1) + (lane >> 3);
+  const int j0 = 4 * cq, t0 = 4 * tg;
 
   if (tid == 0) {
     tc::mbar_init(bar_tma, 1);
@@ -176,13 +187,13 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
   const uint32_t tmem = *tmem_slot;
   const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
 
-  // state: channel threads hold S^T[j][32*ch .. 32*ch+31] in float32
+  // state: hi-lane threads hold S^T[j][32*ch .. 32*ch+31] in float32
   float st[32];
-  if (chan_thread) {
+  if (hi_lanes) {
 #pragma unroll
     for (int x = 0; x < 32; ++x)
       st[x] = A.s_in ? A.s_in[pair * (kN * kN) + static_cast<long long>(32 * ch + x) * kN + j] : 0.f;
-    store_state_tf32(sB4, j, ch, st);
+    store_state_tf32(sB4S, j, ch, st);
   }
 
   uint32_t tma_phase = 0, mma_phase = 0;
@@ -206,7 +217,7 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
 
   for (int c = 0; c < nchunks; ++c) {
     const int Lc = min(C, sb.len - c * C);
-    // ---- P0: this chunk's tiles have landed --------------------------------------------
+    // ---- this chunk's tiles have landed ---------------------------------------------------
     if (tid == 0) {
       if (!tc::mbar_wait_bounded(bar_tma, tma_phase, kMaxPolls)) {
         *abort_flag = 1;
@@ -219,71 +230,121 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
     __syncthreads();
     if (*abort_flag) break;
 
-    // ---- P1: decay products and operands ------------------------------------------------
-    float G[32];   // channel threads: local cumulative products of w over their 32 tokens
-    float GC = 1.f;
-    if (chan_thread) {
-      const int t0 = 32 * ch;
-      float p = 1.f;
+    // ---- P1: decay products and operands (4 channels x 4 tokens per thread) ---------------
+    float G[4][4];  // Gamma_t for t = t0..t0+3 (rows) and channels j0..j0+3 (cols)
+    {
+      float wv[4][4];
 #pragma unroll
-      for (int tt = 0; tt < 32; ++tt) {
-        const int t = t0 + tt;
-        const float wv = t < Lc ? raw_at(raw, RAW_W, t, j) : 1.f;
-        p *= wv;
-        G[tt] = p;
+      for (int tt = 0; tt < 4; ++tt) {
+        if (t0 + tt < Lc) {
+          raw4(smem, RAW_W, t0 + tt, j0, wv[tt]);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) wv[tt][e] = 1.f;
+        }
       }
-      gtot[ch * 64 + j] = p;
-    } else {
-      // V (token m, value channel i) -> B4 element (row i, K = 64 + m); bf16 is exact in tf32.
-      // Lanes walk the 32 channels in a rotated order to spread shared-memory banks.
-      const int rid = (ch * 64) + q * 32 + lane;  // 0..127
-      const int m = rid & 63, ih = rid >> 6;
-#pragma unroll 8
-      for (int x = 0; x < 32; ++x) {
-        const int i = 32 * ih + ((x + lane) & 31);
-        const float vv = m < Lc ? raw_at(raw, RAW_V, m, i) : 0.f;
-        *reinterpret_cast<uint32_t *>(sB4 + kmaj_tf32(64, i, 64 + m)) = __float_as_uint(vv);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        G[0][e] = wv[0][e];
+        G[1][e] = G[0][e] * wv[1][e];
+        G[2][e] = G[1][e] * wv[2][e];
+        G[3][e] = G[2][e] * wv[3][e];
       }
+      *reinterpret_cast<float4 *>(tot + tg * 64 + j0) = make_float4(G[3][0], G[3][1], G[3][2], G[3][3]);
     }
     __syncthreads();
-    if (chan_thread) {
-      const float g0 = gtot[j], g1 = gtot[64 + j];
-      GC = g0 * g1;
-      const float pre = ch ? g0 : 1.f;
-      float Bbar[32], Kbar[32];
+    {
+      float pre[4] = {1.f, 1.f, 1.f, 1.f};
 #pragma unroll
-      for (int tt = 0; tt < 32; ++tt) {
-        const int t = 32 * ch + tt;
-        const bool valid = t < Lc;
-        const float Gt = pre * G[tt];
-        const float Gp = tt == 0 ? pre : pre * G[tt - 1];
-        const float rv = valid ? raw_at(raw, RAW_R, t, j) : 0.f;
-        const float kv = valid ? raw_at(raw, RAW_K, t, j) : 0.f;
-        const float av = valid ? raw_at(raw, RAW_A, t, j) : 0.f;
-        const float bv = valid ? raw_at(raw, RAW_B, t, j) : 0.f;
-        const float inv = __frcp_rn(Gt);
-        const float At = av * Gp;
-        *reinterpret_cast<uint32_t *>(sA1 + kmaj_tf32(128, t, j)) = tc::to_tf32(rv * Gt);
-        *reinterpret_cast<uint32_t *>(sA1 + kmaj_tf32(128, 64 + t, j)) = tc::to_tf32(At);
-        *reinterpret_cast<uint32_t *>(sB1 + kmaj_tf32(128, t, j)) = tc::to_tf32(bv * inv);
-        *reinterpret_cast<uint32_t *>(sB1 + kmaj_tf32(128, 64 + t, j)) = tc::to_tf32(kv * inv);
-        *reinterpret_cast<uint16_t *>(sA3 + mnmaj_bf16(64, t, j)) = float_to_bf16_bits(At);
-        const float ratio = GC * inv;
-        Bbar[tt] = bv * ratio;
-        Kbar[tt] = kv * ratio;
+      for (int g = 0; g < 15; ++g) {
+        if (g < tg) {
+          const float4 u = *reinterpret_cast<const float4 *>(tot + g * 64 + j0);
+          pre[0] *= u.x;
+          pre[1] *= u.y;
+          pre[2] *= u.z;
+          pre[3] *= u.w;
+        }
       }
-      float zeros[32];
+      float rr[4][4], kk[4][4], aa[4][4], bb[4][4], vv[4][4];
 #pragma unroll
-      for (int x = 0; x < 32; ++x) zeros[x] = 0.f;
-      tc::tmem_st32(tmem + lane_base + TM_A2 + 32 * ch, Bbar);
-      tc::tmem_st32(tmem + lane_base + TM_D2 + 64 + 32 * ch, Kbar);
-      tc::tmem_st32(tmem + lane_base + TM_D2 + 32 * ch, zeros);
-      tc::tmem_st_wait();
+      for (int tt = 0; tt < 4; ++tt) {
+        if (t0 + tt < Lc) {
+          raw4(smem, RAW_R, t0 + tt, j0, rr[tt]);
+          raw4(smem, RAW_K, t0 + tt, j0, kk[tt]);
+          raw4(smem, RAW_A, t0 + tt, j0, aa[tt]);
+          raw4(smem, RAW_B, t0 + tt, j0, bb[tt]);
+          raw4(smem, RAW_V, t0 + tt, j0, vv[tt]);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) rr[tt][e] = kk[tt][e] = aa[tt][e] = bb[tt][e] = vv[tt][e] = 0.f;
+        }
+      }
+      float Gp[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) Gp[e] = pre[e];  // Gamma_{t0 - 1}
+#pragma unroll
+      for (int tt = 0; tt < 4; ++tt) {
+        const int t = t0 + tt;
+        float Gt[4], inv[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          Gt[e] = pre[e] * G[tt][e];
+          inv[e] = tc::rcp_approx(Gt[e]);
+        }
+        const uint32_t kofs = (j0 >> 5) * (128 * 128) + ((j0 & 31) >> 2);  // katom base + chunk index
+        uint8_t *a1r = sA1 + (j0 >> 5) * (128 * 128);
+        uint8_t *b1r = sB1 + (j0 >> 5) * (128 * 128);
+        const uint32_t chunk = (j0 & 31) >> 2;
+        (void)kofs;
+        st_tf32x4(a1r + tc::sw128(t, chunk), rr[tt][0] * Gt[0], rr[tt][1] * Gt[1], rr[tt][2] * Gt[2],
+                  rr[tt][3] * Gt[3]);
+        const float At0 = aa[tt][0] * Gp[0], At1 = aa[tt][1] * Gp[1], At2 = aa[tt][2] * Gp[2],
+                    At3 = aa[tt][3] * Gp[3];
+        st_tf32x4(a1r + tc::sw128(64 + t, chunk), At0, At1, At2, At3);
+        st_tf32x4(b1r + tc::sw128(t, chunk), bb[tt][0] * inv[0], bb[tt][1] * inv[1], bb[tt][2] * inv[2],
+                  bb[tt][3] * inv[3]);
+        st_tf32x4(b1r + tc::sw128(64 + t, chunk), kk[tt][0] * inv[0], kk[tt][1] * inv[1], kk[tt][2] * inv[2],
+                  kk[tt][3] * inv[3]);
+        // A3: A~^T as the MN-major bf16 A operand of MMA3 (M = channel, K = token)
+        *reinterpret_cast<uint2 *>(sA3 + mnmaj_bf16(64, t, j0)) =
+            make_uint2(pack_bf16x2(At0, At1), pack_bf16x2(At2, At3));
+#pragma unroll
+        for (int e = 0; e < 4; ++e) Gp[e] = Gt[e];
+      }
+      if (tg == 15) *reinterpret_cast<float4 *>(GCs + j0) = make_float4(Gp[0], Gp[1], Gp[2], Gp[3]);
+      // V -> B4V (row = value channel, K = token), bf16 values are exact in tf32
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        *reinterpret_cast<uint4 *>(sB4V + kmaj_tf32(64, j0 + e, t0)) =
+            make_uint4(__float_as_uint(vv[0][e]), __float_as_uint(vv[1][e]), __float_as_uint(vv[2][e]),
+                       __float_as_uint(vv[3][e]));
     }
     tc::fence_proxy_async_smem();
     __syncthreads();
-    if (!chan_thread) {
-      // Q-part init of D2: row t gets R~[t][32ch .. 32ch+31], read back from A1
+
+    // ---- MMA1 (tf32): D1 = [R~; A~] [B^; K^]^T, and the next chunk's tiles ---------------------
+    if (tid == 0) {
+      if (c + 1 < nchunks) {
+        tc::mbar_arrive_expect_tx(bar_tma, 6 * kTile);
+        for (int i = 0; i < 6; ++i)
+          tc::tma_load_3d(smem + OFF_RAW + i * kTile, &maps.m[i], bar_tma, 0, h,
+                          static_cast<int>(sb.start + static_cast<long long>(c + 1) * C));
+        tma_pending = true;
+      }
+      tc::tc_fence_after();
+      constexpr uint32_t idesc = tc::instr_desc(tc::kFmtTF32, 128, 128, false, false);
+      const uint32_t a0 = smem_u32(sA1), b0 = smem_u32(sB1);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        const uint32_t off = (ks >> 2) * (128 * 128) + (ks & 3) * 32;
+        tc::mma_ss(1, tmem + TM_D1, tc::smem_desc(a0 + off, 16, 1024), tc::smem_desc(b0 + off, 16, 1024), idesc,
+                   ks > 0);
+      }
+      tc::mma_commit(bar_mma);
+    }
+    // D2 and A2 set-up from the operands (overlaps MMA1, which only reads A1 / B1)
+    if (!hi_lanes) {
+      // lanes t = 0..63: Q-part of D2 starts at R~[t][32ch .. 32ch+31] (read back from A1)
       const int t = q * 32 + lane;
       float rt[32];
       const uint8_t *rowblk = sA1 + ch * (128 * 128);
@@ -296,45 +357,36 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
         rt[4 * cc + 3] = __uint_as_float(u.w);
       }
       tc::tmem_st32(tmem + lane_base + TM_D2 + 32 * ch, rt);
-      tc::tmem_st_wait();
-    }
-    tc::tc_fence_before();
-    __syncthreads();
-
-    // ---- MMA1 (tf32): D1 = [R~; A~] [B^; K^]^T ----------------------------------------------
-    if (tid == 0) {
-      tc::tc_fence_after();
-      // the raw tiles are consumed: prefetch the next chunk
-      if (c + 1 < nchunks) {
-        tc::mbar_arrive_expect_tx(bar_tma, 6 * kTile);
-        for (int i = 0; i < 6; ++i)
-          tc::tma_load_3d(smem + OFF_RAW + i * kTile, &maps.m[i], bar_tma, 0, h,
-                          static_cast<int>(sb.start + static_cast<long long>(c + 1) * C));
-        tma_pending = true;
-      }
-      constexpr uint32_t idesc = tc::instr_desc(tc::kFmtTF32, 128, 128, false, false);
-      const uint32_t a0 = smem_u32(sA1), b0 = smem_u32(sB1);
+    } else {
+      // lanes 64+j: B-^T[j][m] = Gamma_C[j] B^[m][j] -> A2; K-^T[j][m] = Gamma_C[j] K^[m][j] -> F-part of D2
+      const float gc = GCs[j];
+      float bv[32], kv[32], zero[32];
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        const uint32_t off = (ks >> 2) * (128 * 128) + (ks & 3) * 32;
-        tc::mma_ss(1, tmem + TM_D1, tc::smem_desc(a0 + off, 16, 1024), tc::smem_desc(b0 + off, 16, 1024), idesc,
-                   ks > 0);
+      for (int x = 0; x < 32; ++x) {
+        const int m = 32 * ch + x;
+        bv[x] = gc * __uint_as_float(*reinterpret_cast<const uint32_t *>(sB1 + kmaj_tf32(128, m, j)));
+        kv[x] = gc * __uint_as_float(*reinterpret_cast<const uint32_t *>(sB1 + kmaj_tf32(128, 64 + m, j)));
+        zero[x] = 0.f;
       }
-      tc::mma_commit(bar_mma);
+      tc::tmem_st32(tmem + lane_base + TM_A2 + 32 * ch, bv);
+      tc::tmem_st32(tmem + lane_base + TM_D2 + 64 + 32 * ch, kv);
+      tc::tmem_st32(tmem + lane_base + TM_D2 + 32 * ch, zero);
     }
+    tc::tmem_st_wait();
     wait_mma();
+    tc::tc_fence_before();
     __syncthreads();
     if (*abort_flag) break;
     tc::tc_fence_after();
 
-    // ---- P3: masks --------------------------------------------------------------------------
+    // ---- P3: masks ------------------------------------------------------------------------------
     {
-      const int t = q * 32 + lane - (chan_thread ? 64 : 0);  // token row of this lane
+      const int t = q * 32 + lane - (hi_lanes ? 64 : 0);  // token row of this lane
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         float v[32];
         tc::tmem_ld32(tmem + lane_base + TM_D1 + 64 * ch + 32 * half, v);
-        if (!chan_thread) {
+        if (!hi_lanes) {
           // lanes 0..63: Mrb (ch 0) / Mrk (ch 1), keep m <= t
 #pragma unroll
           for (int x = 0; x < 32; ++x)
@@ -347,7 +399,8 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
             if (32 * half + x >= t) v[x] = 0.f;
           if (ch == 0) {
 #pragma unroll
-            for (int x = 0; x < 32; ++x) Ls[t * LDS + 32 * half + x] = v[x];
+            for (int x = 0; x < 32; x += 4)
+              *reinterpret_cast<float4 *>(Ls + t * LDL + 32 * half + x) = make_float4(v[x], v[x + 1], v[x + 2], v[x + 3]);
           } else {
             // A3 rows M = 64 + m' (Lak^T), K = t: bf16, one 128-byte row per thread
 #pragma unroll
@@ -362,63 +415,64 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
           }
         }
       }
-      if (!chan_thread) tc::tmem_st_wait();
+      if (!hi_lanes) tc::tmem_st_wait();
     }
     tc::fence_proxy_async_smem();
     tc::tc_fence_before();
     __syncthreads();
 
-    // ---- P4: Tinv = (I - Lab)^-1 --------------------------------------------------------------
-    if (tid < 64) {
-      // diagonal 16x16 blocks, one column per thread, forward substitution
-      const int s = tid >> 4, cix = tid & 15, base = 16 * s;
+    // ---- P4: Tinv = (I - Lab)^-1 -------------------------------------------------------------------
+    if (warp < 2) {
+      // diagonal 16x16 blocks: x = (I - L_ss)^-1 e_c by forward substitution (x_r = [r == c] + sum_{q<r} L_rq x_q)
+      const int s = 2 * warp + (lane >> 4), cix = lane & 15, base = 16 * s;
       float x[16];
 #pragma unroll
       for (int r = 0; r < 16; ++r) {
         float acc = (r == cix) ? 1.f : 0.f;
-        if (r > cix) {
 #pragma unroll
-          for (int qq = 0; qq < 16; ++qq)
-            if (qq >= cix && qq < r) acc = fmaf(Ls[(base + r) * LDS + base + qq], x[qq], acc);
-        }
+        for (int qq = 0; qq < r; ++qq) acc = fmaf(Ls[(base + r) * LDL + base + qq], x[qq], acc);
         x[r] = acc;
       }
 #pragma unroll
-      for (int r = 0; r < 16; ++r) Ts[(base + r) * LDS + base + cix] = x[r];
+      for (int r = 0; r < 16; ++r) Ts[(base + r) * LDT + base + cix] = x[r];
     } else {
       // zero the blocks above the block diagonal
       for (int e = tid - 64; e < 6 * 256; e += kThreads - 64) {
         const int blk = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
         const int sr = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
         const int sc = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
-        Ts[(16 * sr + rr) * LDS + 16 * sc + cc] = 0.f;
+        Ts[(16 * sr + rr) * LDT + 16 * sc + cc] = 0.f;
       }
     }
     __syncthreads();
-    {
-      const int r = tid >> 4, cix = tid & 15;
-      for (int s = 1; s < 4; ++s) {
-        for (int m = 0; m < s; ++m) {
-          float acc = 0.f;
-          for (int qq = 16 * m; qq < 16 * s; ++qq) acc = fmaf(Ls[(16 * s + r) * LDS + qq], Ts[qq * LDS + 16 * m + cix], acc);
-          Zs[(m * 16 + r) * 17 + cix] = acc;
-        }
-        __syncthreads();
-        for (int m = 0; m < s; ++m) {
-          float acc = 0.f;
+    if (warp < 3) {
+      // block column m = warp: T_sm = D_s sum_{q=m}^{s-1} L_sq T_qm, rows s = m+1..3, on warp-level tf32 mma
+      const int m = warp;
+      float *Zw = Zs + warp * (16 * 24);
 #pragma unroll
-          for (int p = 0; p < 16; ++p) acc = fmaf(Ts[(16 * s + r) * LDS + 16 * s + p], Zs[(m * 16 + p) * 17 + cix], acc);
-          Ts[(16 * s + r) * LDS + 16 * m + cix] = acc;
+      for (int s = 1; s < 4; ++s) {
+        if (s > m) {
+          float z[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+          for (int qq = 0; qq < 3; ++qq)
+            if (qq >= m && qq < s)
+              tc::block16_mma(z, Ls + (16 * s) * LDL + 16 * qq, LDL, Ts + (16 * qq) * LDT + 16 * m, LDT, lane);
+          tc::block16_store(Zw, 24, z, lane);
+          __syncwarp();
+          float tb[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+          tc::block16_mma(tb, Ts + (16 * s) * LDT + 16 * s, LDT, Zw, 24, lane);
+          tc::block16_store(Ts + (16 * s) * LDT + 16 * m, LDT, tb, lane);
+          __syncwarp();
         }
-        __syncthreads();
       }
     }
+    __syncthreads();
     {
       // Tinv -> B3 (bf16, K-major: row t, K = m)
       const int t = tid >> 2, m0 = (tid & 3) * 16;
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
-        const float *src = Ts + t * LDS + m0 + 8 * cc;
+        const float *src = Ts + t * LDT + m0 + 8 * cc;
         uint4 u;
         u.x = pack_bf16x2(src[0], src[1]);
         u.y = pack_bf16x2(src[2], src[3]);
@@ -430,7 +484,7 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
     tc::fence_proxy_async_smem();
     __syncthreads();
 
-    // ---- MMA3 (bf16): D3 = [A~^T; Lak^T] Tinv^T ---------------------------------------------
+    // ---- MMA3 (bf16): D3 = [A~^T; Lak^T] Tinv^T ---------------------------------------------------
     if (tid == 0) {
       tc::tc_fence_after();
       constexpr uint32_t idesc = tc::instr_desc(tc::kFmtBF16, 128, 64, true, false);
@@ -446,7 +500,7 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
     if (*abort_flag) break;
     tc::tc_fence_after();
 
-    // ---- P6: D3 -> B2 (tf32 K-major: row n = column of [W~ U~], K = token) -------------------
+    // ---- P6: D3 -> B2 (tf32 K-major: row n = column of [W~ U~], K = token) ---------------------------
     {
       float v[32];
       tc::tmem_ld32(tmem + lane_base + TM_D3 + 32 * ch, v);
@@ -456,15 +510,15 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
     tc::tc_fence_before();
     __syncthreads();
 
-    // ---- MMA2 (tf32, A from TMEM): D2 += [Mrb; B-^T] [W~ U~] ----------------------------------
+    // ---- MMA2 (tf32, A from TMEM): D2 += [Mrb; B-^T] [W~ U~]; then MMA4 ------------------------------
     if (tid == 0) {
       tc::tc_fence_after();
-      constexpr uint32_t idesc = tc::instr_desc(tc::kFmtTF32, 128, 128, false, false);
-      const uint32_t b0 = smem_u32(sB2);
+      constexpr uint32_t idesc2 = tc::instr_desc(tc::kFmtTF32, 128, 128, false, false);
+      const uint32_t b2 = smem_u32(sB2);
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks) {
         const uint32_t off = (ks >> 2) * (128 * 128) + (ks & 3) * 32;
-        tc::mma_ts_tf32(tmem + TM_D2, tmem + TM_A2 + 8 * ks, tc::smem_desc(b0 + off, 16, 1024), idesc, 1);
+        tc::mma_ts_tf32(tmem + TM_D2, tmem + TM_A2 + 8 * ks, tc::smem_desc(b2 + off, 16, 1024), idesc2, 1);
       }
       tc::mma_commit(bar_mma);
     }
@@ -472,15 +526,17 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
     __syncthreads();
     if (*abort_flag) break;
 
-    // ---- MMA4 (tf32, A from TMEM): D4 = [Q P; E F] [S0^T; V] ----------------------------------
+    // ---- MMA4 (tf32, A from TMEM): D4 = [Q P; E F] [S0^T; V] ------------------------------------------
     if (tid == 0) {
       tc::tc_fence_after();
-      constexpr uint32_t idesc = tc::instr_desc(tc::kFmtTF32, 128, 64, false, false);
-      const uint32_t b0 = smem_u32(sB4);
+      constexpr uint32_t idesc4 = tc::instr_desc(tc::kFmtTF32, 128, 64, false, false);
+      const uint32_t bs = smem_u32(sB4S), bvv = smem_u32(sB4V);
 #pragma unroll
       for (int ks = 0; ks < 16; ++ks) {
-        const uint32_t off = (ks >> 2) * (64 * 128) + (ks & 3) * 32;
-        tc::mma_ts_tf32(tmem + TM_D4, tmem + TM_D2 + 8 * ks, tc::smem_desc(b0 + off, 16, 1024), idesc, ks > 0);
+        const uint32_t base = ks < 8 ? bs : bvv;
+        const uint32_t kk = ks & 7;
+        const uint32_t off = (kk >> 2) * (64 * 128) + (kk & 3) * 32;
+        tc::mma_ts_tf32(tmem + TM_D4, tmem + TM_D2 + 8 * ks, tc::smem_desc(base + off, 16, 1024), idesc4, ks > 0);
       }
       tc::mma_commit(bar_mma);
     }
@@ -489,11 +545,11 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
     if (*abort_flag) break;
     tc::tc_fence_after();
 
-    // ---- P8: outputs and state ---------------------------------------------------------------
+    // ---- P8: outputs and state ------------------------------------------------------------------------
     {
       float v[32];
       tc::tmem_ld32(tmem + lane_base + TM_D4 + 32 * ch, v);
-      if (!chan_thread) {
+      if (!hi_lanes) {
         const int t = q * 32 + lane;
         if (t < Lc) {
           const long long tok = sb.start + static_cast<long long>(c) * C + t;
@@ -509,9 +565,10 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
           }
         }
       } else {
+        const float gc = GCs[j];
 #pragma unroll
-        for (int x = 0; x < 32; ++x) st[x] = fmaf(GC, st[x], v[x]);
-        store_state_tf32(sB4, j, ch, st);
+        for (int x = 0; x < 32; ++x) st[x] = fmaf(gc, st[x], v[x]);
+        store_state_tf32(sB4S, j, ch, st);
       }
     }
     tc::fence_proxy_async_smem();
@@ -523,7 +580,7 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
     // an aborted run may leave one tile load in flight: let it land (bounded)
     (void)tc::mbar_wait_bounded(bar_tma, tma_phase, kMaxPolls);
   }
-  if (chan_thread) {
+  if (hi_lanes) {
 #pragma unroll
     for (int x = 0; x < 32; ++x) A.s_out[pair * (kN * kN) + static_cast<long long>(32 * ch + x) * kN + j] = st[x];
   }

@@ -10,7 +10,9 @@
 //   A~ = a*Gamma_{t-1}  R~ = r*Gamma_t  B^ = b/Gamma_t  K^ = k/Gamma_t
 //   B- = b*Gamma_C/Gamma_t  K- = k*Gamma_C/Gamma_t  (Gamma_C: whole chunk)
 //   MMA1 (tf32)  [Mrb Mrk; Lab Lak] = [R~; A~] [B^; K^]^T, causally masked
-//   CUDA cores   Tinv = (I - Lab)^-1 (unit lower triangular)
+//   inverse      Tinv = (I - Lab)^-1 (unit lower triangular; 16x16 diagonal
+//                blocks on CUDA cores, the rest by 2x2 block doubling on
+//                warp-level tf32 mma)
 //   MMA3 (bf16)  [W~ U~]^T = [A~^T; Lak^T] Tinv^T
 //   MMA2 (tf32)  [Q P; E F] = [R~ Mrk; 0 K-^T] + [Mrb; B-^T] [W~ U~]
 //   MMA4 (tf32)  [Y; X] = [Q P; E F] [S0^T; V],   S_C^T = diag(Gamma_C) S0^T + X
@@ -41,16 +43,18 @@ namespace rwkv7 {
 namespace chunk {
 
 constexpr int C = 64;
-constexpr int kThreads = 256;
+constexpr int kComputeThreads = 256;  // 8 compute warps
+constexpr int kThreads = kComputeThreads + 32;  // + one control warp (TMA and MMA issue)
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kMaxPolls = 1u << 22;
 
 // TMEM column map
-constexpr uint32_t TM_D1 = 0;    // 128 cols: [Mrb Mrk] (lanes 0-63), [Lab Lak] (lanes 64-127)
-constexpr uint32_t TM_D2 = 128;  // 128 cols: [Q P] / [E F]
-constexpr uint32_t TM_D3 = 256;  // 64 cols: [W~ U~]^T (lane = column index of W~|U~, col = token)
-constexpr uint32_t TM_D4 = 320;  // 64 cols: Y (lanes 0-63), X (lanes 64-127)
-constexpr uint32_t TM_A2 = 384;  // 64 cols: Mrb (lanes 0-63), B-^T (lanes 64-127)
+constexpr uint32_t TM_D1 = 0;    // 128 cols: [Mrb Mrk] (lanes 0-63) / [Lab Lak] (lanes 64-127);
+                                 // then A2 = [Mrb; B-^T] in cols 0-63 and D3 in cols 64-127
+constexpr uint32_t TM_A2 = 0;
+constexpr uint32_t TM_D3 = 64;   // [W~ U~]^T (lane = column index of W~|U~, col = token)
+constexpr uint32_t TM_D2 = 128;  // 128 cols: [Q P] (lanes 0-63) / [E F] (lanes 64-127)
+constexpr uint32_t TM_D4 = 256;  // 64 cols: Y (lanes 0-63), X (lanes 64-127)
 
 // shared memory map (bytes from a 1024-aligned base)
 constexpr uint32_t kTile = C * kN * 2;            // one bf16 64x64 tile
@@ -59,22 +63,36 @@ constexpr uint32_t OFF_A1 = OFF_RAW + 6 * kTile;  // tf32 K-major [R~; A~] 128x6
 constexpr uint32_t OFF_B1 = OFF_A1 + 32768;       // tf32 K-major [B^; K^] 128x64 (32 KB)
 constexpr uint32_t OFF_A3 = OFF_B1 + 32768;       // bf16 MN-major [A~^T; Lak^T], M=128 x K=64 (16 KB)
 constexpr uint32_t OFF_B4S = OFF_A3 + 16384;      // tf32 K-major S0^T part of the chain B: row i, K = j (16 KB)
-constexpr uint32_t OFF_B4V = OFF_B4S + 16384;     // tf32 K-major V part of the chain B: row i, K = m (16 KB)
-constexpr uint32_t OFF_MISC = OFF_B4V + 16384;
+constexpr uint32_t OFF_B4V = OFF_B4S + 16384;     // 2 x tf32 K-major V part of the chain B: row i, K = m (16 KB each)
+constexpr uint32_t OFF_B2 = OFF_B4V + 2 * 16384;  // tf32 K-major [W~ U~]^T 128x64 (32 KB)
+constexpr uint32_t OFF_MISC = OFF_B2 + 32768;
 // regions reused once MMA1 has consumed A1 / B1
-constexpr int LDL = 68;                           // row stride (floats) of Lab: conflict-free as an mma A operand
-constexpr int LDT = 72;                           // row stride (floats) of Tinv: conflict-free as an mma B operand
-constexpr uint32_t OFF_LS = OFF_A1;               // float [64][LDL]
-constexpr uint32_t OFF_ZS = OFF_A1 + 64 * LDL * 4;  // float [3 warps][16][24]
-constexpr uint32_t OFF_B2 = OFF_A1;               // tf32 K-major [W~ U~]^T 128x64 (after the inverse)
-constexpr uint32_t OFF_TS = OFF_B1;               // float [64][LDT]
-constexpr uint32_t OFF_B3 = OFF_B1 + 19456;       // bf16 K-major Tinv 64x64 (8 KB), 1024-aligned
-constexpr uint32_t MISC_GC = 256;                 // float [64]   Gamma at the chunk end
-constexpr uint32_t MISC_TOT = 512;                // float [16][64] per-token-group decay products
-constexpr uint32_t kSmemBytes = OFF_MISC + MISC_TOT + 16 * 64 * 4 + 1024;
+constexpr int LDL = 68;                             // row stride (floats) of Lab: conflict-free as an mma A operand
+constexpr int LDT = 72;                             // row stride (floats) of Tinv: conflict-free as an mma B operand
+constexpr int LDZ = 24;                             // row stride (floats) of 16x16 scratch blocks
+constexpr uint32_t OFF_LS = OFF_A1;                 // float [64][LDL]
+constexpr uint32_t OFF_ZS = OFF_A1 + 64 * LDL * 4;  // float [6][16][LDZ] scratch blocks of the inverse
+constexpr uint32_t OFF_TS = OFF_B1;                 // float [64][LDT]
+constexpr uint32_t OFF_B3 = OFF_B1 + 19456;         // bf16 K-major Tinv 64x64 (8 KB), 1024-aligned
+constexpr uint32_t MISC_GC = 256;                   // float [64]    Gamma at the chunk end
+constexpr uint32_t MISC_WTOT = 512;                 // float [4][64] decay products of 16-token blocks
+constexpr uint32_t kSmemBytes = OFF_MISC + MISC_WTOT + 4 * 64 * 4 + 1024;
 
-static_assert(OFF_ZS + 3 * 16 * 24 * 4 <= OFF_B1, "inverse scratch overflows A1");
+static_assert(OFF_ZS + 6 * 16 * LDZ * 4 <= OFF_B1, "inverse scratch overflows A1");
 static_assert(OFF_TS + 64 * LDT * 4 <= OFF_B3 && OFF_B3 + 8192 <= OFF_A3, "inverse scratch overflows B1");
+static_assert(kSmemBytes <= 232448, "shared memory over the sm_100 limit");
+
+// Barrier among the 8 compute warps only (the control warp never joins it).
+__device__ __forceinline__ void compute_sync() { asm volatile("bar.sync 1, 256;\n" ::: "memory"); }
+
+// Bounded mbarrier wait that also gives up once the CTA is aborting.
+__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
+  for (uint32_t i = 0; i < kMaxPolls; ++i) {
+    if (tc::mbar_try_wait(bar, parity)) return true;
+    if ((i & 255u) == 255u && *abort_flag) return false;
+  }
+  return false;
+}
 
 struct Maps {
   CUtensorMap m[6];  // r, w, k, a, b, v: dims {64, H, tokens}, box {64, 1, 64}
@@ -93,13 +111,28 @@ struct Args {
 
 enum { RAW_R = 0, RAW_W = 1, RAW_K = 2, RAW_A = 3, RAW_B = 4, RAW_V = 5 };
 
-// byte offset of element (row, k) in a K-major tf32 operand with `rows` rows
+// byte offset of element (row, k) in a K-major 32-bit operand with `rows` rows
 __device__ __forceinline__ uint32_t kmaj_tf32(uint32_t rows, uint32_t row, uint32_t k) {
   return (k >> 5) * (rows * 128u) + tc::sw128(row, (k & 31u) >> 2) + (k & 3u) * 4u;
 }
 // byte offset of element (k, mn) in an MN-major bf16 operand with `krows` K rows
 __device__ __forceinline__ uint32_t mnmaj_bf16(uint32_t krows, uint32_t k, uint32_t mn) {
   return (mn >> 6) * (krows * 128u) + tc::sw128(k, (mn & 63u) >> 3) + (mn & 7u) * 2u;
+}
+
+// One column k = j of 32 consecutive rows row0 .. row0+31 (row0 a multiple of
+// 8) of a K-major 32-bit operand whose K-atoms hold `rows` rows: row row0 + x
+// sits at p[x & 7] + x * 128, so the unrolled accesses need no address math.
+struct ColPtrs {
+  uint8_t *p[8];
+};
+__device__ __forceinline__ ColPtrs col_ptrs(uint8_t *region, uint32_t rows, uint32_t row0, uint32_t j) {
+  ColPtrs c;
+  uint8_t *base = region + (j >> 5) * (rows * 128u) + row0 * 128u + (j & 3u) * 4u;
+  const uint32_t chunk = (j & 31u) >> 2;
+#pragma unroll
+  for (uint32_t r = 0; r < 8; ++r) c.p[r] = base + ((chunk ^ r) << 4);
+  return c;
 }
 
 // four consecutive bf16 channels of one token row of a raw tile
@@ -119,19 +152,144 @@ __device__ __forceinline__ void st_tf32x4(uint8_t *p, float a, float b, float c,
   *reinterpret_cast<uint4 *>(p) = make_uint4(tc::to_tf32(a), tc::to_tf32(b), tc::to_tf32(c), tc::to_tf32(d));
 }
 
-// Writes 32 consecutive float32 values as tf32 into one 128-byte swizzled row.
-__device__ __forceinline__ void store_row_tf32(uint8_t *region_row_block, uint32_t row, const float (&v)[32]) {
+// 32 consecutive values of one 128-byte swizzled row: raw float32 bits / read back
+__device__ __forceinline__ void store_row_f32(uint8_t *blk, uint32_t row, const float (&v)[32]) {
 #pragma unroll
   for (int c = 0; c < 8; ++c)
-    st_tf32x4(region_row_block + tc::sw128(row, c), v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+    *reinterpret_cast<float4 *>(blk + tc::sw128(row, c)) =
+        make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+}
+__device__ __forceinline__ void load_row(const uint8_t *blk, uint32_t row, float (&v)[32]) {
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const float4 u = *reinterpret_cast<const float4 *>(blk + tc::sw128(row, c));
+    v[4 * c] = u.x;
+    v[4 * c + 1] = u.y;
+    v[4 * c + 2] = u.z;
+    v[4 * c + 3] = u.w;
+  }
+}
+// keep v[x] where x <= lim; zero the rest
+__device__ __forceinline__ void mask_upper(float (&v)[32], int lim) {
+#pragma unroll
+  for (int x = 0; x < 32; ++x) v[x] = x <= lim ? v[x] : 0.f;
+}
+__device__ __forceinline__ void zero32(float (&v)[32]) {
+#pragma unroll
+  for (int x = 0; x < 32; ++x) v[x] = 0.f;
 }
 
 // B4S holds S0^T as the K-major B operand of the chain product: row = value
-// channel i, K = key channel j.  A state thread owns S^T[j][32*ch + x].
+// channel i, K = key channel j.  A state thread owns S^T[j][32*ch + x], i.e.
+// column j of rows 32*ch .. 32*ch+31.
 __device__ __forceinline__ void store_state_tf32(uint8_t *sB4S, int j, int ch, const float (&st)[32]) {
+  const ColPtrs cp = col_ptrs(sB4S, 64, 32 * ch, j);
 #pragma unroll
-  for (int x = 0; x < 32; ++x)
-    *reinterpret_cast<uint32_t *>(sB4S + kmaj_tf32(64, 32 * ch + x, j)) = tc::to_tf32(st[x]);
+  for (int x = 0; x < 32; ++x) *reinterpret_cast<uint32_t *>(cp.p[x & 7] + x * 128) = tc::to_tf32(st[x]);
+}
+
+// Stores a 16x16 mma-layout accumulator as bf16 into a K-major bf16 operand
+// (128-byte rows, one K-atom) at rows row0.., K columns col0.. (col0 % 8 == 0).
+__device__ __forceinline__ void block16_store_bf16(uint8_t *op, int row0, int col0, const float (&acc)[2][4],
+                                                   int lane) {
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt) {
+    const int col = col0 + 8 * nt + 2 * t;
+    *reinterpret_cast<uint32_t *>(op + tc::sw128(row0 + g, col >> 3) + (col & 7) * 2) =
+        pack_bf16x2(acc[nt][0], acc[nt][1]);
+    *reinterpret_cast<uint32_t *>(op + tc::sw128(row0 + g + 8, col >> 3) + (col & 7) * 2) =
+        pack_bf16x2(acc[nt][2], acc[nt][3]);
+  }
+}
+
+// Tinv = (I - L)^-1 for the strictly lower 64x64 matrix L in Ls (only entries
+// below the diagonal are read).  Writes Tinv as the bf16 K-major operand B3
+// (row t, K = m; zero above the block diagonal), using Ts (float32) for the
+// blocks later steps read.  Uses the block identity for a lower
+// block-triangular M = I - L:  (M^-1)_BA = (M^-1)_BB L_BA (M^-1)_AA,
+// first for the 16x16 diagonal blocks (forward substitution in registers),
+// then for blocks (1,0), (3,2) and finally the lower-left 32x32 block, each
+// 16x16 product on warp-level tf32 mma.  Every thread of the CTA must call it.
+__device__ __forceinline__ void invert_unit_lower(const float *Ls, float *Ts, float *Zs, uint8_t *sB3, int warp,
+                                                  int lane) {
+  if (warp < 4) {
+    // diagonal block s = warp: column cix of (I - L_ss)^-1, x_r = [r == c] + sum_{q<r} L_rq x_q
+    const int base = 16 * warp, cix = lane & 15;
+    float Lr[120];  // Lr[r(r-1)/2 + q] = L[base + r][base + q] for q < r
+#pragma unroll
+    for (int r = 1; r < 16; ++r) {
+#pragma unroll
+      for (int q4 = 0; q4 < (r + 3) / 4; ++q4) {
+        const float4 u = *reinterpret_cast<const float4 *>(Ls + (base + r) * LDL + base + 4 * q4);
+        const float uu[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (4 * q4 + e < r) Lr[r * (r - 1) / 2 + 4 * q4 + e] = uu[e];
+      }
+    }
+    float x[16];
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+      float acc = (r == cix) ? 1.f : 0.f;
+#pragma unroll
+      for (int q = 0; q < r; ++q) acc = fmaf(Lr[r * (r - 1) / 2 + q], x[q], acc);
+      x[r] = acc;
+    }
+    if (lane < 16) {
+      const int m = base + cix;
+#pragma unroll
+      for (int r = 0; r < 16; ++r) {
+        Ts[(base + r) * LDT + m] = x[r];
+        *reinterpret_cast<uint16_t *>(sB3 + tc::sw128(base + r, m >> 3) + (m & 7) * 2) = float_to_bf16_bits(x[r]);
+      }
+    }
+  } else {
+    // the six 16x16 blocks above the block diagonal are zero: 16 rows x 2 chunks each
+    for (int e = (warp - 4) * 32 + lane; e < 6 * 32; e += 128) {
+      const int blk = e >> 5, rr = (e >> 1) & 15, half = e & 1;
+      const int sr = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
+      const int sc = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
+      *reinterpret_cast<uint4 *>(sB3 + tc::sw128(16 * sr + rr, 2 * sc + half)) = make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+  compute_sync();
+  if (warp < 2) {
+    // T_{s+1,s} = D_{s+1} L_{s+1,s} D_s for s = 0, 2
+    const int s = 2 * warp;
+    float *Z = Zs + warp * (16 * LDZ);
+    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    tc::block16_mma(acc, Ls + (16 * (s + 1)) * LDL + 16 * s, LDL, Ts + (16 * s) * LDT + 16 * s, LDT, lane);
+    tc::block16_store(Z, LDZ, acc, lane);
+    __syncwarp();
+    float t2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    tc::block16_mma(t2, Ts + (16 * (s + 1)) * LDT + 16 * (s + 1), LDT, Z, LDZ, lane);
+    tc::block16_store(Ts + (16 * (s + 1)) * LDT + 16 * s, LDT, t2, lane);
+    block16_store_bf16(sB3, 16 * (s + 1), 16 * s, t2, lane);
+  }
+  compute_sync();
+  // lower-left 32x32 block, one warp per 16x16 tile (s, m), s in {2, 3}, m in {0, 1}
+  const int s = 2 + (warp >> 1), m = warp & 1;
+  if (warp < 4) {
+    // X_sm = sum_{q=m}^{1} L_sq T_qm
+    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+    for (int q = 0; q < 2; ++q)
+      if (q >= m) tc::block16_mma(acc, Ls + (16 * s) * LDL + 16 * q, LDL, Ts + (16 * q) * LDT + 16 * m, LDT, lane);
+    tc::block16_store(Zs + (2 + warp) * (16 * LDZ), LDZ, acc, lane);
+  }
+  compute_sync();
+  if (warp < 4) {
+    // T_sm = sum_{p=2}^{s} T_sp X_pm
+    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+    for (int p = 2; p < 4; ++p)
+      if (p <= s)
+        tc::block16_mma(acc, Ts + (16 * s) * LDT + 16 * p, LDT, Zs + (2 + 2 * (p - 2) + m) * (16 * LDZ), LDZ, lane);
+    block16_store_bf16(sB3, 16 * s, 16 * m, acc, lane);
+  }
+  tc::fence_proxy_async_smem();
+  compute_sync();
 }
 
 __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_constant__ Maps maps, const Args A) {
@@ -147,37 +305,38 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
   float *Ls = reinterpret_cast<float *>(smem + OFF_LS);
   float *Ts = reinterpret_cast<float *>(smem + OFF_TS);
   float *Zs = reinterpret_cast<float *>(smem + OFF_ZS);
-  uint64_t *bar_tma = reinterpret_cast<uint64_t *>(smem + OFF_MISC);
-  uint64_t *bar_mma = bar_tma + 1;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_MISC + 16);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 20);
+  // mbarriers (count 1 each); c = control warp, w = compute warps
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_MISC);
+  uint64_t *bar_tma = bars + 0;    // TMA tiles landed          (tx bytes)
+  uint64_t *bar_p1 = bars + 1;     // w -> c: A1, B1 written; raw tiles consumed
+  uint64_t *bar_m1 = bars + 2;     // c -> w: MMA1 done
+  uint64_t *bar_b3 = bars + 3;     // w -> c: A3 and B3 written
+  uint64_t *bar_m3 = bars + 4;     // c -> w: MMA3 done
+  uint64_t *bar_b2 = bars + 5;     // w -> c: B2, A2 and the D2 initial value written
+  uint64_t *bar_m2 = bars + 6;     // c -> c: MMA2 done
+  uint64_t *bar_st = bars + 7;     // w -> c: state S0^T (B4S) written, D4 read out
+  uint64_t *bar_m4 = bars + 8;     // c -> w: MMA4 done
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_MISC + 80);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 84);
   float *GCs = reinterpret_cast<float *>(smem + OFF_MISC + MISC_GC);
-  float *tot = reinterpret_cast<float *>(smem + OFF_MISC + MISC_TOT);
+  float *wtot = reinterpret_cast<float *>(smem + OFF_MISC + MISC_WTOT);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-  const int q = warp & 3;    // TMEM lane quadrant of this warp
-  const int ch = warp >> 2;  // which half of a 64-column block this warp handles
   const int h = blockIdx.x;
   const int bidx = blockIdx.y;
   const SeqBounds sb = seq_bounds(A.cu_seqlens, bidx, A.T, A.total_T);
   if (sb.len < 0) return;
   const int nchunks = (sb.len + C - 1) / C;
-  const bool hi_lanes = q >= 2;  // owns TMEM lanes 64..127
-  const int j = tid & 63;        // for hi-lane threads: the key channel of its lane
   const long long pair = static_cast<long long>(bidx) * A.H + h;
-  // operand-construction layout: 4 channels x 4 tokens per thread
-  const int cq = 8 * (warp & 1) + (lane & 7), tg = 4 * (warp >> 1) + (lane >> 3);
-  const int j0 = 4 * cq, t0 = 4 * tg;
+  constexpr int kCtrlWarp = kComputeThreads / 32;
 
   if (tid == 0) {
-    tc::mbar_init(bar_tma, 1);
-    tc::mbar_init(bar_mma, 1);
+    for (int i = 0; i < 9; ++i) tc::mbar_init(bars + i, 1);
     tc::fence_mbar_init();
     *abort_flag = 0;
-    for (int i = 0; i < 6; ++i) tc::prefetch_tensormap(&maps.m[i]);
   }
-  if (warp == 0) {
+  if (warp == kCtrlWarp) {
     tc::tmem_alloc(tmem_slot, kTmemCols);
     tc::tmem_relinquish();
   }
@@ -185,409 +344,411 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
 
-  // state: hi-lane threads hold S^T[j][32*ch .. 32*ch+31] in float32
-  float st[32];
-  if (hi_lanes) {
-#pragma unroll
-    for (int x = 0; x < 32; ++x)
-      st[x] = A.s_in ? A.s_in[pair * (kN * kN) + static_cast<long long>(32 * ch + x) * kN + j] : 0.f;
-    store_state_tf32(sB4S, j, ch, st);
-  }
-
-  uint32_t tma_phase = 0, mma_phase = 0;
-  bool tma_pending = false;
-  if (tid == 0 && nchunks > 0) {
-    tc::mbar_arrive_expect_tx(bar_tma, 6 * kTile);
-    for (int i = 0; i < 6; ++i)
-      tc::tma_load_3d(smem + OFF_RAW + i * kTile, &maps.m[i], bar_tma, 0, h, static_cast<int>(sb.start));
-    tma_pending = true;
-  }
-
-  auto wait_mma = [&]() {
-    if (tid == 0) {
-      if (!tc::mbar_wait_bounded(bar_mma, mma_phase, kMaxPolls)) {
+  if (warp == kCtrlWarp) {
+    // ===== control warp: TMA loads and every MMA, issued by one lane =====================
+    if (lane == 0) {
+      auto fail = [&]() {
         *abort_flag = 1;
         report_device_error(A.err, kDevErrTimeout);
-      }
-    }
-    mma_phase ^= 1u;
-  };
-
-  for (int c = 0; c < nchunks; ++c) {
-    const int Lc = min(C, sb.len - c * C);
-    // ---- this chunk's tiles have landed ---------------------------------------------------
-    if (tid == 0) {
-      if (!tc::mbar_wait_bounded(bar_tma, tma_phase, kMaxPolls)) {
-        *abort_flag = 1;
-        report_device_error(A.err, kDevErrTimeout);
-      } else {
-        tma_pending = false;
-      }
-      tma_phase ^= 1u;
-    }
-    __syncthreads();
-    if (*abort_flag) break;
-
-    // ---- P1: decay products and operands (4 channels x 4 tokens per thread) ---------------
-    float G[4][4];  // Gamma_t for t = t0..t0+3 (rows) and channels j0..j0+3 (cols)
-    {
-      float wv[4][4];
-#pragma unroll
-      for (int tt = 0; tt < 4; ++tt) {
-        if (t0 + tt < Lc) {
-          raw4(smem, RAW_W, t0 + tt, j0, wv[tt]);
-        } else {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) wv[tt][e] = 1.f;
-        }
-      }
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        G[0][e] = wv[0][e];
-        G[1][e] = G[0][e] * wv[1][e];
-        G[2][e] = G[1][e] * wv[2][e];
-        G[3][e] = G[2][e] * wv[3][e];
-      }
-      *reinterpret_cast<float4 *>(tot + tg * 64 + j0) = make_float4(G[3][0], G[3][1], G[3][2], G[3][3]);
-    }
-    __syncthreads();
-    {
-      float pre[4] = {1.f, 1.f, 1.f, 1.f};
-#pragma unroll
-      for (int g = 0; g < 15; ++g) {
-        if (g < tg) {
-          const float4 u = *reinterpret_cast<const float4 *>(tot + g * 64 + j0);
-          pre[0] *= u.x;
-          pre[1] *= u.y;
-          pre[2] *= u.z;
-          pre[3] *= u.w;
-        }
-      }
-      float rr[4][4], kk[4][4], aa[4][4], bb[4][4], vv[4][4];
-#pragma unroll
-      for (int tt = 0; tt < 4; ++tt) {
-        if (t0 + tt < Lc) {
-          raw4(smem, RAW_R, t0 + tt, j0, rr[tt]);
-          raw4(smem, RAW_K, t0 + tt, j0, kk[tt]);
-          raw4(smem, RAW_A, t0 + tt, j0, aa[tt]);
-          raw4(smem, RAW_B, t0 + tt, j0, bb[tt]);
-          raw4(smem, RAW_V, t0 + tt, j0, vv[tt]);
-        } else {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) rr[tt][e] = kk[tt][e] = aa[tt][e] = bb[tt][e] = vv[tt][e] = 0.f;
-        }
-      }
-      float Gp[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) Gp[e] = pre[e];  // Gamma_{t0 - 1}
-#pragma unroll
-      for (int tt = 0; tt < 4; ++tt) {
-        const int t = t0 + tt;
-        float Gt[4], inv[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          Gt[e] = pre[e] * G[tt][e];
-          inv[e] = tc::rcp_approx(Gt[e]);
-        }
-        const uint32_t kofs = (j0 >> 5) * (128 * 128) + ((j0 & 31) >> 2);  // katom base + chunk index
-        uint8_t *a1r = sA1 + (j0 >> 5) * (128 * 128);
-        uint8_t *b1r = sB1 + (j0 >> 5) * (128 * 128);
-        const uint32_t chunk = (j0 & 31) >> 2;
-        (void)kofs;
-        st_tf32x4(a1r + tc::sw128(t, chunk), rr[tt][0] * Gt[0], rr[tt][1] * Gt[1], rr[tt][2] * Gt[2],
-                  rr[tt][3] * Gt[3]);
-        const float At0 = aa[tt][0] * Gp[0], At1 = aa[tt][1] * Gp[1], At2 = aa[tt][2] * Gp[2],
-                    At3 = aa[tt][3] * Gp[3];
-        st_tf32x4(a1r + tc::sw128(64 + t, chunk), At0, At1, At2, At3);
-        st_tf32x4(b1r + tc::sw128(t, chunk), bb[tt][0] * inv[0], bb[tt][1] * inv[1], bb[tt][2] * inv[2],
-                  bb[tt][3] * inv[3]);
-        st_tf32x4(b1r + tc::sw128(64 + t, chunk), kk[tt][0] * inv[0], kk[tt][1] * inv[1], kk[tt][2] * inv[2],
-                  kk[tt][3] * inv[3]);
-        // A3: A~^T as the MN-major bf16 A operand of MMA3 (M = channel, K = token)
-        *reinterpret_cast<uint2 *>(sA3 + mnmaj_bf16(64, t, j0)) =
-            make_uint2(pack_bf16x2(At0, At1), pack_bf16x2(At2, At3));
-#pragma unroll
-        for (int e = 0; e < 4; ++e) Gp[e] = Gt[e];
-      }
-      if (tg == 15) *reinterpret_cast<float4 *>(GCs + j0) = make_float4(Gp[0], Gp[1], Gp[2], Gp[3]);
-      // V -> B4V (row = value channel, K = token), bf16 values are exact in tf32
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        *reinterpret_cast<uint4 *>(sB4V + kmaj_tf32(64, j0 + e, t0)) =
-            make_uint4(__float_as_uint(vv[0][e]), __float_as_uint(vv[1][e]), __float_as_uint(vv[2][e]),
-                       __float_as_uint(vv[3][e]));
-    }
-    tc::fence_proxy_async_smem();
-    __syncthreads();
-
-    // ---- MMA1 (tf32): D1 = [R~; A~] [B^; K^]^T, and the next chunk's tiles ---------------------
-    if (tid == 0) {
-      if (c + 1 < nchunks) {
+      };
+      for (int i = 0; i < 6; ++i) tc::prefetch_tensormap(&maps.m[i]);
+      // parity of the last issued phase of each barrier, or -1 when nothing was issued
+      int last_tma = -1, last_m1 = -1, last_m3 = -1, last_m2 = -1, last_m4 = -1;
+      if (nchunks > 0) {
         tc::mbar_arrive_expect_tx(bar_tma, 6 * kTile);
         for (int i = 0; i < 6; ++i)
-          tc::tma_load_3d(smem + OFF_RAW + i * kTile, &maps.m[i], bar_tma, 0, h,
-                          static_cast<int>(sb.start + static_cast<long long>(c + 1) * C));
-        tma_pending = true;
+          tc::tma_load_3d(smem + OFF_RAW + i * kTile, &maps.m[i], bar_tma, 0, h, static_cast<int>(sb.start));
+        last_tma = 0;
       }
-      tc::tc_fence_after();
-      constexpr uint32_t idesc = tc::instr_desc(tc::kFmtTF32, 128, 128, false, false);
-      const uint32_t a0 = smem_u32(sA1), b0 = smem_u32(sB1);
+      for (int c = 0; c < nchunks; ++c) {
+        const uint32_t ph = c & 1;
+        // MMA1 (tf32): D1 = [R~; A~] [B^; K^]^T, once the operands are in place
+        if (!wait_or_abort(bar_p1, ph, abort_flag)) { fail(); break; }
+        if (c + 1 < nchunks) {
+          tc::mbar_arrive_expect_tx(bar_tma, 6 * kTile);
+          for (int i = 0; i < 6; ++i)
+            tc::tma_load_3d(smem + OFF_RAW + i * kTile, &maps.m[i], bar_tma, 0, h,
+                            static_cast<int>(sb.start + static_cast<long long>(c + 1) * C));
+          last_tma = (c + 1) & 1;
+        }
+        tc::tc_fence_after();
+        {
+          constexpr uint32_t idesc = tc::instr_desc(tc::kFmtTF32, 128, 128, false, false);
+          const uint32_t a0 = smem_u32(sA1), b0 = smem_u32(sB1);
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        const uint32_t off = (ks >> 2) * (128 * 128) + (ks & 3) * 32;
-        tc::mma_ss(1, tmem + TM_D1, tc::smem_desc(a0 + off, 16, 1024), tc::smem_desc(b0 + off, 16, 1024), idesc,
-                   ks > 0);
-      }
-      tc::mma_commit(bar_mma);
-    }
-    // D2 and A2 set-up from the operands (overlaps MMA1, which only reads A1 / B1)
-    if (!hi_lanes) {
-      // lanes t = 0..63: Q-part of D2 starts at R~[t][32ch .. 32ch+31] (read back from A1)
-      const int t = q * 32 + lane;
-      float rt[32];
-      const uint8_t *rowblk = sA1 + ch * (128 * 128);
-#pragma unroll
-      for (int cc = 0; cc < 8; ++cc) {
-        const uint4 u = *reinterpret_cast<const uint4 *>(rowblk + tc::sw128(t, cc));
-        rt[4 * cc + 0] = __uint_as_float(u.x);
-        rt[4 * cc + 1] = __uint_as_float(u.y);
-        rt[4 * cc + 2] = __uint_as_float(u.z);
-        rt[4 * cc + 3] = __uint_as_float(u.w);
-      }
-      tc::tmem_st32(tmem + lane_base + TM_D2 + 32 * ch, rt);
-    } else {
-      // lanes 64+j: B-^T[j][m] = Gamma_C[j] B^[m][j] -> A2; K-^T[j][m] = Gamma_C[j] K^[m][j] -> F-part of D2
-      const float gc = GCs[j];
-      float bv[32], kv[32], zero[32];
-#pragma unroll
-      for (int x = 0; x < 32; ++x) {
-        const int m = 32 * ch + x;
-        bv[x] = gc * __uint_as_float(*reinterpret_cast<const uint32_t *>(sB1 + kmaj_tf32(128, m, j)));
-        kv[x] = gc * __uint_as_float(*reinterpret_cast<const uint32_t *>(sB1 + kmaj_tf32(128, 64 + m, j)));
-        zero[x] = 0.f;
-      }
-      tc::tmem_st32(tmem + lane_base + TM_A2 + 32 * ch, bv);
-      tc::tmem_st32(tmem + lane_base + TM_D2 + 64 + 32 * ch, kv);
-      tc::tmem_st32(tmem + lane_base + TM_D2 + 32 * ch, zero);
-    }
-    tc::tmem_st_wait();
-    wait_mma();
-    tc::tc_fence_before();
-    __syncthreads();
-    if (*abort_flag) break;
-    tc::tc_fence_after();
-
-    // ---- P3: masks ------------------------------------------------------------------------------
-    {
-      const int t = q * 32 + lane - (hi_lanes ? 64 : 0);  // token row of this lane
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        float v[32];
-        tc::tmem_ld32(tmem + lane_base + TM_D1 + 64 * ch + 32 * half, v);
-        if (!hi_lanes) {
-          // lanes 0..63: Mrb (ch 0) / Mrk (ch 1), keep m <= t
-#pragma unroll
-          for (int x = 0; x < 32; ++x)
-            if (32 * half + x > t) v[x] = 0.f;
-          tc::tmem_st32(tmem + lane_base + (ch == 0 ? TM_A2 : TM_D2 + 64) + 32 * half, v);
-        } else {
-          // lanes 64..127: Lab (ch 0) / Lak (ch 1), keep m < t
-#pragma unroll
-          for (int x = 0; x < 32; ++x)
-            if (32 * half + x >= t) v[x] = 0.f;
-          if (ch == 0) {
-#pragma unroll
-            for (int x = 0; x < 32; x += 4)
-              *reinterpret_cast<float4 *>(Ls + t * LDL + 32 * half + x) = make_float4(v[x], v[x + 1], v[x + 2], v[x + 3]);
-          } else {
-            // A3 rows M = 64 + m' (Lak^T), K = t: bf16, one 128-byte row per thread
-#pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-              uint4 u;
-              u.x = pack_bf16x2(v[8 * cc + 0], v[8 * cc + 1]);
-              u.y = pack_bf16x2(v[8 * cc + 2], v[8 * cc + 3]);
-              u.z = pack_bf16x2(v[8 * cc + 4], v[8 * cc + 5]);
-              u.w = pack_bf16x2(v[8 * cc + 6], v[8 * cc + 7]);
-              *reinterpret_cast<uint4 *>(sA3 + 64 * 128 + tc::sw128(t, 4 * half + cc)) = u;
-            }
+          for (int ks = 0; ks < 8; ++ks) {
+            const uint32_t off = (ks >> 2) * (128 * 128) + (ks & 3) * 32;
+            tc::mma_ss(1, tmem + TM_D1, tc::smem_desc(a0 + off, 16, 1024), tc::smem_desc(b0 + off, 16, 1024),
+                       idesc, ks > 0);
           }
+          tc::mma_commit(bar_m1);
+          last_m1 = ph;
+        }
+        // MMA3 (bf16): D3 = [A~^T; Lak^T] Tinv^T
+        if (!wait_or_abort(bar_b3, ph, abort_flag)) { fail(); break; }
+        tc::tc_fence_after();
+        {
+          constexpr uint32_t idesc = tc::instr_desc(tc::kFmtBF16, 128, 64, true, false);
+          const uint32_t a0 = smem_u32(sA3), b0 = smem_u32(sB3);
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks)
+            tc::mma_ss(0, tmem + TM_D3, tc::smem_desc(a0 + ks * 2048, 64 * 128, 1024),
+                       tc::smem_desc(b0 + ks * 32, 16, 1024), idesc, ks > 0);
+          tc::mma_commit(bar_m3);
+          last_m3 = ph;
+        }
+        // MMA2 (tf32, A from TMEM): D2 += [Mrb; B-^T] [W~ U~]
+        if (!wait_or_abort(bar_b2, ph, abort_flag)) { fail(); break; }
+        tc::tc_fence_after();
+        {
+          constexpr uint32_t idesc = tc::instr_desc(tc::kFmtTF32, 128, 128, false, false);
+          const uint32_t b2 = smem_u32(sB2);
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks) {
+            const uint32_t off = (ks >> 2) * (128 * 128) + (ks & 3) * 32;
+            tc::mma_ts_tf32(tmem + TM_D2, tmem + TM_A2 + 8 * ks, tc::smem_desc(b2 + off, 16, 1024), idesc, 1);
+          }
+          tc::mma_commit(bar_m2);
+          last_m2 = ph;
+        }
+        if (!wait_or_abort(bar_m2, ph, abort_flag)) { fail(); break; }
+        // MMA4 (tf32, A from TMEM): D4 = [Q P; E F] [S0^T; V], once the state is written
+        if (!wait_or_abort(bar_st, ph, abort_flag)) { fail(); break; }
+        tc::tc_fence_after();
+        {
+          constexpr uint32_t idesc = tc::instr_desc(tc::kFmtTF32, 128, 64, false, false);
+          const uint32_t bs = smem_u32(sB4S), bv = smem_u32(sB4V + (c & 1) * 16384);
+#pragma unroll
+          for (int ks = 0; ks < 16; ++ks) {
+            const uint32_t base = ks < 8 ? bs : bv;
+            const uint32_t kk = ks & 7;
+            const uint32_t off = (kk >> 2) * (64 * 128) + (kk & 3) * 32;
+            tc::mma_ts_tf32(tmem + TM_D4, tmem + TM_D2 + 8 * ks, tc::smem_desc(base + off, 16, 1024), idesc,
+                            ks > 0);
+          }
+          tc::mma_commit(bar_m4);
+          last_m4 = ph;
         }
       }
-      if (!hi_lanes) tc::tmem_st_wait();
+      // every copy and MMA issued here lands before the CTA exits (bounded; phases that
+      // already completed return at once)
+      if (last_tma >= 0) (void)tc::mbar_wait_bounded(bar_tma, last_tma, kMaxPolls);
+      if (last_m1 >= 0) (void)tc::mbar_wait_bounded(bar_m1, last_m1, kMaxPolls);
+      if (last_m3 >= 0) (void)tc::mbar_wait_bounded(bar_m3, last_m3, kMaxPolls);
+      if (last_m2 >= 0) (void)tc::mbar_wait_bounded(bar_m2, last_m2, kMaxPolls);
+      if (last_m4 >= 0) (void)tc::mbar_wait_bounded(bar_m4, last_m4, kMaxPolls);
     }
-    tc::fence_proxy_async_smem();
-    tc::tc_fence_before();
-    __syncthreads();
+  } else {
+    // ===== compute warps ===============================================================
+    const int q = warp & 3;    // TMEM lane quadrant of this warp
+    const int ch = warp >> 2;  // which half of a 64-column block this warp handles
+    const bool hi_lanes = q >= 2;        // owns TMEM lanes 64..127
+    const int j = tid & 63;              // for hi-lane threads: the key channel of its lane
+    const int tl = (q & 1) * 32 + lane;  // the token row of this thread's TMEM lane within its half
+    // operand-construction layout: 4 channels x 4 tokens per thread; the 4 token
+    // groups of a warp sit in lane bits 3..4, the 4 warps of one parity cover 64 tokens
+    const int cq = 8 * (warp & 1) + (lane & 7), tg = 4 * (warp >> 1) + (lane >> 3);
+    const int j0 = 4 * cq, t0 = 4 * tg;
+    const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
 
-    // ---- P4: Tinv = (I - Lab)^-1 -------------------------------------------------------------------
-    if (warp < 2) {
-      // diagonal 16x16 blocks: x = (I - L_ss)^-1 e_c by forward substitution (x_r = [r == c] + sum_{q<r} L_rq x_q)
-      const int s = 2 * warp + (lane >> 4), cix = lane & 15, base = 16 * s;
-      float x[16];
+    // state: hi-lane threads hold S^T[j][32*ch .. 32*ch+31] in float32
+    float st[32];
+    if (hi_lanes) {
 #pragma unroll
-      for (int r = 0; r < 16; ++r) {
-        float acc = (r == cix) ? 1.f : 0.f;
-#pragma unroll
-        for (int qq = 0; qq < r; ++qq) acc = fmaf(Ls[(base + r) * LDL + base + qq], x[qq], acc);
-        x[r] = acc;
-      }
-#pragma unroll
-      for (int r = 0; r < 16; ++r) Ts[(base + r) * LDT + base + cix] = x[r];
-    } else {
-      // zero the blocks above the block diagonal
-      for (int e = tid - 64; e < 6 * 256; e += kThreads - 64) {
-        const int blk = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
-        const int sr = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
-        const int sc = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
-        Ts[(16 * sr + rr) * LDT + 16 * sc + cc] = 0.f;
-      }
+      for (int x = 0; x < 32; ++x)
+        st[x] = A.s_in ? A.s_in[pair * (kN * kN) + static_cast<long long>(32 * ch + x) * kN + j] : 0.f;
+      store_state_tf32(sB4S, j, ch, st);
     }
-    __syncthreads();
-    if (warp < 3) {
-      // block column m = warp: T_sm = D_s sum_{q=m}^{s-1} L_sq T_qm, rows s = m+1..3, on warp-level tf32 mma
-      const int m = warp;
-      float *Zw = Zs + warp * (16 * 24);
-#pragma unroll
-      for (int s = 1; s < 4; ++s) {
-        if (s > m) {
-          float z[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-          for (int qq = 0; qq < 3; ++qq)
-            if (qq >= m && qq < s)
-              tc::block16_mma(z, Ls + (16 * s) * LDL + 16 * qq, LDL, Ts + (16 * qq) * LDT + 16 * m, LDT, lane);
-          tc::block16_store(Zw, 24, z, lane);
-          __syncwarp();
-          float tb[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-          tc::block16_mma(tb, Ts + (16 * s) * LDT + 16 * s, LDT, Zw, 24, lane);
-          tc::block16_store(Ts + (16 * s) * LDT + 16 * m, LDT, tb, lane);
-          __syncwarp();
+    // Wait for the control warp (one thread polls, bounded); false once the CTA aborts.  Thread 0
+    // publishes the decision in a slot chosen by the call parity before the barrier, so every compute
+    // thread reads the same value (a slot is rewritten only two calls later, after all have read it).
+    volatile int *decision = reinterpret_cast<volatile int *>(smem + OFF_MISC + 88);  // [2]
+    uint32_t ncalls = 0;
+    auto wait_ctrl = [&](uint64_t *bar, uint32_t parity) -> bool {
+      const uint32_t slot = ncalls++ & 1u;
+      if (tid == 0) {
+        if (!wait_or_abort(bar, parity, abort_flag)) {
+          *abort_flag = 1;
+          report_device_error(A.err, kDevErrTimeout);
         }
+        decision[slot] = *abort_flag == 0 ? 1 : 0;
       }
-    }
-    __syncthreads();
-    {
-      // Tinv -> B3 (bf16, K-major: row t, K = m)
-      const int t = tid >> 2, m0 = (tid & 3) * 16;
-#pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        const float *src = Ts + t * LDT + m0 + 8 * cc;
-        uint4 u;
-        u.x = pack_bf16x2(src[0], src[1]);
-        u.y = pack_bf16x2(src[2], src[3]);
-        u.z = pack_bf16x2(src[4], src[5]);
-        u.w = pack_bf16x2(src[6], src[7]);
-        *reinterpret_cast<uint4 *>(sB3 + tc::sw128(t, (m0 >> 3) + cc)) = u;
-      }
-    }
-    tc::fence_proxy_async_smem();
-    __syncthreads();
-
-    // ---- MMA3 (bf16): D3 = [A~^T; Lak^T] Tinv^T ---------------------------------------------------
-    if (tid == 0) {
-      tc::tc_fence_after();
-      constexpr uint32_t idesc = tc::instr_desc(tc::kFmtBF16, 128, 64, true, false);
-      const uint32_t a0 = smem_u32(sA3), b0 = smem_u32(sB3);
-#pragma unroll
-      for (int ks = 0; ks < 4; ++ks)
-        tc::mma_ss(0, tmem + TM_D3, tc::smem_desc(a0 + ks * 2048, 64 * 128, 1024),
-                   tc::smem_desc(b0 + ks * 32, 16, 1024), idesc, ks > 0);
-      tc::mma_commit(bar_mma);
-    }
-    wait_mma();
-    __syncthreads();
-    if (*abort_flag) break;
-    tc::tc_fence_after();
-
-    // ---- P6: D3 -> B2 (tf32 K-major: row n = column of [W~ U~], K = token) ---------------------------
-    {
-      float v[32];
-      tc::tmem_ld32(tmem + lane_base + TM_D3 + 32 * ch, v);
-      store_row_tf32(sB2 + ch * (128 * 128), q * 32 + lane, v);
-    }
-    tc::fence_proxy_async_smem();
-    tc::tc_fence_before();
-    __syncthreads();
-
-    // ---- MMA2 (tf32, A from TMEM): D2 += [Mrb; B-^T] [W~ U~]; then MMA4 ------------------------------
-    if (tid == 0) {
-      tc::tc_fence_after();
-      constexpr uint32_t idesc2 = tc::instr_desc(tc::kFmtTF32, 128, 128, false, false);
-      const uint32_t b2 = smem_u32(sB2);
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        const uint32_t off = (ks >> 2) * (128 * 128) + (ks & 3) * 32;
-        tc::mma_ts_tf32(tmem + TM_D2, tmem + TM_A2 + 8 * ks, tc::smem_desc(b2 + off, 16, 1024), idesc2, 1);
-      }
-      tc::mma_commit(bar_mma);
-    }
-    wait_mma();
-    __syncthreads();
-    if (*abort_flag) break;
-
-    // ---- MMA4 (tf32, A from TMEM): D4 = [Q P; E F] [S0^T; V] ------------------------------------------
-    if (tid == 0) {
-      tc::tc_fence_after();
-      constexpr uint32_t idesc4 = tc::instr_desc(tc::kFmtTF32, 128, 64, false, false);
-      const uint32_t bs = smem_u32(sB4S), bvv = smem_u32(sB4V);
-#pragma unroll
-      for (int ks = 0; ks < 16; ++ks) {
-        const uint32_t base = ks < 8 ? bs : bvv;
-        const uint32_t kk = ks & 7;
-        const uint32_t off = (kk >> 2) * (64 * 128) + (kk & 3) * 32;
-        tc::mma_ts_tf32(tmem + TM_D4, tmem + TM_D2 + 8 * ks, tc::smem_desc(base + off, 16, 1024), idesc4, ks > 0);
-      }
-      tc::mma_commit(bar_mma);
-    }
-    wait_mma();
-    __syncthreads();
-    if (*abort_flag) break;
-    tc::tc_fence_after();
-
-    // ---- P8: outputs and state ------------------------------------------------------------------------
-    {
+      compute_sync();
+      return decision[slot] != 0;
+    };
+    bool ok = true;
+    // Read-out of a finished chunk: y rows (lanes 0..63) and the state update
+    // S_C^T = diag(Gamma_C) S0^T + X (lanes 64..127), whose tf32 copy feeds the next MMA4.
+    float gc_done = 1.f;  // Gamma_C[j] of the chunk whose MMA4 is in flight (hi lanes)
+    auto readout = [&](int cidx, int Lcx) {
       float v[32];
       tc::tmem_ld32(tmem + lane_base + TM_D4 + 32 * ch, v);
       if (!hi_lanes) {
-        const int t = q * 32 + lane;
-        if (t < Lc) {
-          const long long tok = sb.start + static_cast<long long>(c) * C + t;
+        if (tl < Lcx) {
+          const long long tok = sb.start + static_cast<long long>(cidx) * C + tl;
           uint16_t *dst = A.y + (tok * A.H + h) * kN + 32 * ch;
 #pragma unroll
           for (int cc = 0; cc < 4; ++cc) {
-            uint4 u;
-            u.x = pack_bf16x2(v[8 * cc + 0], v[8 * cc + 1]);
-            u.y = pack_bf16x2(v[8 * cc + 2], v[8 * cc + 3]);
-            u.z = pack_bf16x2(v[8 * cc + 4], v[8 * cc + 5]);
-            u.w = pack_bf16x2(v[8 * cc + 6], v[8 * cc + 7]);
-            *reinterpret_cast<uint4 *>(dst + 8 * cc) = u;
+            uint4 w4;
+            w4.x = pack_bf16x2(v[8 * cc + 0], v[8 * cc + 1]);
+            w4.y = pack_bf16x2(v[8 * cc + 2], v[8 * cc + 3]);
+            w4.z = pack_bf16x2(v[8 * cc + 4], v[8 * cc + 5]);
+            w4.w = pack_bf16x2(v[8 * cc + 6], v[8 * cc + 7]);
+            *reinterpret_cast<uint4 *>(dst + 8 * cc) = w4;
           }
         }
       } else {
-        const float gc = GCs[j];
 #pragma unroll
-        for (int x = 0; x < 32; ++x) st[x] = fmaf(gc, st[x], v[x]);
+        for (int x = 0; x < 32; ++x) st[x] = fmaf(gc_done, st[x], v[x]);
         store_state_tf32(sB4S, j, ch, st);
       }
-    }
-    tc::fence_proxy_async_smem();
-    tc::tc_fence_before();
-  }
+    };
 
-  __syncthreads();
-  if (tid == 0 && tma_pending) {
-    // an aborted run may leave one tile load in flight: let it land (bounded)
-    (void)tc::mbar_wait_bounded(bar_tma, tma_phase, kMaxPolls);
-  }
-  if (hi_lanes) {
+
+    int Lc_prev = 0;
+    bool have_prev = false;
+    for (int c = 0; c < nchunks; ++c) {
+      const int Lc = min(C, sb.len - c * C);
+      const uint32_t ph = c & 1;
+      uint8_t *sB4Vc = sB4V + (c & 1) * 16384;
+      if (!(ok = wait_ctrl(bar_tma, ph))) break;
+
+      // ---- P1: decay products and operands (4 channels x 4 tokens per thread) ---------------
+      {
+        float G[4][4];        // local products of w over this thread's tokens (rows) per channel (cols)
+        float pre[4], GC[4];  // Gamma before this thread's first token; Gamma at the chunk end
+        {
+          float wv[4][4];
 #pragma unroll
-    for (int x = 0; x < 32; ++x) A.s_out[pair * (kN * kN) + static_cast<long long>(32 * ch + x) * kN + j] = st[x];
+          for (int tt = 0; tt < 4; ++tt) {
+            if (t0 + tt < Lc) {
+              raw4(smem, RAW_W, t0 + tt, j0, wv[tt]);
+            } else {
+#pragma unroll
+              for (int e = 0; e < 4; ++e) wv[tt][e] = 1.f;
+            }
+          }
+          float incl[4], ex[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            G[0][e] = wv[0][e];
+            G[1][e] = G[0][e] * wv[1][e];
+            G[2][e] = G[1][e] * wv[2][e];
+            G[3][e] = G[2][e] * wv[3][e];
+            // inclusive scan over the 4 token groups of this warp (lanes l, l+8, l+16, l+24)
+            incl[e] = G[3][e];
+            float u = __shfl_up_sync(0xffffffffu, incl[e], 8);
+            if (lane >= 8) incl[e] *= u;
+            u = __shfl_up_sync(0xffffffffu, incl[e], 16);
+            if (lane >= 16) incl[e] *= u;
+            ex[e] = __shfl_up_sync(0xffffffffu, incl[e], 8);
+            if (lane < 8) ex[e] = 1.f;
+          }
+          if ((lane >> 3) == 3)
+            *reinterpret_cast<float4 *>(wtot + (warp >> 1) * 64 + j0) =
+                make_float4(incl[0], incl[1], incl[2], incl[3]);
+          compute_sync();
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            pre[e] = ex[e];
+            GC[e] = 1.f;
+          }
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float4 u = *reinterpret_cast<const float4 *>(wtot + k * 64 + j0);
+            GC[0] *= u.x;
+            GC[1] *= u.y;
+            GC[2] *= u.z;
+            GC[3] *= u.w;
+            if (k < (warp >> 1)) {
+              pre[0] *= u.x;
+              pre[1] *= u.y;
+              pre[2] *= u.z;
+              pre[3] *= u.w;
+            }
+          }
+        }
+        float rr[4][4], kk[4][4], aa[4][4], bb[4][4], vv[4][4];
+#pragma unroll
+        for (int tt = 0; tt < 4; ++tt) {
+          if (t0 + tt < Lc) {
+            raw4(smem, RAW_R, t0 + tt, j0, rr[tt]);
+            raw4(smem, RAW_K, t0 + tt, j0, kk[tt]);
+            raw4(smem, RAW_A, t0 + tt, j0, aa[tt]);
+            raw4(smem, RAW_B, t0 + tt, j0, bb[tt]);
+            raw4(smem, RAW_V, t0 + tt, j0, vv[tt]);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) rr[tt][e] = kk[tt][e] = aa[tt][e] = bb[tt][e] = vv[tt][e] = 0.f;
+          }
+        }
+        uint8_t *a1r = sA1 + (j0 >> 5) * (128 * 128);
+        uint8_t *b1r = sB1 + (j0 >> 5) * (128 * 128);
+        const uint32_t chunk = (j0 & 31) >> 2;
+#pragma unroll
+        for (int tt = 0; tt < 4; ++tt) {
+          const int t = t0 + tt;
+          float Gt[4], Gp[4], inv[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            Gp[e] = tt == 0 ? pre[e] : pre[e] * G[tt - 1][e];
+            Gt[e] = pre[e] * G[tt][e];
+            inv[e] = tc::rcp_approx(Gt[e]);
+          }
+          st_tf32x4(a1r + tc::sw128(t, chunk), rr[tt][0] * Gt[0], rr[tt][1] * Gt[1], rr[tt][2] * Gt[2],
+                    rr[tt][3] * Gt[3]);
+          const float At0 = aa[tt][0] * Gp[0], At1 = aa[tt][1] * Gp[1], At2 = aa[tt][2] * Gp[2],
+                      At3 = aa[tt][3] * Gp[3];
+          st_tf32x4(a1r + tc::sw128(64 + t, chunk), At0, At1, At2, At3);
+          st_tf32x4(b1r + tc::sw128(t, chunk), bb[tt][0] * inv[0], bb[tt][1] * inv[1], bb[tt][2] * inv[2],
+                    bb[tt][3] * inv[3]);
+          st_tf32x4(b1r + tc::sw128(64 + t, chunk), kk[tt][0] * inv[0], kk[tt][1] * inv[1], kk[tt][2] * inv[2],
+                    kk[tt][3] * inv[3]);
+          // A3: A~^T as the MN-major bf16 A operand of MMA3 (M = channel, K = token)
+          *reinterpret_cast<uint2 *>(sA3 + mnmaj_bf16(64, t, j0)) =
+              make_uint2(pack_bf16x2(At0, At1), pack_bf16x2(At2, At3));
+        }
+        // V -> B4V (row = value channel, K = token); bf16 values are exact in tf32
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          *reinterpret_cast<uint4 *>(sB4Vc + kmaj_tf32(64, j0 + e, t0)) =
+              make_uint4(__float_as_uint(vv[0][e]), __float_as_uint(vv[1][e]), __float_as_uint(vv[2][e]),
+                         __float_as_uint(vv[3][e]));
+        if (tg == 0) *reinterpret_cast<float4 *>(GCs + j0) = make_float4(GC[0], GC[1], GC[2], GC[3]);
+      }
+      tc::fence_proxy_async_smem();
+      compute_sync();
+      if (tid == 0) tc::mbar_arrive(bar_p1);
+
+      // the previous chunk's MMA4 has run under P1: read it out (y rows, state update)
+      if (have_prev) {
+        if (!(ok = wait_ctrl(bar_m4, ph ^ 1u))) break;
+        tc::tc_fence_after();
+        readout(c - 1, Lc_prev);
+      }
+      // D2 set-up while MMA1 runs (it only reads A1 / B1): Q-part = R~ (lanes 0..63, rows of A1);
+      // E-part = 0 and F-part = K-^T[j][m] = Gamma_C[j] K^[m][j] (lanes 64..127, columns of B1);
+      float gc_cur = 1.f;
+      {
+        float v[32];
+        if (!hi_lanes) {
+          load_row(sA1 + ch * (128 * 128), tl, v);
+          tc::tmem_st32(tmem + lane_base + TM_D2 + 32 * ch, v);
+        } else {
+          gc_cur = GCs[j];
+          const ColPtrs ck = col_ptrs(sB1, 128, 64 + 32 * ch, j);
+#pragma unroll
+          for (int x = 0; x < 32; ++x) v[x] = gc_cur * *reinterpret_cast<const float *>(ck.p[x & 7] + x * 128);
+          tc::tmem_st32(tmem + lane_base + TM_D2 + 64 + 32 * ch, v);
+          zero32(v);
+          tc::tmem_st32(tmem + lane_base + TM_D2 + 32 * ch, v);
+        }
+        tc::tmem_st_wait();
+      }
+      tc::fence_proxy_async_smem();
+      tc::tc_fence_before();
+      compute_sync();
+      if (tid == 0) tc::mbar_arrive(bar_st);
+      if (!(ok = wait_ctrl(bar_m1, ph))) break;
+      tc::tc_fence_after();
+
+      // ---- P3: causal masks; A2 = [Mrb; B-^T] in place, P-part of D2 = Mrk -------------------------
+      // A warp's 32 token rows meet the diagonal in the 32-column half dh; each thread handles the
+      // column half hf = ch of its rows, which lies on (hf == dh), below (hf < dh) or above the diagonal.
+      {
+        const int dh = q & 1, hf = ch;
+        float v[32];
+        if (!hi_lanes) {
+          // rows t of Mrb (in place) and Mrk (moved to the P-part of D2): keep m <= t
+          if (hf == dh) {
+            tc::tmem_ld32(tmem + lane_base + TM_D1 + 32 * hf, v);
+            mask_upper(v, lane);
+            tc::tmem_st32(tmem + lane_base + TM_D1 + 32 * hf, v);
+            tc::tmem_ld32(tmem + lane_base + TM_D1 + 64 + 32 * hf, v);
+            mask_upper(v, lane);
+            tc::tmem_st32(tmem + lane_base + TM_D2 + 64 + 32 * hf, v);
+          } else if (hf > dh) {
+            zero32(v);
+            tc::tmem_st32(tmem + lane_base + TM_D1 + 32 * hf, v);
+            tc::tmem_st32(tmem + lane_base + TM_D2 + 64 + 32 * hf, v);
+          } else {
+            tc::tmem_ld32(tmem + lane_base + TM_D1 + 64 + 32 * hf, v);
+            tc::tmem_st32(tmem + lane_base + TM_D2 + 64 + 32 * hf, v);
+          }
+        } else {
+          // rows t of Lab -> Ls and Lak -> A3 (keep m < t); then B-^T into A2 in place of Lab
+          if (hf <= dh) {
+            tc::tmem_ld32(tmem + lane_base + TM_D1 + 32 * hf, v);
+            if (hf == dh) mask_upper(v, lane - 1);
+            float *row = Ls + tl * LDL + 32 * hf;
+#pragma unroll
+            for (int x = 0; x < 32; x += 4)
+              *reinterpret_cast<float4 *>(row + x) = make_float4(v[x], v[x + 1], v[x + 2], v[x + 3]);
+            tc::tmem_ld32(tmem + lane_base + TM_D1 + 64 + 32 * hf, v);
+            if (hf == dh) mask_upper(v, lane - 1);
+          } else {
+            zero32(v);
+          }
+          {
+            // A2 lower half: B-^T[j][m] = Gamma_C[j] B^[m][j] (columns of B1), in place of Lab
+            float bbar[32];
+            const ColPtrs cb = col_ptrs(sB1, 128, 32 * hf, tl);
+#pragma unroll
+            for (int x = 0; x < 32; ++x) bbar[x] = gc_cur * *reinterpret_cast<const float *>(cb.p[x & 7] + x * 128);
+            tc::tmem_st32(tmem + lane_base + TM_A2 + 32 * hf, bbar);
+          }
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
+            uint4 w4;
+            w4.x = pack_bf16x2(v[8 * cc + 0], v[8 * cc + 1]);
+            w4.y = pack_bf16x2(v[8 * cc + 2], v[8 * cc + 3]);
+            w4.z = pack_bf16x2(v[8 * cc + 4], v[8 * cc + 5]);
+            w4.w = pack_bf16x2(v[8 * cc + 6], v[8 * cc + 7]);
+            *reinterpret_cast<uint4 *>(sA3 + 64 * 128 + tc::sw128(tl, 4 * hf + cc)) = w4;
+          }
+        }
+        tc::tmem_st_wait();
+      }
+      tc::fence_proxy_async_smem();
+      tc::tc_fence_before();
+      compute_sync();
+
+      // ---- P4: Tinv = (I - Lab)^-1 as the bf16 operand B3
+      invert_unit_lower(Ls, Ts, Zs, sB3, warp, lane);
+      if (tid == 0) tc::mbar_arrive(bar_b3);
+      if (!(ok = wait_ctrl(bar_m3, ph))) break;
+      tc::tc_fence_after();
+
+      // ---- P6: D3 -> B2 (K-major: row n = column of [W~ U~], K = token; the tensor core truncates to tf32)
+      {
+        float v[32];
+        tc::tmem_ld32(tmem + lane_base + TM_D3 + 32 * ch, v);
+        store_row_f32(sB2 + ch * (128 * 128), q * 32 + lane, v);
+      }
+      tc::fence_proxy_async_smem();
+      tc::tc_fence_before();
+      compute_sync();
+
+      if (tid == 0) tc::mbar_arrive(bar_b2);
+      gc_done = gc_cur;
+      Lc_prev = Lc;
+      have_prev = true;
+    }
+    // drain: the last chunk's MMA4 and its read-out
+    if (have_prev && ok && wait_ctrl(bar_m4, (nchunks - 1) & 1)) {
+      tc::tc_fence_after();
+      readout(nchunks - 1, Lc_prev);
+    }
+    if (hi_lanes) {
+#pragma unroll
+      for (int x = 0; x < 32; ++x) A.s_out[pair * (kN * kN) + static_cast<long long>(32 * ch + x) * kN + j] = st[x];
+    }
   }
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
-  if (warp == 0) tc::tmem_dealloc(tmem, kTmemCols);
+  if (warp == kCtrlWarp) tc::tmem_dealloc(tmem, kTmemCols);
 }
 
 // ---- host side -----------------------------------------------------------------------------------

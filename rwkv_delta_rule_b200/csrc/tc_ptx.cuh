@@ -178,11 +178,11 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
 }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
 
-// float32 -> tf32 bit pattern, round to nearest (ties away from zero).
+// float32 -> tf32 bit pattern, round to nearest with ties away from zero (the
+// rounding of cvt.rna.tf32.f32), done on the integer pipe: add half an ulp of
+// the 10-bit mantissa to the magnitude bits and clear the 13 dropped bits.
 __device__ __forceinline__ uint32_t to_tf32(float x) {
-  uint32_t r;
-  asm("cvt.rna.tf32.f32 %0, %1;\n" : "=r"(r) : "f"(x));
-  return r;
+  return (__float_as_uint(x) + 0x1000u) & 0xffffe000u;
 }
 
 }  // namespace tc

@@ -14,14 +14,15 @@
 //                blocks on CUDA cores, the rest by 2x2 block doubling on
 //                warp-level tf32 mma)
 //   MMA3 (bf16)  [W~ U~]^T = [A~^T; Lak^T] Tinv^T
-//   MMA2 (tf32)  [Q P; E F] = [R~ Mrk; 0 K-^T] + [Mrb; B-^T] [W~ U~]
+//   MMA2 (bf16)  [Q P; E F] = [R~ Mrk; 0 K-^T] + [Mrb; B-^T] [W~ U~]
 //   MMA4 (tf32)  [Y; X] = [Q P; E F] [S0^T; V],   S_C^T = diag(Gamma_C) S0^T + X
 //
 // Every tf32 operand is K-major: the 128-byte-swizzled MN-major layout is not
 // valid for 32-bit operands (a tf32 MMA given one produced zeros on B200).
 //
 // The products whose rounding reaches y directly (MMA1, the per-chunk state
-// transition MMA4 and its inputs) run in tf32; MMA3 runs in bf16.  The state
+// transition MMA4 and its inputs) run in tf32; MMA3 and MMA2, whose operands
+// only shape the coefficients, run in bf16.  The state
 // is carried in float32 registers across chunks; only its tf32 copy feeds
 // MMA4.  The decay term diag(Gamma_C) S0^T is applied in float32.
 //
@@ -49,23 +50,22 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kMaxPolls = 1u << 22;
 
 // TMEM column map
-constexpr uint32_t TM_D1 = 0;    // 128 cols: [Mrb Mrk] (lanes 0-63) / [Lab Lak] (lanes 64-127);
-                                 // then A2 = [Mrb; B-^T] in cols 0-63 and D3 in cols 64-127
-constexpr uint32_t TM_A2 = 0;
+constexpr uint32_t TM_D1 = 0;    // 128 cols: [Mrb Mrk] (lanes 0-63) / [Lab Lak] (lanes 64-127); then D3 in cols 64-127
 constexpr uint32_t TM_D3 = 64;   // [W~ U~]^T (lane = column index of W~|U~, col = token)
 constexpr uint32_t TM_D2 = 128;  // 128 cols: [Q P] (lanes 0-63) / [E F] (lanes 64-127)
 constexpr uint32_t TM_D4 = 256;  // 64 cols: Y (lanes 0-63), X (lanes 64-127)
+constexpr uint32_t TM_A2 = 320;  // 32 cols: A operand [Mrb; B-^T] of MMA2, bf16 pairs (K = token)
 
 // shared memory map (bytes from a 1024-aligned base)
 constexpr uint32_t kTile = C * kN * 2;            // one bf16 64x64 tile
-constexpr uint32_t OFF_RAW = 0;                   // r w k a b v tiles, row-major [token][channel]
+constexpr uint32_t OFF_RAW = 0;                   // r w k a b v tiles, [token][channel], 128-byte swizzled
 constexpr uint32_t OFF_A1 = OFF_RAW + 6 * kTile;  // tf32 K-major [R~; A~] 128x64 (32 KB)
 constexpr uint32_t OFF_B1 = OFF_A1 + 32768;       // tf32 K-major [B^; K^] 128x64 (32 KB)
 constexpr uint32_t OFF_A3 = OFF_B1 + 32768;       // bf16 MN-major [A~^T; Lak^T], M=128 x K=64 (16 KB)
 constexpr uint32_t OFF_B4S = OFF_A3 + 16384;      // tf32 K-major S0^T part of the chain B: row i, K = j (16 KB)
 constexpr uint32_t OFF_B4V = OFF_B4S + 16384;     // 2 x tf32 K-major V part of the chain B: row i, K = m (16 KB each)
-constexpr uint32_t OFF_B2 = OFF_B4V + 2 * 16384;  // tf32 K-major [W~ U~]^T 128x64 (32 KB)
-constexpr uint32_t OFF_MISC = OFF_B2 + 32768;
+constexpr uint32_t OFF_B2 = OFF_B4V + 2 * 16384;  // bf16 K-major [W~ U~]^T 128x64 (16 KB)
+constexpr uint32_t OFF_MISC = OFF_B2 + 16384;
 // regions reused once MMA1 has consumed A1 / B1
 constexpr int LDL = 68;                             // row stride (floats) of Lab: conflict-free as an mma A operand
 constexpr int LDT = 72;                             // row stride (floats) of Tinv: conflict-free as an mma B operand
@@ -95,7 +95,7 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, vo
 }
 
 struct Maps {
-  CUtensorMap m[6];  // r, w, k, a, b, v: dims {64, H, tokens}, box {64, 1, 64}
+  CUtensorMap m[6];  // r, w, k, a, b, v: dims {64, H, tokens}, box {64, 1, 64}, 128-byte swizzle
 };
 
 struct Args {
@@ -120,6 +120,12 @@ __device__ __forceinline__ uint32_t mnmaj_bf16(uint32_t krows, uint32_t k, uint3
   return (mn >> 6) * (krows * 128u) + tc::sw128(k, (mn & 63u) >> 3) + (mn & 7u) * 2u;
 }
 
+// Row of value channel i in the chain operand B4 = [S0^T; V] (and column of i in D4).  Within each
+// 32-channel half, channel 4l + e sits in row 8e + l: the 8 lanes of a quarter-warp, which store
+// channels 4l + e (l = 0..7) of V, then write 8 rows with distinct (row % 8), i.e. 8 distinct bank
+// groups of the 128-byte swizzle.  Only the order of D4's columns changes; the read-out undoes it.
+__host__ __device__ constexpr int vrow(int i) { return (i & 32) | ((i & 3) << 3) | ((i >> 2) & 7); }
+
 // One column k = j of 32 consecutive rows row0 .. row0+31 (row0 a multiple of
 // 8) of a K-major 32-bit operand whose K-atoms hold `rows` rows: row row0 + x
 // sits at p[x & 7] + x * 128, so the unrolled accesses need no address math.
@@ -135,30 +141,39 @@ __device__ __forceinline__ ColPtrs col_ptrs(uint8_t *region, uint32_t rows, uint
   return c;
 }
 
-// four consecutive bf16 channels of one token row of a raw tile
+// four consecutive bf16 channels (j0 % 4 == 0) of one token row of a raw tile; the tiles land
+// 128-byte swizzled (16-byte chunk c of row t at chunk c ^ (t % 8)), so the four token groups
+// of a warp, four rows apart, read from two disjoint bank halves
 __device__ __forceinline__ void raw4(const uint8_t *smem, int tile, int t, int j0, float (&o)[4]) {
-  const uint2 u = *reinterpret_cast<const uint2 *>(smem + OFF_RAW + tile * kTile + (t * kN + j0) * 2);
+  const uint32_t byte = static_cast<uint32_t>(j0) * 2u;
+  const uint2 u = *reinterpret_cast<const uint2 *>(smem + OFF_RAW + tile * kTile + tc::sw128(t, byte >> 4) +
+                                                   (byte & 15u));
   o[0] = __uint_as_float(u.x << 16);
   o[1] = __uint_as_float(u.x & 0xffff0000u);
   o[2] = __uint_as_float(u.y << 16);
   o[3] = __uint_as_float(u.y & 0xffff0000u);
 }
 
+// two floats -> one bf16x2 word (round to nearest even; lo in the low half), one cvt instruction
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  return static_cast<uint32_t>(float_to_bf16_bits(lo)) | (static_cast<uint32_t>(float_to_bf16_bits(hi)) << 16);
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;\n" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// 32 consecutive K values of one A-operand row -> 16 TMEM columns of bf16 pairs
+__device__ __forceinline__ void tmem_st_bf16x32(uint32_t taddr, const float (&v)[32]) {
+  float p[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) p[i] = __uint_as_float(pack_bf16x2(v[2 * i], v[2 * i + 1]));
+  tc::tmem_st16(taddr, p);
 }
 
 __device__ __forceinline__ void st_tf32x4(uint8_t *p, float a, float b, float c, float d) {
   *reinterpret_cast<uint4 *>(p) = make_uint4(tc::to_tf32(a), tc::to_tf32(b), tc::to_tf32(c), tc::to_tf32(d));
 }
 
-// 32 consecutive values of one 128-byte swizzled row: raw float32 bits / read back
-__device__ __forceinline__ void store_row_f32(uint8_t *blk, uint32_t row, const float (&v)[32]) {
-#pragma unroll
-  for (int c = 0; c < 8; ++c)
-    *reinterpret_cast<float4 *>(blk + tc::sw128(row, c)) =
-        make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
-}
+// 32 consecutive float32 values of one 128-byte swizzled row
 __device__ __forceinline__ void load_row(const uint8_t *blk, uint32_t row, float (&v)[32]) {
 #pragma unroll
   for (int c = 0; c < 8; ++c) {
@@ -179,13 +194,16 @@ __device__ __forceinline__ void zero32(float (&v)[32]) {
   for (int x = 0; x < 32; ++x) v[x] = 0.f;
 }
 
-// B4S holds S0^T as the K-major B operand of the chain product: row = value
-// channel i, K = key channel j.  A state thread owns S^T[j][32*ch + x], i.e.
+// B4S holds S0^T as the K-major B operand of the chain product: row = vrow(value
+// channel i), K = key channel j.  A state thread owns S^T[j][32*ch + x], i.e.
 // column j of rows 32*ch .. 32*ch+31.
 __device__ __forceinline__ void store_state_tf32(uint8_t *sB4S, int j, int ch, const float (&st)[32]) {
   const ColPtrs cp = col_ptrs(sB4S, 64, 32 * ch, j);
 #pragma unroll
-  for (int x = 0; x < 32; ++x) *reinterpret_cast<uint32_t *>(cp.p[x & 7] + x * 128) = tc::to_tf32(st[x]);
+  for (int x = 0; x < 32; ++x) {
+    const int row = vrow(x);  // value channel 32*ch + x, permuted within its half
+    *reinterpret_cast<uint32_t *>(cp.p[row & 7] + row * 128) = tc::to_tf32(st[x]);
+  }
 }
 
 // Stores a 16x16 mma-layout accumulator as bf16 into a K-major bf16 operand
@@ -228,13 +246,15 @@ __device__ __forceinline__ void invert_unit_lower(const float *Ls, float *Ts, fl
           if (4 * q4 + e < r) Lr[r * (r - 1) / 2 + 4 * q4 + e] = uu[e];
       }
     }
+    // column sweep: once x_q is final it is pushed into every later row, so the 15 updates of a
+    // step are independent (each row still sums its terms in increasing q)
     float x[16];
 #pragma unroll
-    for (int r = 0; r < 16; ++r) {
-      float acc = (r == cix) ? 1.f : 0.f;
+    for (int r = 0; r < 16; ++r) x[r] = (r == cix) ? 1.f : 0.f;
 #pragma unroll
-      for (int q = 0; q < r; ++q) acc = fmaf(Lr[r * (r - 1) / 2 + q], x[q], acc);
-      x[r] = acc;
+    for (int q = 0; q < 15; ++q) {
+#pragma unroll
+      for (int r = q + 1; r < 16; ++r) x[r] = fmaf(Lr[r * (r - 1) / 2 + q], x[q], x[r]);
     }
     if (lane < 16) {
       const int m = base + cix;
@@ -365,13 +385,6 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
         const uint32_t ph = c & 1;
         // MMA1 (tf32): D1 = [R~; A~] [B^; K^]^T, once the operands are in place
         if (!wait_or_abort(bar_p1, ph, abort_flag)) { fail(); break; }
-        if (c + 1 < nchunks) {
-          tc::mbar_arrive_expect_tx(bar_tma, 6 * kTile);
-          for (int i = 0; i < 6; ++i)
-            tc::tma_load_3d(smem + OFF_RAW + i * kTile, &maps.m[i], bar_tma, 0, h,
-                            static_cast<int>(sb.start + static_cast<long long>(c + 1) * C));
-          last_tma = (c + 1) & 1;
-        }
         tc::tc_fence_after();
         {
           constexpr uint32_t idesc = tc::instr_desc(tc::kFmtTF32, 128, 128, false, false);
@@ -384,6 +397,15 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
           }
           tc::mma_commit(bar_m1);
           last_m1 = ph;
+        }
+        // the next chunk's tiles (P1 has consumed the raw tiles), issued after MMA1: six TMA issues
+        // take longer than MMA1 itself
+        if (c + 1 < nchunks) {
+          tc::mbar_arrive_expect_tx(bar_tma, 6 * kTile);
+          for (int i = 0; i < 6; ++i)
+            tc::tma_load_3d(smem + OFF_RAW + i * kTile, &maps.m[i], bar_tma, 0, h,
+                            static_cast<int>(sb.start + static_cast<long long>(c + 1) * C));
+          last_tma = (c + 1) & 1;
         }
         // MMA3 (bf16): D3 = [A~^T; Lak^T] Tinv^T
         if (!wait_or_abort(bar_b3, ph, abort_flag)) { fail(); break; }
@@ -398,17 +420,15 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
           tc::mma_commit(bar_m3);
           last_m3 = ph;
         }
-        // MMA2 (tf32, A from TMEM): D2 += [Mrb; B-^T] [W~ U~]
+        // MMA2 (bf16, A from TMEM): D2 += [Mrb; B-^T] [W~ U~]
         if (!wait_or_abort(bar_b2, ph, abort_flag)) { fail(); break; }
         tc::tc_fence_after();
         {
-          constexpr uint32_t idesc = tc::instr_desc(tc::kFmtTF32, 128, 128, false, false);
+          constexpr uint32_t idesc = tc::instr_desc(tc::kFmtBF16, 128, 128, false, false);
           const uint32_t b2 = smem_u32(sB2);
 #pragma unroll
-          for (int ks = 0; ks < 8; ++ks) {
-            const uint32_t off = (ks >> 2) * (128 * 128) + (ks & 3) * 32;
-            tc::mma_ts_tf32(tmem + TM_D2, tmem + TM_A2 + 8 * ks, tc::smem_desc(b2 + off, 16, 1024), idesc, 1);
-          }
+          for (int ks = 0; ks < 4; ++ks)
+            tc::mma_ts_bf16(tmem + TM_D2, tmem + TM_A2 + 8 * ks, tc::smem_desc(b2 + ks * 32, 16, 1024), idesc, 1);
           tc::mma_commit(bar_m2);
           last_m2 = ph;
         }
@@ -480,6 +500,7 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
     bool ok = true;
     // Read-out of a finished chunk: y rows (lanes 0..63) and the state update
     // S_C^T = diag(Gamma_C) S0^T + X (lanes 64..127), whose tf32 copy feeds the next MMA4.
+    // D4 column vrow(i) holds value channel i.
     float gc_done = 1.f;  // Gamma_C[j] of the chunk whose MMA4 is in flight (hi lanes)
     auto readout = [&](int cidx, int Lcx) {
       float v[32];
@@ -491,16 +512,16 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
 #pragma unroll
           for (int cc = 0; cc < 4; ++cc) {
             uint4 w4;
-            w4.x = pack_bf16x2(v[8 * cc + 0], v[8 * cc + 1]);
-            w4.y = pack_bf16x2(v[8 * cc + 2], v[8 * cc + 3]);
-            w4.z = pack_bf16x2(v[8 * cc + 4], v[8 * cc + 5]);
-            w4.w = pack_bf16x2(v[8 * cc + 6], v[8 * cc + 7]);
+            w4.x = pack_bf16x2(v[vrow(8 * cc + 0)], v[vrow(8 * cc + 1)]);
+            w4.y = pack_bf16x2(v[vrow(8 * cc + 2)], v[vrow(8 * cc + 3)]);
+            w4.z = pack_bf16x2(v[vrow(8 * cc + 4)], v[vrow(8 * cc + 5)]);
+            w4.w = pack_bf16x2(v[vrow(8 * cc + 6)], v[vrow(8 * cc + 7)]);
             *reinterpret_cast<uint4 *>(dst + 8 * cc) = w4;
           }
         }
       } else {
 #pragma unroll
-        for (int x = 0; x < 32; ++x) st[x] = fmaf(gc_done, st[x], v[x]);
+        for (int x = 0; x < 32; ++x) st[x] = fmaf(gc_done, st[x], v[vrow(x)]);
         store_state_tf32(sB4S, j, ch, st);
       }
     };
@@ -609,10 +630,10 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
           *reinterpret_cast<uint2 *>(sA3 + mnmaj_bf16(64, t, j0)) =
               make_uint2(pack_bf16x2(At0, At1), pack_bf16x2(At2, At3));
         }
-        // V -> B4V (row = value channel, K = token); bf16 values are exact in tf32
+        // V -> B4V (row = vrow(value channel), K = token); bf16 values are exact in tf32
 #pragma unroll
         for (int e = 0; e < 4; ++e)
-          *reinterpret_cast<uint4 *>(sB4Vc + kmaj_tf32(64, j0 + e, t0)) =
+          *reinterpret_cast<uint4 *>(sB4Vc + kmaj_tf32(64, vrow(j0 + e), t0)) =
               make_uint4(__float_as_uint(vv[0][e]), __float_as_uint(vv[1][e]), __float_as_uint(vv[2][e]),
                          __float_as_uint(vv[3][e]));
         if (tg == 0) *reinterpret_cast<float4 *>(GCs + j0) = make_float4(GC[0], GC[1], GC[2], GC[3]);
@@ -660,24 +681,34 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
         const int dh = q & 1, hf = ch;
         float v[32];
         if (!hi_lanes) {
-          // rows t of Mrb (in place) and Mrk (moved to the P-part of D2): keep m <= t
+          // rows t of Mrb (to A2 as bf16) and Mrk (moved to the P-part of D2): keep m <= t
           if (hf == dh) {
             tc::tmem_ld32(tmem + lane_base + TM_D1 + 32 * hf, v);
             mask_upper(v, lane);
-            tc::tmem_st32(tmem + lane_base + TM_D1 + 32 * hf, v);
+            tmem_st_bf16x32(tmem + lane_base + TM_A2 + 16 * hf, v);
             tc::tmem_ld32(tmem + lane_base + TM_D1 + 64 + 32 * hf, v);
             mask_upper(v, lane);
             tc::tmem_st32(tmem + lane_base + TM_D2 + 64 + 32 * hf, v);
           } else if (hf > dh) {
             zero32(v);
-            tc::tmem_st32(tmem + lane_base + TM_D1 + 32 * hf, v);
+            tmem_st_bf16x32(tmem + lane_base + TM_A2 + 16 * hf, v);
             tc::tmem_st32(tmem + lane_base + TM_D2 + 64 + 32 * hf, v);
           } else {
+            tc::tmem_ld32(tmem + lane_base + TM_D1 + 32 * hf, v);
+            tmem_st_bf16x32(tmem + lane_base + TM_A2 + 16 * hf, v);
             tc::tmem_ld32(tmem + lane_base + TM_D1 + 64 + 32 * hf, v);
             tc::tmem_st32(tmem + lane_base + TM_D2 + 64 + 32 * hf, v);
           }
         } else {
-          // rows t of Lab -> Ls and Lak -> A3 (keep m < t); then B-^T into A2 in place of Lab
+          // B-^T -> A2 (bf16); rows t of Lab -> Ls and Lak -> A3 (keep m < t)
+          {
+            // A2 lower half: B-^T[j][m] = Gamma_C[j] B^[m][j] (columns of B1)
+            float bbar[32];
+            const ColPtrs cb = col_ptrs(sB1, 128, 32 * hf, tl);
+#pragma unroll
+            for (int x = 0; x < 32; ++x) bbar[x] = gc_cur * *reinterpret_cast<const float *>(cb.p[x & 7] + x * 128);
+            tmem_st_bf16x32(tmem + lane_base + TM_A2 + 16 * hf, bbar);
+          }
           if (hf <= dh) {
             tc::tmem_ld32(tmem + lane_base + TM_D1 + 32 * hf, v);
             if (hf == dh) mask_upper(v, lane - 1);
@@ -689,14 +720,6 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
             if (hf == dh) mask_upper(v, lane - 1);
           } else {
             zero32(v);
-          }
-          {
-            // A2 lower half: B-^T[j][m] = Gamma_C[j] B^[m][j] (columns of B1), in place of Lab
-            float bbar[32];
-            const ColPtrs cb = col_ptrs(sB1, 128, 32 * hf, tl);
-#pragma unroll
-            for (int x = 0; x < 32; ++x) bbar[x] = gc_cur * *reinterpret_cast<const float *>(cb.p[x & 7] + x * 128);
-            tc::tmem_st32(tmem + lane_base + TM_A2 + 32 * hf, bbar);
           }
 #pragma unroll
           for (int cc = 0; cc < 4; ++cc) {
@@ -720,11 +743,20 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
       if (!(ok = wait_ctrl(bar_m3, ph))) break;
       tc::tc_fence_after();
 
-      // ---- P6: D3 -> B2 (K-major: row n = column of [W~ U~], K = token; the tensor core truncates to tf32)
+      // ---- P6: D3 -> B2 (bf16, K-major: row n = column of [W~ U~], K = token)
       {
         float v[32];
         tc::tmem_ld32(tmem + lane_base + TM_D3 + 32 * ch, v);
-        store_row_f32(sB2 + ch * (128 * 128), q * 32 + lane, v);
+        const uint32_t n = q * 32 + lane;
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          uint4 w4;
+          w4.x = pack_bf16x2(v[8 * cc + 0], v[8 * cc + 1]);
+          w4.y = pack_bf16x2(v[8 * cc + 2], v[8 * cc + 3]);
+          w4.z = pack_bf16x2(v[8 * cc + 4], v[8 * cc + 5]);
+          w4.w = pack_bf16x2(v[8 * cc + 6], v[8 * cc + 7]);
+          *reinterpret_cast<uint4 *>(sB2 + tc::sw128(n, 4 * ch + cc)) = w4;
+        }
       }
       tc::fence_proxy_async_smem();
       tc::tc_fence_before();
@@ -780,7 +812,7 @@ static bool make_map(CUtensorMap *map, const void *base, long long tokens, int H
   const cuuint32_t box[3] = {static_cast<cuuint32_t>(kN), 1, static_cast<cuuint32_t>(C)};
   const cuuint32_t estr[3] = {1, 1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 

@@ -55,6 +55,7 @@ constexpr uint32_t TM_D3 = 64;   // [W~ U~]^T (lane = column index of W~|U~, col
 constexpr uint32_t TM_D2 = 128;  // 128 cols: [Q P] (lanes 0-63) / [E F] (lanes 64-127)
 constexpr uint32_t TM_D4 = 256;  // 64 cols: Y (lanes 0-63), X (lanes 64-127)
 constexpr uint32_t TM_A2 = 320;  // 32 cols: A operand [Mrb; B-^T] of MMA2, bf16 pairs (K = token)
+constexpr uint32_t TM_S = 384;   // 64 cols, lanes 64-127: the float32 state S^T (lane 64 + j, column vrow(i))
 
 // shared memory map (bytes from a 1024-aligned base)
 constexpr uint32_t kTile = C * kN * 2;            // one bf16 64x64 tile
@@ -65,25 +66,30 @@ constexpr uint32_t OFF_A3 = OFF_B1 + 32768;       // bf16 MN-major [A~^T; Lak^T]
 constexpr uint32_t OFF_B4S = OFF_A3 + 16384;      // tf32 K-major S0^T part of the chain B: row i, K = j (16 KB)
 constexpr uint32_t OFF_B4V = OFF_B4S + 16384;     // 2 x tf32 K-major V part of the chain B: row i, K = m (16 KB each)
 constexpr uint32_t OFF_B2 = OFF_B4V + 2 * 16384;  // bf16 K-major [W~ U~]^T 128x64 (16 KB)
-constexpr uint32_t OFF_MISC = OFF_B2 + 16384;
-// regions reused once MMA1 has consumed A1 / B1
-constexpr int LDL = 68;                             // row stride (floats) of Lab: conflict-free as an mma A operand
-constexpr int LDT = 72;                             // row stride (floats) of Tinv: conflict-free as an mma B operand
-constexpr int LDZ = 24;                             // row stride (floats) of 16x16 scratch blocks
-constexpr uint32_t OFF_LS = OFF_A1;                 // float [64][LDL]
-constexpr uint32_t OFF_ZS = OFF_A1 + 64 * LDL * 4;  // float [6][16][LDZ] scratch blocks of the inverse
-constexpr uint32_t OFF_TS = OFF_B1;                 // float [64][LDT]
-constexpr uint32_t OFF_B3 = OFF_B1 + 19456;         // bf16 K-major Tinv 64x64 (8 KB), 1024-aligned
-constexpr uint32_t MISC_GC = 256;                   // float [64]    Gamma at the chunk end
-constexpr uint32_t MISC_WTOT = 512;                 // float [4][64] decay products of 16-token blocks
-constexpr uint32_t kSmemBytes = OFF_MISC + MISC_WTOT + 4 * 64 * 4 + 1024;
+constexpr uint32_t OFF_MISC = OFF_B2 + 16384;      // mbarriers, slots, Gamma_C, block decay products (2 KB)
+// scratch of the inverse: it runs while other warps still read R~ (A1) and K^ (B1), so it lives in
+// its own region (Lab and the fp32 blocks of Tinv) and in B2, which is idle until MMA3 has run
+constexpr int LDL = 68;   // row stride (floats) of Lab: conflict-free as an mma A operand
+constexpr int LDTB = 24;  // row stride (floats) of the 16x16 fp32 blocks of Tinv (conflict-free as a B operand)
+constexpr int LDZ = 20;   // row stride (floats) of the 16x16 scratch products
+constexpr uint32_t OFF_LS = OFF_MISC + 2048;              // float [64][LDL]
+constexpr uint32_t OFF_TS = OFF_LS + 64 * LDL * 4;        // float [6][16][LDTB]: Tinv blocks (s,s), (1,0), (3,2)
+constexpr uint32_t OFF_B3 = OFF_B2;                       // bf16 K-major Tinv 64x64 (8 KB), 1024-aligned
+constexpr uint32_t OFF_ZS = OFF_B2 + 8192;                // float [6][16][LDZ]
+constexpr uint32_t MISC_GC = 256;                         // float [64]    Gamma at the chunk end
+constexpr uint32_t MISC_WTOT = 512;                       // float [4][64] decay products of 16-token blocks
+constexpr uint32_t kSmemBytes = OFF_TS + 6 * 16 * LDTB * 4 + 1024;
 
-static_assert(OFF_ZS + 6 * 16 * LDZ * 4 <= OFF_B1, "inverse scratch overflows A1");
-static_assert(OFF_TS + 64 * LDT * 4 <= OFF_B3 && OFF_B3 + 8192 <= OFF_A3, "inverse scratch overflows B1");
+static_assert(MISC_WTOT + 4 * 64 * 4 <= 2048, "misc region overflow");
+static_assert(OFF_ZS + 6 * 16 * LDZ * 4 <= OFF_B2 + 16384, "inverse scratch overflows B2");
 static_assert(kSmemBytes <= 232448, "shared memory over the sm_100 limit");
 
 // Barrier among the 8 compute warps only (the control warp never joins it).
 __device__ __forceinline__ void compute_sync() { asm volatile("bar.sync 1, 256;\n" ::: "memory"); }
+// Barriers of the two compute groups while they work apart: warps 0-3 (the inverse) and warps 4-7
+// (read-out and set-up).
+__device__ __forceinline__ void group_sync_lo() { asm volatile("bar.sync 2, 128;\n" ::: "memory"); }
+__device__ __forceinline__ void group_sync_hi() { asm volatile("bar.sync 3, 128;\n" ::: "memory"); }
 
 // Bounded mbarrier wait that also gives up once the CTA is aborting.
 __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
@@ -194,16 +200,12 @@ __device__ __forceinline__ void zero32(float (&v)[32]) {
   for (int x = 0; x < 32; ++x) v[x] = 0.f;
 }
 
-// B4S holds S0^T as the K-major B operand of the chain product: row = vrow(value
-// channel i), K = key channel j.  A state thread owns S^T[j][32*ch + x], i.e.
-// column j of rows 32*ch .. 32*ch+31.
-__device__ __forceinline__ void store_state_tf32(uint8_t *sB4S, int j, int ch, const float (&st)[32]) {
-  const ColPtrs cp = col_ptrs(sB4S, 64, 32 * ch, j);
+// B4S holds S0^T as the K-major B operand of the chain product: row p = vrow(value channel i),
+// K = key channel j.  Stores rows 32*hh .. 32*hh+31 of column j (tf32).
+__device__ __forceinline__ void store_state_rows_tf32(uint8_t *sB4S, int j, int hh, const float (&v)[32]) {
+  const ColPtrs cp = col_ptrs(sB4S, 64, 32 * hh, j);
 #pragma unroll
-  for (int x = 0; x < 32; ++x) {
-    const int row = vrow(x);  // value channel 32*ch + x, permuted within its half
-    *reinterpret_cast<uint32_t *>(cp.p[row & 7] + row * 128) = tc::to_tf32(st[x]);
-  }
+  for (int x = 0; x < 32; ++x) *reinterpret_cast<uint32_t *>(cp.p[x & 7] + x * 128) = tc::to_tf32(v[x]);
 }
 
 // Stores a 16x16 mma-layout accumulator as bf16 into a K-major bf16 operand
@@ -221,6 +223,11 @@ __device__ __forceinline__ void block16_store_bf16(uint8_t *op, int row0, int co
   }
 }
 
+// fp32 block (r, c) of Tinv in the compact scratch: the diagonal blocks, (1,0) and (3,2)
+__device__ __forceinline__ float *ts_block(float *Ts, int r, int c) {
+  return Ts + ((r == c) ? r : (r == 1 ? 4 : 5)) * (16 * LDTB);
+}
+
 // Tinv = (I - L)^-1 for the strictly lower 64x64 matrix L in Ls (only entries
 // below the diagonal are read).  Writes Tinv as the bf16 K-major operand B3
 // (row t, K = m; zero above the block diagonal), using Ts (float32) for the
@@ -228,10 +235,21 @@ __device__ __forceinline__ void block16_store_bf16(uint8_t *op, int row0, int co
 // block-triangular M = I - L:  (M^-1)_BA = (M^-1)_BB L_BA (M^-1)_AA,
 // first for the 16x16 diagonal blocks (forward substitution in registers),
 // then for blocks (1,0), (3,2) and finally the lower-left 32x32 block, each
-// 16x16 product on warp-level tf32 mma.  Every thread of the CTA must call it.
+// 16x16 product on warp-level tf32 mma.  Called by warps 0-3 only (they
+// synchronise among themselves); ends with B3 visible to the tensor core.
 __device__ __forceinline__ void invert_unit_lower(const float *Ls, float *Ts, float *Zs, uint8_t *sB3, int warp,
                                                   int lane) {
-  if (warp < 4) {
+  {
+    // the six 16x16 blocks above the block diagonal are zero: 16 rows x 2 chunks each
+    const int e = warp * 32 + lane;
+    for (int k = e; k < 6 * 32; k += 128) {
+      const int blk = k >> 5, rr = (k >> 1) & 15, half = k & 1;
+      const int sr = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
+      const int sc = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
+      *reinterpret_cast<uint4 *>(sB3 + tc::sw128(16 * sr + rr, 2 * sc + half)) = make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+  {
     // diagonal block s = warp: column cix of (I - L_ss)^-1, x_r = [r == c] + sum_{q<r} L_rq x_q
     const int base = 16 * warp, cix = lane & 15;
     float Lr[120];  // Lr[r(r-1)/2 + q] = L[base + r][base + q] for q < r
@@ -258,58 +276,51 @@ __device__ __forceinline__ void invert_unit_lower(const float *Ls, float *Ts, fl
     }
     if (lane < 16) {
       const int m = base + cix;
+      float *D = ts_block(Ts, warp, warp);
 #pragma unroll
       for (int r = 0; r < 16; ++r) {
-        Ts[(base + r) * LDT + m] = x[r];
+        D[r * LDTB + cix] = x[r];
         *reinterpret_cast<uint16_t *>(sB3 + tc::sw128(base + r, m >> 3) + (m & 7) * 2) = float_to_bf16_bits(x[r]);
       }
     }
-  } else {
-    // the six 16x16 blocks above the block diagonal are zero: 16 rows x 2 chunks each
-    for (int e = (warp - 4) * 32 + lane; e < 6 * 32; e += 128) {
-      const int blk = e >> 5, rr = (e >> 1) & 15, half = e & 1;
-      const int sr = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
-      const int sc = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
-      *reinterpret_cast<uint4 *>(sB3 + tc::sw128(16 * sr + rr, 2 * sc + half)) = make_uint4(0u, 0u, 0u, 0u);
-    }
   }
-  compute_sync();
+  group_sync_lo();
   if (warp < 2) {
     // T_{s+1,s} = D_{s+1} L_{s+1,s} D_s for s = 0, 2
     const int s = 2 * warp;
     float *Z = Zs + warp * (16 * LDZ);
     float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-    tc::block16_mma(acc, Ls + (16 * (s + 1)) * LDL + 16 * s, LDL, Ts + (16 * s) * LDT + 16 * s, LDT, lane);
+    tc::block16_mma(acc, Ls + (16 * (s + 1)) * LDL + 16 * s, LDL, ts_block(Ts, s, s), LDTB, lane);
     tc::block16_store(Z, LDZ, acc, lane);
     __syncwarp();
     float t2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-    tc::block16_mma(t2, Ts + (16 * (s + 1)) * LDT + 16 * (s + 1), LDT, Z, LDZ, lane);
-    tc::block16_store(Ts + (16 * (s + 1)) * LDT + 16 * s, LDT, t2, lane);
+    tc::block16_mma(t2, ts_block(Ts, s + 1, s + 1), LDTB, Z, LDZ, lane);
+    tc::block16_store(ts_block(Ts, s + 1, s), LDTB, t2, lane);
     block16_store_bf16(sB3, 16 * (s + 1), 16 * s, t2, lane);
   }
-  compute_sync();
+  group_sync_lo();
   // lower-left 32x32 block, one warp per 16x16 tile (s, m), s in {2, 3}, m in {0, 1}
   const int s = 2 + (warp >> 1), m = warp & 1;
-  if (warp < 4) {
+  {
     // X_sm = sum_{q=m}^{1} L_sq T_qm
     float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
     for (int q = 0; q < 2; ++q)
-      if (q >= m) tc::block16_mma(acc, Ls + (16 * s) * LDL + 16 * q, LDL, Ts + (16 * q) * LDT + 16 * m, LDT, lane);
+      if (q >= m) tc::block16_mma(acc, Ls + (16 * s) * LDL + 16 * q, LDL, ts_block(Ts, q, m), LDTB, lane);
     tc::block16_store(Zs + (2 + warp) * (16 * LDZ), LDZ, acc, lane);
   }
-  compute_sync();
-  if (warp < 4) {
+  group_sync_lo();
+  {
     // T_sm = sum_{p=2}^{s} T_sp X_pm
     float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
     for (int p = 2; p < 4; ++p)
       if (p <= s)
-        tc::block16_mma(acc, Ts + (16 * s) * LDT + 16 * p, LDT, Zs + (2 + 2 * (p - 2) + m) * (16 * LDZ), LDZ, lane);
+        tc::block16_mma(acc, ts_block(Ts, s, p), LDTB, Zs + (2 + 2 * (p - 2) + m) * (16 * LDZ), LDZ, lane);
     block16_store_bf16(sB3, 16 * s, 16 * m, acc, lane);
   }
   tc::fence_proxy_async_smem();
-  compute_sync();
+  group_sync_lo();
 }
 
 __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_constant__ Maps maps, const Args A) {
@@ -472,13 +483,16 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
     const int j0 = 4 * cq, t0 = 4 * tg;
     const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
 
-    // state: hi-lane threads hold S^T[j][32*ch .. 32*ch+31] in float32
-    float st[32];
+    // The float32 state S^T lives in TMEM (lane 64 + j, column vrow(i)); the hi-lane warps own those
+    // lanes (column half ch each) and keep its tf32 copy in B4S.
     if (hi_lanes) {
+      float v[32];
 #pragma unroll
       for (int x = 0; x < 32; ++x)
-        st[x] = A.s_in ? A.s_in[pair * (kN * kN) + static_cast<long long>(32 * ch + x) * kN + j] : 0.f;
-      store_state_tf32(sB4S, j, ch, st);
+        v[vrow(x)] = A.s_in ? A.s_in[pair * (kN * kN) + static_cast<long long>(32 * ch + x) * kN + j] : 0.f;
+      tc::tmem_st32(tmem + lane_base + TM_S + 32 * ch, v);
+      store_state_rows_tf32(sB4S, j, ch, v);
+      tc::tmem_st_wait();
     }
     // Wait for the control warp (one thread polls, bounded); false once the CTA aborts.  Thread 0
     // publishes the decision in a slot chosen by the call parity before the barrier, so every compute
@@ -499,30 +513,36 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
     };
     bool ok = true;
     // Read-out of a finished chunk: y rows (lanes 0..63) and the state update
-    // S_C^T = diag(Gamma_C) S0^T + X (lanes 64..127), whose tf32 copy feeds the next MMA4.
-    // D4 column vrow(i) holds value channel i.
+    // S_C^T = diag(Gamma_C) S0^T + X (lanes 64..127), whose tf32 copy feeds the next MMA4; each warp
+    // takes the column half ch.  D4 column vrow(i) holds value channel i, like the state in TMEM.
     float gc_done = 1.f;  // Gamma_C[j] of the chunk whose MMA4 is in flight (hi lanes)
     auto readout = [&](int cidx, int Lcx) {
-      float v[32];
-      tc::tmem_ld32(tmem + lane_base + TM_D4 + 32 * ch, v);
-      if (!hi_lanes) {
-        if (tl < Lcx) {
-          const long long tok = sb.start + static_cast<long long>(cidx) * C + tl;
-          uint16_t *dst = A.y + (tok * A.H + h) * kN + 32 * ch;
+      {
+        const int hh = ch;
+        float v[32];
+        tc::tmem_ld32(tmem + lane_base + TM_D4 + 32 * hh, v);
+        if (!hi_lanes) {
+          if (tl < Lcx) {
+            const long long tok = sb.start + static_cast<long long>(cidx) * C + tl;
+            uint16_t *dst = A.y + (tok * A.H + h) * kN + 32 * hh;
 #pragma unroll
-          for (int cc = 0; cc < 4; ++cc) {
-            uint4 w4;
-            w4.x = pack_bf16x2(v[vrow(8 * cc + 0)], v[vrow(8 * cc + 1)]);
-            w4.y = pack_bf16x2(v[vrow(8 * cc + 2)], v[vrow(8 * cc + 3)]);
-            w4.z = pack_bf16x2(v[vrow(8 * cc + 4)], v[vrow(8 * cc + 5)]);
-            w4.w = pack_bf16x2(v[vrow(8 * cc + 6)], v[vrow(8 * cc + 7)]);
-            *reinterpret_cast<uint4 *>(dst + 8 * cc) = w4;
+            for (int cc = 0; cc < 4; ++cc) {
+              uint4 w4;
+              w4.x = pack_bf16x2(v[vrow(8 * cc + 0)], v[vrow(8 * cc + 1)]);
+              w4.y = pack_bf16x2(v[vrow(8 * cc + 2)], v[vrow(8 * cc + 3)]);
+              w4.z = pack_bf16x2(v[vrow(8 * cc + 4)], v[vrow(8 * cc + 5)]);
+              w4.w = pack_bf16x2(v[vrow(8 * cc + 6)], v[vrow(8 * cc + 7)]);
+              *reinterpret_cast<uint4 *>(dst + 8 * cc) = w4;
+            }
           }
-        }
-      } else {
+        } else {
+          float sv[32];
+          tc::tmem_ld32(tmem + lane_base + TM_S + 32 * hh, sv);
 #pragma unroll
-        for (int x = 0; x < 32; ++x) st[x] = fmaf(gc_done, st[x], v[vrow(x)]);
-        store_state_tf32(sB4S, j, ch, st);
+          for (int x = 0; x < 32; ++x) sv[x] = fmaf(gc_done, sv[x], v[x]);
+          tc::tmem_st32(tmem + lane_base + TM_S + 32 * hh, sv);
+          store_state_rows_tf32(sB4S, j, hh, sv);
+        }
       }
     };
 
@@ -641,40 +661,16 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
       tc::fence_proxy_async_smem();
       compute_sync();
       if (tid == 0) tc::mbar_arrive(bar_p1);
-
-      // the previous chunk's MMA4 has run under P1: read it out (y rows, state update)
+      // while MMA1 runs: the previous chunk's MMA4 (which ran under P1) is read out
       if (have_prev) {
         if (!(ok = wait_ctrl(bar_m4, ph ^ 1u))) break;
         tc::tc_fence_after();
         readout(c - 1, Lc_prev);
       }
-      // D2 set-up while MMA1 runs (it only reads A1 / B1): Q-part = R~ (lanes 0..63, rows of A1);
-      // E-part = 0 and F-part = K-^T[j][m] = Gamma_C[j] K^[m][j] (lanes 64..127, columns of B1);
-      float gc_cur = 1.f;
-      {
-        float v[32];
-        if (!hi_lanes) {
-          load_row(sA1 + ch * (128 * 128), tl, v);
-          tc::tmem_st32(tmem + lane_base + TM_D2 + 32 * ch, v);
-        } else {
-          gc_cur = GCs[j];
-          const ColPtrs ck = col_ptrs(sB1, 128, 64 + 32 * ch, j);
-#pragma unroll
-          for (int x = 0; x < 32; ++x) v[x] = gc_cur * *reinterpret_cast<const float *>(ck.p[x & 7] + x * 128);
-          tc::tmem_st32(tmem + lane_base + TM_D2 + 64 + 32 * ch, v);
-          zero32(v);
-          tc::tmem_st32(tmem + lane_base + TM_D2 + 32 * ch, v);
-        }
-        tc::tmem_st_wait();
-      }
-      tc::fence_proxy_async_smem();
-      tc::tc_fence_before();
-      compute_sync();
-      if (tid == 0) tc::mbar_arrive(bar_st);
       if (!(ok = wait_ctrl(bar_m1, ph))) break;
       tc::tc_fence_after();
 
-      // ---- P3: causal masks; A2 = [Mrb; B-^T] in place, P-part of D2 = Mrk -------------------------
+      // ---- P3: causal masks; A2 = [Mrb; B-^T] (bf16), P-part of D2 = Mrk ----------------------------
       // A warp's 32 token rows meet the diagonal in the 32-column half dh; each thread handles the
       // column half hf = ch of its rows, which lies on (hf == dh), below (hf < dh) or above the diagonal.
       {
@@ -702,11 +698,12 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
         } else {
           // B-^T -> A2 (bf16); rows t of Lab -> Ls and Lak -> A3 (keep m < t)
           {
-            // A2 lower half: B-^T[j][m] = Gamma_C[j] B^[m][j] (columns of B1)
+            // A2 lower half: B-^T[j][m] = Gamma_C[j] B^[m][j] (columns of B1), j = tl
             float bbar[32];
+            const float gcj = GCs[tl];
             const ColPtrs cb = col_ptrs(sB1, 128, 32 * hf, tl);
 #pragma unroll
-            for (int x = 0; x < 32; ++x) bbar[x] = gc_cur * *reinterpret_cast<const float *>(cb.p[x & 7] + x * 128);
+            for (int x = 0; x < 32; ++x) bbar[x] = gcj * *reinterpret_cast<const float *>(cb.p[x & 7] + x * 128);
             tmem_st_bf16x32(tmem + lane_base + TM_A2 + 16 * hf, bbar);
           }
           if (hf <= dh) {
@@ -737,9 +734,36 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
       tc::tc_fence_before();
       compute_sync();
 
-      // ---- P4: Tinv = (I - Lab)^-1 as the bf16 operand B3
-      invert_unit_lower(Ls, Ts, Zs, sB3, warp, lane);
-      if (tid == 0) tc::mbar_arrive(bar_b3);
+      // The two groups work apart until MMA3 is done: warps 0-3 invert, warps 4-7 set up D2 (Q-part =
+      // R~, rows of A1; E-part = 0 and F-part = K-^T[j][m] = Gamma_C[j] K^[m][j], columns of B1).  The
+      // inverse's scratch lies outside A1 and B1.
+      const float gc_cur = hi_lanes ? GCs[j] : 1.f;  // Gamma_C[j] of this chunk (hi lanes)
+      if (warp < 4) {
+        // ---- P4: Tinv = (I - Lab)^-1 as the bf16 operand B3
+        invert_unit_lower(Ls, Ts, Zs, sB3, warp, lane);
+        if (tid == 0) tc::mbar_arrive(bar_b3);
+      } else {
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          float v[32];
+          if (!hi_lanes) {
+            load_row(sA1 + hh * (128 * 128), tl, v);
+            tc::tmem_st32(tmem + lane_base + TM_D2 + 32 * hh, v);
+          } else {
+            const ColPtrs ck = col_ptrs(sB1, 128, 64 + 32 * hh, j);
+#pragma unroll
+            for (int x = 0; x < 32; ++x) v[x] = gc_cur * *reinterpret_cast<const float *>(ck.p[x & 7] + x * 128);
+            tc::tmem_st32(tmem + lane_base + TM_D2 + 64 + 32 * hh, v);
+            zero32(v);
+            tc::tmem_st32(tmem + lane_base + TM_D2 + 32 * hh, v);
+          }
+        }
+        tc::tmem_st_wait();
+        tc::fence_proxy_async_smem();
+        tc::tc_fence_before();
+        group_sync_hi();
+        if (tid == 128) tc::mbar_arrive(bar_st);
+      }
       if (!(ok = wait_ctrl(bar_m3, ph))) break;
       tc::tc_fence_after();
 
@@ -773,8 +797,12 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
       readout(nchunks - 1, Lc_prev);
     }
     if (hi_lanes) {
+      tc::tmem_st_wait();
+      float v[32];
+      tc::tmem_ld32(tmem + lane_base + TM_S + 32 * ch, v);
 #pragma unroll
-      for (int x = 0; x < 32; ++x) A.s_out[pair * (kN * kN) + static_cast<long long>(32 * ch + x) * kN + j] = st[x];
+      for (int x = 0; x < 32; ++x)
+        A.s_out[pair * (kN * kN) + static_cast<long long>(32 * ch + x) * kN + j] = v[vrow(x)];
     }
   }
   tc::tc_fence_before();

@@ -76,9 +76,10 @@ constexpr uint32_t OFF_LS = OFF_MISC + 2048;              // float [64][LDL]
 constexpr uint32_t OFF_TS = OFF_LS + 64 * LDL * 4;        // float [6][16][LDTB]: Tinv blocks (s,s), (1,0), (3,2)
 constexpr uint32_t OFF_B3 = OFF_B2;                       // bf16 K-major Tinv 64x64 (8 KB), 1024-aligned
 constexpr uint32_t OFF_ZS = OFF_B2 + 8192;                // float [6][16][LDZ]
-constexpr uint32_t MISC_GC = 256;                         // float [64]    Gamma at the chunk end
-constexpr uint32_t MISC_WTOT = 512;                       // float [4][64] decay products of 16-token blocks
-constexpr uint32_t kSmemBytes = OFF_TS + 6 * 16 * LDTB * 4 + 1024;
+constexpr uint32_t OFF_PRE = OFF_TS + 6 * 16 * LDTB * 4;  // float [16][64]: Gamma before each 4-token group
+constexpr uint32_t MISC_GC = 256;                         // float [2][64] Gamma at the chunk end, by chunk parity
+constexpr uint32_t MISC_WTOT = 768;                       // float [4][64] decay products of 16-token blocks
+constexpr uint32_t kSmemBytes = OFF_PRE + 16 * 64 * 4 + 1024;
 
 static_assert(MISC_WTOT + 4 * 64 * 4 <= 2048, "misc region overflow");
 static_assert(OFF_ZS + 6 * 16 * LDZ * 4 <= OFF_B2 + 16384, "inverse scratch overflows B2");
@@ -323,6 +324,109 @@ __device__ __forceinline__ void invert_unit_lower(const float *Ls, float *Ts, fl
   group_sync_lo();
 }
 
+// Work of warps 4-7 on the chunk after the current one, done while warps 0-3 invert (tid4 = tid -
+// 128): the decay scan (pre4[g][j] = product of w over the tokens before 4-token group g; GCn[j] =
+// product over the chunk), the MMA1 B operand [B^; K^] = [b; k] / Gamma_t (tf32) and the MMA4 V^T
+// operand.  Each thread covers 4 channels x 8 tokens; tokens at or past Lcn act as w = 1, b = k =
+// v = 0.  Gamma_t is formed as pre4[g] times the running product inside the group, exactly as the
+// operand construction of R~ and A~ forms it.  Warps 4-7 synchronise among themselves.
+__device__ __forceinline__ void prep_next(const uint8_t *smem, uint8_t *sB1, uint8_t *sB4Vn, float *pre4, float *GCn,
+                                          float *wtot, int tid4, int Lcn) {
+  const int lane = tid4 & 31, wq = tid4 >> 5;
+  const int cq = tid4 & 15, to = tid4 >> 4;  // channel quad; token octet (2 per warp)
+  const int j0 = 4 * cq, tb = 8 * to;
+  float G[8][4];  // running products of w inside each 4-token group
+#pragma unroll
+  for (int tt = 0; tt < 8; ++tt) {
+    if (tb + tt < Lcn) {
+      raw4(smem, RAW_W, tb + tt, j0, G[tt]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) G[tt][e] = 1.f;
+    }
+  }
+#pragma unroll
+  for (int g = 0; g < 2; ++g)
+#pragma unroll
+    for (int k = 1; k < 4; ++k)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) G[4 * g + k][e] *= G[4 * g + k - 1][e];
+  float oct[4], exo[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    oct[e] = G[3][e] * G[7][e];
+    const float u = __shfl_up_sync(0xffffffffu, oct[e], 16);  // the even octet of this warp
+    exo[e] = lane >= 16 ? u : 1.f;
+  }
+  if (lane >= 16)
+    *reinterpret_cast<float4 *>(wtot + wq * 64 + j0) =
+        make_float4(exo[0] * oct[0], exo[1] * oct[1], exo[2] * oct[2], exo[3] * oct[3]);
+  group_sync_hi();
+  float p0[4], p1[4], gc[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    p0[e] = 1.f;
+    gc[e] = 1.f;
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float4 u = *reinterpret_cast<const float4 *>(wtot + k * 64 + j0);
+    const float uu[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      gc[e] *= uu[e];
+      if (k < wq) p0[e] *= uu[e];
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    p0[e] *= exo[e];
+    p1[e] = p0[e] * G[3][e];
+  }
+  *reinterpret_cast<float4 *>(pre4 + (2 * to) * 64 + j0) = make_float4(p0[0], p0[1], p0[2], p0[3]);
+  *reinterpret_cast<float4 *>(pre4 + (2 * to + 1) * 64 + j0) = make_float4(p1[0], p1[1], p1[2], p1[3]);
+  if (to == 0) *reinterpret_cast<float4 *>(GCn + j0) = make_float4(gc[0], gc[1], gc[2], gc[3]);
+  // [B^; K^] rows (K-major tf32; K = channel)
+  uint8_t *b1r = sB1 + (j0 >> 5) * (128 * 128);
+  const uint32_t chunk = (j0 & 31) >> 2;
+#pragma unroll
+  for (int tt = 0; tt < 8; ++tt) {
+    const int t = tb + tt;
+    float bb[4], kk[4], inv[4];
+    if (t < Lcn) {
+      raw4(smem, RAW_B, t, j0, bb);
+      raw4(smem, RAW_K, t, j0, kk);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) bb[e] = kk[e] = 0.f;
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) inv[e] = tc::rcp_approx((tt < 4 ? p0[e] : p1[e]) * G[tt][e]);
+    st_tf32x4(b1r + tc::sw128(t, chunk), bb[0] * inv[0], bb[1] * inv[1], bb[2] * inv[2], bb[3] * inv[3]);
+    st_tf32x4(b1r + tc::sw128(64 + t, chunk), kk[0] * inv[0], kk[1] * inv[1], kk[2] * inv[2], kk[3] * inv[3]);
+  }
+  // V^T (row = vrow(value channel), K = token); bf16 values are exact in tf32
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    float vv[4][4];
+#pragma unroll
+    for (int tt = 0; tt < 4; ++tt) {
+      if (tb + 4 * h + tt < Lcn) {
+        raw4(smem, RAW_V, tb + 4 * h + tt, j0, vv[tt]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) vv[tt][e] = 0.f;
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      *reinterpret_cast<uint4 *>(sB4Vn + kmaj_tf32(64, vrow(j0 + e), tb + 4 * h)) =
+          make_uint4(__float_as_uint(vv[0][e]), __float_as_uint(vv[1][e]), __float_as_uint(vv[2][e]),
+                     __float_as_uint(vv[3][e]));
+  }
+  tc::fence_proxy_async_smem();
+}
+
 __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_constant__ Maps maps, const Args A) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -349,7 +453,8 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
   uint64_t *bar_m4 = bars + 8;     // c -> w: MMA4 done
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_MISC + 80);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 84);
-  float *GCs = reinterpret_cast<float *>(smem + OFF_MISC + MISC_GC);
+  float *GCs = reinterpret_cast<float *>(smem + OFF_MISC + MISC_GC);  // [2][64]
+  float *pre4 = reinterpret_cast<float *>(smem + OFF_PRE);
   float *wtot = reinterpret_cast<float *>(smem + OFF_MISC + MISC_WTOT);
 
   const int tid = threadIdx.x;
@@ -418,6 +523,10 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
                             static_cast<int>(sb.start + static_cast<long long>(c + 1) * C));
           last_tma = (c + 1) & 1;
         }
+        // warm L2 with the chunk after that, so its TMA is an L2 hit when warps 4-7 need it early
+        if (c + 2 < nchunks)
+          for (int i = 0; i < 6; ++i)
+            tc::tma_prefetch_l2_3d(&maps.m[i], 0, h, static_cast<int>(sb.start + static_cast<long long>(c + 2) * C));
         // MMA3 (bf16): D3 = [A~^T; Lak^T] Tinv^T
         if (!wait_or_abort(bar_b3, ph, abort_flag)) { fail(); break; }
         tc::tc_fence_after();
@@ -511,6 +620,21 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
       compute_sync();
       return decision[slot] != 0;
     };
+    // The same for warps 4-7 alone (thread 128 polls; slots of their own).
+    volatile int *decision_hi = reinterpret_cast<volatile int *>(smem + OFF_MISC + 96);  // [2]
+    uint32_t ncalls_hi = 0;
+    auto wait_group_hi = [&](uint64_t *bar, uint32_t parity) -> bool {
+      const uint32_t slot = ncalls_hi++ & 1u;
+      if (tid == 128) {
+        if (!wait_or_abort(bar, parity, abort_flag)) {
+          *abort_flag = 1;
+          report_device_error(A.err, kDevErrTimeout);
+        }
+        decision_hi[slot] = *abort_flag == 0 ? 1 : 0;
+      }
+      group_sync_hi();
+      return decision_hi[slot] != 0;
+    };
     bool ok = true;
     // Read-out of a finished chunk: y rows (lanes 0..63) and the state update
     // S_C^T = diag(Gamma_C) S0^T + X (lanes 64..127), whose tf32 copy feeds the next MMA4; each warp
@@ -547,116 +671,66 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
     };
 
 
+    // the first chunk's decay scan, [B^; K^] and V^T
+    if (nchunks > 0 && warp >= 4 && wait_group_hi(bar_tma, 0))
+      prep_next(smem, sB1, sB4V, pre4, GCs, wtot, tid - 128, min(C, sb.len));
+    compute_sync();
+
     int Lc_prev = 0;
     bool have_prev = false;
     for (int c = 0; c < nchunks; ++c) {
       const int Lc = min(C, sb.len - c * C);
       const uint32_t ph = c & 1;
-      uint8_t *sB4Vc = sB4V + (c & 1) * 16384;
-      if (!(ok = wait_ctrl(bar_tma, ph))) break;
-
-      // ---- P1: decay products and operands (4 channels x 4 tokens per thread) ---------------
+      // ---- P1: the A operand [R~; A~] of MMA1 and A~^T of MMA3 (4 channels x 4 tokens per thread);
+      // the decay scan, [B^; K^] and V^T of this chunk were prepared by warps 4-7 beforehand
       {
-        float G[4][4];        // local products of w over this thread's tokens (rows) per channel (cols)
-        float pre[4], GC[4];  // Gamma before this thread's first token; Gamma at the chunk end
-        {
-          float wv[4][4];
+        const float4 pv = *reinterpret_cast<const float4 *>(pre4 + tg * 64 + j0);
+        const float pre[4] = {pv.x, pv.y, pv.z, pv.w};  // Gamma before this thread's first token
+        float G[4][4];  // running products of w over this thread's tokens (rows) per channel (cols)
 #pragma unroll
-          for (int tt = 0; tt < 4; ++tt) {
-            if (t0 + tt < Lc) {
-              raw4(smem, RAW_W, t0 + tt, j0, wv[tt]);
-            } else {
+        for (int tt = 0; tt < 4; ++tt) {
+          if (t0 + tt < Lc) {
+            raw4(smem, RAW_W, t0 + tt, j0, G[tt]);
+          } else {
 #pragma unroll
-              for (int e = 0; e < 4; ++e) wv[tt][e] = 1.f;
-            }
-          }
-          float incl[4], ex[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            G[0][e] = wv[0][e];
-            G[1][e] = G[0][e] * wv[1][e];
-            G[2][e] = G[1][e] * wv[2][e];
-            G[3][e] = G[2][e] * wv[3][e];
-            // inclusive scan over the 4 token groups of this warp (lanes l, l+8, l+16, l+24)
-            incl[e] = G[3][e];
-            float u = __shfl_up_sync(0xffffffffu, incl[e], 8);
-            if (lane >= 8) incl[e] *= u;
-            u = __shfl_up_sync(0xffffffffu, incl[e], 16);
-            if (lane >= 16) incl[e] *= u;
-            ex[e] = __shfl_up_sync(0xffffffffu, incl[e], 8);
-            if (lane < 8) ex[e] = 1.f;
-          }
-          if ((lane >> 3) == 3)
-            *reinterpret_cast<float4 *>(wtot + (warp >> 1) * 64 + j0) =
-                make_float4(incl[0], incl[1], incl[2], incl[3]);
-          compute_sync();
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            pre[e] = ex[e];
-            GC[e] = 1.f;
-          }
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const float4 u = *reinterpret_cast<const float4 *>(wtot + k * 64 + j0);
-            GC[0] *= u.x;
-            GC[1] *= u.y;
-            GC[2] *= u.z;
-            GC[3] *= u.w;
-            if (k < (warp >> 1)) {
-              pre[0] *= u.x;
-              pre[1] *= u.y;
-              pre[2] *= u.z;
-              pre[3] *= u.w;
-            }
+            for (int e = 0; e < 4; ++e) G[tt][e] = 1.f;
           }
         }
-        float rr[4][4], kk[4][4], aa[4][4], bb[4][4], vv[4][4];
+#pragma unroll
+        for (int k = 1; k < 4; ++k)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) G[k][e] *= G[k - 1][e];
+        float rr[4][4], aa[4][4];
 #pragma unroll
         for (int tt = 0; tt < 4; ++tt) {
           if (t0 + tt < Lc) {
             raw4(smem, RAW_R, t0 + tt, j0, rr[tt]);
-            raw4(smem, RAW_K, t0 + tt, j0, kk[tt]);
             raw4(smem, RAW_A, t0 + tt, j0, aa[tt]);
-            raw4(smem, RAW_B, t0 + tt, j0, bb[tt]);
-            raw4(smem, RAW_V, t0 + tt, j0, vv[tt]);
           } else {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) rr[tt][e] = kk[tt][e] = aa[tt][e] = bb[tt][e] = vv[tt][e] = 0.f;
+            for (int e = 0; e < 4; ++e) rr[tt][e] = aa[tt][e] = 0.f;
           }
         }
         uint8_t *a1r = sA1 + (j0 >> 5) * (128 * 128);
-        uint8_t *b1r = sB1 + (j0 >> 5) * (128 * 128);
         const uint32_t chunk = (j0 & 31) >> 2;
 #pragma unroll
         for (int tt = 0; tt < 4; ++tt) {
           const int t = t0 + tt;
-          float Gt[4], Gp[4], inv[4];
+          float Gt[4], Gp[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             Gp[e] = tt == 0 ? pre[e] : pre[e] * G[tt - 1][e];
             Gt[e] = pre[e] * G[tt][e];
-            inv[e] = tc::rcp_approx(Gt[e]);
           }
           st_tf32x4(a1r + tc::sw128(t, chunk), rr[tt][0] * Gt[0], rr[tt][1] * Gt[1], rr[tt][2] * Gt[2],
                     rr[tt][3] * Gt[3]);
           const float At0 = aa[tt][0] * Gp[0], At1 = aa[tt][1] * Gp[1], At2 = aa[tt][2] * Gp[2],
                       At3 = aa[tt][3] * Gp[3];
           st_tf32x4(a1r + tc::sw128(64 + t, chunk), At0, At1, At2, At3);
-          st_tf32x4(b1r + tc::sw128(t, chunk), bb[tt][0] * inv[0], bb[tt][1] * inv[1], bb[tt][2] * inv[2],
-                    bb[tt][3] * inv[3]);
-          st_tf32x4(b1r + tc::sw128(64 + t, chunk), kk[tt][0] * inv[0], kk[tt][1] * inv[1], kk[tt][2] * inv[2],
-                    kk[tt][3] * inv[3]);
           // A3: A~^T as the MN-major bf16 A operand of MMA3 (M = channel, K = token)
           *reinterpret_cast<uint2 *>(sA3 + mnmaj_bf16(64, t, j0)) =
               make_uint2(pack_bf16x2(At0, At1), pack_bf16x2(At2, At3));
         }
-        // V -> B4V (row = vrow(value channel), K = token); bf16 values are exact in tf32
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          *reinterpret_cast<uint4 *>(sB4Vc + kmaj_tf32(64, vrow(j0 + e), t0)) =
-              make_uint4(__float_as_uint(vv[0][e]), __float_as_uint(vv[1][e]), __float_as_uint(vv[2][e]),
-                         __float_as_uint(vv[3][e]));
-        if (tg == 0) *reinterpret_cast<float4 *>(GCs + j0) = make_float4(GC[0], GC[1], GC[2], GC[3]);
       }
       tc::fence_proxy_async_smem();
       compute_sync();
@@ -700,7 +774,7 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
           {
             // A2 lower half: B-^T[j][m] = Gamma_C[j] B^[m][j] (columns of B1), j = tl
             float bbar[32];
-            const float gcj = GCs[tl];
+            const float gcj = GCs[(c & 1) * 64 + tl];
             const ColPtrs cb = col_ptrs(sB1, 128, 32 * hf, tl);
 #pragma unroll
             for (int x = 0; x < 32; ++x) bbar[x] = gcj * *reinterpret_cast<const float *>(cb.p[x & 7] + x * 128);
@@ -737,7 +811,7 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
       // The two groups work apart until MMA3 is done: warps 0-3 invert, warps 4-7 set up D2 (Q-part =
       // R~, rows of A1; E-part = 0 and F-part = K-^T[j][m] = Gamma_C[j] K^[m][j], columns of B1).  The
       // inverse's scratch lies outside A1 and B1.
-      const float gc_cur = hi_lanes ? GCs[j] : 1.f;  // Gamma_C[j] of this chunk (hi lanes)
+      const float gc_cur = hi_lanes ? GCs[(c & 1) * 64 + j] : 1.f;  // Gamma_C[j] of this chunk (hi lanes)
       if (warp < 4) {
         // ---- P4: Tinv = (I - Lab)^-1 as the bf16 operand B3
         invert_unit_lower(Ls, Ts, Zs, sB3, warp, lane);
@@ -763,6 +837,11 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
         tc::tc_fence_before();
         group_sync_hi();
         if (tid == 128) tc::mbar_arrive(bar_st);
+        // then the next chunk's decay scan, [B^; K^] and V^T (its tiles were loaded after MMA1); A1/B1
+        // are free: MMA1 is done, P3 and the set-up above have read B1 and A1
+        if (c + 1 < nchunks && wait_group_hi(bar_tma, (c + 1) & 1))
+          prep_next(smem, sB1, sB4V + ((c + 1) & 1) * 16384, pre4, GCs + ((c + 1) & 1) * 64, wtot, tid - 128,
+                    min(C, sb.len - (c + 1) * C));
       }
       if (!(ok = wait_ctrl(bar_m3, ph))) break;
       tc::tc_fence_after();

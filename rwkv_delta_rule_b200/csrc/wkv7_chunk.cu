@@ -445,7 +445,7 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
   uint64_t *bar_tma = bars + 0;    // TMA tiles landed          (tx bytes)
   uint64_t *bar_p1 = bars + 1;     // w -> c: A1, B1 written; raw tiles consumed
   uint64_t *bar_m1 = bars + 2;     // c -> w: MMA1 done
-  uint64_t *bar_b3 = bars + 3;     // w -> c: A3 and B3 written
+  uint64_t *bar_b3 = bars + 3;     // w -> c: A3 and B3 written (one arrival per compute group)
   uint64_t *bar_m3 = bars + 4;     // c -> w: MMA3 done
   uint64_t *bar_b2 = bars + 5;     // w -> c: B2, A2 and the D2 initial value written
   uint64_t *bar_m2 = bars + 6;     // c -> c: MMA2 done
@@ -468,7 +468,7 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
   constexpr int kCtrlWarp = kComputeThreads / 32;
 
   if (tid == 0) {
-    for (int i = 0; i < 9; ++i) tc::mbar_init(bars + i, 1);
+    for (int i = 0; i < 9; ++i) tc::mbar_init(bars + i, i == 3 ? 2 : 1);  // b3: both compute groups
     tc::fence_mbar_init();
     *abort_flag = 0;
   }
@@ -552,8 +552,9 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
           tc::mma_commit(bar_m2);
           last_m2 = ph;
         }
-        if (!wait_or_abort(bar_m2, ph, abort_flag)) { fail(); break; }
-        // MMA4 (tf32, A from TMEM): D4 = [Q P; E F] [S0^T; V], once the state is written
+        // MMA4 (tf32, A from TMEM): D4 = [Q P; E F] [S0^T; V], once the state is written.  It reads
+        // MMA2's accumulator as its A operand with no wait in between: MMAs issued by one thread
+        // execute in issue order.
         if (!wait_or_abort(bar_st, ph, abort_flag)) { fail(); break; }
         tc::tc_fence_after();
         {
@@ -735,110 +736,120 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
       tc::fence_proxy_async_smem();
       compute_sync();
       if (tid == 0) tc::mbar_arrive(bar_p1);
-      // while MMA1 runs: the previous chunk's MMA4 (which ran under P1) is read out
+      // ---- while MMA1 runs: the previous chunk's read-out (its MMA4 ran under P1), then the D2 set-up:
+      // Q-part = R~ (rows of A1), E-part = 0, F-part = K-^T[j][m] = Gamma_C[j] K^[m][j] (columns of B1)
+      const float gc_cur = hi_lanes ? GCs[(c & 1) * 64 + j] : 1.f;  // Gamma_C[j] of this chunk (hi lanes)
       if (have_prev) {
         if (!(ok = wait_ctrl(bar_m4, ph ^ 1u))) break;
         tc::tc_fence_after();
         readout(c - 1, Lc_prev);
       }
-      if (!(ok = wait_ctrl(bar_m1, ph))) break;
-      tc::tc_fence_after();
-
-      // ---- P3: causal masks; A2 = [Mrb; B-^T] (bf16), P-part of D2 = Mrk ----------------------------
-      // A warp's 32 token rows meet the diagonal in the 32-column half dh; each thread handles the
-      // column half hf = ch of its rows, which lies on (hf == dh), below (hf < dh) or above the diagonal.
       {
-        const int dh = q & 1, hf = ch;
         float v[32];
         if (!hi_lanes) {
-          // rows t of Mrb (to A2 as bf16) and Mrk (moved to the P-part of D2): keep m <= t
-          if (hf == dh) {
-            tc::tmem_ld32(tmem + lane_base + TM_D1 + 32 * hf, v);
-            mask_upper(v, lane);
-            tmem_st_bf16x32(tmem + lane_base + TM_A2 + 16 * hf, v);
-            tc::tmem_ld32(tmem + lane_base + TM_D1 + 64 + 32 * hf, v);
-            mask_upper(v, lane);
-            tc::tmem_st32(tmem + lane_base + TM_D2 + 64 + 32 * hf, v);
-          } else if (hf > dh) {
-            zero32(v);
-            tmem_st_bf16x32(tmem + lane_base + TM_A2 + 16 * hf, v);
-            tc::tmem_st32(tmem + lane_base + TM_D2 + 64 + 32 * hf, v);
-          } else {
-            tc::tmem_ld32(tmem + lane_base + TM_D1 + 32 * hf, v);
-            tmem_st_bf16x32(tmem + lane_base + TM_A2 + 16 * hf, v);
-            tc::tmem_ld32(tmem + lane_base + TM_D1 + 64 + 32 * hf, v);
-            tc::tmem_st32(tmem + lane_base + TM_D2 + 64 + 32 * hf, v);
-          }
+          load_row(sA1 + ch * (128 * 128), tl, v);
+          tc::tmem_st32(tmem + lane_base + TM_D2 + 32 * ch, v);
         } else {
-          // B-^T -> A2 (bf16); rows t of Lab -> Ls and Lak -> A3 (keep m < t)
-          {
-            // A2 lower half: B-^T[j][m] = Gamma_C[j] B^[m][j] (columns of B1), j = tl
-            float bbar[32];
-            const float gcj = GCs[(c & 1) * 64 + tl];
-            const ColPtrs cb = col_ptrs(sB1, 128, 32 * hf, tl);
+          const ColPtrs ck = col_ptrs(sB1, 128, 64 + 32 * ch, j);
 #pragma unroll
-            for (int x = 0; x < 32; ++x) bbar[x] = gcj * *reinterpret_cast<const float *>(cb.p[x & 7] + x * 128);
-            tmem_st_bf16x32(tmem + lane_base + TM_A2 + 16 * hf, bbar);
-          }
-          if (hf <= dh) {
-            tc::tmem_ld32(tmem + lane_base + TM_D1 + 32 * hf, v);
-            if (hf == dh) mask_upper(v, lane - 1);
-            float *row = Ls + tl * LDL + 32 * hf;
-#pragma unroll
-            for (int x = 0; x < 32; x += 4)
-              *reinterpret_cast<float4 *>(row + x) = make_float4(v[x], v[x + 1], v[x + 2], v[x + 3]);
-            tc::tmem_ld32(tmem + lane_base + TM_D1 + 64 + 32 * hf, v);
-            if (hf == dh) mask_upper(v, lane - 1);
-          } else {
-            zero32(v);
-          }
-#pragma unroll
-          for (int cc = 0; cc < 4; ++cc) {
-            uint4 w4;
-            w4.x = pack_bf16x2(v[8 * cc + 0], v[8 * cc + 1]);
-            w4.y = pack_bf16x2(v[8 * cc + 2], v[8 * cc + 3]);
-            w4.z = pack_bf16x2(v[8 * cc + 4], v[8 * cc + 5]);
-            w4.w = pack_bf16x2(v[8 * cc + 6], v[8 * cc + 7]);
-            *reinterpret_cast<uint4 *>(sA3 + 64 * 128 + tc::sw128(tl, 4 * hf + cc)) = w4;
-          }
+          for (int x = 0; x < 32; ++x) v[x] = gc_cur * *reinterpret_cast<const float *>(ck.p[x & 7] + x * 128);
+          tc::tmem_st32(tmem + lane_base + TM_D2 + 64 + 32 * ch, v);
+          zero32(v);
+          tc::tmem_st32(tmem + lane_base + TM_D2 + 32 * ch, v);
         }
         tc::tmem_st_wait();
       }
       tc::fence_proxy_async_smem();
       tc::tc_fence_before();
       compute_sync();
+      if (tid == 0) tc::mbar_arrive(bar_st);
+      if (!(ok = wait_ctrl(bar_m1, ph))) break;
+      tc::tc_fence_after();
 
-      // The two groups work apart until MMA3 is done: warps 0-3 invert, warps 4-7 set up D2 (Q-part =
-      // R~, rows of A1; E-part = 0 and F-part = K-^T[j][m] = Gamma_C[j] K^[m][j], columns of B1).  The
-      // inverse's scratch lies outside A1 and B1.
-      const float gc_cur = hi_lanes ? GCs[(c & 1) * 64 + j] : 1.f;  // Gamma_C[j] of this chunk (hi lanes)
+      // ---- The two groups work apart until MMA3 is done.  Warps 0-3: Lab -> Ls (warps 2 and 3 own its
+      // TMEM lanes), then the inverse.  Warps 4-7: the rest of the causal masks for all 128 lanes (A2 =
+      // [Mrb; B-^T] as bf16, the P-part of D2 = Mrk, the lower half of A3 = Lak^T), then the next chunk's
+      // decay scan, [B^; K^] and V^T.  MMA3 waits for both groups (its barrier counts two arrivals).
+      // The rows of quadrant q meet the diagonal in the 32-column half dh; column half hf lies on
+      // (hf == dh), below (hf < dh) or above it.  The inverse's scratch lies outside A1 and B1.
+      const int dh = q & 1;
       if (warp < 4) {
+        if (hi_lanes) {
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            if (hf <= dh) {
+              float v[32];
+              tc::tmem_ld32(tmem + lane_base + TM_D1 + 32 * hf, v);
+              if (hf == dh) mask_upper(v, lane - 1);
+              float *row = Ls + tl * LDL + 32 * hf;
+#pragma unroll
+              for (int x = 0; x < 32; x += 4)
+                *reinterpret_cast<float4 *>(row + x) = make_float4(v[x], v[x + 1], v[x + 2], v[x + 3]);
+            }
+          }
+        }
+        group_sync_lo();
         // ---- P4: Tinv = (I - Lab)^-1 as the bf16 operand B3
         invert_unit_lower(Ls, Ts, Zs, sB3, warp, lane);
         if (tid == 0) tc::mbar_arrive(bar_b3);
       } else {
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
+        for (int hf = 0; hf < 2; ++hf) {
           float v[32];
           if (!hi_lanes) {
-            load_row(sA1 + hh * (128 * 128), tl, v);
-            tc::tmem_st32(tmem + lane_base + TM_D2 + 32 * hh, v);
+            // rows t of Mrb (to A2 as bf16) and Mrk (to the P-part of D2): keep m <= t
+            if (hf == dh) {
+              tc::tmem_ld32(tmem + lane_base + TM_D1 + 32 * hf, v);
+              mask_upper(v, lane);
+              tmem_st_bf16x32(tmem + lane_base + TM_A2 + 16 * hf, v);
+              tc::tmem_ld32(tmem + lane_base + TM_D1 + 64 + 32 * hf, v);
+              mask_upper(v, lane);
+              tc::tmem_st32(tmem + lane_base + TM_D2 + 64 + 32 * hf, v);
+            } else if (hf > dh) {
+              zero32(v);
+              tmem_st_bf16x32(tmem + lane_base + TM_A2 + 16 * hf, v);
+              tc::tmem_st32(tmem + lane_base + TM_D2 + 64 + 32 * hf, v);
+            } else {
+              tc::tmem_ld32(tmem + lane_base + TM_D1 + 32 * hf, v);
+              tmem_st_bf16x32(tmem + lane_base + TM_A2 + 16 * hf, v);
+              tc::tmem_ld32(tmem + lane_base + TM_D1 + 64 + 32 * hf, v);
+              tc::tmem_st32(tmem + lane_base + TM_D2 + 64 + 32 * hf, v);
+            }
           } else {
-            const ColPtrs ck = col_ptrs(sB1, 128, 64 + 32 * hh, j);
+            {
+              // A2 lower half: B-^T[j][m] = Gamma_C[j] B^[m][j] (columns of B1), j = tl
+              float bbar[32];
+              const ColPtrs cb = col_ptrs(sB1, 128, 32 * hf, tl);
 #pragma unroll
-            for (int x = 0; x < 32; ++x) v[x] = gc_cur * *reinterpret_cast<const float *>(ck.p[x & 7] + x * 128);
-            tc::tmem_st32(tmem + lane_base + TM_D2 + 64 + 32 * hh, v);
-            zero32(v);
-            tc::tmem_st32(tmem + lane_base + TM_D2 + 32 * hh, v);
+              for (int x = 0; x < 32; ++x)
+                bbar[x] = gc_cur * *reinterpret_cast<const float *>(cb.p[x & 7] + x * 128);
+              tmem_st_bf16x32(tmem + lane_base + TM_A2 + 16 * hf, bbar);
+            }
+            // rows t of Lak -> A3 (keep m < t)
+            if (hf <= dh) {
+              tc::tmem_ld32(tmem + lane_base + TM_D1 + 64 + 32 * hf, v);
+              if (hf == dh) mask_upper(v, lane - 1);
+            } else {
+              zero32(v);
+            }
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+              uint4 w4;
+              w4.x = pack_bf16x2(v[8 * cc + 0], v[8 * cc + 1]);
+              w4.y = pack_bf16x2(v[8 * cc + 2], v[8 * cc + 3]);
+              w4.z = pack_bf16x2(v[8 * cc + 4], v[8 * cc + 5]);
+              w4.w = pack_bf16x2(v[8 * cc + 6], v[8 * cc + 7]);
+              *reinterpret_cast<uint4 *>(sA3 + 64 * 128 + tc::sw128(tl, 4 * hf + cc)) = w4;
+            }
           }
         }
         tc::tmem_st_wait();
         tc::fence_proxy_async_smem();
         tc::tc_fence_before();
         group_sync_hi();
-        if (tid == 128) tc::mbar_arrive(bar_st);
-        // then the next chunk's decay scan, [B^; K^] and V^T (its tiles were loaded after MMA1); A1/B1
-        // are free: MMA1 is done, P3 and the set-up above have read B1 and A1
+        if (tid == 128) tc::mbar_arrive(bar_b3);
+        // then the next chunk's decay scan, [B^; K^] and V^T (its tiles were loaded after MMA1); B1 is
+        // free: MMA1 is done and the masks above have read its B^ columns
         if (c + 1 < nchunks && wait_group_hi(bar_tma, (c + 1) & 1))
           prep_next(smem, sB1, sB4V + ((c + 1) & 1) * 16384, pre4, GCs + ((c + 1) & 1) * 64, wtot, tid - 128,
                     min(C, sb.len - (c + 1) * C));

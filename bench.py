@@ -63,7 +63,7 @@ def load_peaks():
 # capture at B=4 (48 CTAs, 178 MB of operands, larger than L2) scaled by B to the B=8 workload; the
 # figure holds only for the kernel source it was taken on (sha256 prefix of wkv7_chunk.cu), and the
 # line reports null for any other build.  The capture is summarised under profiles/.
-MEASURED_TRAFFIC = {"source_sha256": "2833fea516e1d4b2", "bytes_per_token_head": (151876352 + 15380736) / (4 * 4096 * 12)}
+MEASURED_TRAFFIC = {"source_sha256": "d214f418d1afffb3", "bytes_per_token_head": (151908864 + 15943168) / (4 * 4096 * 12)}
 
 
 def measured_traffic(B, T, H, path):

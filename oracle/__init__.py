@@ -133,5 +133,34 @@ def wkv7_varlen(r, w, k, v, a, b, cu_seqlens, s_in=None, *, nthreads: Optional[i
     return y, s_out
 
 
+def x070_prologue(xw, k, xa, k_k) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """The x070 operand prologue in float64 (RWKV-7 G0 7.2B walkthrough, lshu.cn/news/198401,
+    section 7.1): the decay comes from its pre-activation as ``exp(-exp(w'))`` with
+    ``w' = -softplus(-xw) - 0.5``; the in-context learning rate is ``sigmoid(xa)``; the key is
+    scaled by ``k_k`` and L2-normalised over the head (``x / max(||x||, 1e-12)``) into ``kk``; the
+    kernel operands are ``a = -kk`` and ``b = kk * sigmoid(xa)``.
+
+    ``xw, k, xa``: ``[..., N]``; ``k_k``: ``[H, N]`` broadcast over the leading dims, or None for
+    ones.  Returns float64 ``(w, a, b)`` of the same shape."""
+    xw = _as_np(xw, np.float64)
+    k = _as_np(k, np.float64)
+    xa = _as_np(xa, np.float64)
+    softplus_neg = np.log1p(np.exp(-np.abs(-xw))) + np.maximum(-xw, 0.0)  # softplus(-xw), stable form
+    w = np.exp(-np.exp(-softplus_neg - 0.5))
+    rate = 1.0 / (1.0 + np.exp(-xa))
+    kx = k if k_k is None else k * _as_np(k_k, np.float64)
+    norm = np.sqrt(np.sum(kx * kx, axis=-1, keepdims=True))
+    kk = kx / np.maximum(norm, 1e-12)
+    return w, -kk, kk * rate
+
+
+def wkv7_model_native(r, xw, k, v, xa, k_k, s_in=None, *, nthreads: Optional[int] = None):
+    """The recurrence on model-native inputs: the prologue above, then ``wkv7`` in float64
+    (``k`` itself enters the recurrence unchanged)."""
+    w, a, b = x070_prologue(xw, k, xa, k_k)
+    return wkv7(_as_np(r, np.float64), w, _as_np(k, np.float64), _as_np(v, np.float64), a, b, s_in,
+                nthreads=nthreads, precision="f64")
+
+
 def real_bytes(real: str = "double") -> int:
     return int(_lib(real).wkv7_oracle_real_bytes())

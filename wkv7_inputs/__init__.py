@@ -113,6 +113,40 @@ def draw(B: int, T: int, H: int, N: int = N_HEAD, *, seed: int, dtype: str = "bf
     return out
 
 
+def draw_model_native(B: int, T: int, H: int, N: int = N_HEAD, *, seed: int, z_mean: float = 0.0,
+                      s0_std: Optional[float] = None) -> Dict[str, torch.Tensor]:
+    """Draw model-native inputs for the fused operand prologue (no prologue arithmetic here).
+
+    Returns bf16 ``[B, T, H, N]`` tensors ``r`` ~ N(0,1), ``xw`` (decay pre-activation) ~
+    N(z_mean, 1), ``k`` = unit vector per (b, t, h) times U(0.5, 1.5) per channel, ``v`` ~ N(0,1)
+    and ``xa`` (in-context learning-rate pre-activation) ~ N(0,1); ``<name>_f32`` copies; ``k_k``:
+    float32 ``[H, N]`` ~ U(0.5, 1.5); ``s0``: float32 ``[B, H, N, N]`` or None.
+    """
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    shp = (B, T, H, N)
+    f32 = torch.float32
+    r = torch.randn(shp, generator=g, dtype=f32)
+    xw = torch.randn(shp, generator=g, dtype=f32) + float(z_mean)
+    kh = torch.randn(shp, generator=g, dtype=f32)
+    s = torch.rand(shp, generator=g, dtype=f32) + 0.5
+    v = torch.randn(shp, generator=g, dtype=f32)
+    xa = torch.randn(shp, generator=g, dtype=f32)
+    k_k = torch.rand((H, N), generator=g, dtype=f32) + 0.5
+    s0 = None
+    if s0_std is not None:
+        s0 = torch.randn((B, H, N, N), generator=g, dtype=f32) * float(s0_std)
+    k = kh / kh.norm(dim=-1, keepdim=True) * s
+    out: Dict[str, torch.Tensor] = {}
+    for nm, x in (("r", r), ("xw", xw), ("k", k), ("v", v), ("xa", xa)):
+        xs = x.to(torch.bfloat16).contiguous()
+        out[nm] = xs
+        out[nm + "_f32"] = xs.to(f32)
+    out["k_k"] = k_k.contiguous()
+    out["s0"] = s0
+    return out
+
+
 def draw_case(case: Case, *, T: Optional[int] = None, B: Optional[int] = None) -> Dict[str, torch.Tensor]:
     """Draw a named workload, optionally at a reduced B or T (same recipe, same seed)."""
     return draw(case.B if B is None else B, case.T if T is None else T, case.H, case.N,

@@ -299,6 +299,81 @@ def bench_decode(lib7, dev, steps_target: int = 1024, layers: int = 24):
             "achieved_gbs": byts / step_s / 1e9, "launches": nsteps}
 
 
+NATIVE = ("r", "xw", "k", "v", "xa")
+
+
+def bench_model_native(lib7, dev, B, T, H, steps, decode_steps=1024, layers=24):
+    """The model-native entry points (operand prologue in the kernels) on the same shapes: prefill
+    launch time and HBM roofline (five input tensors + y + state), and decode steps/s."""
+    case = wi.CASES[WORKLOAD]
+    d = wi.draw_model_native(B, T, H, seed=case.seed, s0_std=case.s0_std)
+    dd = {n: d[n].to(dev) for n in NATIVE}
+    kk = d["k_k"].to(dev)
+    s0 = d["s0"].to(dev)
+    y = torch.empty_like(dd["r"])
+    s_out = torch.empty_like(s0)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        lib7.rwkv7_wkv_prefill_fused_bf16(lib7.RWKV7_PATH_AUTO, *[dd[n] for n in NATIVE], kk, s0, y, s_out, stream)
+
+    for _ in range(5):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    assert lib7.rwkv7_get_last_error() == 0
+    ms = e0.elapsed_time(e1) / steps
+    byts = 6 * B * T * H * N * 2 + 2 * B * H * N * N * 4
+    peaks, _ = load_peaks()
+    pre = {"launch_ms": ms, "tokens_per_s": B * T / (ms / 1e3), "algorithmic_bytes_per_launch": byts,
+           "achieved_gbs": byts / (ms / 1e3) / 1e9, "frac": byts / (ms / 1e3) / 1e9 / peaks["hbm_gbs"]}
+    del dd, y, s_out
+    # decode at the L24-D1024 shape, rotating `layers` distinct states inside a CUDA graph
+    dc = wi.CASES["decode_l24_d1024_b256_1024steps"]
+    Bd, Hd, ntok = dc.B, dc.H, 8
+    dn = wi.draw_model_native(Bd, ntok, Hd, seed=dc.seed)
+    toks = [{n: dn[n][:, t].contiguous().to(dev) for n in NATIVE} for t in range(ntok)]
+    kkd = dn["k_k"].to(dev)
+    states = torch.zeros(layers, Bd, Hd, N, N, device=dev)
+    ys = [torch.empty(Bd, Hd, N, dtype=torch.bfloat16, device=dev) for _ in range(layers)]
+    per_graph = layers * 4
+
+    def one_pass():
+        for i in range(per_graph):
+            tk = toks[i % ntok]
+            lib7.rwkv7_wkv_decode_fused_bf16(*[tk[n] for n in NATIVE], kkd, states[i % layers], ys[i % layers])
+
+    sd = torch.cuda.Stream(device=dev)
+    sd.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(sd):
+        one_pass()
+    torch.cuda.current_stream().wait_stream(sd)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        one_pass()
+    reps = max(1, (decode_steps + per_graph - 1) // per_graph)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(reps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    step_s = e0.elapsed_time(e1) / 1e3 / (reps * per_graph)
+    dbytes = Bd * Hd * (2 * N * N * 4 + 6 * N * 2)
+    dec = {"workload": "decode_l24_d1024_b256", "steps_per_s": 1.0 / step_s, "us_per_step": step_s * 1e6,
+           "bytes_per_step": dbytes, "achieved_gbs": dbytes / step_s / 1e9,
+           "frac": dbytes / step_s / 1e9 / peaks["hbm_gbs"]}
+    return {"prefill": pre, "decode": dec,
+            "inputs": "bf16 r, x_w, k, v, x_a [B,T,H,64] + float32 k_k [H,64]; w, a, b formed in-kernel"}
+
+
 def run_ours(args):
     world, rank, local = dist_setup()
     dev = torch.device("cuda", local)
@@ -402,6 +477,11 @@ def run_ours(args):
         decode["frac"] = decode["achieved_gbs"] / peaks["hbm_gbs"]
         assert lib7.rwkv7_get_last_error() == 0
 
+    native = None
+    if not args.no_native and args.path == "auto":
+        native = bench_model_native(lib7, dev, B, T, H, steps=min(args.steps, 50),
+                                    decode_steps=0 if args.no_decode else args.decode_steps)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
         T_s = min(T, args.ref_tokens)
@@ -425,6 +505,7 @@ def run_ours(args):
         "clocks": clocks.summary(),
         "cpu_baseline": cpu,
         "decode": decode,
+        "model_native": native,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -445,6 +526,7 @@ def main():
     ap.add_argument("--batch", type=int, default=0, help="override B (profiling runs only)")
     ap.add_argument("--seqlen", type=int, default=0, help="override T (profiling runs only)")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-native", action="store_true", help="skip the model-native entry points' lines")
     ap.add_argument("--decode-steps", type=int, default=1024)
     ap.add_argument("--decode-layers", type=int, default=24, help="distinct decode states rotated over")
     ap.add_argument("--no-e2e", action="store_true")

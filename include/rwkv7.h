@@ -136,6 +136,30 @@ RWKV7_API rwkv7_status rwkv7_wkv_decode_bf16(int B, int H, int N, const uint16_t
                                    const uint16_t *b, float *s_inout, uint16_t *y,
                                    rwkv7_stream_t stream);
 
+/* ---- model-native inputs (operand prologue fused into the kernels) ------------
+ *
+ * The same recurrence, but the caller passes what the x070 time-mix produces before its operand
+ * prologue (RWKV-7 G0 7.2B walkthrough, lshu.cn/news/198401, section 7.1), and the kernels form
+ * the operands in float32:
+ *   w = exp(-exp(-softplus(-xw) - 0.5))          (decay in (0.5452, 1))
+ *   kk = normalize(k * k_k) over the 64 channels   (x / max(|x|, 1e-12))
+ *   a = -kk,  b = kk * sigmoid(xa)
+ * and k enters the recurrence as given.  Five token tensors instead of six.
+ *
+ * r, xw, k, v, xa: bf16 bit patterns [B,T,H,64] (prefill) / [B,H,64] (decode), 16-byte aligned.
+ * k_k: float32 [H,64] key scale, or NULL for ones (16-byte aligned when given; device memory).
+ * Everything else (state, y, ownership, errors, paths) as for the bf16 entry points above; the
+ * CHUNK path has no extra domain condition here, since every decay is >= 0.5452. */
+RWKV7_API rwkv7_status rwkv7_wkv_prefill_fused_bf16(int path, int B, int T, int H, int N, const uint16_t *r,
+                                                    const uint16_t *xw, const uint16_t *k, const uint16_t *v,
+                                                    const uint16_t *xa, const float *k_k, const float *s_in,
+                                                    uint16_t *y, float *s_out, rwkv7_stream_t stream);
+
+RWKV7_API rwkv7_status rwkv7_wkv_decode_fused_bf16(int B, int H, int N, const uint16_t *r, const uint16_t *xw,
+                                                   const uint16_t *k, const uint16_t *v, const uint16_t *xa,
+                                                   const float *k_k, float *s_inout, uint16_t *y,
+                                                   rwkv7_stream_t stream);
+
 /* ---- status ---------------------------------------------------------------- */
 
 /* Static English description of a status code (never NULL). */

@@ -24,8 +24,9 @@ import torch
 __all__ = [
     "RWKV7_PATH_AUTO", "RWKV7_PATH_SCAN", "RWKV7_PATH_CHUNK", "Rwkv7Error", "library_path", "load_library",
     "rwkv7_wkv_prefill", "rwkv7_wkv_prefill_bf16", "rwkv7_wkv_prefill_bf16_path", "rwkv7_wkv_prefill_varlen_bf16",
-    "rwkv7_wkv_decode", "rwkv7_wkv_decode_bf16", "rwkv7_status_string", "rwkv7_get_last_error", "rwkv7_version",
-    "prefill", "decode_", "EXPORTED_SYMBOLS",
+    "rwkv7_wkv_decode", "rwkv7_wkv_decode_bf16", "rwkv7_wkv_prefill_fused_bf16", "rwkv7_wkv_decode_fused_bf16",
+    "rwkv7_status_string", "rwkv7_get_last_error", "rwkv7_version",
+    "prefill", "decode_", "prefill_model_native", "decode_model_native_", "EXPORTED_SYMBOLS",
 ]
 
 RWKV7_PATH_AUTO, RWKV7_PATH_SCAN, RWKV7_PATH_CHUNK = 0, 1, 2
@@ -33,7 +34,8 @@ N_HEAD = 64
 
 EXPORTED_SYMBOLS = (
     "rwkv7_wkv_prefill", "rwkv7_wkv_prefill_bf16", "rwkv7_wkv_prefill_bf16_path", "rwkv7_wkv_prefill_varlen_bf16",
-    "rwkv7_wkv_decode", "rwkv7_wkv_decode_bf16", "rwkv7_status_string", "rwkv7_get_last_error", "rwkv7_version",
+    "rwkv7_wkv_decode", "rwkv7_wkv_decode_bf16", "rwkv7_wkv_prefill_fused_bf16", "rwkv7_wkv_decode_fused_bf16",
+    "rwkv7_status_string", "rwkv7_get_last_error", "rwkv7_version",
 )
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -68,6 +70,8 @@ def load_library() -> ctypes.CDLL:
         ("rwkv7_wkv_prefill_varlen_bf16", [ci, ci, ci, ci, ci, ci, vp] + [vp] * 6 + [vp, vp, vp, vp]),
         ("rwkv7_wkv_decode", [ci, ci, ci] + [vp] * 6 + [vp, vp, vp]),
         ("rwkv7_wkv_decode_bf16", [ci, ci, ci] + [vp] * 6 + [vp, vp, vp]),
+        ("rwkv7_wkv_prefill_fused_bf16", [ci, ci, ci, ci, ci] + [vp] * 6 + [vp, vp, vp, vp]),
+        ("rwkv7_wkv_decode_fused_bf16", [ci, ci, ci] + [vp] * 6 + [vp, vp, vp]),
     ):
         fn = getattr(lib, name)
         fn.argtypes = args
@@ -179,6 +183,30 @@ def rwkv7_wkv_decode_bf16(r, w, k, v, a, b, s_inout, y, stream=None) -> None:
     _decode_common("rwkv7_wkv_decode_bf16", torch.bfloat16, r, w, k, v, a, b, s_inout, y, stream)
 
 
+def rwkv7_wkv_prefill_fused_bf16(path, r, xw, k, v, xa, k_k, s_in, y, s_out, stream=None) -> None:
+    """Prefill on model-native inputs: bf16 ``r, xw, k, v, xa`` / y ``[B,T,H,64]``, float32 ``k_k``
+    ``[H,64]`` or None (ones); w, a and b are formed in the kernels."""
+    B, T, H, N = r.shape
+    for nm, t in (("r", r), ("xw", xw), ("k", k), ("v", v), ("xa", xa), ("y", y)):
+        _check(t, nm, torch.bfloat16, (B, T, H, N))
+    _check(k_k, "k_k", torch.float32, (H, N), allow_none=True)
+    _check(s_in, "s_in", torch.float32, (B, H, N, N), allow_none=True)
+    _check(s_out, "s_out", torch.float32, (B, H, N, N))
+    _call("rwkv7_wkv_prefill_fused_bf16", int(path), B, T, H, N,
+          *[_ptr(t) for t in (r, xw, k, v, xa, k_k, s_in, y, s_out)], _stream(stream))
+
+
+def rwkv7_wkv_decode_fused_bf16(r, xw, k, v, xa, k_k, s_inout, y, stream=None) -> None:
+    """One decode step on model-native inputs ``[B,H,64]`` (bf16), ``k_k`` ``[H,64]`` float32 or None."""
+    B, H, N = r.shape
+    for nm, t in (("r", r), ("xw", xw), ("k", k), ("v", v), ("xa", xa), ("y", y)):
+        _check(t, nm, torch.bfloat16, (B, H, N))
+    _check(k_k, "k_k", torch.float32, (H, N), allow_none=True)
+    _check(s_inout, "s_inout", torch.float32, (B, H, N, N))
+    _call("rwkv7_wkv_decode_fused_bf16", B, H, N, *[_ptr(t) for t in (r, xw, k, v, xa, k_k, s_inout, y)],
+          _stream(stream))
+
+
 def rwkv7_status_string(status: int) -> str:
     return load_library().rwkv7_status_string(int(status)).decode()
 
@@ -215,4 +243,21 @@ def decode_(r, w, k, v, a, b, state, y=None, *, stream=None):
         rwkv7_wkv_decode(r, w, k, v, a, b, state, y, stream)
     else:
         rwkv7_wkv_decode_bf16(r, w, k, v, a, b, state, y, stream)
+    return y
+
+
+def prefill_model_native(r, xw, k, v, xa, k_k=None, s_in=None, *, path: int = RWKV7_PATH_AUTO, stream=None):
+    """Allocate ``y`` and ``s_out`` and run the prefill on model-native inputs; returns ``(y, s_out)``."""
+    B, T, H, N = r.shape
+    y = torch.empty_like(r)
+    s_out = torch.empty((B, H, N, N), dtype=torch.float32, device=r.device)
+    rwkv7_wkv_prefill_fused_bf16(path, r, xw, k, v, xa, k_k, s_in, y, s_out, stream)
+    return y, s_out
+
+
+def decode_model_native_(r, xw, k, v, xa, k_k, state, y=None, *, stream=None):
+    """One decode step on model-native inputs, updating ``state`` in place; returns ``y``."""
+    if y is None:
+        y = torch.empty_like(r)
+    rwkv7_wkv_decode_fused_bf16(r, xw, k, v, xa, k_k, state, y, stream)
     return y

@@ -51,6 +51,17 @@ template <> struct Elem<uint16_t> {
   }
 };
 
+// ---- the x070 operand prologue for model-native inputs --------------------------
+// RWKV-7 G0 7.2B walkthrough, lshu.cn/news/198401, section 7.1: the decay comes from its
+// pre-activation x as exp(-exp(-softplus(-x) - 0.5)), which equals exp(-e^-0.5 sigmoid(x)) because
+// exp(-softplus(-x)) = sigmoid(x); the in-context learning rate is sigmoid(x_a); the key scaled by
+// k_k and L2-normalised over the head gives kk, and the recurrence takes a = -kk, b = kk * rate
+// (k itself enters unchanged).  Computed in float32 from the bf16 inputs.
+__device__ __forceinline__ float x070_sigmoid(float x) { return __fdividef(1.f, 1.f + __expf(-x)); }
+__device__ __forceinline__ float x070_decay(float xw) { return __expf(-0.60653065971263342f * x070_sigmoid(xw)); }
+// 1 / max(||x||, 1e-12) from the sum of squares (the divisor of the L2 normalisation)
+__device__ __forceinline__ float x070_inv_norm(float sumsq) { return rsqrtf(fmaxf(sumsq, 1e-24f)); }
+
 // ---- cp.async (16-byte, L2-only) ---------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

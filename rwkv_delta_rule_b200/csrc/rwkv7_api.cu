@@ -153,4 +153,31 @@ rwkv7_status rwkv7_wkv_decode_bf16(int B, int H, int N, const uint16_t *r, const
       launch_decode<uint16_t>(r, w, k, v, a, b, s_inout, y, B, H, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+rwkv7_status rwkv7_wkv_prefill_fused_bf16(int path, int B, int T, int H, int N, const uint16_t *r,
+                                          const uint16_t *xw, const uint16_t *k, const uint16_t *v,
+                                          const uint16_t *xa, const float *k_k, const float *s_in, uint16_t *y,
+                                          float *s_out, rwkv7_stream_t stream) {
+  if (path != RWKV7_PATH_AUTO && path != RWKV7_PATH_SCAN && path != RWKV7_PATH_CHUNK) return RWKV7_ERR_INVALID;
+  // the b slot of the shared checks is filled with xa: model-native calls have no b
+  const rwkv7_status st = check_prefill(B, T, H, N, r, xw, k, v, xa, xa, s_in, y, s_out);
+  if (st != RWKV7_OK) return st;
+  if (!aligned16(k_k)) return RWKV7_ERR_ALIGN;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  const long long total = static_cast<long long>(B) * T;
+  if (use_chunk(path, T))
+    return from_cuda(
+        launch_chunk_fused(r, xw, k, v, xa, k_k, s_in, y, s_out, nullptr, B, T, total, H, error_word_ptr(), cs));
+  return from_cuda(launch_scan_fused(r, xw, k, v, xa, k_k, s_in, y, s_out, nullptr, B, T, total, H, cs));
+}
+
+rwkv7_status rwkv7_wkv_decode_fused_bf16(int B, int H, int N, const uint16_t *r, const uint16_t *xw,
+                                         const uint16_t *k, const uint16_t *v, const uint16_t *xa, const float *k_k,
+                                         float *s_inout, uint16_t *y, rwkv7_stream_t stream) {
+  if (N != kN) return RWKV7_ERR_UNSUPPORTED;
+  if (B <= 0 || H <= 0 || !none_null(r, xw, k, v, xa, s_inout, y)) return RWKV7_ERR_INVALID;
+  if (!all_aligned(r, xw, k, v, xa, k_k, s_inout, y)) return RWKV7_ERR_ALIGN;
+  return from_cuda(
+      launch_decode_fused(r, xw, k, v, xa, k_k, s_inout, y, B, H, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

@@ -79,7 +79,8 @@ constexpr uint32_t OFF_ZS = OFF_B2 + 8192;                // float [6][16][LDZ]
 constexpr uint32_t OFF_PRE = OFF_TS + 6 * 16 * LDTB * 4;  // float [16][64]: Gamma before each 4-token group
 constexpr uint32_t MISC_GC = 256;                         // float [2][64] Gamma at the chunk end, by chunk parity
 constexpr uint32_t MISC_WTOT = 768;                       // float [4][64] decay products of 16-token blocks
-constexpr uint32_t kSmemBytes = OFF_PRE + 16 * 64 * 4 + 1024;
+constexpr uint32_t OFF_KX = OFF_PRE + 16 * 64 * 4;  // model-native inputs: float [64] k_k, float [64] 1/|k k_k|
+constexpr uint32_t kSmemBytes = OFF_KX + 2 * 64 * 4 + 1024;
 
 static_assert(MISC_WTOT + 4 * 64 * 4 <= 2048, "misc region overflow");
 static_assert(OFF_ZS + 6 * 16 * LDZ * 4 <= OFF_B2 + 16384, "inverse scratch overflows B2");
@@ -114,6 +115,7 @@ struct Args {
   long long total_T;
   int H;
   int *err;
+  const float *k_k;  // model-native inputs: [H, 64] key scale, nullptr = ones
 };
 
 enum { RAW_R = 0, RAW_W = 1, RAW_K = 2, RAW_A = 3, RAW_B = 4, RAW_V = 5 };
@@ -330,8 +332,9 @@ __device__ __forceinline__ void invert_unit_lower(const float *Ls, float *Ts, fl
 // operand.  Each thread covers 4 channels x 8 tokens; tokens at or past Lcn act as w = 1, b = k =
 // v = 0.  Gamma_t is formed as pre4[g] times the running product inside the group, exactly as the
 // operand construction of R~ and A~ forms it.  Warps 4-7 synchronise among themselves.
-__device__ __forceinline__ void prep_next(const uint8_t *smem, uint8_t *sB1, uint8_t *sB4Vn, float *pre4, float *GCn,
-                                          float *wtot, int tid4, int Lcn) {
+template <bool kFused>
+__device__ __forceinline__ void prep_next(const uint8_t *smem, uint8_t *sA1, uint8_t *sB1, uint8_t *sB4Vn, float *pre4,
+                                          float *GCn, float *wtot, const float *kkw, float *invn, int tid4, int Lcn) {
   const int lane = tid4 & 31, wq = tid4 >> 5;
   const int cq = tid4 & 15, to = tid4 >> 4;  // channel quad; token octet (2 per warp)
   const int j0 = 4 * cq, tb = 8 * to;
@@ -340,9 +343,35 @@ __device__ __forceinline__ void prep_next(const uint8_t *smem, uint8_t *sB1, uin
   for (int tt = 0; tt < 8; ++tt) {
     if (tb + tt < Lcn) {
       raw4(smem, RAW_W, tb + tt, j0, G[tt]);
+      if (kFused) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) G[tt][e] = x070_decay(G[tt][e]);  // the tile holds x_w
+      }
     } else {
 #pragma unroll
       for (int e = 0; e < 4; ++e) G[tt][e] = 1.f;
+    }
+  }
+  float kks[4] = {1.f, 1.f, 1.f, 1.f}, inv[8];
+  if (kFused) {
+    // 1 / |k * k_k| per token: the 16 lanes of a half-warp hold the 64 channels of its tokens
+#pragma unroll
+    for (int e = 0; e < 4; ++e) kks[e] = kkw[j0 + e];
+#pragma unroll
+    for (int tt = 0; tt < 8; ++tt) {
+      float kv[4], ss = 0.f;
+      if (tb + tt < Lcn) {
+        raw4(smem, RAW_K, tb + tt, j0, kv);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) kv[e] = 0.f;
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) ss = fmaf(kv[e] * kks[e], kv[e] * kks[e], ss);
+#pragma unroll
+      for (int off = 8; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+      inv[tt] = x070_inv_norm(ss);
+      if (cq == 0) invn[tb + tt] = inv[tt];
     }
   }
 #pragma unroll
@@ -386,24 +415,38 @@ __device__ __forceinline__ void prep_next(const uint8_t *smem, uint8_t *sB1, uin
   *reinterpret_cast<float4 *>(pre4 + (2 * to) * 64 + j0) = make_float4(p0[0], p0[1], p0[2], p0[3]);
   *reinterpret_cast<float4 *>(pre4 + (2 * to + 1) * 64 + j0) = make_float4(p1[0], p1[1], p1[2], p1[3]);
   if (to == 0) *reinterpret_cast<float4 *>(GCn + j0) = make_float4(gc[0], gc[1], gc[2], gc[3]);
-  // [B^; K^] rows (K-major tf32; K = channel)
+  // [B^; K^] rows (K-major tf32; K = channel), and Gamma_t itself (float32) where the operand
+  // construction will put R~ = r Gamma_t: it reads Gamma_t there and overwrites it in place
   uint8_t *b1r = sB1 + (j0 >> 5) * (128 * 128);
+  uint8_t *a1r = sA1 + (j0 >> 5) * (128 * 128);
   const uint32_t chunk = (j0 & 31) >> 2;
 #pragma unroll
   for (int tt = 0; tt < 8; ++tt) {
     const int t = tb + tt;
-    float bb[4], kk[4], inv[4];
+    float bb[4], kk[4], ig[4];
     if (t < Lcn) {
-      raw4(smem, RAW_B, t, j0, bb);
       raw4(smem, RAW_K, t, j0, kk);
+      if (kFused) {
+        // b = kk * sigmoid(x_a), kk = k * k_k / |k * k_k| (the tile in the a slot holds x_a)
+        raw4(smem, RAW_A, t, j0, bb);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) bb[e] = kk[e] * kks[e] * inv[tt] * x070_sigmoid(bb[e]);
+      } else {
+        raw4(smem, RAW_B, t, j0, bb);
+      }
     } else {
 #pragma unroll
       for (int e = 0; e < 4; ++e) bb[e] = kk[e] = 0.f;
     }
+    float gt[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) inv[e] = tc::rcp_approx((tt < 4 ? p0[e] : p1[e]) * G[tt][e]);
-    st_tf32x4(b1r + tc::sw128(t, chunk), bb[0] * inv[0], bb[1] * inv[1], bb[2] * inv[2], bb[3] * inv[3]);
-    st_tf32x4(b1r + tc::sw128(64 + t, chunk), kk[0] * inv[0], kk[1] * inv[1], kk[2] * inv[2], kk[3] * inv[3]);
+    for (int e = 0; e < 4; ++e) {
+      gt[e] = (tt < 4 ? p0[e] : p1[e]) * G[tt][e];
+      ig[e] = tc::rcp_approx(gt[e]);
+    }
+    *reinterpret_cast<float4 *>(a1r + tc::sw128(t, chunk)) = make_float4(gt[0], gt[1], gt[2], gt[3]);
+    st_tf32x4(b1r + tc::sw128(t, chunk), bb[0] * ig[0], bb[1] * ig[1], bb[2] * ig[2], bb[3] * ig[3]);
+    st_tf32x4(b1r + tc::sw128(64 + t, chunk), kk[0] * ig[0], kk[1] * ig[1], kk[2] * ig[2], kk[3] * ig[3]);
   }
   // V^T (row = vrow(value channel), K = token); bf16 values are exact in tf32
 #pragma unroll
@@ -427,6 +470,10 @@ __device__ __forceinline__ void prep_next(const uint8_t *smem, uint8_t *sB1, uin
   tc::fence_proxy_async_smem();
 }
 
+// kFused: model-native inputs -- the w, a and b tiles hold x_w, x_a and nothing; w = decay(x_w),
+// a = -kk and b = kk * sigmoid(x_a) with kk = k * k_k / |k * k_k| are formed where the operands are
+// built (the decay-scan / [B^; K^] preparation and P1), and only five tiles are loaded per chunk.
+template <bool kFused>
 __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_constant__ Maps maps, const Args A) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -455,6 +502,8 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 84);
   float *GCs = reinterpret_cast<float *>(smem + OFF_MISC + MISC_GC);  // [2][64]
   float *pre4 = reinterpret_cast<float *>(smem + OFF_PRE);
+  float *kkw = reinterpret_cast<float *>(smem + OFF_KX);        // [64] key scale of this head
+  float *invn = reinterpret_cast<float *>(smem + OFF_KX + 256);  // [64] 1 / |k * k_k| per token of a chunk
   float *wtot = reinterpret_cast<float *>(smem + OFF_MISC + MISC_WTOT);
 
   const int tid = threadIdx.x;
@@ -492,9 +541,10 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
       // parity of the last issued phase of each barrier, or -1 when nothing was issued
       int last_tma = -1, last_m1 = -1, last_m3 = -1, last_m2 = -1, last_m4 = -1;
       if (nchunks > 0) {
-        tc::mbar_arrive_expect_tx(bar_tma, 6 * kTile);
+        tc::mbar_arrive_expect_tx(bar_tma, (kFused ? 5 : 6) * kTile);
         for (int i = 0; i < 6; ++i)
-          tc::tma_load_3d(smem + OFF_RAW + i * kTile, &maps.m[i], bar_tma, 0, h, static_cast<int>(sb.start));
+          if (!kFused || i != RAW_B)
+            tc::tma_load_3d(smem + OFF_RAW + i * kTile, &maps.m[i], bar_tma, 0, h, static_cast<int>(sb.start));
         last_tma = 0;
       }
       for (int c = 0; c < nchunks; ++c) {
@@ -517,16 +567,19 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
         // the next chunk's tiles (P1 has consumed the raw tiles), issued after MMA1: six TMA issues
         // take longer than MMA1 itself
         if (c + 1 < nchunks) {
-          tc::mbar_arrive_expect_tx(bar_tma, 6 * kTile);
+          tc::mbar_arrive_expect_tx(bar_tma, (kFused ? 5 : 6) * kTile);
           for (int i = 0; i < 6; ++i)
-            tc::tma_load_3d(smem + OFF_RAW + i * kTile, &maps.m[i], bar_tma, 0, h,
-                            static_cast<int>(sb.start + static_cast<long long>(c + 1) * C));
+            if (!kFused || i != RAW_B)
+              tc::tma_load_3d(smem + OFF_RAW + i * kTile, &maps.m[i], bar_tma, 0, h,
+                              static_cast<int>(sb.start + static_cast<long long>(c + 1) * C));
           last_tma = (c + 1) & 1;
         }
         // warm L2 with the chunk after that, so its TMA is an L2 hit when warps 4-7 need it early
         if (c + 2 < nchunks)
           for (int i = 0; i < 6; ++i)
-            tc::tma_prefetch_l2_3d(&maps.m[i], 0, h, static_cast<int>(sb.start + static_cast<long long>(c + 2) * C));
+            if (!kFused || i != RAW_B)
+              tc::tma_prefetch_l2_3d(&maps.m[i], 0, h,
+                                     static_cast<int>(sb.start + static_cast<long long>(c + 2) * C));
         // MMA3 (bf16): D3 = [A~^T; Lak^T] Tinv^T
         if (!wait_or_abort(bar_b3, ph, abort_flag)) { fail(); break; }
         tc::tc_fence_after();
@@ -672,9 +725,10 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
     };
 
 
-    // the first chunk's decay scan, [B^; K^] and V^T
+    // the key scale of this head (model-native inputs), then the first chunk's decay scan, [B^; K^] and V^T
+    if (kFused && tid >= 128 && tid < 192) kkw[tid - 128] = A.k_k ? A.k_k[h * kN + (tid - 128)] : 1.f;
     if (nchunks > 0 && warp >= 4 && wait_group_hi(bar_tma, 0))
-      prep_next(smem, sB1, sB4V, pre4, GCs, wtot, tid - 128, min(C, sb.len));
+      prep_next<kFused>(smem, sA1, sB1, sB4V, pre4, GCs, wtot, kkw, invn, tid - 128, min(C, sb.len));
     compute_sync();
 
     int Lc_prev = 0;
@@ -687,41 +741,44 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
       {
         const float4 pv = *reinterpret_cast<const float4 *>(pre4 + tg * 64 + j0);
         const float pre[4] = {pv.x, pv.y, pv.z, pv.w};  // Gamma before this thread's first token
-        float G[4][4];  // running products of w over this thread's tokens (rows) per channel (cols)
+        uint8_t *a1r = sA1 + (j0 >> 5) * (128 * 128);
+        const uint32_t chunk = (j0 & 31) >> 2;
+        float G[4][4];  // Gamma_t of this thread's tokens (rows) and channels (cols), left in A1 by the preparation
 #pragma unroll
         for (int tt = 0; tt < 4; ++tt) {
-          if (t0 + tt < Lc) {
-            raw4(smem, RAW_W, t0 + tt, j0, G[tt]);
-          } else {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) G[tt][e] = 1.f;
-          }
+          const float4 u = *reinterpret_cast<const float4 *>(a1r + tc::sw128(t0 + tt, chunk));
+          G[tt][0] = u.x;
+          G[tt][1] = u.y;
+          G[tt][2] = u.z;
+          G[tt][3] = u.w;
         }
-#pragma unroll
-        for (int k = 1; k < 4; ++k)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) G[k][e] *= G[k - 1][e];
         float rr[4][4], aa[4][4];
 #pragma unroll
         for (int tt = 0; tt < 4; ++tt) {
           if (t0 + tt < Lc) {
             raw4(smem, RAW_R, t0 + tt, j0, rr[tt]);
-            raw4(smem, RAW_A, t0 + tt, j0, aa[tt]);
+            if (kFused) {
+              // a = -kk = -(k * k_k) / |k * k_k|; the norms come from the preparation of this chunk
+              raw4(smem, RAW_K, t0 + tt, j0, aa[tt]);
+              const float in = invn[t0 + tt];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) aa[tt][e] = -(aa[tt][e] * kkw[j0 + e] * in);
+            } else {
+              raw4(smem, RAW_A, t0 + tt, j0, aa[tt]);
+            }
           } else {
 #pragma unroll
             for (int e = 0; e < 4; ++e) rr[tt][e] = aa[tt][e] = 0.f;
           }
         }
-        uint8_t *a1r = sA1 + (j0 >> 5) * (128 * 128);
-        const uint32_t chunk = (j0 & 31) >> 2;
 #pragma unroll
         for (int tt = 0; tt < 4; ++tt) {
           const int t = t0 + tt;
           float Gt[4], Gp[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            Gp[e] = tt == 0 ? pre[e] : pre[e] * G[tt - 1][e];
-            Gt[e] = pre[e] * G[tt][e];
+            Gp[e] = tt == 0 ? pre[e] : G[tt - 1][e];
+            Gt[e] = G[tt][e];
           }
           st_tf32x4(a1r + tc::sw128(t, chunk), rr[tt][0] * Gt[0], rr[tt][1] * Gt[1], rr[tt][2] * Gt[2],
                     rr[tt][3] * Gt[3]);
@@ -851,7 +908,8 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
         // then the next chunk's decay scan, [B^; K^] and V^T (its tiles were loaded after MMA1); B1 is
         // free: MMA1 is done and the masks above have read its B^ columns
         if (c + 1 < nchunks && wait_group_hi(bar_tma, (c + 1) & 1))
-          prep_next(smem, sB1, sB4V + ((c + 1) & 1) * 16384, pre4, GCs + ((c + 1) & 1) * 64, wtot, tid - 128,
+          prep_next<kFused>(smem, sA1, sB1, sB4V + ((c + 1) & 1) * 16384, pre4, GCs + ((c + 1) & 1) * 64, wtot, kkw,
+                            invn, tid - 128,
                     min(C, sb.len - (c + 1) * C));
       }
       if (!(ok = wait_ctrl(bar_m3, ph))) break;
@@ -950,12 +1008,34 @@ cudaError_t launch_chunk(const uint16_t *r, const uint16_t *w, const uint16_t *k
     if (!make_map(&maps.m[i], ops[i] ? ops[i] : static_cast<const void *>(s_out), tokens, H))
       return cudaErrorInvalidValue;
   }
-  Args args{y, s_in, s_out, cu_seqlens, T, total_T, H, err_word};
-  cudaError_t e = cudaFuncSetAttribute(wkv7_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  Args args{y, s_in, s_out, cu_seqlens, T, total_T, H, err_word, nullptr};
+  cudaError_t e = cudaFuncSetAttribute(wkv7_chunk_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(kSmemBytes));
   if (e != cudaSuccess) return e;
   dim3 grid(H, B);
-  wkv7_chunk_kernel<<<grid, kThreads, kSmemBytes, stream>>>(maps, args);
+  wkv7_chunk_kernel<false><<<grid, kThreads, kSmemBytes, stream>>>(maps, args);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_chunk_fused(const uint16_t *r, const uint16_t *xw, const uint16_t *k, const uint16_t *v,
+                               const uint16_t *xa, const float *k_k, const float *s_in, uint16_t *y, float *s_out,
+                               const int32_t *cu_seqlens, int B, int T, long long total_T, int H, int *err_word,
+                               cudaStream_t stream) {
+  using namespace chunk;
+  if (total_T > 0x7fffffffLL || H > 0xffff || B > 65535) return cudaErrorInvalidValue;
+  Maps maps;
+  const void *ops[6] = {r, xw, k, xa, nullptr, v};  // the b slot is never loaded
+  const long long tokens = total_T > 0 ? total_T : 1;
+  for (int i = 0; i < 6; ++i) {
+    if (!make_map(&maps.m[i], ops[i] ? ops[i] : static_cast<const void *>(s_out), tokens, H))
+      return cudaErrorInvalidValue;
+  }
+  Args args{y, s_in, s_out, cu_seqlens, T, total_T, H, err_word, k_k};
+  cudaError_t e = cudaFuncSetAttribute(wkv7_chunk_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kSmemBytes));
+  if (e != cudaSuccess) return e;
+  dim3 grid(H, B);
+  wkv7_chunk_kernel<true><<<grid, kThreads, kSmemBytes, stream>>>(maps, args);
   return cudaGetLastError();
 }
 

@@ -11,21 +11,27 @@
 // t/16 + 16*m (m = 0..3): four 16-byte loads per thread, issued together,
 // and a warp covers two whole 256-byte rows per load.  The row sums S a and
 // S r are finished with four xor-shuffles inside each 16-lane half-warp.
+//
+// The fused variant takes model-native inputs (decay pre-activation x_w in place of w, the key k,
+// the learning-rate pre-activation x_a in place of a, and the per-channel key scale k_k) and forms
+// w, a = -kk and b = kk * sigmoid(x_a) in-kernel; the key norm is one more 16-lane reduction.
 #include "common.cuh"
 #include "launch.h"
 
 namespace rwkv7 {
 
 template <typename TIn> struct DecodeArgs {
-  const TIn *r, *w, *k, *v, *a, *b;
+  const TIn *r, *w, *k, *v, *a, *b;  // fused: w = x_w, a = x_a, b unused
   float *s;
   TIn *y;
+  const float *k_k;  // fused: [H, 64] key scale, nullptr = ones
+  int H;
 };
 
 __device__ __forceinline__ float4 ld_state(const float *p) { return *reinterpret_cast<const float4 *>(p); }
 __device__ __forceinline__ void st_state(float *p, float4 x) { *reinterpret_cast<float4 *>(p) = x; }
 
-template <typename TIn>
+template <typename TIn, bool kFused>
 __global__ void __launch_bounds__(256) wkv7_decode_kernel(DecodeArgs<TIn> A) {
   const long long pair = blockIdx.x;  // b * H + h
   const int tid = threadIdx.x;
@@ -42,24 +48,57 @@ __global__ void __launch_bounds__(256) wkv7_decode_kernel(DecodeArgs<TIn> A) {
   Elem<TIn>::load4(A.w + vb + 4 * c4, ww);
   Elem<TIn>::load4(A.k + vb + 4 * c4, kk);
   Elem<TIn>::load4(A.a + vb + 4 * c4, aa);
-  Elem<TIn>::load4(A.b + vb + 4 * c4, bb);
+  if (!kFused) Elem<TIn>::load4(A.b + vb + 4 * c4, bb);
   Elem<TIn>::load4(A.r + vb + 4 * c4, rr);
-#pragma unroll
-  for (int m = 0; m < 4; ++m) vv[m] = Elem<TIn>::load(A.v + vb + rg + 16 * m);
-
   float sa[4];
+  if (kFused) {
+    // x070 prologue: kk = normalise(k * k_k) over the 64 channels, a = -kk, b = kk * rate, decay from
+    // x_w.  S a = -(S kx) / |kx| with kx = k * k_k: the row sums of S kx and |kx|^2 share the shuffles.
+    const int h = static_cast<int>(pair % A.H);
+    float kx[4], ss = 0.f;
 #pragma unroll
-  for (int m = 0; m < 4; ++m) {
-    float p = st[m].x * aa[0];
-    p = fmaf(st[m].y, aa[1], p);
-    p = fmaf(st[m].z, aa[2], p);
-    p = fmaf(st[m].w, aa[3], p);
-    sa[m] = p;
+    for (int e = 0; e < 4; ++e) {
+      kx[e] = A.k_k ? kk[e] * A.k_k[h * kN + 4 * c4 + e] : kk[e];
+      ss = fmaf(kx[e], kx[e], ss);
+    }
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      float p = st[m].x * kx[0];
+      p = fmaf(st[m].y, kx[1], p);
+      p = fmaf(st[m].z, kx[2], p);
+      p = fmaf(st[m].w, kx[3], p);
+      sa[m] = p;
+    }
+#pragma unroll
+    for (int off = 8; off >= 1; off >>= 1) {
+      ss += __shfl_xor_sync(0xffffffffu, ss, off);
+#pragma unroll
+      for (int m = 0; m < 4; ++m) sa[m] += __shfl_xor_sync(0xffffffffu, sa[m], off);
+    }
+    const float inv = x070_inv_norm(ss);
+#pragma unroll
+    for (int m = 0; m < 4; ++m) sa[m] *= -inv;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      bb[e] = kx[e] * inv * x070_sigmoid(aa[e]);
+      ww[e] = x070_decay(ww[e]);
+    }
+  } else {
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      float p = st[m].x * aa[0];
+      p = fmaf(st[m].y, aa[1], p);
+      p = fmaf(st[m].z, aa[2], p);
+      p = fmaf(st[m].w, aa[3], p);
+      sa[m] = p;
+    }
+#pragma unroll
+    for (int off = 8; off >= 1; off >>= 1)
+#pragma unroll
+      for (int m = 0; m < 4; ++m) sa[m] += __shfl_xor_sync(0xffffffffu, sa[m], off);
   }
 #pragma unroll
-  for (int off = 8; off >= 1; off >>= 1)
-#pragma unroll
-    for (int m = 0; m < 4; ++m) sa[m] += __shfl_xor_sync(0xffffffffu, sa[m], off);
+  for (int m = 0; m < 4; ++m) vv[m] = Elem<TIn>::load(A.v + vb + rg + 16 * m);
 
   float yv[4];
 #pragma unroll
@@ -91,10 +130,20 @@ __global__ void __launch_bounds__(256) wkv7_decode_kernel(DecodeArgs<TIn> A) {
 template <typename TIn>
 cudaError_t launch_decode(const TIn *r, const TIn *w, const TIn *k, const TIn *v, const TIn *a, const TIn *b,
                           float *s, TIn *y, int B, int H, cudaStream_t stream) {
-  DecodeArgs<TIn> A{r, w, k, v, a, b, s, y};
+  DecodeArgs<TIn> A{r, w, k, v, a, b, s, y, nullptr, H};
   const long long pairs = static_cast<long long>(B) * H;
   if (pairs > 0x7fffffffLL) return cudaErrorInvalidValue;
-  wkv7_decode_kernel<TIn><<<static_cast<unsigned>(pairs), 256, 0, stream>>>(A);
+  wkv7_decode_kernel<TIn, false><<<static_cast<unsigned>(pairs), 256, 0, stream>>>(A);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode_fused(const uint16_t *r, const uint16_t *xw, const uint16_t *k, const uint16_t *v,
+                                const uint16_t *xa, const float *k_k, float *s, uint16_t *y, int B, int H,
+                                cudaStream_t stream) {
+  DecodeArgs<uint16_t> A{r, xw, k, v, xa, nullptr, s, y, k_k, H};
+  const long long pairs = static_cast<long long>(B) * H;
+  if (pairs > 0x7fffffffLL) return cudaErrorInvalidValue;
+  wkv7_decode_kernel<uint16_t, true><<<static_cast<unsigned>(pairs), 256, 0, stream>>>(A);
   return cudaGetLastError();
 }
 

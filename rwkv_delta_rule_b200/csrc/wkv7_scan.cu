@@ -17,6 +17,10 @@
 // Per-token operands are staged into shared memory in tiles of TT tokens
 // with cp.async, double-buffered, and y is staged per tile and written back
 // as contiguous runs of ROWS elements.
+//
+// The fused variant takes model-native inputs (x_w in place of w, x_a in place of a, no b, and the
+// per-channel key scale k_k) and forms w, a = -kk and b = kk * sigmoid(x_a) per token in registers;
+// the key norm is two more xor-shuffles inside the quad, which holds all 64 columns of a row.
 #include "common.cuh"
 #include "launch.h"
 
@@ -38,7 +42,7 @@ template <typename TIn, int ROWS> struct ScanCfg {
 };
 
 template <typename TIn> struct ScanArgs {
-  const TIn *r, *w, *k, *v, *a, *b;
+  const TIn *r, *w, *k, *v, *a, *b;  // fused: w = x_w, a = x_a, b unused
   const float *s_in;
   TIn *y;
   float *s_out;
@@ -46,9 +50,10 @@ template <typename TIn> struct ScanArgs {
   int T;
   long long total_T;
   int H;
+  const float *k_k;  // fused: [H, 64] key scale, nullptr = ones
 };
 
-template <typename TIn, int ROWS>
+template <typename TIn, int ROWS, bool kFused>
 __device__ __forceinline__ void scan_load_tile(const ScanArgs<TIn> &A, TIn *buf, long long tok0, int ntok, int h,
                                                int row0) {
   using C = ScanCfg<TIn, ROWS>;
@@ -59,6 +64,7 @@ __device__ __forceinline__ void scan_load_tile(const ScanArgs<TIn> &A, TIn *buf,
     TIn *dst = buf + tt * C::kTokElems;
     if (cc < 5 * C::kChunksVec) {
       const int vid = cc / C::kChunksVec, part = cc - vid * C::kChunksVec;
+      if (kFused && vid == 4) continue;  // no b
       const TIn *src = vid == 0 ? A.r : vid == 1 ? A.w : vid == 2 ? A.k : vid == 3 ? A.a : A.b;
       cp_async16(dst + vid * kN + part * C::kEPC, src + base + part * C::kEPC);
     } else {
@@ -68,7 +74,7 @@ __device__ __forceinline__ void scan_load_tile(const ScanArgs<TIn> &A, TIn *buf,
   }
 }
 
-template <typename TIn, int ROWS>
+template <typename TIn, int ROWS, bool kFused>
 __global__ void __launch_bounds__(ScanCfg<TIn, ROWS>::kThreads) wkv7_scan_kernel(ScanArgs<TIn> A) {
   using C = ScanCfg<TIn, ROWS>;
   constexpr int kSplits = kN / ROWS;
@@ -95,9 +101,15 @@ __global__ void __launch_bounds__(ScanCfg<TIn, ROWS>::kThreads) wkv7_scan_kernel
     s[4 * m + 0] = x.x; s[4 * m + 1] = x.y; s[4 * m + 2] = x.z; s[4 * m + 3] = x.w;
   }
 
+  float kkr[16];  // fused: key scale of this thread's 16 columns
+#pragma unroll
+  for (int m = 0; m < 4; ++m)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) kkr[4 * m + e] = (kFused && A.k_k) ? A.k_k[h * kN + 16 * m + 4 * q + e] : 1.f;
+
   const int ntiles = (sb.len + C::kTT - 1) / C::kTT;
   if (ntiles > 0) {
-    scan_load_tile<TIn, ROWS>(A, bufs, sb.start, min(C::kTT, sb.len), h, row0);
+    scan_load_tile<TIn, ROWS, kFused>(A, bufs, sb.start, min(C::kTT, sb.len), h, row0);
     cp_async_commit();
   }
   for (int tile = 0; tile < ntiles; ++tile) {
@@ -105,8 +117,8 @@ __global__ void __launch_bounds__(ScanCfg<TIn, ROWS>::kThreads) wkv7_scan_kernel
     const int ntok = min(C::kTT, sb.len - t0);
     if (tile + 1 < ntiles) {
       const int t1 = t0 + C::kTT;
-      scan_load_tile<TIn, ROWS>(A, bufs + ((tile + 1) & 1) * C::kBufElems, sb.start + t1, min(C::kTT, sb.len - t1),
-                                h, row0);
+      scan_load_tile<TIn, ROWS, kFused>(A, bufs + ((tile + 1) & 1) * C::kBufElems, sb.start + t1,
+                                        min(C::kTT, sb.len - t1), h, row0);
       cp_async_commit();
       cp_async_wait<1>();
     } else {
@@ -126,9 +138,25 @@ __global__ void __launch_bounds__(ScanCfg<TIn, ROWS>::kThreads) wkv7_scan_kernel
         Elem<TIn>::load4(tok + 1 * kN + col, ww + 4 * m);
         Elem<TIn>::load4(tok + 2 * kN + col, kk + 4 * m);
         Elem<TIn>::load4(tok + 3 * kN + col, aa + 4 * m);
-        Elem<TIn>::load4(tok + 4 * kN + col, bb + 4 * m);
+        if (!kFused) Elem<TIn>::load4(tok + 4 * kN + col, bb + 4 * m);
       }
       const float vi = Elem<TIn>::load(tok + C::kVecElems + rloc);
+      if (kFused) {
+        // x070 prologue: kk = normalise(k * k_k) over the quad's 64 columns, a = -kk, b = kk * rate
+        float ss = 0.f;
+#pragma unroll
+        for (int c = 0; c < 16; ++c) ss = fmaf(kk[c] * kkr[c], kk[c] * kkr[c], ss);
+        ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+        ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+        const float inv = x070_inv_norm(ss);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const float kkv = kk[c] * kkr[c] * inv;
+          bb[c] = kkv * x070_sigmoid(aa[c]);
+          aa[c] = -kkv;
+          ww[c] = x070_decay(ww[c]);
+        }
+      }
 
       // sa = S a (state before this token), four partial sums then the quad
       float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
@@ -177,10 +205,10 @@ __global__ void __launch_bounds__(ScanCfg<TIn, ROWS>::kThreads) wkv7_scan_kernel
         make_float4(s[4 * m + 0], s[4 * m + 1], s[4 * m + 2], s[4 * m + 3]);
 }
 
-template <typename TIn, int ROWS>
+template <typename TIn, int ROWS, bool kFused = false>
 static cudaError_t launch_scan_rows(const ScanArgs<TIn> &A, int B, cudaStream_t stream) {
   using C = ScanCfg<TIn, ROWS>;
-  auto kern = wkv7_scan_kernel<TIn, ROWS>;
+  auto kern = wkv7_scan_kernel<TIn, ROWS, kFused>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(C::kSmemBytes));
   if (e != cudaSuccess) return e;
@@ -193,8 +221,16 @@ template <typename TIn>
 cudaError_t launch_scan(const TIn *r, const TIn *w, const TIn *k, const TIn *v, const TIn *a, const TIn *b,
                         const float *s_in, TIn *y, float *s_out, const int32_t *cu_seqlens, int B, int T,
                         long long total_T, int H, cudaStream_t stream) {
-  ScanArgs<TIn> A{r, w, k, v, a, b, s_in, y, s_out, cu_seqlens, T, total_T, H};
+  ScanArgs<TIn> A{r, w, k, v, a, b, s_in, y, s_out, cu_seqlens, T, total_T, H, nullptr};
   return launch_scan_rows<TIn, 16>(A, B, stream);
+}
+
+cudaError_t launch_scan_fused(const uint16_t *r, const uint16_t *xw, const uint16_t *k, const uint16_t *v,
+                              const uint16_t *xa, const float *k_k, const float *s_in, uint16_t *y, float *s_out,
+                              const int32_t *cu_seqlens, int B, int T, long long total_T, int H,
+                              cudaStream_t stream) {
+  ScanArgs<uint16_t> A{r, xw, k, v, xa, nullptr, s_in, y, s_out, cu_seqlens, T, total_T, H, k_k};
+  return launch_scan_rows<uint16_t, 16, true>(A, B, stream);
 }
 
 template cudaError_t launch_scan<float>(const float *, const float *, const float *, const float *, const float *,

@@ -35,6 +35,14 @@ template <typename TIn, bool kFused>
 __global__ void __launch_bounds__(256) wkv7_decode_kernel(DecodeArgs<TIn> A) {
   const long long pair = blockIdx.x;  // b * H + h
   const int tid = threadIdx.x;
+  // fused: the decay and the learning rate of each of the 64 channels, computed once per CTA (the 16
+  // row groups share them) by threads 0..63 while the state loads are in flight
+  __shared__ float s_w[kFused ? kN : 1], s_rate[kFused ? kN : 1];
+  if (kFused && tid < kN) {
+    const long long vbase = pair * kN;
+    s_w[tid] = x070_decay(Elem<TIn>::load(A.w + vbase + tid));
+    s_rate[tid] = x070_sigmoid(Elem<TIn>::load(A.a + vbase + tid));
+  }
   const int c4 = tid & 15;   // column chunk: columns 4*c4 .. 4*c4+3
   const int rg = tid >> 4;   // rows rg + 16*m
   float *S = A.s + pair * (kN * kN);
@@ -45,10 +53,12 @@ __global__ void __launch_bounds__(256) wkv7_decode_kernel(DecodeArgs<TIn> A) {
 
   const long long vb = pair * kN;
   float ww[4], kk[4], aa[4], bb[4], rr[4], vv[4];
-  Elem<TIn>::load4(A.w + vb + 4 * c4, ww);
   Elem<TIn>::load4(A.k + vb + 4 * c4, kk);
-  Elem<TIn>::load4(A.a + vb + 4 * c4, aa);
-  if (!kFused) Elem<TIn>::load4(A.b + vb + 4 * c4, bb);
+  if (!kFused) {
+    Elem<TIn>::load4(A.w + vb + 4 * c4, ww);
+    Elem<TIn>::load4(A.a + vb + 4 * c4, aa);
+    Elem<TIn>::load4(A.b + vb + 4 * c4, bb);
+  }
   Elem<TIn>::load4(A.r + vb + 4 * c4, rr);
   float sa[4];
   if (kFused) {
@@ -78,10 +88,11 @@ __global__ void __launch_bounds__(256) wkv7_decode_kernel(DecodeArgs<TIn> A) {
     const float inv = x070_inv_norm(ss);
 #pragma unroll
     for (int m = 0; m < 4; ++m) sa[m] *= -inv;
+    __syncthreads();  // s_w / s_rate
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      bb[e] = kx[e] * inv * x070_sigmoid(aa[e]);
-      ww[e] = x070_decay(ww[e]);
+      bb[e] = kx[e] * inv * s_rate[4 * c4 + e];
+      ww[e] = s_w[4 * c4 + e];
     }
   } else {
 #pragma unroll

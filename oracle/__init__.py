@@ -162,5 +162,24 @@ def wkv7_model_native(r, xw, k, v, xa, k_k, s_in=None, *, nthreads: Optional[int
                 nthreads=nthreads, precision="f64")
 
 
+LN_EPS = 64e-5  # the GroupNorm eps of the x070 ln_x (the page marks it as not to be changed)
+
+
+def group_norm_heads(y, ln_w=None, ln_b=None, eps: float = LN_EPS) -> np.ndarray:
+    """The x070 ``ln_x`` epilogue in float64 (RWKV-7 G0 7.2B walkthrough, lshu.cn/news/198401, section
+    7.1: GroupNorm with eps 64e-5, one group per head): for every token and head, the 64 channels of
+    ``y`` minus their mean, divided by ``sqrt(var + eps)`` (variance over the 64 channels, divisor
+    64), times ``ln_w`` plus ``ln_b`` (``[H, N]``; None means ones / zeros).  ``y``: ``[..., H, N]``."""
+    y = _as_np(y, np.float64)
+    mu = y.mean(axis=-1, keepdims=True)
+    var = ((y - mu) ** 2).mean(axis=-1, keepdims=True)
+    out = (y - mu) / np.sqrt(var + eps)
+    if ln_w is not None:
+        out = out * _as_np(ln_w, np.float64)
+    if ln_b is not None:
+        out = out + _as_np(ln_b, np.float64)
+    return out
+
+
 def real_bytes(real: str = "double") -> int:
     return int(_lib(real).wkv7_oracle_real_bytes())

@@ -302,20 +302,27 @@ def bench_decode(lib7, dev, steps_target: int = 1024, layers: int = 24):
 NATIVE = ("r", "xw", "k", "v", "xa")
 
 
-def bench_model_native(lib7, dev, B, T, H, steps, decode_steps=1024, layers=24):
-    """The model-native entry points (operand prologue in the kernels) on the same shapes: prefill
-    launch time and HBM roofline (five input tensors + y + state), and decode steps/s."""
+def bench_options(lib7, dev, B, T, H, steps, *, native, group_norm, decode_steps=1024, layers=24):
+    """The option entry points on the same shapes -- model-native inputs (operand prologue in the
+    kernels) and / or the ln_x GroupNorm epilogue: prefill launch time and HBM roofline (input tensors
+    + y + state in and out), and decode steps/s at the L24-D1024 shape."""
     case = wi.CASES[WORKLOAD]
-    d = wi.draw_model_native(B, T, H, seed=case.seed, s0_std=case.s0_std)
-    dd = {n: d[n].to(dev) for n in NATIVE}
-    kk = d["k_k"].to(dev)
+    names = NATIVE if native else OPS
+    d = (wi.draw_model_native if native else wi.draw)(B, T, H, seed=case.seed, s0_std=case.s0_std)
+    dd = {n: d[n].to(dev) for n in names}
+    kk = d["k_k"].to(dev) if native else None
+    ln = {k: t.to(dev) for k, t in wi.draw_group_norm(H, seed=case.seed + 1).items()} if group_norm else {}
+    opt = dict(model_native=native, k_k=kk, group_norm=group_norm, ln_w=ln.get("ln_w"), ln_b=ln.get("ln_b"))
     s0 = d["s0"].to(dev)
     y = torch.empty_like(dd["r"])
     s_out = torch.empty_like(s0)
     stream = torch.cuda.current_stream(dev)
 
+    def ops(src):
+        return [src[n] for n in names] + ([None] if native else [])
+
     def step():
-        lib7.rwkv7_wkv_prefill_fused_bf16(lib7.RWKV7_PATH_AUTO, *[dd[n] for n in NATIVE], kk, s0, y, s_out, stream)
+        lib7.rwkv7_wkv_prefill_ext_bf16(lib7.RWKV7_PATH_AUTO, *ops(dd), s0, y, s_out, stream=stream, **opt)
 
     for _ in range(5):
         step()
@@ -328,50 +335,56 @@ def bench_model_native(lib7, dev, B, T, H, steps, decode_steps=1024, layers=24):
     torch.cuda.synchronize()
     assert lib7.rwkv7_get_last_error() == 0
     ms = e0.elapsed_time(e1) / steps
-    byts = 6 * B * T * H * N * 2 + 2 * B * H * N * N * 4
+    byts = (len(names) + 1) * B * T * H * N * 2 + 2 * B * H * N * N * 4
     peaks, _ = load_peaks()
     pre = {"launch_ms": ms, "tokens_per_s": B * T / (ms / 1e3), "algorithmic_bytes_per_launch": byts,
            "achieved_gbs": byts / (ms / 1e3) / 1e9, "frac": byts / (ms / 1e3) / 1e9 / peaks["hbm_gbs"]}
     del dd, y, s_out
-    # decode at the L24-D1024 shape, rotating `layers` distinct states inside a CUDA graph
-    dc = wi.CASES["decode_l24_d1024_b256_1024steps"]
-    Bd, Hd, ntok = dc.B, dc.H, 8
-    dn = wi.draw_model_native(Bd, ntok, Hd, seed=dc.seed)
-    toks = [{n: dn[n][:, t].contiguous().to(dev) for n in NATIVE} for t in range(ntok)]
-    kkd = dn["k_k"].to(dev)
-    states = torch.zeros(layers, Bd, Hd, N, N, device=dev)
-    ys = [torch.empty(Bd, Hd, N, dtype=torch.bfloat16, device=dev) for _ in range(layers)]
-    per_graph = layers * 4
+    out = {"prefill": pre}
+    if decode_steps:
+        dc = wi.CASES["decode_l24_d1024_b256_1024steps"]
+        Bd, Hd, ntok = dc.B, dc.H, 8
+        dn = (wi.draw_model_native if native else wi.draw)(Bd, ntok, Hd, seed=dc.seed)
+        toks = [{n: dn[n][:, t].contiguous().to(dev) for n in names} for t in range(ntok)]
+        dopt = dict(opt, k_k=dn["k_k"].to(dev) if native else None)
+        if group_norm:
+            lnd = wi.draw_group_norm(Hd, seed=dc.seed + 1)
+            dopt.update(ln_w=lnd["ln_w"].to(dev), ln_b=lnd["ln_b"].to(dev))
+        states = torch.zeros(layers, Bd, Hd, N, N, device=dev)
+        ys = [torch.empty(Bd, Hd, N, dtype=torch.bfloat16, device=dev) for _ in range(layers)]
+        per_graph = layers * 4
 
-    def one_pass():
-        for i in range(per_graph):
-            tk = toks[i % ntok]
-            lib7.rwkv7_wkv_decode_fused_bf16(*[tk[n] for n in NATIVE], kkd, states[i % layers], ys[i % layers])
+        def one_pass():
+            for i in range(per_graph):
+                lib7.rwkv7_wkv_decode_ext_bf16(*ops(toks[i % ntok]), states[i % layers], ys[i % layers], **dopt)
 
-    sd = torch.cuda.Stream(device=dev)
-    sd.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(sd):
-        one_pass()
-    torch.cuda.current_stream().wait_stream(sd)
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g):
-        one_pass()
-    reps = max(1, (decode_steps + per_graph - 1) // per_graph)
-    for _ in range(3):
-        g.replay()
-    torch.cuda.synchronize()
-    e0.record()
-    for _ in range(reps):
-        g.replay()
-    e1.record()
-    torch.cuda.synchronize()
-    step_s = e0.elapsed_time(e1) / 1e3 / (reps * per_graph)
-    dbytes = Bd * Hd * (2 * N * N * 4 + 6 * N * 2)
-    dec = {"workload": "decode_l24_d1024_b256", "steps_per_s": 1.0 / step_s, "us_per_step": step_s * 1e6,
-           "bytes_per_step": dbytes, "achieved_gbs": dbytes / step_s / 1e9,
-           "frac": dbytes / step_s / 1e9 / peaks["hbm_gbs"]}
-    return {"prefill": pre, "decode": dec,
-            "inputs": "bf16 r, x_w, k, v, x_a [B,T,H,64] + float32 k_k [H,64]; w, a, b formed in-kernel"}
+        sd = torch.cuda.Stream(device=dev)
+        sd.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(sd):
+            one_pass()
+        torch.cuda.current_stream().wait_stream(sd)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            one_pass()
+        reps = max(1, (decode_steps + per_graph - 1) // per_graph)
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(reps):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        assert lib7.rwkv7_get_last_error() == 0
+        step_s = e0.elapsed_time(e1) / 1e3 / (reps * per_graph)
+        dbytes = Bd * Hd * (2 * N * N * 4 + (len(names) + 1) * N * 2)
+        out["decode"] = {"workload": "decode_l24_d1024_b256", "steps_per_s": 1.0 / step_s,
+                         "us_per_step": step_s * 1e6, "bytes_per_step": dbytes, "achieved_gbs": dbytes / step_s / 1e9,
+                         "frac": dbytes / step_s / 1e9 / peaks["hbm_gbs"]}
+    out["inputs"] = (("bf16 r, x_w, k, v, x_a [B,T,H,64] + float32 k_k [H,64]; w, a, b formed in-kernel"
+                      if native else "bf16 r, w, k, v, a, b [B,T,H,64]")
+                     + ("; y through the ln_x GroupNorm (float32 ln_w, ln_b [H,64])" if group_norm else ""))
+    return out
 
 
 def run_ours(args):
@@ -479,8 +492,10 @@ def run_ours(args):
 
     native = None
     if not args.no_native and args.path == "auto":
-        native = bench_model_native(lib7, dev, B, T, H, steps=min(args.steps, 50),
-                                    decode_steps=0 if args.no_decode else args.decode_steps)
+        native = {key: bench_options(lib7, dev, B, T, H, steps=min(args.steps, 50), native=nat, group_norm=gn,
+                                     decode_steps=0 if args.no_decode else args.decode_steps)
+                  for key, nat, gn in (("model_native", True, False), ("group_norm", False, True),
+                                       ("model_native_group_norm", True, True))}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -505,7 +520,7 @@ def run_ours(args):
         "clocks": clocks.summary(),
         "cpu_baseline": cpu,
         "decode": decode,
-        "model_native": native,
+        "options": native,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -526,7 +541,8 @@ def main():
     ap.add_argument("--batch", type=int, default=0, help="override B (profiling runs only)")
     ap.add_argument("--seqlen", type=int, default=0, help="override T (profiling runs only)")
     ap.add_argument("--no-decode", action="store_true")
-    ap.add_argument("--no-native", action="store_true", help="skip the model-native entry points' lines")
+    ap.add_argument("--no-native", action="store_true",
+                    help="skip the option entry points' lines (model-native inputs, GroupNorm epilogue)")
     ap.add_argument("--decode-steps", type=int, default=1024)
     ap.add_argument("--decode-layers", type=int, default=24, help="distinct decode states rotated over")
     ap.add_argument("--no-e2e", action="store_true")

@@ -160,6 +160,38 @@ RWKV7_API rwkv7_status rwkv7_wkv_decode_fused_bf16(int B, int H, int N, const ui
                                                    const float *k_k, float *s_inout, uint16_t *y,
                                                    rwkv7_stream_t stream);
 
+/* ---- options: model-native inputs and the ln_x epilogue, in any combination ----
+ *
+ * A host struct read during the call; zero-initialise it for none of the parts, or pass NULL.
+ *   model_native = 1: the w and a arguments hold the pre-activations x_w and x_a, b is ignored (may
+ *                     be NULL) and k_k is the key scale (see the fused entry points above).
+ *   group_norm = 1:   the x070 ln_x epilogue (RWKV-7 G0 7.2B walkthrough, lshu.cn/news/198401,
+ *                     section 7.1: GroupNorm with one group per head, eps 64e-5) is applied to y:
+ *                     y = (y - mean) / sqrt(var + 64e-5) * ln_w + ln_b over each token-head's 64
+ *                     channels (variance with divisor 64).  ln_w / ln_b: float32 [H,64] device
+ *                     buffers, 16-byte aligned, NULL meaning ones / zeros.
+ * The state is not affected by group_norm. */
+typedef struct rwkv7_options {
+  int model_native;
+  const float *k_k;
+  int group_norm;
+  const float *ln_w;
+  const float *ln_b;
+} rwkv7_options;
+
+/* bf16 prefill with options (NULL = none); other arguments as for rwkv7_wkv_prefill_bf16_path. */
+RWKV7_API rwkv7_status rwkv7_wkv_prefill_ext_bf16(int path, int B, int T, int H, int N, const uint16_t *r,
+                                                  const uint16_t *w, const uint16_t *k, const uint16_t *v,
+                                                  const uint16_t *a, const uint16_t *b, const rwkv7_options *opt,
+                                                  const float *s_in, uint16_t *y, float *s_out,
+                                                  rwkv7_stream_t stream);
+
+/* bf16 decode step with options (NULL = none); other arguments as for rwkv7_wkv_decode_bf16. */
+RWKV7_API rwkv7_status rwkv7_wkv_decode_ext_bf16(int B, int H, int N, const uint16_t *r, const uint16_t *w,
+                                                 const uint16_t *k, const uint16_t *v, const uint16_t *a,
+                                                 const uint16_t *b, const rwkv7_options *opt, float *s_inout,
+                                                 uint16_t *y, rwkv7_stream_t stream);
+
 /* ---- status ---------------------------------------------------------------- */
 
 /* Static English description of a status code (never NULL). */

@@ -62,6 +62,24 @@ __device__ __forceinline__ float x070_decay(float xw) { return __expf(-0.6065306
 // 1 / max(||x||, 1e-12) from the sum of squares (the divisor of the L2 normalisation)
 __device__ __forceinline__ float x070_inv_norm(float sumsq) { return rsqrtf(fmaxf(sumsq, 1e-24f)); }
 
+// ---- the x070 ln_x epilogue: GroupNorm with one group per head, eps 64e-5 ----------
+// (lshu.cn/news/198401, section 7.1).  y_n = (y - mean) / sqrt(var + eps) * ln_w + ln_b over the 64
+// channels of a token-head, variance with divisor 64.
+constexpr float kLnEps = 64e-5f;
+
+// Mean and variance of the 64 values held two per lane (x0, x1) by a full warp.
+__device__ __forceinline__ void warp_mean_var64(float x0, float x1, float &mean, float &var) {
+  float s = x0 + x1;
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+  mean = s * (1.f / 64.f);
+  const float d0 = x0 - mean, d1 = x1 - mean;
+  float q = d0 * d0 + d1 * d1;
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) q += __shfl_xor_sync(0xffffffffu, q, off);
+  var = q * (1.f / 64.f);
+}
+
 // ---- cp.async (16-byte, L2-only) ---------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -14,23 +14,27 @@ cudaError_t launch_scan(const TIn *r, const TIn *w, const TIn *k, const TIn *v, 
                         const float *s_in, TIn *y, float *s_out, const int32_t *cu_seqlens, int B, int T,
                         long long total_T, int H, cudaStream_t stream);
 
-// The scan on model-native inputs (x_w, k, x_a and the key scale k_k, [H,64] float32 or nullptr
-// for ones): w, a and b are formed per token in-kernel.
-cudaError_t launch_scan_fused(const uint16_t *r, const uint16_t *xw, const uint16_t *k, const uint16_t *v,
-                              const uint16_t *xa, const float *k_k, const float *s_in, uint16_t *y, float *s_out,
-                              const int32_t *cu_seqlens, int B, int T, long long total_T, int H,
-                              cudaStream_t stream);
+// The bf16 scan with the optional parts: model-native inputs (w, a slots hold x_w, x_a; b unused;
+// key scale k_k [H,64] float32 or nullptr for ones) and the GroupNorm epilogue on y (ln_w, ln_b
+// [H,64] float32 or nullptr for ones / zeros).
+cudaError_t launch_scan_ext(const uint16_t *r, const uint16_t *w, const uint16_t *k, const uint16_t *v,
+                            const uint16_t *a, const uint16_t *b, bool model_native, const float *k_k,
+                            bool group_norm, const float *ln_w, const float *ln_b, const float *s_in, uint16_t *y,
+                            float *s_out, const int32_t *cu_seqlens, int B, int T, long long total_T, int H,
+                            cudaStream_t stream);
 
 // One decode step over [B,H,64], state updated in place.
 template <typename TIn>
 cudaError_t launch_decode(const TIn *r, const TIn *w, const TIn *k, const TIn *v, const TIn *a, const TIn *b,
                           float *s, TIn *y, int B, int H, cudaStream_t stream);
 
-// The same step on model-native inputs (x_w, k, x_a and the key scale k_k, [H,64] float32 or
-// nullptr for ones): w, a and b are formed in-kernel.
-cudaError_t launch_decode_fused(const uint16_t *r, const uint16_t *xw, const uint16_t *k, const uint16_t *v,
-                                const uint16_t *xa, const float *k_k, float *s, uint16_t *y, int B, int H,
-                                cudaStream_t stream);
+// The bf16 step with the optional parts: model-native inputs (w, a slots hold x_w, x_a; b unused;
+// key scale k_k [H,64] float32 or nullptr for ones) and the GroupNorm epilogue on y (ln_w, ln_b
+// [H,64] float32 or nullptr for ones / zeros).
+cudaError_t launch_decode_ext(const uint16_t *r, const uint16_t *w, const uint16_t *k, const uint16_t *v,
+                              const uint16_t *a, const uint16_t *b, bool model_native, const float *k_k,
+                              bool group_norm, const float *ln_w, const float *ln_b, float *s, uint16_t *y, int B,
+                              int H, cudaStream_t stream);
 
 // Chunked tensor-core prefill (bfloat16 operands), same layouts as
 // launch_scan.  err_word: device word that bounded waits report into.
@@ -39,11 +43,13 @@ cudaError_t launch_chunk(const uint16_t *r, const uint16_t *w, const uint16_t *k
                          const int32_t *cu_seqlens, int B, int T, long long total_T, int H, int *err_word,
                          cudaStream_t stream);
 
-// The chunked prefill on model-native inputs (x_w, k, x_a and the key scale k_k, [H,64] float32 or
-// nullptr for ones): w, a and b are formed in-kernel; five tiles are loaded per chunk.
-cudaError_t launch_chunk_fused(const uint16_t *r, const uint16_t *xw, const uint16_t *k, const uint16_t *v,
-                               const uint16_t *xa, const float *k_k, const float *s_in, uint16_t *y, float *s_out,
-                               const int32_t *cu_seqlens, int B, int T, long long total_T, int H, int *err_word,
-                               cudaStream_t stream);
+// The chunked prefill with the optional parts: model-native inputs (w, a slots hold x_w, x_a; b
+// unused; key scale k_k [H,64] float32 or nullptr for ones) and the GroupNorm epilogue on y (ln_w,
+// ln_b [H,64] float32 or nullptr for ones / zeros).
+cudaError_t launch_chunk_ext(const uint16_t *r, const uint16_t *w, const uint16_t *k, const uint16_t *v,
+                             const uint16_t *a, const uint16_t *b, bool model_native, const float *k_k,
+                             bool group_norm, const float *ln_w, const float *ln_b, const float *s_in, uint16_t *y,
+                             float *s_out, const int32_t *cu_seqlens, int B, int T, long long total_T, int H,
+                             int *err_word, cudaStream_t stream);
 
 }  // namespace rwkv7

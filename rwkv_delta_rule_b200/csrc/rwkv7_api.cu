@@ -149,35 +149,61 @@ rwkv7_status rwkv7_wkv_decode_bf16(int B, int H, int N, const uint16_t *r, const
   if (N != kN) return RWKV7_ERR_UNSUPPORTED;
   if (B <= 0 || H <= 0 || !none_null(r, w, k, v, a, b, s_inout, y)) return RWKV7_ERR_INVALID;
   if (!all_aligned(r, w, k, v, a, b, s_inout, y)) return RWKV7_ERR_ALIGN;
+  return from_cuda(launch_decode_ext(r, w, k, v, a, b, false, nullptr, false, nullptr, nullptr, s_inout, y, B, H,
+                                     reinterpret_cast<cudaStream_t>(stream)));
+}
+
+rwkv7_status rwkv7_wkv_prefill_ext_bf16(int path, int B, int T, int H, int N, const uint16_t *r, const uint16_t *w,
+                                        const uint16_t *k, const uint16_t *v, const uint16_t *a, const uint16_t *b,
+                                        const rwkv7_options *opt, const float *s_in, uint16_t *y, float *s_out,
+                                        rwkv7_stream_t stream) {
+  if (path != RWKV7_PATH_AUTO && path != RWKV7_PATH_SCAN && path != RWKV7_PATH_CHUNK) return RWKV7_ERR_INVALID;
+  const bool native = opt != nullptr && opt->model_native != 0;
+  const bool ln = opt != nullptr && opt->group_norm != 0;
+  const float *k_k = native ? opt->k_k : nullptr;
+  const float *ln_w = ln ? opt->ln_w : nullptr, *ln_b = ln ? opt->ln_b : nullptr;
+  // model-native calls have no b: the shared checks see a in its place
+  const rwkv7_status st = check_prefill(B, T, H, N, r, w, k, v, a, native ? a : b, s_in, y, s_out);
+  if (st != RWKV7_OK) return st;
+  if (!all_aligned(k_k, ln_w, ln_b)) return RWKV7_ERR_ALIGN;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  const long long total = static_cast<long long>(B) * T;
+  if (use_chunk(path, T))
+    return from_cuda(launch_chunk_ext(r, w, k, v, a, b, native, k_k, ln, ln_w, ln_b, s_in, y, s_out, nullptr, B, T,
+                                      total, H, error_word_ptr(), cs));
   return from_cuda(
-      launch_decode<uint16_t>(r, w, k, v, a, b, s_inout, y, B, H, reinterpret_cast<cudaStream_t>(stream)));
+      launch_scan_ext(r, w, k, v, a, b, native, k_k, ln, ln_w, ln_b, s_in, y, s_out, nullptr, B, T, total, H, cs));
+}
+
+rwkv7_status rwkv7_wkv_decode_ext_bf16(int B, int H, int N, const uint16_t *r, const uint16_t *w, const uint16_t *k,
+                                       const uint16_t *v, const uint16_t *a, const uint16_t *b,
+                                       const rwkv7_options *opt, float *s_inout, uint16_t *y,
+                                       rwkv7_stream_t stream) {
+  const bool native = opt != nullptr && opt->model_native != 0;
+  const bool ln = opt != nullptr && opt->group_norm != 0;
+  const float *k_k = native ? opt->k_k : nullptr;
+  const float *ln_w = ln ? opt->ln_w : nullptr, *ln_b = ln ? opt->ln_b : nullptr;
+  if (N != kN) return RWKV7_ERR_UNSUPPORTED;
+  if (B <= 0 || H <= 0 || !none_null(r, w, k, v, a, s_inout, y) || (!native && b == nullptr))
+    return RWKV7_ERR_INVALID;
+  if (!all_aligned(r, w, k, v, a, b, s_inout, y, k_k, ln_w, ln_b)) return RWKV7_ERR_ALIGN;
+  return from_cuda(launch_decode_ext(r, w, k, v, a, b, native, k_k, ln, ln_w, ln_b, s_inout, y, B, H,
+                                     reinterpret_cast<cudaStream_t>(stream)));
 }
 
 rwkv7_status rwkv7_wkv_prefill_fused_bf16(int path, int B, int T, int H, int N, const uint16_t *r,
                                           const uint16_t *xw, const uint16_t *k, const uint16_t *v,
                                           const uint16_t *xa, const float *k_k, const float *s_in, uint16_t *y,
                                           float *s_out, rwkv7_stream_t stream) {
-  if (path != RWKV7_PATH_AUTO && path != RWKV7_PATH_SCAN && path != RWKV7_PATH_CHUNK) return RWKV7_ERR_INVALID;
-  // the b slot of the shared checks is filled with xa: model-native calls have no b
-  const rwkv7_status st = check_prefill(B, T, H, N, r, xw, k, v, xa, xa, s_in, y, s_out);
-  if (st != RWKV7_OK) return st;
-  if (!aligned16(k_k)) return RWKV7_ERR_ALIGN;
-  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  const long long total = static_cast<long long>(B) * T;
-  if (use_chunk(path, T))
-    return from_cuda(
-        launch_chunk_fused(r, xw, k, v, xa, k_k, s_in, y, s_out, nullptr, B, T, total, H, error_word_ptr(), cs));
-  return from_cuda(launch_scan_fused(r, xw, k, v, xa, k_k, s_in, y, s_out, nullptr, B, T, total, H, cs));
+  const rwkv7_options opt{1, k_k, 0, nullptr, nullptr};
+  return rwkv7_wkv_prefill_ext_bf16(path, B, T, H, N, r, xw, k, v, xa, nullptr, &opt, s_in, y, s_out, stream);
 }
 
 rwkv7_status rwkv7_wkv_decode_fused_bf16(int B, int H, int N, const uint16_t *r, const uint16_t *xw,
                                          const uint16_t *k, const uint16_t *v, const uint16_t *xa, const float *k_k,
                                          float *s_inout, uint16_t *y, rwkv7_stream_t stream) {
-  if (N != kN) return RWKV7_ERR_UNSUPPORTED;
-  if (B <= 0 || H <= 0 || !none_null(r, xw, k, v, xa, s_inout, y)) return RWKV7_ERR_INVALID;
-  if (!all_aligned(r, xw, k, v, xa, k_k, s_inout, y)) return RWKV7_ERR_ALIGN;
-  return from_cuda(
-      launch_decode_fused(r, xw, k, v, xa, k_k, s_inout, y, B, H, reinterpret_cast<cudaStream_t>(stream)));
+  const rwkv7_options opt{1, k_k, 0, nullptr, nullptr};
+  return rwkv7_wkv_decode_ext_bf16(B, H, N, r, xw, k, v, xa, nullptr, &opt, s_inout, y, stream);
 }
 
 }  // extern "C"

@@ -80,11 +80,15 @@ constexpr uint32_t OFF_PRE = OFF_TS + 6 * 16 * LDTB * 4;  // float [16][64]: Gam
 constexpr uint32_t MISC_GC = 256;                         // float [2][64] Gamma at the chunk end, by chunk parity
 constexpr uint32_t MISC_WTOT = 768;                       // float [4][64] decay products of 16-token blocks
 constexpr uint32_t OFF_KX = OFF_PRE + 16 * 64 * 4;  // model-native inputs: float [64] k_k, float [64] 1/|k k_k|
-constexpr uint32_t kSmemBytes = OFF_KX + 2 * 64 * 4 + 1024;
+constexpr uint32_t OFF_LN = OFF_KX + 2 * 64 * 4;     // group norm: float [2][64] ln_w, ln_b; float2 [2][64] stats
+constexpr uint32_t kSmemBytes = OFF_LN + 2 * 64 * 4 + 2 * 64 * 8 + 1024;
 
 static_assert(MISC_WTOT + 4 * 64 * 4 <= 2048, "misc region overflow");
 static_assert(OFF_ZS + 6 * 16 * LDZ * 4 <= OFF_B2 + 16384, "inverse scratch overflows B2");
 static_assert(kSmemBytes <= 232448, "shared memory over the sm_100 limit");
+
+// Barrier of the four lo-lane compute warps (0, 1, 4, 5: TMEM lanes 0..63, the token rows of y).
+__device__ __forceinline__ void lo_lane_sync() { asm volatile("bar.sync 4, 128;\n" ::: "memory"); }
 
 // Barrier among the 8 compute warps only (the control warp never joins it).
 __device__ __forceinline__ void compute_sync() { asm volatile("bar.sync 1, 256;\n" ::: "memory"); }
@@ -116,6 +120,7 @@ struct Args {
   int H;
   int *err;
   const float *k_k;  // model-native inputs: [H, 64] key scale, nullptr = ones
+  const float *ln_w, *ln_b;  // group-norm epilogue: [H, 64] weight / bias, nullptr = ones / zeros
 };
 
 enum { RAW_R = 0, RAW_W = 1, RAW_K = 2, RAW_A = 3, RAW_B = 4, RAW_V = 5 };
@@ -473,7 +478,9 @@ __device__ __forceinline__ void prep_next(const uint8_t *smem, uint8_t *sA1, uin
 // kFused: model-native inputs -- the w, a and b tiles hold x_w, x_a and nothing; w = decay(x_w),
 // a = -kk and b = kk * sigmoid(x_a) with kk = k * k_k / |k * k_k| are formed where the operands are
 // built (the decay-scan / [B^; K^] preparation and P1), and only five tiles are loaded per chunk.
-template <bool kFused>
+// kLN: the x070 ln_x epilogue (GroupNorm over each token-head's 64 channels, eps 64e-5) is applied
+// to y before it is stored.
+template <bool kFused, bool kLN>
 __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_constant__ Maps maps, const Args A) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -504,6 +511,8 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
   float *pre4 = reinterpret_cast<float *>(smem + OFF_PRE);
   float *kkw = reinterpret_cast<float *>(smem + OFF_KX);        // [64] key scale of this head
   float *invn = reinterpret_cast<float *>(smem + OFF_KX + 256);  // [64] 1 / |k * k_k| per token of a chunk
+  float *lnw = reinterpret_cast<float *>(smem + OFF_LN);         // [2][64] ln_w, ln_b of this head
+  float2 *lnst = reinterpret_cast<float2 *>(smem + OFF_LN + 512);  // [2][64] (mean, M2) of each half-row of y
   float *wtot = reinterpret_cast<float *>(smem + OFF_MISC + MISC_WTOT);
 
   const int tid = threadIdx.x;
@@ -700,6 +709,29 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
         float v[32];
         tc::tmem_ld32(tmem + lane_base + TM_D4 + 32 * hh, v);
         if (!hi_lanes) {
+          if (kLN) {
+            // ln_x: each half-row's mean and squared deviation, exchanged between the two warps of a
+            // token row, combined with Chan's pairwise formula (M2 = M2a + M2b + 32 (ma - mb)^2 / 2)
+            float mh = 0.f;
+#pragma unroll
+            for (int x = 0; x < 32; ++x) mh += v[x];
+            mh *= (1.f / 32.f);
+            float m2 = 0.f;
+#pragma unroll
+            for (int x = 0; x < 32; ++x) m2 = fmaf(v[x] - mh, v[x] - mh, m2);
+            lnst[hh * 64 + tl] = make_float2(mh, m2);
+            lo_lane_sync();
+            const float2 o = lnst[(hh ^ 1) * 64 + tl];
+            const float dm = mh - o.x;
+            const float mean = 0.5f * (mh + o.x);
+            const float var = (m2 + o.y + 16.f * dm * dm) * (1.f / 64.f);
+            const float rs = rsqrtf(var + kLnEps);
+#pragma unroll
+            for (int x = 0; x < 32; ++x) {
+              const int cidx2 = 32 * hh + x;  // value channel of logical position x (D4 column vrow(x))
+              v[vrow(x)] = fmaf((v[vrow(x)] - mean) * rs, lnw[cidx2], lnw[64 + cidx2]);
+            }
+          }
           if (tl < Lcx) {
             const long long tok = sb.start + static_cast<long long>(cidx) * C + tl;
             uint16_t *dst = A.y + (tok * A.H + h) * kN + 32 * hh;
@@ -727,6 +759,10 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
 
     // the key scale of this head (model-native inputs), then the first chunk's decay scan, [B^; K^] and V^T
     if (kFused && tid >= 128 && tid < 192) kkw[tid - 128] = A.k_k ? A.k_k[h * kN + (tid - 128)] : 1.f;
+    if (kLN && tid >= 128) {
+      const int e = tid - 128;  // 0..127: ln_w then ln_b
+      lnw[e] = e < 64 ? (A.ln_w ? A.ln_w[h * kN + e] : 1.f) : (A.ln_b ? A.ln_b[h * kN + e - 64] : 0.f);
+    }
     if (nchunks > 0 && warp >= 4 && wait_group_hi(bar_tma, 0))
       prep_next<kFused>(smem, sA1, sB1, sB4V, pre4, GCs, wtot, kkw, invn, tid - 128, min(C, sb.len));
     compute_sync();
@@ -994,49 +1030,48 @@ static bool make_map(CUtensorMap *map, const void *base, long long tokens, int H
 
 }  // namespace chunk
 
-cudaError_t launch_chunk(const uint16_t *r, const uint16_t *w, const uint16_t *k, const uint16_t *v,
-                         const uint16_t *a, const uint16_t *b, const float *s_in, uint16_t *y, float *s_out,
-                         const int32_t *cu_seqlens, int B, int T, long long total_T, int H, int *err_word,
-                         cudaStream_t stream) {
+namespace chunk {
+
+template <bool kFused, bool kLN>
+static cudaError_t launch_variant(const Maps &maps, const Args &args, int B, int H, cudaStream_t stream) {
+  cudaError_t e = cudaFuncSetAttribute(wkv7_chunk_kernel<kFused, kLN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kSmemBytes));
+  if (e != cudaSuccess) return e;
+  dim3 grid(H, B);
+  wkv7_chunk_kernel<kFused, kLN><<<grid, kThreads, kSmemBytes, stream>>>(maps, args);
+  return cudaGetLastError();
+}
+
+}  // namespace chunk
+
+cudaError_t launch_chunk_ext(const uint16_t *r, const uint16_t *w, const uint16_t *k, const uint16_t *v,
+                             const uint16_t *a, const uint16_t *b, bool model_native, const float *k_k,
+                             bool group_norm, const float *ln_w, const float *ln_b, const float *s_in, uint16_t *y,
+                             float *s_out, const int32_t *cu_seqlens, int B, int T, long long total_T, int H,
+                             int *err_word, cudaStream_t stream) {
   using namespace chunk;
   if (total_T > 0x7fffffffLL || H > 0xffff || B > 65535) return cudaErrorInvalidValue;
   Maps maps;
-  const void *ops[6] = {r, w, k, a, b, v};
+  const void *ops[6] = {r, w, k, a, model_native ? nullptr : b, v};  // model-native: the b slot is never loaded
   const long long tokens = total_T > 0 ? total_T : 1;
   for (int i = 0; i < 6; ++i) {
     // a zero-token call still needs a valid map; it never issues a load
     if (!make_map(&maps.m[i], ops[i] ? ops[i] : static_cast<const void *>(s_out), tokens, H))
       return cudaErrorInvalidValue;
   }
-  Args args{y, s_in, s_out, cu_seqlens, T, total_T, H, err_word, nullptr};
-  cudaError_t e = cudaFuncSetAttribute(wkv7_chunk_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(kSmemBytes));
-  if (e != cudaSuccess) return e;
-  dim3 grid(H, B);
-  wkv7_chunk_kernel<false><<<grid, kThreads, kSmemBytes, stream>>>(maps, args);
-  return cudaGetLastError();
+  Args args{y, s_in, s_out, cu_seqlens, T, total_T, H, err_word, k_k, ln_w, ln_b};
+  if (model_native && group_norm) return launch_variant<true, true>(maps, args, B, H, stream);
+  if (model_native) return launch_variant<true, false>(maps, args, B, H, stream);
+  if (group_norm) return launch_variant<false, true>(maps, args, B, H, stream);
+  return launch_variant<false, false>(maps, args, B, H, stream);
 }
 
-cudaError_t launch_chunk_fused(const uint16_t *r, const uint16_t *xw, const uint16_t *k, const uint16_t *v,
-                               const uint16_t *xa, const float *k_k, const float *s_in, uint16_t *y, float *s_out,
-                               const int32_t *cu_seqlens, int B, int T, long long total_T, int H, int *err_word,
-                               cudaStream_t stream) {
-  using namespace chunk;
-  if (total_T > 0x7fffffffLL || H > 0xffff || B > 65535) return cudaErrorInvalidValue;
-  Maps maps;
-  const void *ops[6] = {r, xw, k, xa, nullptr, v};  // the b slot is never loaded
-  const long long tokens = total_T > 0 ? total_T : 1;
-  for (int i = 0; i < 6; ++i) {
-    if (!make_map(&maps.m[i], ops[i] ? ops[i] : static_cast<const void *>(s_out), tokens, H))
-      return cudaErrorInvalidValue;
-  }
-  Args args{y, s_in, s_out, cu_seqlens, T, total_T, H, err_word, k_k};
-  cudaError_t e = cudaFuncSetAttribute(wkv7_chunk_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(kSmemBytes));
-  if (e != cudaSuccess) return e;
-  dim3 grid(H, B);
-  wkv7_chunk_kernel<true><<<grid, kThreads, kSmemBytes, stream>>>(maps, args);
-  return cudaGetLastError();
+cudaError_t launch_chunk(const uint16_t *r, const uint16_t *w, const uint16_t *k, const uint16_t *v,
+                         const uint16_t *a, const uint16_t *b, const float *s_in, uint16_t *y, float *s_out,
+                         const int32_t *cu_seqlens, int B, int T, long long total_T, int H, int *err_word,
+                         cudaStream_t stream) {
+  return launch_chunk_ext(r, w, k, v, a, b, false, nullptr, false, nullptr, nullptr, s_in, y, s_out, cu_seqlens, B,
+                          T, total_T, H, err_word, stream);
 }
 
 }  // namespace rwkv7

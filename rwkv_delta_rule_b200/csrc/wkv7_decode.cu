@@ -26,12 +26,13 @@ template <typename TIn> struct DecodeArgs {
   TIn *y;
   const float *k_k;  // fused: [H, 64] key scale, nullptr = ones
   int H;
+  const float *ln_w, *ln_b;  // group-norm epilogue: [H, 64] weight / bias, nullptr = ones / zeros
 };
 
 __device__ __forceinline__ float4 ld_state(const float *p) { return *reinterpret_cast<const float4 *>(p); }
 __device__ __forceinline__ void st_state(float *p, float4 x) { *reinterpret_cast<float4 *>(p) = x; }
 
-template <typename TIn, bool kFused>
+template <typename TIn, bool kFused, bool kLN>
 __global__ void __launch_bounds__(256) wkv7_decode_kernel(DecodeArgs<TIn> A) {
   const long long pair = blockIdx.x;  // b * H + h
   const int tid = threadIdx.x;
@@ -132,29 +133,55 @@ __global__ void __launch_bounds__(256) wkv7_decode_kernel(DecodeArgs<TIn> A) {
   for (int off = 8; off >= 1; off >>= 1)
 #pragma unroll
     for (int m = 0; m < 4; ++m) yv[m] += __shfl_xor_sync(0xffffffffu, yv[m], off);
-  if (c4 == 0) {
+  if (!kLN) {
+    if (c4 == 0) {
 #pragma unroll
-    for (int m = 0; m < 4; ++m) Elem<TIn>::store(A.y + vb + rg + 16 * m, yv[m]);
+      for (int m = 0; m < 4; ++m) Elem<TIn>::store(A.y + vb + rg + 16 * m, yv[m]);
+    }
+  } else {
+    // ln_x: GroupNorm over the head's 64 channels of y, by warp 0 (two channels per lane)
+    __shared__ float s_y[kLN ? kN : 1];
+    if (c4 == 0) {
+#pragma unroll
+      for (int m = 0; m < 4; ++m) s_y[rg + 16 * m] = yv[m];
+    }
+    __syncthreads();
+    if (tid < 32) {
+      const float y0 = s_y[tid], y1 = s_y[tid + 32];
+      float mean, var;
+      warp_mean_var64(y0, y1, mean, var);
+      const float rs = rsqrtf(var + kLnEps);
+      const int h = static_cast<int>(pair % A.H);
+      const float w0 = A.ln_w ? A.ln_w[h * kN + tid] : 1.f, w1 = A.ln_w ? A.ln_w[h * kN + tid + 32] : 1.f;
+      const float b0 = A.ln_b ? A.ln_b[h * kN + tid] : 0.f, b1 = A.ln_b ? A.ln_b[h * kN + tid + 32] : 0.f;
+      Elem<TIn>::store(A.y + vb + tid, fmaf((y0 - mean) * rs, w0, b0));
+      Elem<TIn>::store(A.y + vb + tid + 32, fmaf((y1 - mean) * rs, w1, b1));
+    }
   }
 }
 
 template <typename TIn>
 cudaError_t launch_decode(const TIn *r, const TIn *w, const TIn *k, const TIn *v, const TIn *a, const TIn *b,
                           float *s, TIn *y, int B, int H, cudaStream_t stream) {
-  DecodeArgs<TIn> A{r, w, k, v, a, b, s, y, nullptr, H};
+  DecodeArgs<TIn> A{r, w, k, v, a, b, s, y, nullptr, H, nullptr, nullptr};
   const long long pairs = static_cast<long long>(B) * H;
   if (pairs > 0x7fffffffLL) return cudaErrorInvalidValue;
-  wkv7_decode_kernel<TIn, false><<<static_cast<unsigned>(pairs), 256, 0, stream>>>(A);
+  wkv7_decode_kernel<TIn, false, false><<<static_cast<unsigned>(pairs), 256, 0, stream>>>(A);
   return cudaGetLastError();
 }
 
-cudaError_t launch_decode_fused(const uint16_t *r, const uint16_t *xw, const uint16_t *k, const uint16_t *v,
-                                const uint16_t *xa, const float *k_k, float *s, uint16_t *y, int B, int H,
-                                cudaStream_t stream) {
-  DecodeArgs<uint16_t> A{r, xw, k, v, xa, nullptr, s, y, k_k, H};
+cudaError_t launch_decode_ext(const uint16_t *r, const uint16_t *w, const uint16_t *k, const uint16_t *v,
+                              const uint16_t *a, const uint16_t *b, bool model_native, const float *k_k,
+                              bool group_norm, const float *ln_w, const float *ln_b, float *s, uint16_t *y, int B,
+                              int H, cudaStream_t stream) {
+  DecodeArgs<uint16_t> A{r, w, k, v, a, b, s, y, k_k, H, ln_w, ln_b};
   const long long pairs = static_cast<long long>(B) * H;
   if (pairs > 0x7fffffffLL) return cudaErrorInvalidValue;
-  wkv7_decode_kernel<uint16_t, true><<<static_cast<unsigned>(pairs), 256, 0, stream>>>(A);
+  const unsigned g = static_cast<unsigned>(pairs);
+  if (model_native && group_norm) wkv7_decode_kernel<uint16_t, true, true><<<g, 256, 0, stream>>>(A);
+  else if (model_native) wkv7_decode_kernel<uint16_t, true, false><<<g, 256, 0, stream>>>(A);
+  else if (group_norm) wkv7_decode_kernel<uint16_t, false, true><<<g, 256, 0, stream>>>(A);
+  else wkv7_decode_kernel<uint16_t, false, false><<<g, 256, 0, stream>>>(A);
   return cudaGetLastError();
 }
 

@@ -21,6 +21,10 @@
 // The fused variant takes model-native inputs (x_w in place of w, x_a in place of a, no b, and the
 // per-channel key scale k_k) and forms w, a = -kk and b = kk * sigmoid(x_a) per token in registers;
 // the key norm is two more xor-shuffles inside the quad, which holds all 64 columns of a row.
+//
+// The group-norm variant (x070 ln_x on y) runs one CTA of 256 threads per (b, h) (ROWS = 64), so
+// every token's 64 channels of y meet in one tile of shared memory; one warp per token normalises
+// them on the way out.
 #include "common.cuh"
 #include "launch.h"
 
@@ -51,6 +55,7 @@ template <typename TIn> struct ScanArgs {
   long long total_T;
   int H;
   const float *k_k;  // fused: [H, 64] key scale, nullptr = ones
+  const float *ln_w, *ln_b;  // group-norm epilogue: [H, 64] weight / bias, nullptr = ones / zeros
 };
 
 template <typename TIn, int ROWS, bool kFused>
@@ -74,8 +79,9 @@ __device__ __forceinline__ void scan_load_tile(const ScanArgs<TIn> &A, TIn *buf,
   }
 }
 
-template <typename TIn, int ROWS, bool kFused>
+template <typename TIn, int ROWS, bool kFused, bool kLN>
 __global__ void __launch_bounds__(ScanCfg<TIn, ROWS>::kThreads) wkv7_scan_kernel(ScanArgs<TIn> A) {
+  static_assert(!kLN || ROWS == kN, "the group-norm epilogue needs all 64 rows in one CTA");
   using C = ScanCfg<TIn, ROWS>;
   constexpr int kSplits = kN / ROWS;
   extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -190,10 +196,26 @@ __global__ void __launch_bounds__(ScanCfg<TIn, ROWS>::kThreads) wkv7_scan_kernel
       if (q == 0) ys[tt * ROWS + rloc] = y;
     }
     __syncthreads();
-    for (int e = tid; e < ntok * ROWS; e += C::kThreads) {
-      const int tt = e / ROWS, rr_ = e - tt * ROWS;
-      const long long yi = ((sb.start + t0 + tt) * A.H + h) * kN + row0 + rr_;
-      Elem<TIn>::store(A.y + yi, ys[e]);
+    if (!kLN) {
+      for (int e = tid; e < ntok * ROWS; e += C::kThreads) {
+        const int tt = e / ROWS, rr_ = e - tt * ROWS;
+        const long long yi = ((sb.start + t0 + tt) * A.H + h) * kN + row0 + rr_;
+        Elem<TIn>::store(A.y + yi, ys[e]);
+      }
+    } else {
+      // ln_x: one warp per token, channels lane and lane + 32
+      const int lane = tid & 31;
+      const float w0 = A.ln_w ? A.ln_w[h * kN + lane] : 1.f, w1 = A.ln_w ? A.ln_w[h * kN + lane + 32] : 1.f;
+      const float b0 = A.ln_b ? A.ln_b[h * kN + lane] : 0.f, b1 = A.ln_b ? A.ln_b[h * kN + lane + 32] : 0.f;
+      for (int tt = tid >> 5; tt < ntok; tt += C::kThreads / 32) {
+        const float y0 = ys[tt * ROWS + lane], y1 = ys[tt * ROWS + lane + 32];
+        float mean, var;
+        warp_mean_var64(y0, y1, mean, var);
+        const float rs = rsqrtf(var + kLnEps);
+        const long long yi = ((sb.start + t0 + tt) * A.H + h) * kN;
+        Elem<TIn>::store(A.y + yi + lane, fmaf((y0 - mean) * rs, w0, b0));
+        Elem<TIn>::store(A.y + yi + lane + 32, fmaf((y1 - mean) * rs, w1, b1));
+      }
     }
     // the next iteration's first __syncthreads orders these reads of ys
     // before the next tile's writes to it
@@ -205,10 +227,10 @@ __global__ void __launch_bounds__(ScanCfg<TIn, ROWS>::kThreads) wkv7_scan_kernel
         make_float4(s[4 * m + 0], s[4 * m + 1], s[4 * m + 2], s[4 * m + 3]);
 }
 
-template <typename TIn, int ROWS, bool kFused = false>
+template <typename TIn, int ROWS, bool kFused = false, bool kLN = false>
 static cudaError_t launch_scan_rows(const ScanArgs<TIn> &A, int B, cudaStream_t stream) {
   using C = ScanCfg<TIn, ROWS>;
-  auto kern = wkv7_scan_kernel<TIn, ROWS, kFused>;
+  auto kern = wkv7_scan_kernel<TIn, ROWS, kFused, kLN>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(C::kSmemBytes));
   if (e != cudaSuccess) return e;
@@ -221,16 +243,20 @@ template <typename TIn>
 cudaError_t launch_scan(const TIn *r, const TIn *w, const TIn *k, const TIn *v, const TIn *a, const TIn *b,
                         const float *s_in, TIn *y, float *s_out, const int32_t *cu_seqlens, int B, int T,
                         long long total_T, int H, cudaStream_t stream) {
-  ScanArgs<TIn> A{r, w, k, v, a, b, s_in, y, s_out, cu_seqlens, T, total_T, H, nullptr};
+  ScanArgs<TIn> A{r, w, k, v, a, b, s_in, y, s_out, cu_seqlens, T, total_T, H, nullptr, nullptr, nullptr};
   return launch_scan_rows<TIn, 16>(A, B, stream);
 }
 
-cudaError_t launch_scan_fused(const uint16_t *r, const uint16_t *xw, const uint16_t *k, const uint16_t *v,
-                              const uint16_t *xa, const float *k_k, const float *s_in, uint16_t *y, float *s_out,
-                              const int32_t *cu_seqlens, int B, int T, long long total_T, int H,
-                              cudaStream_t stream) {
-  ScanArgs<uint16_t> A{r, xw, k, v, xa, nullptr, s_in, y, s_out, cu_seqlens, T, total_T, H, k_k};
-  return launch_scan_rows<uint16_t, 16, true>(A, B, stream);
+cudaError_t launch_scan_ext(const uint16_t *r, const uint16_t *w, const uint16_t *k, const uint16_t *v,
+                            const uint16_t *a, const uint16_t *b, bool model_native, const float *k_k,
+                            bool group_norm, const float *ln_w, const float *ln_b, const float *s_in, uint16_t *y,
+                            float *s_out, const int32_t *cu_seqlens, int B, int T, long long total_T, int H,
+                            cudaStream_t stream) {
+  ScanArgs<uint16_t> A{r, w, k, v, a, b, s_in, y, s_out, cu_seqlens, T, total_T, H, k_k, ln_w, ln_b};
+  if (model_native && group_norm) return launch_scan_rows<uint16_t, 64, true, true>(A, B, stream);
+  if (model_native) return launch_scan_rows<uint16_t, 16, true, false>(A, B, stream);
+  if (group_norm) return launch_scan_rows<uint16_t, 64, false, true>(A, B, stream);
+  return launch_scan_rows<uint16_t, 16, false, false>(A, B, stream);
 }
 
 template cudaError_t launch_scan<float>(const float *, const float *, const float *, const float *, const float *,

@@ -147,6 +147,16 @@ def draw_model_native(B: int, T: int, H: int, N: int = N_HEAD, *, seed: int, z_m
     return out
 
 
+def draw_group_norm(H: int, N: int = N_HEAD, *, seed: int) -> Dict[str, torch.Tensor]:
+    """Draw the per-head GroupNorm affine parameters: ``ln_w`` float32 ``[H, N]`` ~ U(0.5, 1.5) and
+    ``ln_b`` float32 ``[H, N]`` ~ N(0, 0.1^2)."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    ln_w = torch.rand((H, N), generator=g, dtype=torch.float32) + 0.5
+    ln_b = torch.randn((H, N), generator=g, dtype=torch.float32) * 0.1
+    return {"ln_w": ln_w.contiguous(), "ln_b": ln_b.contiguous()}
+
+
 def draw_case(case: Case, *, T: Optional[int] = None, B: Optional[int] = None) -> Dict[str, torch.Tensor]:
     """Draw a named workload, optionally at a reduced B or T (same recipe, same seed)."""
     return draw(case.B if B is None else B, case.T if T is None else T, case.H, case.N,

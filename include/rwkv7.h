@@ -170,13 +170,24 @@ RWKV7_API rwkv7_status rwkv7_wkv_decode_fused_bf16(int B, int H, int N, const ui
  *                     y = (y - mean) / sqrt(var + 64e-5) * ln_w + ln_b over each token-head's 64
  *                     channels (variance with divisor 64).  ln_w / ln_b: float32 [H,64] device
  *                     buffers, 16-byte aligned, NULL meaning ones / zeros.
- * The state is not affected by group_norm. */
+ * The state is not affected by group_norm.
+ *   chunk_schedule:   how the CHUNK path spreads its work (prefill only; results are the same up
+ *                     to float32 rounding order):
+ *                     0 = chosen from the shape;
+ *                     1 = one CTA per (b, h), walking its chunks with the state on chip;
+ *                     2 = every chunk of every (b, h) is a task, spread over all SMs; each chunk
+ *                         takes its start state from s_out, where the previous chunk of the same
+ *                         (b, h) left it (flags in library-owned device memory order the two).
+ *                         Needs B*H <= 65536 (else RWKV7_ERR_CUDA).  Up to 4 such launches may
+ *                         run at once on a device.
+ */
 typedef struct rwkv7_options {
   int model_native;
   const float *k_k;
   int group_norm;
   const float *ln_w;
   const float *ln_b;
+  int chunk_schedule;
 } rwkv7_options;
 
 /* bf16 prefill with options (NULL = none); other arguments as for rwkv7_wkv_prefill_bf16_path. */

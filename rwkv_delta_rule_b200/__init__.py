@@ -22,7 +22,8 @@ from typing import Optional
 import torch
 
 __all__ = [
-    "RWKV7_PATH_AUTO", "RWKV7_PATH_SCAN", "RWKV7_PATH_CHUNK", "Rwkv7Error", "library_path", "load_library",
+    "RWKV7_PATH_AUTO", "RWKV7_PATH_SCAN", "RWKV7_PATH_CHUNK", "RWKV7_SCHED_AUTO", "RWKV7_SCHED_PAIR",
+    "RWKV7_SCHED_TASKS", "Rwkv7Error", "library_path", "load_library",
     "rwkv7_wkv_prefill", "rwkv7_wkv_prefill_bf16", "rwkv7_wkv_prefill_bf16_path", "rwkv7_wkv_prefill_varlen_bf16",
     "rwkv7_wkv_decode", "rwkv7_wkv_decode_bf16", "rwkv7_wkv_prefill_fused_bf16", "rwkv7_wkv_decode_fused_bf16",
     "rwkv7_wkv_prefill_ext_bf16", "rwkv7_wkv_decode_ext_bf16", "Options",
@@ -32,6 +33,8 @@ __all__ = [
 ]
 
 RWKV7_PATH_AUTO, RWKV7_PATH_SCAN, RWKV7_PATH_CHUNK = 0, 1, 2
+# chunk-path schedules (rwkv7_options.chunk_schedule)
+RWKV7_SCHED_AUTO, RWKV7_SCHED_PAIR, RWKV7_SCHED_TASKS = 0, 1, 2
 N_HEAD = 64
 
 EXPORTED_SYMBOLS = (
@@ -49,7 +52,7 @@ class Options(ctypes.Structure):
     """``rwkv7_options`` of include/rwkv7.h (host struct; the pointers are device addresses)."""
 
     _fields_ = [("model_native", ctypes.c_int), ("k_k", ctypes.c_void_p), ("group_norm", ctypes.c_int),
-                ("ln_w", ctypes.c_void_p), ("ln_b", ctypes.c_void_p)]
+                ("ln_w", ctypes.c_void_p), ("ln_b", ctypes.c_void_p), ("chunk_schedule", ctypes.c_int)]
 
 
 class Rwkv7Error(RuntimeError):
@@ -219,27 +222,28 @@ def rwkv7_wkv_decode_fused_bf16(r, xw, k, v, xa, k_k, s_inout, y, stream=None) -
           _stream(stream))
 
 
-def _options(model_native: bool, k_k, group_norm: bool, ln_w, ln_b, H: int, N: int) -> Options:
+def _options(model_native: bool, k_k, group_norm: bool, ln_w, ln_b, H: int, N: int, schedule: int = 0) -> Options:
     if model_native:
         _check(k_k, "k_k", torch.float32, (H, N), allow_none=True)
     if group_norm:
         _check(ln_w, "ln_w", torch.float32, (H, N), allow_none=True)
         _check(ln_b, "ln_b", torch.float32, (H, N), allow_none=True)
     return Options(int(bool(model_native)), _ptr(k_k) if model_native else None, int(bool(group_norm)),
-                   _ptr(ln_w) if group_norm else None, _ptr(ln_b) if group_norm else None)
+                   _ptr(ln_w) if group_norm else None, _ptr(ln_b) if group_norm else None, int(schedule))
 
 
 def rwkv7_wkv_prefill_ext_bf16(path, r, w, k, v, a, b, s_in, y, s_out, *, model_native=False, k_k=None,
-                               group_norm=False, ln_w=None, ln_b=None, stream=None) -> None:
-    """bf16 prefill with options: model-native inputs (``w``, ``a`` hold x_w, x_a; ``b`` None) and / or the
-    ln_x GroupNorm epilogue on ``y`` (``ln_w`` / ``ln_b`` ``[H,64]`` float32 or None)."""
+                               group_norm=False, ln_w=None, ln_b=None, schedule=0, stream=None) -> None:
+    """bf16 prefill with options: model-native inputs (``w``, ``a`` hold x_w, x_a; ``b`` None), the
+    ln_x GroupNorm epilogue on ``y`` (``ln_w`` / ``ln_b`` ``[H,64]`` float32 or None), and the chunk
+    path's schedule (``RWKV7_SCHED_*``)."""
     B, T, H, N = r.shape
     names = (("r", r), ("w", w), ("k", k), ("v", v), ("a", a), ("y", y)) + (() if model_native else (("b", b),))
     for nm, t in names:
         _check(t, nm, torch.bfloat16, (B, T, H, N))
     _check(s_in, "s_in", torch.float32, (B, H, N, N), allow_none=True)
     _check(s_out, "s_out", torch.float32, (B, H, N, N))
-    opt = _options(model_native, k_k, group_norm, ln_w, ln_b, H, N)
+    opt = _options(model_native, k_k, group_norm, ln_w, ln_b, H, N, schedule)
     _call("rwkv7_wkv_prefill_ext_bf16", int(path), B, T, H, N,
           *[_ptr(t) for t in (r, w, k, v, a, None if model_native else b)], ctypes.byref(opt),
           _ptr(s_in), _ptr(y), _ptr(s_out), _stream(stream))
@@ -315,13 +319,13 @@ def decode_model_native_(r, xw, k, v, xa, k_k, state, y=None, *, stream=None):
 
 
 def prefill_ext(r, w, k, v, a, b=None, s_in=None, *, path: int = RWKV7_PATH_AUTO, model_native=False, k_k=None,
-                group_norm=False, ln_w=None, ln_b=None, stream=None):
+                group_norm=False, ln_w=None, ln_b=None, schedule=0, stream=None):
     """Allocate ``y`` and ``s_out`` and run the prefill with options; returns ``(y, s_out)``."""
     B, T, H, N = r.shape
     y = torch.empty_like(r)
     s_out = torch.empty((B, H, N, N), dtype=torch.float32, device=r.device)
     rwkv7_wkv_prefill_ext_bf16(path, r, w, k, v, a, b, s_in, y, s_out, model_native=model_native, k_k=k_k,
-                               group_norm=group_norm, ln_w=ln_w, ln_b=ln_b, stream=stream)
+                               group_norm=group_norm, ln_w=ln_w, ln_b=ln_b, schedule=schedule, stream=stream)
     return y, s_out
 
 

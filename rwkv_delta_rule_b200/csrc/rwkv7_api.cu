@@ -162,6 +162,8 @@ rwkv7_status rwkv7_wkv_prefill_ext_bf16(int path, int B, int T, int H, int N, co
   const bool ln = opt != nullptr && opt->group_norm != 0;
   const float *k_k = native ? opt->k_k : nullptr;
   const float *ln_w = ln ? opt->ln_w : nullptr, *ln_b = ln ? opt->ln_b : nullptr;
+  const int schedule = opt != nullptr ? opt->chunk_schedule : 0;
+  if (schedule < 0 || schedule > 2) return RWKV7_ERR_INVALID;
   // model-native calls have no b: the shared checks see a in its place
   const rwkv7_status st = check_prefill(B, T, H, N, r, w, k, v, a, native ? a : b, s_in, y, s_out);
   if (st != RWKV7_OK) return st;
@@ -170,7 +172,7 @@ rwkv7_status rwkv7_wkv_prefill_ext_bf16(int path, int B, int T, int H, int N, co
   const long long total = static_cast<long long>(B) * T;
   if (use_chunk(path, T))
     return from_cuda(launch_chunk_ext(r, w, k, v, a, b, native, k_k, ln, ln_w, ln_b, s_in, y, s_out, nullptr, B, T,
-                                      total, H, error_word_ptr(), cs));
+                                      total, H, schedule, error_word_ptr(), cs));
   return from_cuda(
       launch_scan_ext(r, w, k, v, a, b, native, k_k, ln, ln_w, ln_b, s_in, y, s_out, nullptr, B, T, total, H, cs));
 }
@@ -195,14 +197,14 @@ rwkv7_status rwkv7_wkv_prefill_fused_bf16(int path, int B, int T, int H, int N, 
                                           const uint16_t *xw, const uint16_t *k, const uint16_t *v,
                                           const uint16_t *xa, const float *k_k, const float *s_in, uint16_t *y,
                                           float *s_out, rwkv7_stream_t stream) {
-  const rwkv7_options opt{1, k_k, 0, nullptr, nullptr};
+  const rwkv7_options opt{1, k_k, 0, nullptr, nullptr, 0};
   return rwkv7_wkv_prefill_ext_bf16(path, B, T, H, N, r, xw, k, v, xa, nullptr, &opt, s_in, y, s_out, stream);
 }
 
 rwkv7_status rwkv7_wkv_decode_fused_bf16(int B, int H, int N, const uint16_t *r, const uint16_t *xw,
                                          const uint16_t *k, const uint16_t *v, const uint16_t *xa, const float *k_k,
                                          float *s_inout, uint16_t *y, rwkv7_stream_t stream) {
-  const rwkv7_options opt{1, k_k, 0, nullptr, nullptr};
+  const rwkv7_options opt{1, k_k, 0, nullptr, nullptr, 0};
   return rwkv7_wkv_decode_ext_bf16(B, H, N, r, xw, k, v, xa, nullptr, &opt, s_inout, y, stream);
 }
 

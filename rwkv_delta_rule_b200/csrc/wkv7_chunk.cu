@@ -36,6 +36,9 @@
 // model's decay exp(-e^-0.5 sigmoid(x)) is always >= 0.5452.
 #include <cuda.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "common.cuh"
 #include "launch.h"
 #include "tc_ptx.cuh"
@@ -80,8 +83,8 @@ constexpr uint32_t OFF_PRE = OFF_TS + 6 * 16 * LDTB * 4;  // float [16][64]: Gam
 constexpr uint32_t MISC_GC = 256;                         // float [2][64] Gamma at the chunk end, by chunk parity
 constexpr uint32_t MISC_WTOT = 768;                       // float [4][64] decay products of 16-token blocks
 constexpr uint32_t OFF_KX = OFF_PRE + 16 * 64 * 4;  // model-native inputs: float [64] k_k, float [64] 1/|k k_k|
-constexpr uint32_t OFF_LN = OFF_KX + 2 * 64 * 4;     // group norm: float [2][64] ln_w, ln_b; float2 [2][64] stats
-constexpr uint32_t kSmemBytes = OFF_LN + 2 * 64 * 4 + 2 * 64 * 8 + 1024;
+constexpr uint32_t OFF_LN = OFF_KX + 2 * 64 * 4;     // group norm: float [2][128] ln_w, ln_b by task parity
+constexpr uint32_t kSmemBytes = OFF_LN + 2 * 128 * 4 + 1024;
 
 static_assert(MISC_WTOT + 4 * 64 * 4 <= 2048, "misc region overflow");
 static_assert(OFF_ZS + 6 * 16 * LDZ * 4 <= OFF_B2 + 16384, "inverse scratch overflows B2");
@@ -108,6 +111,9 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, vo
 
 struct Maps {
   CUtensorMap m[6];  // r, w, k, a, b, v: dims {64, H, tokens}, box {64, 1, 64}, 128-byte swizzle
+  // task-parallel schedule: the state a chunk starts from, float32 rows of 64 (box {32, 64},
+  // 128-byte swizzle): s_in (or a zero block), and s_out, where every chunk leaves its end state
+  CUtensorMap s_in, s_out;
 };
 
 struct Args {
@@ -121,7 +127,87 @@ struct Args {
   int *err;
   const float *k_k;  // model-native inputs: [H, 64] key scale, nullptr = ones
   const float *ln_w, *ln_b;  // group-norm epilogue: [H, 64] weight / bias, nullptr = ones / zeros
+  // task-parallel schedule: task n = chunk n / BH of pair n % BH; CTA x of G takes x, x + G, ...
+  long long ntasks, BH;
+  unsigned long long *flags;  // [BH]: (epoch << 32) | chunks of the pair whose end state is in s_out
+  unsigned epoch;             // unique per launch: flags of other launches never match
+  int s_in_zero;              // the s_in map covers one zero block (row 0 for every pair)
 };
+
+// One unit of work: chunk c of the (b, h) pair bh.
+struct Task {
+  long long n;     // chunk index (one pair per CTA) or task index (task-parallel)
+  long long bh;    // b * H + h
+  long long tok0;  // token row of the chunk's first token in the [tokens, H, 64] operands
+  int c, h, Lc;    // chunk of the sequence, head, tokens in the chunk (1..64)
+};
+
+// Fills t with chunk c of pair bh (task index n); false for a chunk past the end of its sequence.
+// kTask: bh < 65536, so b = bh / H is a 32-bit division; else the pair is (blockIdx.y, blockIdx.x).
+template <bool kTask>
+__device__ __forceinline__ bool task_set(const Args &A, long long n, int c, long long bh, Task &t) {
+  int b, h;
+  if (kTask) {
+    b = static_cast<int>(static_cast<unsigned>(bh) / static_cast<unsigned>(A.H));
+    h = static_cast<int>(bh) - b * A.H;
+  } else {
+    b = blockIdx.y;
+    h = blockIdx.x;
+  }
+  const SeqBounds sb = seq_bounds(A.cu_seqlens, b, A.T, A.total_T);
+  if (sb.len <= 0 || static_cast<long long>(c) * C >= sb.len) return false;
+  t.n = n;
+  t.bh = bh;
+  t.c = c;
+  t.h = h;
+  t.tok0 = sb.start + static_cast<long long>(c) * C;
+  t.Lc = min(C, sb.len - c * C);
+  return true;
+}
+// One pair per CTA: its chunks in order.
+__device__ __forceinline__ bool pair_first(const Args &A, Task &t) {
+  return task_set<false>(A, 0, 0, static_cast<long long>(blockIdx.y) * A.H + blockIdx.x, t);
+}
+// Advances t to the pair's next chunk; false (t unchanged) past the last one.
+__device__ __forceinline__ bool pair_next(const Args &A, Task &t) { return task_set<false>(A, t.n + 1, t.c + 1, t.bh, t); }
+
+// Task-parallel schedule: CTA x of G takes the tasks x, x + G, x + 2G, ... in order (a static
+// assignment: measured faster here than claiming tasks from a global counter, which lets a pair's next
+// chunk start before its predecessor can finish).  *next is the CTA's next candidate index; empty
+// tasks (chunks past a ragged sequence's end) are skipped.  False when none is left.
+__device__ __forceinline__ bool claim_task(const Args &A, long long *next, Task &t) {
+  for (long long n = *next; n < A.ntasks; n += gridDim.x) {
+    const int c = static_cast<int>(n / A.BH);
+    if (task_set<true>(A, n, c, n - static_cast<long long>(c) * A.BH, t)) {
+      *next = n + gridDim.x;
+      return true;
+    }
+  }
+  *next = A.ntasks;
+  return false;
+}
+
+// Whether (chain_ready: one look; wait_chain: bounded wait) the end state of chunk c - 1 of pair bh
+// is in s_out: the flag word carries this launch's epoch and a count of at least c.  Acquire at GPU
+// scope, then an async-proxy fence, so the TMA load that follows sees the state another CTA stored.
+__device__ __forceinline__ bool chain_ready(const unsigned long long *flag, unsigned epoch, int c) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];\n" : "=l"(v) : "l"(flag) : "memory");
+  if (static_cast<unsigned>(v >> 32) == epoch && static_cast<unsigned>(v) >= static_cast<unsigned>(c)) {
+    tc::fence_proxy_async_global();
+    return true;
+  }
+  return false;
+}
+__device__ __forceinline__ bool wait_chain(const unsigned long long *flag, unsigned epoch, int c,
+                                           volatile int *abort_flag) {
+  for (uint32_t i = 0; i < kMaxPolls; ++i) {
+    if (chain_ready(flag, epoch, c)) return true;
+    if ((i & 63u) == 63u && *abort_flag) return false;
+    __nanosleep(64);
+  }
+  return false;
+}
 
 enum { RAW_R = 0, RAW_W = 1, RAW_K = 2, RAW_A = 3, RAW_B = 4, RAW_V = 5 };
 
@@ -139,6 +225,12 @@ __device__ __forceinline__ uint32_t mnmaj_bf16(uint32_t krows, uint32_t k, uint3
 // channels 4l + e (l = 0..7) of V, then write 8 rows with distinct (row % 8), i.e. 8 distinct bank
 // groups of the 128-byte swizzle.  Only the order of D4's columns changes; the read-out undoes it.
 __host__ __device__ constexpr int vrow(int i) { return (i & 32) | ((i & 3) << 3) | ((i >> 2) & 7); }
+// The row order in use: vrow when the state lives in TMEM (one pair per CTA); the natural order in the
+// task-parallel schedule, where the state arrives by TMA as rows of s_out.
+template <bool kTask>
+__host__ __device__ constexpr int vr(int i) {
+  return kTask ? i : vrow(i);
+}
 
 // One column k = j of 32 consecutive rows row0 .. row0+31 (row0 a multiple of
 // 8) of a K-major 32-bit operand whose K-atoms hold `rows` rows: row row0 + x
@@ -337,7 +429,7 @@ __device__ __forceinline__ void invert_unit_lower(const float *Ls, float *Ts, fl
 // operand.  Each thread covers 4 channels x 8 tokens; tokens at or past Lcn act as w = 1, b = k =
 // v = 0.  Gamma_t is formed as pre4[g] times the running product inside the group, exactly as the
 // operand construction of R~ and A~ forms it.  Warps 4-7 synchronise among themselves.
-template <bool kFused>
+template <bool kFused, bool kTask>
 __device__ __forceinline__ void prep_next(const uint8_t *smem, uint8_t *sA1, uint8_t *sB1, uint8_t *sB4Vn, float *pre4,
                                           float *GCn, float *wtot, const float *kkw, float *invn, int tid4, int Lcn) {
   const int lane = tid4 & 31, wq = tid4 >> 5;
@@ -453,7 +545,7 @@ __device__ __forceinline__ void prep_next(const uint8_t *smem, uint8_t *sA1, uin
     st_tf32x4(b1r + tc::sw128(t, chunk), bb[0] * ig[0], bb[1] * ig[1], bb[2] * ig[2], bb[3] * ig[3]);
     st_tf32x4(b1r + tc::sw128(64 + t, chunk), kk[0] * ig[0], kk[1] * ig[1], kk[2] * ig[2], kk[3] * ig[3]);
   }
-  // V^T (row = vrow(value channel), K = token); bf16 values are exact in tf32
+  // V^T (row = vr(value channel), K = token); bf16 values are exact in tf32
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     float vv[4][4];
@@ -468,7 +560,7 @@ __device__ __forceinline__ void prep_next(const uint8_t *smem, uint8_t *sA1, uin
     }
 #pragma unroll
     for (int e = 0; e < 4; ++e)
-      *reinterpret_cast<uint4 *>(sB4Vn + kmaj_tf32(64, vrow(j0 + e), tb + 4 * h)) =
+      *reinterpret_cast<uint4 *>(sB4Vn + kmaj_tf32(64, vr<kTask>(j0 + e), tb + 4 * h)) =
           make_uint4(__float_as_uint(vv[0][e]), __float_as_uint(vv[1][e]), __float_as_uint(vv[2][e]),
                      __float_as_uint(vv[3][e]));
   }
@@ -480,7 +572,13 @@ __device__ __forceinline__ void prep_next(const uint8_t *smem, uint8_t *sA1, uin
 // built (the decay-scan / [B^; K^] preparation and P1), and only five tiles are loaded per chunk.
 // kLN: the x070 ln_x epilogue (GroupNorm over each token-head's 64 channels, eps 64e-5) is applied
 // to y before it is stored.
-template <bool kFused, bool kLN>
+// kTask: the task-parallel schedule.  Chunk c of pair bh is task c * BH + bh; CTA x (of G, all
+// resident) takes tasks x, x + G, ...  The work of a chunk that does not involve its start state
+// (everything up to MMA2) runs while other CTAs finish earlier chunks of the same pair; before MMA4
+// the control lane waits for the pair's flag, then loads the start state from s_out (s_in for chunk
+// 0) by TMA.  The read-out stores the end state to s_out and publishes it with a release store of
+// the flag.  Without kTask one CTA owns a pair and keeps its state in TMEM across the chunks.
+template <bool kFused, bool kLN, bool kTask>
 __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_constant__ Maps maps, const Args A) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -503,32 +601,34 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
   uint64_t *bar_m3 = bars + 4;     // c -> w: MMA3 done
   uint64_t *bar_b2 = bars + 5;     // w -> c: B2, A2 and the D2 initial value written
   uint64_t *bar_m2 = bars + 6;     // c -> c: MMA2 done
-  uint64_t *bar_st = bars + 7;     // w -> c: state S0^T (B4S) written, D4 read out
+  uint64_t *bar_st = bars + 7;     // w -> c: D4 read out (and, one pair per CTA, the state S0^T in B4S)
   uint64_t *bar_m4 = bars + 8;     // c -> w: MMA4 done
+  uint64_t *bar_sin = bars + 9;    // task-parallel: the start state landed in B4S (tx bytes)
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_MISC + 80);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 84);
   float *GCs = reinterpret_cast<float *>(smem + OFF_MISC + MISC_GC);  // [2][64]
   float *pre4 = reinterpret_cast<float *>(smem + OFF_PRE);
-  float *kkw = reinterpret_cast<float *>(smem + OFF_KX);        // [64] key scale of this head
+  float *kkw = reinterpret_cast<float *>(smem + OFF_KX);        // [64] key scale of the head being prepared
   float *invn = reinterpret_cast<float *>(smem + OFF_KX + 256);  // [64] 1 / |k * k_k| per token of a chunk
-  float *lnw = reinterpret_cast<float *>(smem + OFF_LN);         // [2][64] ln_w, ln_b of this head
-  float2 *lnst = reinterpret_cast<float2 *>(smem + OFF_LN + 512);  // [2][64] (mean, M2) of each half-row of y
+  float *lnw = reinterpret_cast<float *>(smem + OFF_LN);         // [2][128] ln_w, ln_b of a task's head, by parity
   float *wtot = reinterpret_cast<float *>(smem + OFF_MISC + MISC_WTOT);
+  // task-parallel: the task of the next iteration, by iteration parity, written by the control lane
+  // before its bar_tma arrival for that iteration (n = -1: none)
+  Task *task_slot = reinterpret_cast<Task *>(smem + OFF_MISC + 112);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-  const int h = blockIdx.x;
-  const int bidx = blockIdx.y;
-  const SeqBounds sb = seq_bounds(A.cu_seqlens, bidx, A.T, A.total_T);
-  if (sb.len < 0) return;
-  const int nchunks = (sb.len + C - 1) / C;
-  const long long pair = static_cast<long long>(bidx) * A.H + h;
+  if (!kTask) {
+    const SeqBounds sb0 = seq_bounds(A.cu_seqlens, blockIdx.y, A.T, A.total_T);
+    if (sb0.len < 0) return;
+  }
   constexpr int kCtrlWarp = kComputeThreads / 32;
 
   if (tid == 0) {
-    for (int i = 0; i < 9; ++i) tc::mbar_init(bars + i, i == 3 ? 2 : 1);  // b3: both compute groups
+    for (int i = 0; i < 10; ++i) tc::mbar_init(bars + i, i == 3 ? 2 : 1);  // b3: both compute groups
     tc::fence_mbar_init();
     *abort_flag = 0;
+    task_slot[0].n = task_slot[1].n = -1;
   }
   if (warp == kCtrlWarp) {
     tc::tmem_alloc(tmem_slot, kTmemCols);
@@ -547,17 +647,82 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
         report_device_error(A.err, kDevErrTimeout);
       };
       for (int i = 0; i < 6; ++i) tc::prefetch_tensormap(&maps.m[i]);
+      if (kTask) {
+        tc::prefetch_tensormap(&maps.s_in);
+        tc::prefetch_tensormap(&maps.s_out);
+      }
       // parity of the last issued phase of each barrier, or -1 when nothing was issued
-      int last_tma = -1, last_m1 = -1, last_m3 = -1, last_m2 = -1, last_m4 = -1;
-      if (nchunks > 0) {
+      int last_tma = -1, last_m1 = -1, last_m3 = -1, last_m2 = -1, last_m4 = -1, last_sin = -1;
+      // Stores the end state of a finished task, which the compute warps left in B4S before arriving
+      // on bar_st (this lane's wait on it acquired their writes), to s_out by TMA; once the store has
+      // completed, raises the pair's flag (async-proxy fence, GPU-scope fence, then the flag word).
+      // B4S is free again when this returns.  Done here, where the lane idles until the window ends.
+      auto publish = [&](const Task &pt) {
+        tc::fence_proxy_async_smem();
+        const int row = static_cast<int>(pt.bh * kN);
+        tc::tma_store_2d(&maps.s_out, sB4S, 0, row);
+        tc::tma_store_2d(&maps.s_out, sB4S + 64 * 128, 32, row);
+        tc::bulk_commit_group();
+        tc::bulk_wait_all();
+        tc::fence_proxy_async_global();
+        const unsigned long long val = (static_cast<unsigned long long>(A.epoch) << 32) |
+                                       static_cast<unsigned>(pt.c + 1);
+        asm volatile("fence.acq_rel.gpu;\n\tst.relaxed.gpu.global.u64 [%0], %1;\n" ::"l"(A.flags + pt.bh), "l"(val)
+                     : "memory");
+      };
+      // The start state of task t into B4S (s_in for a first chunk, else s_out once the flag is up).
+      // Looked for without blocking after bar_st and after MMA3; waited for before MMA4.
+      bool state_issued = false;
+      auto load_state = [&](const Task &t, uint32_t ph) {
+        const CUtensorMap *sm = t.c > 0 ? &maps.s_out : &maps.s_in;
+        const int row = (t.c == 0 && A.s_in_zero) ? 0 : static_cast<int>(t.bh * kN);
+        tc::mbar_arrive_expect_tx(bar_sin, kN * kN * 4);
+        tc::tma_load_2d(sB4S, sm, bar_sin, 0, row);
+        tc::tma_load_2d(sB4S + 64 * 128, sm, bar_sin, 32, row);
+        state_issued = true;
+        last_sin = static_cast<int>(ph);
+      };
+      auto load_raw = [&](const Task &t) {
         tc::mbar_arrive_expect_tx(bar_tma, (kFused ? 5 : 6) * kTile);
         for (int i = 0; i < 6; ++i)
           if (!kFused || i != RAW_B)
-            tc::tma_load_3d(smem + OFF_RAW + i * kTile, &maps.m[i], bar_tma, 0, h, static_cast<int>(sb.start));
+            tc::tma_load_3d(smem + OFF_RAW + i * kTile, &maps.m[i], bar_tma, 0, t.h, static_cast<int>(t.tok0));
+      };
+      auto prefetch_l2 = [&](const Task &t) {
+        for (int i = 0; i < 6; ++i)
+          if (!kFused || i != RAW_B) tc::tma_prefetch_l2_3d(&maps.m[i], 0, t.h, static_cast<int>(t.tok0));
+      };
+      // the current task, the next one (its tiles load during this iteration) and, task-parallel, the
+      // one after (claimed ahead so its tiles can be warmed in L2)
+      Task t, nt, nn, pt;
+      Task none;
+      none.n = -1;
+      bool have = false, have_n = false, have_nn = false;
+      long long next_task = blockIdx.x;
+      uint32_t nit = 0;  // iterations completed
+      if constexpr (kTask) {
+        have = claim_task(A, &next_task, t);
+        if (have) have_n = claim_task(A, &next_task, nt);
+        if (have_n) have_nn = claim_task(A, &next_task, nn);
+        task_slot[0] = have ? t : none;
+        if (have) {
+          load_raw(t);
+          if (have_n) prefetch_l2(nt);
+        } else {
+          tc::mbar_arrive(bar_tma);  // releases the compute warps, who find no task
+        }
         last_tma = 0;
+      } else {
+        have = pair_first(A, t);
+        if (have) {
+          load_raw(t);
+          last_tma = 0;
+          nt = t;
+          have_n = pair_next(A, nt);
+        }
       }
-      for (int c = 0; c < nchunks; ++c) {
-        const uint32_t ph = c & 1;
+      for (uint32_t it = 0; have; ++it) {
+        const uint32_t ph = it & 1;
         // MMA1 (tf32): D1 = [R~; A~] [B^; K^]^T, once the operands are in place
         if (!wait_or_abort(bar_p1, ph, abort_flag)) { fail(); break; }
         tc::tc_fence_after();
@@ -573,22 +738,31 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
           tc::mma_commit(bar_m1);
           last_m1 = ph;
         }
-        // the next chunk's tiles (P1 has consumed the raw tiles), issued after MMA1: six TMA issues
-        // take longer than MMA1 itself
-        if (c + 1 < nchunks) {
-          tc::mbar_arrive_expect_tx(bar_tma, (kFused ? 5 : 6) * kTile);
-          for (int i = 0; i < 6; ++i)
-            if (!kFused || i != RAW_B)
-              tc::tma_load_3d(smem + OFF_RAW + i * kTile, &maps.m[i], bar_tma, 0, h,
-                              static_cast<int>(sb.start + static_cast<long long>(c + 1) * C));
-          last_tma = (c + 1) & 1;
+        // the next task's tiles (P1 has consumed the raw tiles), issued after MMA1: six TMA issues
+        // take longer than MMA1 itself; then warm L2 with the task after that
+        if constexpr (kTask) {
+          task_slot[(it + 1) & 1] = have_n ? nt : none;
+          if (have_n) {
+            load_raw(nt);
+            if (have_nn) prefetch_l2(nn);
+          } else {
+            tc::mbar_arrive(bar_tma);  // no next task: the compute warps read the empty slot
+          }
+          last_tma = (it + 1) & 1;
+        } else if (have_n) {
+          load_raw(nt);
+          last_tma = (it + 1) & 1;
+          Task n2 = nt;
+          if (pair_next(A, n2)) prefetch_l2(n2);
         }
-        // warm L2 with the chunk after that, so its TMA is an L2 hit when warps 4-7 need it early
-        if (c + 2 < nchunks)
-          for (int i = 0; i < 6; ++i)
-            if (!kFused || i != RAW_B)
-              tc::tma_prefetch_l2_3d(&maps.m[i], 0, h,
-                                     static_cast<int>(sb.start + static_cast<long long>(c + 2) * C));
+        if (kTask) {
+          // the start state, into B4S once the previous read-out is done with it
+          // the previous task's end state out of B4S, then (if already there) this task's start state in
+          if (!wait_or_abort(bar_st, ph, abort_flag)) { fail(); break; }
+          if (it > 0) publish(pt);
+          state_issued = false;
+          if (t.c == 0 || chain_ready(A.flags + t.bh, A.epoch, t.c)) load_state(t, ph);
+        }
         // MMA3 (bf16): D3 = [A~^T; Lak^T] Tinv^T
         if (!wait_or_abort(bar_b3, ph, abort_flag)) { fail(); break; }
         tc::tc_fence_after();
@@ -602,6 +776,7 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
           tc::mma_commit(bar_m3);
           last_m3 = ph;
         }
+        if (kTask && !state_issued && chain_ready(A.flags + t.bh, A.epoch, t.c)) load_state(t, ph);
         // MMA2 (bf16, A from TMEM): D2 += [Mrb; B-^T] [W~ U~]
         if (!wait_or_abort(bar_b2, ph, abort_flag)) { fail(); break; }
         tc::tc_fence_after();
@@ -614,14 +789,18 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
           tc::mma_commit(bar_m2);
           last_m2 = ph;
         }
-        // MMA4 (tf32, A from TMEM): D4 = [Q P; E F] [S0^T; V], once the state is written.  It reads
+        // MMA4 (tf32, A from TMEM): D4 = [Q P; E F] [S0^T; V], once the state is in B4S.  It reads
         // MMA2's accumulator as its A operand with no wait in between: MMAs issued by one thread
         // execute in issue order.
-        if (!wait_or_abort(bar_st, ph, abort_flag)) { fail(); break; }
+        if (kTask && !state_issued) {
+          if (!wait_chain(A.flags + t.bh, A.epoch, t.c, abort_flag)) { fail(); break; }
+          load_state(t, ph);
+        }
+        if (!wait_or_abort(kTask ? bar_sin : bar_st, ph, abort_flag)) { fail(); break; }
         tc::tc_fence_after();
         {
           constexpr uint32_t idesc = tc::instr_desc(tc::kFmtTF32, 128, 64, false, false);
-          const uint32_t bs = smem_u32(sB4S), bv = smem_u32(sB4V + (c & 1) * 16384);
+          const uint32_t bs = smem_u32(sB4S), bv = smem_u32(sB4V + ph * 16384);
 #pragma unroll
           for (int ks = 0; ks < 16; ++ks) {
             const uint32_t base = ks < 8 ? bs : bv;
@@ -633,10 +812,25 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
           tc::mma_commit(bar_m4);
           last_m4 = ph;
         }
+        pt = t;
+        nit = it + 1;
+        t = nt;
+        have = have_n;
+        if constexpr (kTask) {
+          nt = nn;
+          have_n = have_nn;
+          have_nn = have_n && claim_task(A, &next_task, nn);
+        } else if (have) {
+          nt = t;
+          have_n = pair_next(A, nt);
+        }
       }
+      // the last task's flag, once the compute warps' final read-out has stored its end state
+      if (kTask && nit > 0 && !*abort_flag && wait_or_abort(bar_st, nit & 1, abort_flag)) publish(pt);
       // every copy and MMA issued here lands before the CTA exits (bounded; phases that
       // already completed return at once)
       if (last_tma >= 0) (void)tc::mbar_wait_bounded(bar_tma, last_tma, kMaxPolls);
+      if (last_sin >= 0) (void)tc::mbar_wait_bounded(bar_sin, last_sin, kMaxPolls);
       if (last_m1 >= 0) (void)tc::mbar_wait_bounded(bar_m1, last_m1, kMaxPolls);
       if (last_m3 >= 0) (void)tc::mbar_wait_bounded(bar_m3, last_m3, kMaxPolls);
       if (last_m2 >= 0) (void)tc::mbar_wait_bounded(bar_m2, last_m2, kMaxPolls);
@@ -655,9 +849,19 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
     const int j0 = 4 * cq, t0 = 4 * tg;
     const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
 
-    // The float32 state S^T lives in TMEM (lane 64 + j, column vrow(i)); the hi-lane warps own those
-    // lanes (column half ch each) and keep its tf32 copy in B4S.
-    if (hi_lanes) {
+    if (kTask && A.cu_seqlens != nullptr) {
+      // empty sequences of a ragged batch have no task: their end state is the start state
+      for (long long bh = blockIdx.x; bh < A.BH; bh += gridDim.x) {
+        const int b = static_cast<int>(bh / A.H);
+        if (seq_bounds(A.cu_seqlens, b, A.T, A.total_T).len != 0) continue;
+        for (int e = tid; e < kN * kN; e += kComputeThreads)
+          A.s_out[bh * (kN * kN) + e] = A.s_in ? A.s_in[bh * (kN * kN) + e] : 0.f;
+      }
+    }
+    // One pair per CTA: the float32 state S^T lives in TMEM (lane 64 + j, column vrow(i)); the hi-lane
+    // warps own those lanes (column half ch each) and keep its tf32 copy in B4S.
+    if (!kTask && hi_lanes) {
+      const long long pair = static_cast<long long>(blockIdx.y) * A.H + blockIdx.x;
       float v[32];
 #pragma unroll
       for (int x = 0; x < 32; ++x)
@@ -698,80 +902,116 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
       group_sync_hi();
       return decision_hi[slot] != 0;
     };
+    // The per-head parameters of a task, loaded by warps 4-7 (tid4 = tid - 128) before its
+    // preparation: the key scale (model-native inputs) and ln_w, ln_b into buffer `par`.
+    auto load_head = [&](int hd, uint32_t par, int tid4) {
+      if (kFused && tid4 < 64) kkw[tid4] = A.k_k ? A.k_k[hd * kN + tid4] : 1.f;
+      if (kLN)
+        lnw[par * 128 + tid4] = tid4 < 64 ? (A.ln_w ? A.ln_w[hd * kN + tid4] : 1.f)
+                                          : (A.ln_b ? A.ln_b[hd * kN + tid4 - 64] : 0.f);
+    };
     bool ok = true;
     // Read-out of a finished chunk: y rows (lanes 0..63) and the state update
-    // S_C^T = diag(Gamma_C) S0^T + X (lanes 64..127), whose tf32 copy feeds the next MMA4; each warp
-    // takes the column half ch.  D4 column vrow(i) holds value channel i, like the state in TMEM.
+    // S_C^T = diag(Gamma_C) S0^T + X (lanes 64..127); each warp takes the column half ch.  D4 column
+    // vr(i) holds value channel i.  One pair per CTA: the new state goes to TMEM and, as tf32, to B4S
+    // for the next MMA4.  Task-parallel: S0 is the float32 copy in B4S and the new state replaces it
+    // there; after the next bar_st arrival the control lane stores it to s_out and raises the flag.
     float gc_done = 1.f;  // Gamma_C[j] of the chunk whose MMA4 is in flight (hi lanes)
-    auto readout = [&](int cidx, int Lcx) {
-      {
-        const int hh = ch;
-        float v[32];
-        tc::tmem_ld32(tmem + lane_base + TM_D4 + 32 * hh, v);
-        if (!hi_lanes) {
-          if (kLN) {
-            // ln_x: each half-row's mean and squared deviation, exchanged between the two warps of a
-            // token row, combined with Chan's pairwise formula (M2 = M2a + M2b + 32 (ma - mb)^2 / 2)
-            float mh = 0.f;
+    auto readout = [&](const Task &pt, uint32_t par) {
+      const int hh = ch;
+      float v[32];
+      tc::tmem_ld32(tmem + lane_base + TM_D4 + 32 * hh, v);
+      if (!hi_lanes) {
+        if (kLN) {
+          // ln_x: each half-row's mean and squared deviation, exchanged between the two warps of a
+          // token row, combined with Chan's pairwise formula (M2 = M2a + M2b + 32 (ma - mb)^2 / 2)
+          const float *lp = lnw + par * 128;
+          float2 *lnst = reinterpret_cast<float2 *>(Ls);  // the inverse's scratch is idle here
+          float mh = 0.f;
 #pragma unroll
-            for (int x = 0; x < 32; ++x) mh += v[x];
-            mh *= (1.f / 32.f);
-            float m2 = 0.f;
+          for (int x = 0; x < 32; ++x) mh += v[x];
+          mh *= (1.f / 32.f);
+          float m2 = 0.f;
 #pragma unroll
-            for (int x = 0; x < 32; ++x) m2 = fmaf(v[x] - mh, v[x] - mh, m2);
-            lnst[hh * 64 + tl] = make_float2(mh, m2);
-            lo_lane_sync();
-            const float2 o = lnst[(hh ^ 1) * 64 + tl];
-            const float dm = mh - o.x;
-            const float mean = 0.5f * (mh + o.x);
-            const float var = (m2 + o.y + 16.f * dm * dm) * (1.f / 64.f);
-            const float rs = rsqrtf(var + kLnEps);
+          for (int x = 0; x < 32; ++x) m2 = fmaf(v[x] - mh, v[x] - mh, m2);
+          lnst[hh * 64 + tl] = make_float2(mh, m2);
+          lo_lane_sync();
+          const float2 o = lnst[(hh ^ 1) * 64 + tl];
+          const float dm = mh - o.x;
+          const float mean = 0.5f * (mh + o.x);
+          const float var = (m2 + o.y + 16.f * dm * dm) * (1.f / 64.f);
+          const float rs = rsqrtf(var + kLnEps);
 #pragma unroll
-            for (int x = 0; x < 32; ++x) {
-              const int cidx2 = 32 * hh + x;  // value channel of logical position x (D4 column vrow(x))
-              v[vrow(x)] = fmaf((v[vrow(x)] - mean) * rs, lnw[cidx2], lnw[64 + cidx2]);
-            }
+          for (int x = 0; x < 32; ++x) {
+            const int cidx2 = 32 * hh + x;  // value channel of logical position x (D4 column vr(x))
+            v[vr<kTask>(x)] = fmaf((v[vr<kTask>(x)] - mean) * rs, lp[cidx2], lp[64 + cidx2]);
           }
-          if (tl < Lcx) {
-            const long long tok = sb.start + static_cast<long long>(cidx) * C + tl;
-            uint16_t *dst = A.y + (tok * A.H + h) * kN + 32 * hh;
-#pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-              uint4 w4;
-              w4.x = pack_bf16x2(v[vrow(8 * cc + 0)], v[vrow(8 * cc + 1)]);
-              w4.y = pack_bf16x2(v[vrow(8 * cc + 2)], v[vrow(8 * cc + 3)]);
-              w4.z = pack_bf16x2(v[vrow(8 * cc + 4)], v[vrow(8 * cc + 5)]);
-              w4.w = pack_bf16x2(v[vrow(8 * cc + 6)], v[vrow(8 * cc + 7)]);
-              *reinterpret_cast<uint4 *>(dst + 8 * cc) = w4;
-            }
-          }
-        } else {
-          float sv[32];
-          tc::tmem_ld32(tmem + lane_base + TM_S + 32 * hh, sv);
-#pragma unroll
-          for (int x = 0; x < 32; ++x) sv[x] = fmaf(gc_done, sv[x], v[x]);
-          tc::tmem_st32(tmem + lane_base + TM_S + 32 * hh, sv);
-          store_state_rows_tf32(sB4S, j, hh, sv);
         }
+        if (tl < pt.Lc) {
+          uint16_t *dst = A.y + ((pt.tok0 + tl) * A.H + pt.h) * kN + 32 * hh;
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
+            uint4 w4;
+            w4.x = pack_bf16x2(v[vr<kTask>(8 * cc + 0)], v[vr<kTask>(8 * cc + 1)]);
+            w4.y = pack_bf16x2(v[vr<kTask>(8 * cc + 2)], v[vr<kTask>(8 * cc + 3)]);
+            w4.z = pack_bf16x2(v[vr<kTask>(8 * cc + 4)], v[vr<kTask>(8 * cc + 5)]);
+            w4.w = pack_bf16x2(v[vr<kTask>(8 * cc + 6)], v[vr<kTask>(8 * cc + 7)]);
+            *reinterpret_cast<uint4 *>(dst + 8 * cc) = w4;
+          }
+        }
+      } else if (!kTask) {
+        float sv[32];
+        tc::tmem_ld32(tmem + lane_base + TM_S + 32 * hh, sv);
+#pragma unroll
+        for (int x = 0; x < 32; ++x) sv[x] = fmaf(gc_done, sv[x], v[x]);
+        tc::tmem_st32(tmem + lane_base + TM_S + 32 * hh, sv);
+        store_state_rows_tf32(sB4S, j, hh, sv);
+      } else {
+        // S_C[i][j] = Gamma_C[j] S0[i][j] + X[j][i], rows i = 32 hh + x, in place in B4S (float32),
+        // from where the control lane stores it to s_out by TMA
+        // (all 32 loads first: stores through these pointers would otherwise order every later load)
+        const ColPtrs cp = col_ptrs(sB4S, 64, 32 * hh, j);
+        float s0[32];
+#pragma unroll
+        for (int x = 0; x < 32; ++x) s0[x] = *reinterpret_cast<const float *>(cp.p[x & 7] + x * 128);
+#pragma unroll
+        for (int x = 0; x < 32; ++x) *reinterpret_cast<float *>(cp.p[x & 7] + x * 128) = fmaf(gc_done, s0[x], v[x]);
       }
     };
 
-
-    // the key scale of this head (model-native inputs), then the first chunk's decay scan, [B^; K^] and V^T
-    if (kFused && tid >= 128 && tid < 192) kkw[tid - 128] = A.k_k ? A.k_k[h * kN + (tid - 128)] : 1.f;
-    if (kLN && tid >= 128) {
-      const int e = tid - 128;  // 0..127: ln_w then ln_b
-      lnw[e] = e < 64 ? (A.ln_w ? A.ln_w[h * kN + e] : 1.f) : (A.ln_b ? A.ln_b[h * kN + e - 64] : 0.f);
+    // the first task's head parameters (one pair per CTA: both buffers, the head never changes), then
+    // its decay scan, [B^; K^] and V^T.  Task-parallel: the control lane names the task in its slot.
+    Task t;
+    bool have;
+    if constexpr (kTask) {
+      if (warp >= 4 && wait_group_hi(bar_tma, 0)) {
+        const Task t0 = task_slot[0];
+        if (t0.n >= 0) {
+          load_head(t0.h, 0, tid - 128);
+          group_sync_hi();
+          prep_next<kFused, kTask>(smem, sA1, sB1, sB4V, pre4, GCs, wtot, kkw, invn, tid - 128, t0.Lc);
+        }
+      }
+      compute_sync();
+      t = task_slot[0];
+      have = t.n >= 0;
+    } else {
+      have = pair_first(A, t);
+      if (warp >= 4) {
+        load_head(have ? t.h : 0, 0, tid - 128);
+        load_head(have ? t.h : 0, 1, tid - 128);
+      }
+      if (have && warp >= 4 && wait_group_hi(bar_tma, 0))
+        prep_next<kFused, kTask>(smem, sA1, sB1, sB4V, pre4, GCs, wtot, kkw, invn, tid - 128, t.Lc);
+      compute_sync();
     }
-    if (nchunks > 0 && warp >= 4 && wait_group_hi(bar_tma, 0))
-      prep_next<kFused>(smem, sA1, sB1, sB4V, pre4, GCs, wtot, kkw, invn, tid - 128, min(C, sb.len));
-    compute_sync();
 
-    int Lc_prev = 0;
+    Task pt;
     bool have_prev = false;
-    for (int c = 0; c < nchunks; ++c) {
-      const int Lc = min(C, sb.len - c * C);
-      const uint32_t ph = c & 1;
+    uint32_t it = 0;
+    for (; have; ++it) {
+      const int Lc = t.Lc;
+      const uint32_t ph = it & 1;
       // ---- P1: the A operand [R~; A~] of MMA1 and A~^T of MMA3 (4 channels x 4 tokens per thread);
       // the decay scan, [B^; K^] and V^T of this chunk were prepared by warps 4-7 beforehand
       {
@@ -809,20 +1049,20 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
         }
 #pragma unroll
         for (int tt = 0; tt < 4; ++tt) {
-          const int t = t0 + tt;
+          const int tk = t0 + tt;
           float Gt[4], Gp[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             Gp[e] = tt == 0 ? pre[e] : G[tt - 1][e];
             Gt[e] = G[tt][e];
           }
-          st_tf32x4(a1r + tc::sw128(t, chunk), rr[tt][0] * Gt[0], rr[tt][1] * Gt[1], rr[tt][2] * Gt[2],
+          st_tf32x4(a1r + tc::sw128(tk, chunk), rr[tt][0] * Gt[0], rr[tt][1] * Gt[1], rr[tt][2] * Gt[2],
                     rr[tt][3] * Gt[3]);
           const float At0 = aa[tt][0] * Gp[0], At1 = aa[tt][1] * Gp[1], At2 = aa[tt][2] * Gp[2],
                       At3 = aa[tt][3] * Gp[3];
-          st_tf32x4(a1r + tc::sw128(64 + t, chunk), At0, At1, At2, At3);
+          st_tf32x4(a1r + tc::sw128(64 + tk, chunk), At0, At1, At2, At3);
           // A3: A~^T as the MN-major bf16 A operand of MMA3 (M = channel, K = token)
-          *reinterpret_cast<uint2 *>(sA3 + mnmaj_bf16(64, t, j0)) =
+          *reinterpret_cast<uint2 *>(sA3 + mnmaj_bf16(64, tk, j0)) =
               make_uint2(pack_bf16x2(At0, At1), pack_bf16x2(At2, At3));
         }
       }
@@ -831,11 +1071,11 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
       if (tid == 0) tc::mbar_arrive(bar_p1);
       // ---- while MMA1 runs: the previous chunk's read-out (its MMA4 ran under P1), then the D2 set-up:
       // Q-part = R~ (rows of A1), E-part = 0, F-part = K-^T[j][m] = Gamma_C[j] K^[m][j] (columns of B1)
-      const float gc_cur = hi_lanes ? GCs[(c & 1) * 64 + j] : 1.f;  // Gamma_C[j] of this chunk (hi lanes)
+      const float gc_cur = hi_lanes ? GCs[ph * 64 + j] : 1.f;  // Gamma_C[j] of this chunk (hi lanes)
       if (have_prev) {
         if (!(ok = wait_ctrl(bar_m4, ph ^ 1u))) break;
         tc::tc_fence_after();
-        readout(c - 1, Lc_prev);
+        readout(pt, ph ^ 1u);
       }
       {
         float v[32];
@@ -861,7 +1101,7 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
 
       // ---- The two groups work apart until MMA3 is done.  Warps 0-3: Lab -> Ls (warps 2 and 3 own its
       // TMEM lanes), then the inverse.  Warps 4-7: the rest of the causal masks for all 128 lanes (A2 =
-      // [Mrb; B-^T] as bf16, the P-part of D2 = Mrk, the lower half of A3 = Lak^T), then the next chunk's
+      // [Mrb; B-^T] as bf16, the P-part of D2 = Mrk, the lower half of A3 = Lak^T), then the next task's
       // decay scan, [B^; K^] and V^T.  MMA3 waits for both groups (its barrier counts two arrivals).
       // The rows of quadrant q meet the diagonal in the 32-column half dh; column half hf lies on
       // (hf == dh), below (hf < dh) or above it.  The inverse's scratch lies outside A1 and B1.
@@ -941,12 +1181,25 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
         tc::tc_fence_before();
         group_sync_hi();
         if (tid == 128) tc::mbar_arrive(bar_b3);
-        // then the next chunk's decay scan, [B^; K^] and V^T (its tiles were loaded after MMA1); B1 is
-        // free: MMA1 is done and the masks above have read its B^ columns
-        if (c + 1 < nchunks && wait_group_hi(bar_tma, (c + 1) & 1))
-          prep_next<kFused>(smem, sA1, sB1, sB4V + ((c + 1) & 1) * 16384, pre4, GCs + ((c + 1) & 1) * 64, wtot, kkw,
-                            invn, tid - 128,
-                    min(C, sb.len - (c + 1) * C));
+        // then the next task's decay scan, [B^; K^] and V^T (its tiles were loaded after MMA1); B1 is
+        // free: MMA1 is done and the masks above have read its B^ columns.  A task of another head
+        // first brings its key scale and ln_x parameters (the previous read-out is done with them).
+        if constexpr (kTask) {
+          if (wait_group_hi(bar_tma, (it + 1) & 1)) {
+            const Task nt = task_slot[(it + 1) & 1];
+            if (nt.n >= 0) {
+              load_head(nt.h, (it + 1) & 1, tid - 128);
+              group_sync_hi();
+              prep_next<kFused, kTask>(smem, sA1, sB1, sB4V + ((it + 1) & 1) * 16384, pre4,
+                                       GCs + ((it + 1) & 1) * 64, wtot, kkw, invn, tid - 128, nt.Lc);
+            }
+          }
+        } else {
+          Task nt = t;
+          if (pair_next(A, nt) && wait_group_hi(bar_tma, (it + 1) & 1))
+            prep_next<kFused, kTask>(smem, sA1, sB1, sB4V + ((it + 1) & 1) * 16384, pre4, GCs + ((it + 1) & 1) * 64,
+                                     wtot, kkw, invn, tid - 128, nt.Lc);
+        }
       }
       if (!(ok = wait_ctrl(bar_m3, ph))) break;
       tc::tc_fence_after();
@@ -972,15 +1225,27 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
 
       if (tid == 0) tc::mbar_arrive(bar_b2);
       gc_done = gc_cur;
-      Lc_prev = Lc;
+      pt = t;
       have_prev = true;
+      if constexpr (kTask) {
+        t = task_slot[(it + 1) & 1];
+        have = t.n >= 0;
+      } else {
+        have = pair_next(A, t);
+      }
     }
     // drain: the last chunk's MMA4 and its read-out
-    if (have_prev && ok && wait_ctrl(bar_m4, (nchunks - 1) & 1)) {
+    if (have_prev && ok && wait_ctrl(bar_m4, (it - 1) & 1)) {
       tc::tc_fence_after();
-      readout(nchunks - 1, Lc_prev);
+      readout(pt, (it - 1) & 1);
+      if (kTask) {
+        // the last task's end state is stored: hand the flag to the control lane
+        compute_sync();
+        if (tid == 0) tc::mbar_arrive(bar_st);
+      }
     }
-    if (hi_lanes) {
+    if (!kTask && hi_lanes) {
+      const long long pair = static_cast<long long>(blockIdx.y) * A.H + blockIdx.x;
       tc::tmem_st_wait();
       float v[32];
       tc::tmem_ld32(tmem + lane_base + TM_S + 32 * ch, v);
@@ -1028,17 +1293,90 @@ static bool make_map(CUtensorMap *map, const void *base, long long tokens, int H
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-}  // namespace chunk
+static bool make_state_map(CUtensorMap *map, const void *base, long long rows) {
+  PFN_encodeTiled enc = get_encode();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kN), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kN) * 4};
+  const cuuint32_t box[2] = {32, static_cast<cuuint32_t>(kN)};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void *>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
-namespace chunk {
+// Scratch of the task-parallel schedule, in static device memory (the library allocates nothing):
+// per-pair flags in kFlagSlots slots, taken in turn by successive launches, so up to kFlagSlots
+// launches may run at once on one device; and a zero state block for s_in == NULL.
+constexpr int kFlagSlots = 4;
+constexpr long long kMaxChainPairs = 1 << 16;
+__device__ unsigned long long g_chain_flags[kFlagSlots * kMaxChainPairs];
+__device__ __align__(1024) float g_zero_state[kN * kN];
+
+struct DeviceScratch {
+  int sms = 0;
+  unsigned long long *flags = nullptr;
+  const float *zeros = nullptr;
+};
+
+static bool device_scratch(DeviceScratch &ds) {
+  static DeviceScratch cache[64];
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  std::lock_guard<std::mutex> lock(mu);
+  DeviceScratch &c = cache[dev];
+  if (c.sms == 0) {
+    int sms = 0;
+    void *f = nullptr, *z = nullptr;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) return false;
+    if (cudaGetSymbolAddress(&f, g_chain_flags) != cudaSuccess) return false;
+    if (cudaGetSymbolAddress(&z, g_zero_state) != cudaSuccess) return false;
+    c.flags = static_cast<unsigned long long *>(f);
+    c.zeros = static_cast<const float *>(z);
+    c.sms = sms;
+  }
+  ds = c;
+  return true;
+}
+
+// A fresh epoch per launch (never 0, so zeroed flags match no launch).
+static unsigned next_epoch() {
+  static std::atomic<unsigned> counter{0};
+  unsigned e;
+  do {
+    e = counter.fetch_add(1) + 1;
+  } while (e == 0);
+  return e;
+}
 
 template <bool kFused, bool kLN>
-static cudaError_t launch_variant(const Maps &maps, const Args &args, int B, int H, cudaStream_t stream) {
-  cudaError_t e = cudaFuncSetAttribute(wkv7_chunk_kernel<kFused, kLN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(kSmemBytes));
+static cudaError_t launch_variant(const Maps &maps, const Args &args, int B, int H, bool task, int grid_tasks,
+                                  cudaStream_t stream) {
+  if (!task) {
+    cudaError_t e = cudaFuncSetAttribute(wkv7_chunk_kernel<kFused, kLN, false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemBytes));
+    if (e != cudaSuccess) return e;
+    dim3 grid(H, B);
+    wkv7_chunk_kernel<kFused, kLN, false><<<grid, kThreads, kSmemBytes, stream>>>(maps, args);
+    return cudaGetLastError();
+  }
+  cudaError_t e = cudaFuncSetAttribute(wkv7_chunk_kernel<kFused, kLN, true>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemBytes));
   if (e != cudaSuccess) return e;
-  dim3 grid(H, B);
-  wkv7_chunk_kernel<kFused, kLN><<<grid, kThreads, kSmemBytes, stream>>>(maps, args);
+  // every CTA resident at once (a CTA may wait for a chunk another CTA holds): cooperative launch
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid_tasks));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, wkv7_chunk_kernel<kFused, kLN, true>, maps, args);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -1048,7 +1386,7 @@ cudaError_t launch_chunk_ext(const uint16_t *r, const uint16_t *w, const uint16_
                              const uint16_t *a, const uint16_t *b, bool model_native, const float *k_k,
                              bool group_norm, const float *ln_w, const float *ln_b, const float *s_in, uint16_t *y,
                              float *s_out, const int32_t *cu_seqlens, int B, int T, long long total_T, int H,
-                             int *err_word, cudaStream_t stream) {
+                             int schedule, int *err_word, cudaStream_t stream) {
   using namespace chunk;
   if (total_T > 0x7fffffffLL || H > 0xffff || B > 65535) return cudaErrorInvalidValue;
   Maps maps;
@@ -1059,11 +1397,36 @@ cudaError_t launch_chunk_ext(const uint16_t *r, const uint16_t *w, const uint16_
     if (!make_map(&maps.m[i], ops[i] ? ops[i] : static_cast<const void *>(s_out), tokens, H))
       return cudaErrorInvalidValue;
   }
-  Args args{y, s_in, s_out, cu_seqlens, T, total_T, H, err_word, k_k, ln_w, ln_b};
-  if (model_native && group_norm) return launch_variant<true, true>(maps, args, B, H, stream);
-  if (model_native) return launch_variant<true, false>(maps, args, B, H, stream);
-  if (group_norm) return launch_variant<false, true>(maps, args, B, H, stream);
-  return launch_variant<false, false>(maps, args, B, H, stream);
+  const long long BH = static_cast<long long>(B) * H;
+  // chunk rows of the task list: every chunk of the longest sequence (a ragged batch: bounded by
+  // total_T, so rows of any length are covered; tasks past a sequence's end are skipped)
+  const long long rows = (cu_seqlens == nullptr ? static_cast<long long>(T) : total_T) + C - 1;
+  const long long ntasks = (rows / C) * BH;
+  Args args{y, s_in, s_out, cu_seqlens, T, total_T, H, err_word, k_k, ln_w, ln_b, ntasks, BH, nullptr, 0, 0};
+  // The task-parallel schedule pays when one CTA per pair would leave many SMs idle: measured on B200,
+  // 48 and 96 pairs ran 1.2x and 1.1x faster, 1 and 2 pairs 1.6x; at 128 pairs and above the pair
+  // schedule was as fast or faster.
+  DeviceScratch ds;
+  bool task = false;
+  int grid_tasks = 0;
+  if (schedule != 1 && ntasks > 0 && ntasks < (1LL << 31) && BH <= kMaxChainPairs && device_scratch(ds)) {
+    task = schedule == 2 || 4 * BH <= 3 * static_cast<long long>(ds.sms);
+    grid_tasks = static_cast<int>(ntasks < ds.sms ? ntasks : ds.sms);
+  }
+  if (schedule == 2 && !task) return cudaErrorInvalidValue;
+  if (task) {
+    const unsigned epoch = next_epoch();
+    args.flags = ds.flags + static_cast<long long>(epoch % kFlagSlots) * kMaxChainPairs;
+    args.epoch = epoch;
+    args.s_in_zero = s_in == nullptr ? 1 : 0;
+    if (!make_state_map(&maps.s_in, s_in ? static_cast<const void *>(s_in) : ds.zeros, s_in ? BH * kN : kN) ||
+        !make_state_map(&maps.s_out, s_out, BH * kN))
+      return cudaErrorInvalidValue;
+  }
+  if (model_native && group_norm) return launch_variant<true, true>(maps, args, B, H, task, grid_tasks, stream);
+  if (model_native) return launch_variant<true, false>(maps, args, B, H, task, grid_tasks, stream);
+  if (group_norm) return launch_variant<false, true>(maps, args, B, H, task, grid_tasks, stream);
+  return launch_variant<false, false>(maps, args, B, H, task, grid_tasks, stream);
 }
 
 cudaError_t launch_chunk(const uint16_t *r, const uint16_t *w, const uint16_t *k, const uint16_t *v,
@@ -1071,7 +1434,7 @@ cudaError_t launch_chunk(const uint16_t *r, const uint16_t *w, const uint16_t *k
                          const int32_t *cu_seqlens, int B, int T, long long total_T, int H, int *err_word,
                          cudaStream_t stream) {
   return launch_chunk_ext(r, w, k, v, a, b, false, nullptr, false, nullptr, nullptr, s_in, y, s_out, cu_seqlens, B,
-                          T, total_T, H, err_word, stream);
+                          T, total_T, H, 0, err_word, stream);
 }
 
 }  // namespace rwkv7

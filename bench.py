@@ -60,10 +60,11 @@ def load_peaks():
 
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one chunk-kernel launch, from one ncu
-# capture at B=4 (48 CTAs, 178 MB of operands, larger than L2) scaled by B to the B=8 workload; the
+# capture at B=4 (48 pairs on the task-parallel schedule, as at B=8; 178 MB of operands, larger than
+# L2) scaled by B to the B=8 workload; the
 # figure holds only for the kernel source it was taken on (sha256 prefix of wkv7_chunk.cu), and the
 # line reports null for any other build.  The capture is summarised under profiles/.
-MEASURED_TRAFFIC = {"source_sha256": "d214f418d1afffb3", "bytes_per_token_head": (151908864 + 15943168) / (4 * 4096 * 12)}
+MEASURED_TRAFFIC = {"source_sha256": "013ea9f230dd5411", "bytes_per_token_head": (152044032 + 14690304) / (4 * 4096 * 12)}
 
 
 def measured_traffic(B, T, H, path):

@@ -6,7 +6,9 @@ imports nothing from the CUDA library: the two share only the seeded input
 generator ``wkv7_inputs``.
 
 The arithmetic lives in ``wkv7_oracle.c`` (token-by-token definition, see its
-header for the passages it follows).  This module compiles it with gcc
+header for the passages it follows) and ``wkv7_oracle_bwd.c`` (its gradients by the chain rule:
+the pages give no backward, so that file is pinned by finite differences and by torch autograd of
+an independent loop, ``tests/test_oracle_backward.py``).  This module compiles it with gcc
 (``-O2 -ffp-contract=off``, no fast-math) and wraps it with ctypes.
 
 Pins: every function here is checked by ``tests/test_oracle_pins.py`` against
@@ -26,6 +28,7 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "wkv7_oracle.c")
+_SRC_BWD = os.path.join(_HERE, "wkv7_oracle_bwd.c")
 _BUILD = os.path.join(_HERE, "_build")
 _LIBS = {"double": "liboracle_wkv7.so", "long double": "liboracle_wkv7_ld.so"}
 _lock = threading.Lock()
@@ -44,6 +47,12 @@ def build(force: bool = False) -> None:
                "-fno-fast-math", f"-DORACLE_REAL={real}", _SRC, "-o", tmp]
         subprocess.run(cmd, check=True)
         os.replace(tmp, out)
+    out = os.path.join(_BUILD, "liboracle_wkv7_bwd.so")
+    if force or not os.path.exists(out) or os.path.getmtime(out) < os.path.getmtime(_SRC_BWD):
+        tmp = out + ".tmp%d" % os.getpid()
+        subprocess.run(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread", "-ffp-contract=off",
+                        "-fno-fast-math", _SRC_BWD, "-o", tmp], check=True)
+        os.replace(tmp, out)
 
 
 def _lib(real: str = "double") -> ctypes.CDLL:
@@ -61,6 +70,19 @@ def _lib(real: str = "double") -> ctypes.CDLL:
             lib.wkv7_oracle_real_bytes.restype = ci
             _loaded[real] = lib
         return _loaded[real]
+
+
+def _lib_bwd() -> ctypes.CDLL:
+    with _lock:
+        if "bwd" not in _loaded:
+            build()
+            lib = ctypes.CDLL(os.path.join(_BUILD, "liboracle_wkv7_bwd.so"))
+            dp = ctypes.POINTER(ctypes.c_double)
+            ci = ctypes.c_int
+            lib.wkv7_oracle_bwd_f64.argtypes = [ci, ci, ci, ci] + [dp] * 9 + [dp] * 7 + [ci]
+            lib.wkv7_oracle_bwd_f64.restype = ci
+            _loaded["bwd"] = lib
+        return _loaded["bwd"]
 
 
 def _as_np(x, dt) -> np.ndarray:
@@ -183,3 +205,28 @@ def group_norm_heads(y, ln_w=None, ln_b=None, eps: float = LN_EPS) -> np.ndarray
 
 def real_bytes(real: str = "double") -> int:
     return int(_lib(real).wkv7_oracle_real_bytes())
+
+
+def wkv7_backward(r, w, k, v, a, b, s_in, dy, ds_out=None, *, nthreads: Optional[int] = None):
+    """Gradients of ``L = sum <dy, y> + <ds_out, s_out>`` for the recurrence of ``wkv7`` (float64,
+    token-by-token chain rule; see ``wkv7_oracle_bwd.c``).  Token tensors ``[B, T, H, N]``, states
+    ``[B, H, N, N]``; ``s_in`` / ``ds_out`` None mean zero.  Returns float64 arrays
+    ``(dr, dw, dk, dv, da, db, ds_in)``."""
+    ops = [_as_np(x, np.float64) for x in (r, w, k, v, a, b)]
+    B, T, H, N = ops[0].shape
+    dyn = _as_np(dy, np.float64)
+    assert dyn.shape == (B, T, H, N)
+    s0 = None if s_in is None else _as_np(s_in, np.float64)
+    dso = None if ds_out is None else _as_np(ds_out, np.float64)
+    outs = [np.zeros((B, T, H, N)) for _ in range(6)]
+    ds_in = np.zeros((B, H, N, N))
+    dp = ctypes.POINTER(ctypes.c_double)
+
+    def ptr(x):
+        return None if x is None else x.ctypes.data_as(dp)
+
+    st = _lib_bwd().wkv7_oracle_bwd_f64(B, T, H, N, *[ptr(x) for x in ops], ptr(s0), ptr(dyn), ptr(dso),
+                                        *[ptr(x) for x in outs], ptr(ds_in), int(nthreads or default_threads()))
+    if st != 0:
+        raise RuntimeError(f"oracle backward failed ({st})")
+    return tuple(outs) + (ds_in,)

@@ -28,8 +28,9 @@ __all__ = [
     "rwkv7_wkv_decode", "rwkv7_wkv_decode_bf16", "rwkv7_wkv_prefill_fused_bf16", "rwkv7_wkv_decode_fused_bf16",
     "rwkv7_wkv_prefill_ext_bf16", "rwkv7_wkv_decode_ext_bf16", "Options",
     "rwkv7_status_string", "rwkv7_get_last_error", "rwkv7_version",
+    "rwkv7_wkv_prefill_save_bf16", "rwkv7_wkv_backward_bf16",
     "prefill", "decode_", "prefill_model_native", "decode_model_native_", "prefill_ext", "decode_ext_",
-    "EXPORTED_SYMBOLS",
+    "prefill_save", "backward", "EXPORTED_SYMBOLS",
 ]
 
 RWKV7_PATH_AUTO, RWKV7_PATH_SCAN, RWKV7_PATH_CHUNK = 0, 1, 2
@@ -41,6 +42,7 @@ EXPORTED_SYMBOLS = (
     "rwkv7_wkv_prefill", "rwkv7_wkv_prefill_bf16", "rwkv7_wkv_prefill_bf16_path", "rwkv7_wkv_prefill_varlen_bf16",
     "rwkv7_wkv_decode", "rwkv7_wkv_decode_bf16", "rwkv7_wkv_prefill_fused_bf16", "rwkv7_wkv_decode_fused_bf16",
     "rwkv7_wkv_prefill_ext_bf16", "rwkv7_wkv_decode_ext_bf16",
+    "rwkv7_wkv_prefill_save_bf16", "rwkv7_wkv_backward_bf16",
     "rwkv7_status_string", "rwkv7_get_last_error", "rwkv7_version",
 )
 
@@ -87,6 +89,8 @@ def load_library() -> ctypes.CDLL:
         ("rwkv7_wkv_decode_fused_bf16", [ci, ci, ci] + [vp] * 6 + [vp, vp, vp]),
         ("rwkv7_wkv_prefill_ext_bf16", [ci, ci, ci, ci, ci] + [vp] * 6 + [ctypes.POINTER(Options), vp, vp, vp, vp]),
         ("rwkv7_wkv_decode_ext_bf16", [ci, ci, ci] + [vp] * 6 + [ctypes.POINTER(Options), vp, vp, vp]),
+        ("rwkv7_wkv_prefill_save_bf16", [ci, ci, ci, ci] + [vp] * 6 + [vp, vp, vp, vp, vp]),
+        ("rwkv7_wkv_backward_bf16", [ci, ci, ci, ci] + [vp] * 6 + [vp, vp, vp] + [vp] * 7 + [vp]),
     ):
         fn = getattr(lib, name)
         fn.argtypes = args
@@ -262,6 +266,40 @@ def rwkv7_wkv_decode_ext_bf16(r, w, k, v, a, b, s_inout, y, *, model_native=Fals
           ctypes.byref(opt), _ptr(s_inout), _ptr(y), _stream(stream))
 
 
+def n_checkpoints(T: int) -> int:
+    """Saved states per (b, h) of ``rwkv7_wkv_prefill_save_bf16``: one before every 64th token."""
+    return (int(T) + 63) // 64
+
+
+def rwkv7_wkv_prefill_save_bf16(r, w, k, v, a, b, s_in, y, s_out, states, stream=None) -> None:
+    """bf16 prefill (sequential scan) that also writes ``states`` float32 ``[B, H, ceil(T/64), 64, 64]``,
+    the state before every 64th token, for ``rwkv7_wkv_backward_bf16``."""
+    B, T, H, N = r.shape
+    for nm, t in (("r", r), ("w", w), ("k", k), ("v", v), ("a", a), ("b", b), ("y", y)):
+        _check(t, nm, torch.bfloat16, (B, T, H, N))
+    _check(s_in, "s_in", torch.float32, (B, H, N, N), allow_none=True)
+    _check(s_out, "s_out", torch.float32, (B, H, N, N))
+    _check(states, "states", torch.float32, (B, H, n_checkpoints(T), N, N))
+    _call("rwkv7_wkv_prefill_save_bf16", B, T, H, N, *[_ptr(t) for t in (r, w, k, v, a, b, s_in, y, s_out, states)],
+          _stream(stream))
+
+
+def rwkv7_wkv_backward_bf16(r, w, k, v, a, b, states, dy, ds_out, dr, dw, dk, dv, da, db, ds_in,
+                            stream=None) -> None:
+    """Gradients (float32) of a loss with dL/dy = ``dy`` (bf16) and dL/ds_out = ``ds_out`` (float32 or
+    None) with respect to r, w, k, v, a, b (``[B, T, H, 64]``) and s_in (``ds_in`` or None)."""
+    B, T, H, N = r.shape
+    for nm, t in (("r", r), ("w", w), ("k", k), ("v", v), ("a", a), ("b", b), ("dy", dy)):
+        _check(t, nm, torch.bfloat16, (B, T, H, N))
+    for nm, t in (("dr", dr), ("dw", dw), ("dk", dk), ("dv", dv), ("da", da), ("db", db)):
+        _check(t, nm, torch.float32, (B, T, H, N))
+    _check(states, "states", torch.float32, (B, H, n_checkpoints(T), N, N))
+    _check(ds_out, "ds_out", torch.float32, (B, H, N, N), allow_none=True)
+    _check(ds_in, "ds_in", torch.float32, (B, H, N, N), allow_none=True)
+    _call("rwkv7_wkv_backward_bf16", B, T, H, N, *[_ptr(t) for t in (r, w, k, v, a, b, states, dy, ds_out)],
+          *[_ptr(t) for t in (dr, dw, dk, dv, da, db, ds_in)], _stream(stream))
+
+
 def rwkv7_status_string(status: int) -> str:
     return load_library().rwkv7_status_string(int(status)).decode()
 
@@ -337,3 +375,22 @@ def decode_ext_(r, w, k, v, a, b, state, y=None, *, model_native=False, k_k=None
     rwkv7_wkv_decode_ext_bf16(r, w, k, v, a, b, state, y, model_native=model_native, k_k=k_k,
                               group_norm=group_norm, ln_w=ln_w, ln_b=ln_b, stream=stream)
     return y
+
+
+def prefill_save(r, w, k, v, a, b, s_in=None, *, stream=None):
+    """Allocate and run the checkpointing prefill; returns ``(y, s_out, states)``."""
+    B, T, H, N = r.shape
+    y = torch.empty_like(r)
+    s_out = torch.empty((B, H, N, N), dtype=torch.float32, device=r.device)
+    states = torch.empty((B, H, n_checkpoints(T), N, N), dtype=torch.float32, device=r.device)
+    rwkv7_wkv_prefill_save_bf16(r, w, k, v, a, b, s_in, y, s_out, states, stream=stream)
+    return y, s_out, states
+
+
+def backward(r, w, k, v, a, b, states, dy, ds_out=None, *, stream=None):
+    """Allocate and run the backward; returns float32 ``(dr, dw, dk, dv, da, db, ds_in)``."""
+    B, T, H, N = r.shape
+    g = [torch.empty((B, T, H, N), dtype=torch.float32, device=r.device) for _ in range(6)]
+    ds_in = torch.empty((B, H, N, N), dtype=torch.float32, device=r.device)
+    rwkv7_wkv_backward_bf16(r, w, k, v, a, b, states, dy, ds_out, *g, ds_in, stream=stream)
+    return tuple(g) + (ds_in,)

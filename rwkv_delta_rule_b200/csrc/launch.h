@@ -23,6 +23,19 @@ cudaError_t launch_scan_ext(const uint16_t *r, const uint16_t *w, const uint16_t
                             float *s_out, const int32_t *cu_seqlens, int B, int T, long long total_T, int H,
                             cudaStream_t stream);
 
+// The bf16 scan (dense T) that also writes the state before every 64th token into states
+// [B, H, ceil(T/64), 64, 64] (the checkpoints the backward starts from).
+cudaError_t launch_scan_save(const uint16_t *r, const uint16_t *w, const uint16_t *k, const uint16_t *v,
+                             const uint16_t *a, const uint16_t *b, const float *s_in, uint16_t *y, float *s_out,
+                             float *states, int B, int T, int H, cudaStream_t stream);
+
+// Gradients of the recurrence (see wkv7_backward.cu); dr, dw, dk, da, db must be zero on entry
+// (they are accumulated), dv and ds_in (optional) are written.
+cudaError_t launch_backward(const uint16_t *r, const uint16_t *w, const uint16_t *k, const uint16_t *v,
+                            const uint16_t *a, const uint16_t *b, const float *states, const uint16_t *dy,
+                            const float *ds_out, float *dr, float *dw, float *dk, float *dv, float *da, float *db,
+                            float *ds_in, int B, int T, int H, cudaStream_t stream);
+
 // One decode step over [B,H,64], state updated in place.
 template <typename TIn>
 cudaError_t launch_decode(const TIn *r, const TIn *w, const TIn *k, const TIn *v, const TIn *a, const TIn *b,

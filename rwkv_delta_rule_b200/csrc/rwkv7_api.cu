@@ -208,4 +208,43 @@ rwkv7_status rwkv7_wkv_decode_fused_bf16(int B, int H, int N, const uint16_t *r,
   return rwkv7_wkv_decode_ext_bf16(B, H, N, r, xw, k, v, xa, nullptr, &opt, s_inout, y, stream);
 }
 
+rwkv7_status rwkv7_wkv_prefill_save_bf16(int B, int T, int H, int N, const uint16_t *r, const uint16_t *w,
+                                         const uint16_t *k, const uint16_t *v, const uint16_t *a, const uint16_t *b,
+                                         const float *s_in, uint16_t *y, float *s_out, float *states,
+                                         rwkv7_stream_t stream) {
+  const rwkv7_status st = check_prefill(B, T, H, N, r, w, k, v, a, b, s_in, y, s_out);
+  if (st != RWKV7_OK) return st;
+  if (T > 0 && states == nullptr) return RWKV7_ERR_INVALID;
+  if (!aligned16(states)) return RWKV7_ERR_ALIGN;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  return from_cuda(launch_scan_save(r, w, k, v, a, b, s_in, y, s_out, states, B, T, H, cs));
+}
+
+rwkv7_status rwkv7_wkv_backward_bf16(int B, int T, int H, int N, const uint16_t *r, const uint16_t *w,
+                                     const uint16_t *k, const uint16_t *v, const uint16_t *a, const uint16_t *b,
+                                     const float *states, const uint16_t *dy, const float *ds_out, float *dr,
+                                     float *dw, float *dk, float *dv, float *da, float *db, float *ds_in,
+                                     rwkv7_stream_t stream) {
+  if (N != kN) return RWKV7_ERR_UNSUPPORTED;
+  if (B <= 0 || H <= 0 || T < 0 || B > 65535 || H > 0xffff) return RWKV7_ERR_INVALID;
+  if (T > 0 && !none_null(r, w, k, v, a, b, states, dy, dr, dw, dk, dv, da, db)) return RWKV7_ERR_INVALID;
+  if (!all_aligned(r, w, k, v, a, b, dy, dr, dw, dk, dv, da, db) || !all_aligned(states, ds_out, ds_in))
+    return RWKV7_ERR_ALIGN;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  const size_t bytes = sizeof(float) * static_cast<size_t>(B) * T * H * kN;
+  if (T > 0) {
+    // the column sums arrive from several row groups: these five are accumulated
+    for (float *g : {dr, dw, dk, da, db})
+      if (cudaMemsetAsync(g, 0, bytes, cs) != cudaSuccess) return RWKV7_ERR_CUDA;
+  } else if (ds_in != nullptr) {
+    const size_t sb = sizeof(float) * static_cast<size_t>(B) * H * kN * kN;
+    const cudaError_t e = ds_out ? cudaMemcpyAsync(ds_in, ds_out, sb, cudaMemcpyDeviceToDevice, cs)
+                                 : cudaMemsetAsync(ds_in, 0, sb, cs);
+    return from_cuda(e);
+  } else {
+    return RWKV7_OK;
+  }
+  return from_cuda(launch_backward(r, w, k, v, a, b, states, dy, ds_out, dr, dw, dk, dv, da, db, ds_in, B, T, H, cs));
+}
+
 }  // extern "C"

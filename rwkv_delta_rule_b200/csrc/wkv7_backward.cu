@@ -1,0 +1,291 @@
+// wkv7_backward.cu -- gradients of the x070 recurrence for training (sequential form).
+//
+// The forward (RWKV-7 G0 7.2B walkthrough, lshu.cn/news/198401, section 7.1) is, per (b, h),
+//   sa = S a_t;   S' = S diag(w_t) + sa b_t^T + v_t k_t^T;   y_t = S' r_t.
+// The pages give no backward; this is the chain rule applied to that loop, for a loss whose
+// gradients dy (per token) and ds_out (final state) are given.  Walking the tokens backwards with
+// G = dL/dS' (starting from ds_out):
+//   G += dy_t r_t^T;   dr_t = S'^T dy_t;   dv_t = G k_t;   dk_t = G^T v_t;
+//   db_t = G^T sa;     g = G b_t;          dw_t = colsum(G .* S);   da_t = S^T g;
+//   G <- G diag(w_t) + g a_t^T            (= dL/dS, carried to the token before),
+// and ds_in = G at the start.
+//
+// Rows of S (value channels) are independent in the forward and in the walk back: row i of G and
+// of S only meet the shared vectors.  A (b, h) pair is split into 4 row groups of 16 rows, one CTA
+// of 128 threads each; every row is spread over 8 lanes holding 8 columns.  Row sums (sa, g, dv)
+// are three xor-shuffles inside the 8 lanes; the column sums (dr, dk, db, dw, da: sums over rows)
+// are two xor-shuffles over the 4 rows of a warp, then the 4 warps' partials in shared memory, then
+// float32 atomics across the 4 row groups (the caller zeroes those outputs first).
+//
+// The states S before every token are recomputed from the checkpoints the forward saved (the state
+// before every 64th token): per 64-token chunk, walked from the last, a forward pass from the
+// checkpoint keeps the state before each 8-token sub-block in shared memory; then each sub-block,
+// from the last, recomputes its 9 states into registers and walks its tokens back.  Per-token
+// operands are staged 8 tokens at a time by cp.async, double-buffered, in the order the schedule
+// visits them.
+#include "common.cuh"
+#include "launch.h"
+
+namespace rwkv7 {
+namespace bwd {
+
+constexpr int kRows = 16;                 // state rows per CTA (4 CTAs per (b, h))
+constexpr int kThreads = kRows * 8;       // 8 lanes per row: 128 threads, 4 warps of 4 rows
+constexpr int kSub = 8;                   // tokens per sub-block
+constexpr int kChunk = 64;                // tokens per saved state
+constexpr int kSubs = kChunk / kSub;      // sub-blocks per chunk
+constexpr int kTokVec = 7;                // staged per token: r, w, k, a, b, v, dy (64 bf16 each)
+constexpr int kStageElems = kSub * kTokVec * kN;
+enum { V_R = 0, V_W = 1, V_K = 2, V_A = 3, V_B = 4, V_V = 5, V_DY = 6 };
+
+constexpr size_t kSmemSubck = sizeof(float) * kSubs * kRows * kN;   // 32 KB
+constexpr size_t kSmemStage = sizeof(uint16_t) * 2 * kStageElems;   // 14 KB
+constexpr size_t kSmemPart = sizeof(float) * 2 * 4 * 5 * kN;         // 10 KB
+constexpr size_t kSmemBytes = kSmemSubck + kSmemStage + kSmemPart;
+
+struct Args {
+  const uint16_t *r, *w, *k, *v, *a, *b, *dy;
+  const float *states;  // [B, H, ceil(T/64), 64, 64]
+  const float *ds_out;  // [B, H, 64, 64] or nullptr
+  float *dr, *dw, *dk, *dv, *da, *db;  // [B, T, H, 64]; dr dw dk da db accumulated
+  float *ds_in;                        // [B, H, 64, 64] or nullptr
+  int T, H;
+};
+
+// One visit of the schedule: sub-block s of chunk c, in the forward pass (fwd) or the walk back.
+struct Visit {
+  int c, s, fwd;
+};
+// Chunks from the last; each contributes its forward sub-blocks 0..n-1, then n-1..0 backwards.
+__device__ __forceinline__ Visit visit_at(int kk, int nck, int nsub_last) {
+  Visit v;
+  int j, nsub;
+  if (kk < 2 * nsub_last) {
+    v.c = nck - 1;
+    j = kk;
+    nsub = nsub_last;
+  } else {
+    const int k2 = kk - 2 * nsub_last;
+    v.c = nck - 2 - k2 / (2 * kSubs);
+    j = k2 % (2 * kSubs);
+    nsub = kSubs;
+  }
+  v.fwd = j < nsub ? 1 : 0;
+  v.s = v.fwd ? j : 2 * nsub - 1 - j;
+  return v;
+}
+
+__device__ __forceinline__ void stage_visit(const Args &A, uint16_t *buf, long long tok0, int ntok, int h) {
+  const int total = ntok * kTokVec * 8;  // 16-byte pieces
+  for (int c = threadIdx.x; c < total; c += kThreads) {
+    const int tt = c / (kTokVec * 8), rem = c - tt * (kTokVec * 8);
+    const int vid = rem >> 3, part = rem & 7;
+    const uint16_t *src = vid == V_R   ? A.r
+                          : vid == V_W ? A.w
+                          : vid == V_K ? A.k
+                          : vid == V_A ? A.a
+                          : vid == V_B ? A.b
+                          : vid == V_V ? A.v
+                                       : A.dy;
+    cp_async16(buf + (tt * kTokVec + vid) * kN + part * 8, src + ((tok0 + tt) * A.H + h) * kN + part * 8);
+  }
+}
+
+__device__ __forceinline__ void ld8(const uint16_t *p, float (&o)[8]) {
+  const uint4 u = *reinterpret_cast<const uint4 *>(p);
+  o[0] = __uint_as_float(u.x << 16);
+  o[1] = __uint_as_float(u.x & 0xffff0000u);
+  o[2] = __uint_as_float(u.y << 16);
+  o[3] = __uint_as_float(u.y & 0xffff0000u);
+  o[4] = __uint_as_float(u.z << 16);
+  o[5] = __uint_as_float(u.z & 0xffff0000u);
+  o[6] = __uint_as_float(u.w << 16);
+  o[7] = __uint_as_float(u.w & 0xffff0000u);
+}
+
+__device__ __forceinline__ float rowsum8(float x) {
+  x += __shfl_xor_sync(0xffffffffu, x, 1);
+  x += __shfl_xor_sync(0xffffffffu, x, 2);
+  x += __shfl_xor_sync(0xffffffffu, x, 4);
+  return x;
+}
+
+// One forward token on this thread's 8 columns (c0 ..) of row `row`: S <- S diag(w) + (S a) b^T + v k^T.
+__device__ __forceinline__ void fwd_token(float (&S)[8], const uint16_t *tk, int c0, int row) {
+  float w8[8], k8[8], a8[8], b8[8];
+  ld8(tk + V_W * kN + c0, w8);
+  ld8(tk + V_K * kN + c0, k8);
+  ld8(tk + V_A * kN + c0, a8);
+  ld8(tk + V_B * kN + c0, b8);
+  const float vi = bf16_bits_to_float(tk[V_V * kN + row]);
+  float sa = 0.f;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) sa = fmaf(S[e], a8[e], sa);
+  sa = rowsum8(sa);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) S[e] = fmaf(S[e], w8[e], fmaf(sa, b8[e], vi * k8[e]));
+}
+
+__global__ void __launch_bounds__(kThreads) wkv7_backward_kernel(const Args A) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  float *subck = reinterpret_cast<float *>(smem_raw);
+  uint16_t *stage = reinterpret_cast<uint16_t *>(smem_raw + kSmemSubck);
+  float *part = reinterpret_cast<float *>(smem_raw + kSmemSubck + kSmemStage);
+
+  constexpr int kSplits = kN / kRows;
+  const int h = blockIdx.x / kSplits;
+  const int row0 = (blockIdx.x - h * kSplits) * kRows;
+  const int bidx = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int rl = tid >> 3, c0 = 8 * (tid & 7);
+  const int row = row0 + rl;  // state row (value channel) of this thread
+  const int T = A.T;
+  const long long pair = static_cast<long long>(bidx) * A.H + h;
+  const long long tok_base = static_cast<long long>(bidx) * T;  // token row of t = 0
+  const int nck = (T + kChunk - 1) / kChunk;
+  const int nsub_last = nck > 0 ? (T - (nck - 1) * kChunk + kSub - 1) / kSub : 0;
+  const int nvisits = nck > 0 ? 2 * nsub_last + 2 * kSubs * (nck - 1) : 0;
+  float *grads[5] = {A.dr, A.dk, A.db, A.dw, A.da};
+
+  float G[8];  // dL/dS for this thread's columns of its row
+#pragma unroll
+  for (int e = 0; e < 8; ++e) G[e] = A.ds_out ? A.ds_out[pair * (kN * kN) + row * kN + c0 + e] : 0.f;
+  float S[8];  // running state of the forward passes
+#pragma unroll
+  for (int e = 0; e < 8; ++e) S[e] = 0.f;
+
+  int pbuf = 0;
+  if (nvisits > 0) {
+    const Visit v0 = visit_at(0, nck, nsub_last);
+    const int t0 = v0.c * kChunk + v0.s * kSub;
+    stage_visit(A, stage, tok_base + t0, min(kSub, T - t0), h);
+    cp_async_commit();
+  }
+  for (int kk = 0; kk < nvisits; ++kk) {
+    const Visit vis = visit_at(kk, nck, nsub_last);
+    if (kk + 1 < nvisits) {
+      const Visit vn = visit_at(kk + 1, nck, nsub_last);
+      const int tn = vn.c * kChunk + vn.s * kSub;
+      stage_visit(A, stage + ((kk + 1) & 1) * kStageElems, tok_base + tn, min(kSub, T - tn), h);
+      cp_async_commit();
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    const uint16_t *buf = stage + (kk & 1) * kStageElems;
+    const int t0 = vis.c * kChunk + vis.s * kSub;
+    const int Ls = min(kSub, T - t0);
+    float *sck = subck + (vis.s * kRows + rl) * kN + c0;
+
+    if (vis.fwd) {
+      // forward from the chunk's checkpoint, keeping the state before each sub-block
+      if (vis.s == 0) {
+        const float *ck = A.states + (pair * nck + vis.c) * (kN * kN) + row * kN + c0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) S[e] = ck[e];
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) sck[e] = S[e];
+      for (int u = 0; u < Ls; ++u) fwd_token(S, buf + u * kTokVec * kN, c0, row);
+    } else {
+      // this sub-block's states: St[u] before token t0 + u, St[u + 1] after it
+      float St[kSub + 1][8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) St[0][e] = sck[e];
+#pragma unroll
+      for (int u = 0; u < kSub; ++u) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) St[u + 1][e] = St[u][e];
+        if (u < Ls) fwd_token(St[u + 1], buf + u * kTokVec * kN, c0, row);
+      }
+#pragma unroll
+      for (int u = kSub - 1; u >= 0; --u) {
+        if (u >= Ls) continue;  // uniform across the CTA
+        const uint16_t *tk = buf + u * kTokVec * kN;
+        float r8[8], w8[8], k8[8], a8[8], b8[8];
+        ld8(tk + V_R * kN + c0, r8);
+        ld8(tk + V_W * kN + c0, w8);
+        ld8(tk + V_K * kN + c0, k8);
+        ld8(tk + V_A * kN + c0, a8);
+        ld8(tk + V_B * kN + c0, b8);
+        const float vi = bf16_bits_to_float(tk[V_V * kN + row]);
+        const float dyi = bf16_bits_to_float(tk[V_DY * kN + row]);
+        // y_t = S' r_t
+#pragma unroll
+        for (int e = 0; e < 8; ++e) G[e] = fmaf(dyi, r8[e], G[e]);
+        float p[5][8];  // column partials: dr, dk, db, dw, da
+        float dv = 0.f, sa = 0.f, g = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          p[0][e] = St[u + 1][e] * dyi;
+          dv = fmaf(G[e], k8[e], dv);
+          p[1][e] = G[e] * vi;
+          sa = fmaf(St[u][e], a8[e], sa);
+          g = fmaf(G[e], b8[e], g);
+          p[3][e] = G[e] * St[u][e];
+        }
+        dv = rowsum8(dv);
+        sa = rowsum8(sa);
+        g = rowsum8(g);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          p[2][e] = G[e] * sa;
+          p[4][e] = St[u][e] * g;
+          G[e] = fmaf(G[e], w8[e], g * a8[e]);
+        }
+        // sums over the warp's 4 rows (lane bits 3, 4)
+#pragma unroll
+        for (int q = 0; q < 5; ++q)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            p[q][e] += __shfl_xor_sync(0xffffffffu, p[q][e], 8);
+            p[q][e] += __shfl_xor_sync(0xffffffffu, p[q][e], 16);
+          }
+        const long long tok = tok_base + t0 + u;
+        float *pw = part + pbuf * (4 * 5 * kN);
+        if (lane < 8) {
+#pragma unroll
+          for (int q = 0; q < 5; ++q) {
+            float *dst = pw + (warp * 5 + q) * kN + c0;
+            *reinterpret_cast<float4 *>(dst) = make_float4(p[q][0], p[q][1], p[q][2], p[q][3]);
+            *reinterpret_cast<float4 *>(dst + 4) = make_float4(p[q][4], p[q][5], p[q][6], p[q][7]);
+          }
+        }
+        if ((tid & 7) == 0) A.dv[(tok * A.H + h) * kN + row] = dv;
+        __syncthreads();
+        // the 4 warps' partials, then the 4 row groups through float32 atomics
+        for (int idx = tid; idx < 5 * kN; idx += kThreads) {
+          const int q = idx >> 6, col = idx & 63;
+          const float sum = (pw[(0 * 5 + q) * kN + col] + pw[(1 * 5 + q) * kN + col]) +
+                            (pw[(2 * 5 + q) * kN + col] + pw[(3 * 5 + q) * kN + col]);
+          atomicAdd(grads[q] + (tok * A.H + h) * kN + col, sum);
+        }
+        pbuf ^= 1;
+      }
+    }
+    // every thread is done with this staging buffer before the next visit refills it
+    __syncthreads();
+  }
+  if (A.ds_in != nullptr)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) A.ds_in[pair * (kN * kN) + row * kN + c0 + e] = G[e];
+}
+
+}  // namespace bwd
+
+cudaError_t launch_backward(const uint16_t *r, const uint16_t *w, const uint16_t *k, const uint16_t *v,
+                            const uint16_t *a, const uint16_t *b, const float *states, const uint16_t *dy,
+                            const float *ds_out, float *dr, float *dw, float *dk, float *dv, float *da, float *db,
+                            float *ds_in, int B, int T, int H, cudaStream_t stream) {
+  using namespace bwd;
+  Args A{r, w, k, v, a, b, dy, states, ds_out, dr, dw, dk, dv, da, db, ds_in, T, H};
+  cudaError_t e = cudaFuncSetAttribute(wkv7_backward_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kSmemBytes));
+  if (e != cudaSuccess) return e;
+  dim3 grid(H * (kN / kRows), B);
+  wkv7_backward_kernel<<<grid, kThreads, kSmemBytes, stream>>>(A);
+  return cudaGetLastError();
+}
+
+}  // namespace rwkv7

@@ -56,6 +56,7 @@ template <typename TIn> struct ScanArgs {
   int H;
   const float *k_k;  // fused: [H, 64] key scale, nullptr = ones
   const float *ln_w, *ln_b;  // group-norm epilogue: [H, 64] weight / bias, nullptr = ones / zeros
+  float *states;  // nullptr, or [B, H, ceil(T / 64), 64, 64]: the state before every 64th token (dense T)
 };
 
 template <typename TIn, int ROWS, bool kFused>
@@ -147,6 +148,16 @@ __global__ void __launch_bounds__(ScanCfg<TIn, ROWS>::kThreads) wkv7_scan_kernel
         if (!kFused) Elem<TIn>::load4(tok + 4 * kN + col, bb + 4 * m);
       }
       const float vi = Elem<TIn>::load(tok + C::kVecElems + rloc);
+      if (A.states != nullptr && ((t0 + tt) & 63) == 0) {
+        // checkpoint for the backward: this thread's 16 columns of the state before the token
+        const int nck = (A.T + 63) >> 6;
+        float *ck = A.states + ((static_cast<long long>(bidx) * A.H + h) * nck + ((t0 + tt) >> 6)) * (kN * kN) +
+                    static_cast<long long>(row) * kN;
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+          *reinterpret_cast<float4 *>(ck + 16 * m + 4 * q) =
+              make_float4(s[4 * m + 0], s[4 * m + 1], s[4 * m + 2], s[4 * m + 3]);
+      }
       if (kFused) {
         // x070 prologue: kk = normalise(k * k_k) over the quad's 64 columns, a = -kk, b = kk * rate
         float ss = 0.f;
@@ -243,8 +254,16 @@ template <typename TIn>
 cudaError_t launch_scan(const TIn *r, const TIn *w, const TIn *k, const TIn *v, const TIn *a, const TIn *b,
                         const float *s_in, TIn *y, float *s_out, const int32_t *cu_seqlens, int B, int T,
                         long long total_T, int H, cudaStream_t stream) {
-  ScanArgs<TIn> A{r, w, k, v, a, b, s_in, y, s_out, cu_seqlens, T, total_T, H, nullptr, nullptr, nullptr};
+  ScanArgs<TIn> A{r, w, k, v, a, b, s_in, y, s_out, cu_seqlens, T, total_T, H, nullptr, nullptr, nullptr, nullptr};
   return launch_scan_rows<TIn, 16>(A, B, stream);
+}
+
+cudaError_t launch_scan_save(const uint16_t *r, const uint16_t *w, const uint16_t *k, const uint16_t *v,
+                             const uint16_t *a, const uint16_t *b, const float *s_in, uint16_t *y, float *s_out,
+                             float *states, int B, int T, int H, cudaStream_t stream) {
+  ScanArgs<uint16_t> A{r, w, k, v, a, b, s_in, y, s_out, nullptr, T, static_cast<long long>(B) * T, H,
+                       nullptr, nullptr, nullptr, states};
+  return launch_scan_rows<uint16_t, 16>(A, B, stream);
 }
 
 cudaError_t launch_scan_ext(const uint16_t *r, const uint16_t *w, const uint16_t *k, const uint16_t *v,
@@ -252,7 +271,7 @@ cudaError_t launch_scan_ext(const uint16_t *r, const uint16_t *w, const uint16_t
                             bool group_norm, const float *ln_w, const float *ln_b, const float *s_in, uint16_t *y,
                             float *s_out, const int32_t *cu_seqlens, int B, int T, long long total_T, int H,
                             cudaStream_t stream) {
-  ScanArgs<uint16_t> A{r, w, k, v, a, b, s_in, y, s_out, cu_seqlens, T, total_T, H, k_k, ln_w, ln_b};
+  ScanArgs<uint16_t> A{r, w, k, v, a, b, s_in, y, s_out, cu_seqlens, T, total_T, H, k_k, ln_w, ln_b, nullptr};
   if (model_native && group_norm) return launch_scan_rows<uint16_t, 64, true, true>(A, B, stream);
   if (model_native) return launch_scan_rows<uint16_t, 16, true, false>(A, B, stream);
   if (group_norm) return launch_scan_rows<uint16_t, 64, false, true>(A, B, stream);

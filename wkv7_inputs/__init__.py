@@ -157,6 +157,19 @@ def draw_group_norm(H: int, N: int = N_HEAD, *, seed: int) -> Dict[str, torch.Te
     return {"ln_w": ln_w.contiguous(), "ln_b": ln_b.contiguous()}
 
 
+def draw_grads(B: int, T: int, H: int, N: int = N_HEAD, *, seed: int, ds_std: Optional[float] = 1.0
+               ) -> Dict[str, torch.Tensor]:
+    """Draw the incoming gradients of a backward call: ``dy`` bf16 ``[B, T, H, N]`` ~ N(0, 1) (with a
+    ``dy_f32`` copy) and ``ds_out`` float32 ``[B, H, N, N]`` ~ N(0, ds_std^2), or None."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    dy = torch.randn((B, T, H, N), generator=g, dtype=torch.float32).to(torch.bfloat16).contiguous()
+    ds = None
+    if ds_std is not None:
+        ds = (torch.randn((B, H, N, N), generator=g, dtype=torch.float32) * float(ds_std)).contiguous()
+    return {"dy": dy, "dy_f32": dy.to(torch.float32), "ds_out": ds}
+
+
 def draw_case(case: Case, *, T: Optional[int] = None, B: Optional[int] = None) -> Dict[str, torch.Tensor]:
     """Draw a named workload, optionally at a reduced B or T (same recipe, same seed)."""
     return draw(case.B if B is None else B, case.T if T is None else T, case.H, case.N,

@@ -388,6 +388,48 @@ def bench_options(lib7, dev, B, T, H, steps, *, native, group_norm, decode_steps
     return out
 
 
+def bench_backward(lib7, dev, B, T, H, steps=5):
+    """The training pair on the same shapes: the checkpointing forward (scan with a saved state every
+    64 tokens) and the backward (float32 gradients of r, w, k, v, a, b and the initial state).
+    Reports ms per call and tokens/s; the backward is bound by its per-token CUDA-core work."""
+    case = wi.CASES[WORKLOAD]
+    d = wi.draw(B, T, H, seed=case.seed, s0_std=case.s0_std)
+    gr = wi.draw_grads(B, T, H, seed=case.seed + 2)
+    dd = {n: d[n].to(dev) for n in OPS}
+    s0 = d["s0"].to(dev)
+    dy, ds = gr["dy"].to(dev), gr["ds_out"].to(dev)
+    y = torch.empty_like(dd["r"])
+    s_out = torch.empty_like(s0)
+    states = torch.empty((B, H, lib7.n_checkpoints(T), N, N), dtype=torch.float32, device=dev)
+    g = [torch.empty((B, T, H, N), dtype=torch.float32, device=dev) for _ in range(6)]
+    ds_in = torch.empty_like(s0)
+    stream = torch.cuda.current_stream(dev)
+
+    def fwd():
+        lib7.rwkv7_wkv_prefill_save_bf16(*[dd[n] for n in OPS], s0, y, s_out, states, stream)
+
+    def bwd():
+        lib7.rwkv7_wkv_backward_bf16(*[dd[n] for n in OPS], states, dy, ds, *g, ds_in, stream)
+
+    out = {}
+    for name, fn in (("forward_save", fwd), ("backward", bwd)):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / steps
+        out[name] = {"ms": ms, "tokens_per_s": B * T / (ms / 1e3)}
+    assert lib7.rwkv7_get_last_error() == 0
+    out["workload"] = WORKLOAD
+    out["outputs"] = "float32 dr, dw, dk, dv, da, db [B,T,H,64] and ds_in; dy bf16, ds_out float32"
+    return out
+
+
 def run_ours(args):
     world, rank, local = dist_setup()
     dev = torch.device("cuda", local)
@@ -498,6 +540,10 @@ def run_ours(args):
                   for key, nat, gn in (("model_native", True, False), ("group_norm", False, True),
                                        ("model_native_group_norm", True, True))}
 
+    train = None
+    if not args.no_backward and args.path == "auto":
+        train = bench_backward(lib7, dev, B, T, H)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
         T_s = min(T, args.ref_tokens)
@@ -522,6 +568,7 @@ def run_ours(args):
         "cpu_baseline": cpu,
         "decode": decode,
         "options": native,
+        "training": train,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -544,6 +591,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-native", action="store_true",
                     help="skip the option entry points' lines (model-native inputs, GroupNorm epilogue)")
+    ap.add_argument("--no-backward", action="store_true", help="skip the training (forward-save + backward) line")
     ap.add_argument("--decode-steps", type=int, default=1024)
     ap.add_argument("--decode-layers", type=int, default=24, help="distinct decode states rotated over")
     ap.add_argument("--no-e2e", action="store_true")

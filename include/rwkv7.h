@@ -213,16 +213,16 @@ RWKV7_API rwkv7_status rwkv7_wkv_decode_ext_bf16(int B, int H, int N, const uint
  *   g = G b_t;  dw_t[j] = sum_i G[i][j] S[i][j];  da_t = S^T g;  G <- G diag(w_t) + g a_t^T,
  * and ds_in = G at the start.
  *
- * rwkv7_wkv_prefill_save_bf16: rwkv7_wkv_prefill_bf16 (sequential scan) that also writes the state
- *   before every 64th token: states float32 [B, H, ceil(T/64), 64, 64] (device, 16-byte aligned,
- *   caller-owned; states[b,h,c] = the state before token 64c, so states[b,h,0] = s_in or zeros).
+ * rwkv7_wkv_prefill_save_bf16: rwkv7_wkv_prefill_bf16_path that also writes the state before every
+ *   64th token: states float32 [B, H, ceil(T/64), 64, 64] (device, 16-byte aligned, caller-owned;
+ *   states[b,h,c] = the state before token 64c, so states[b,h,0] = s_in or zeros).
  * rwkv7_wkv_backward_bf16: r, w, k, v, a, b, dy bf16 [B,T,H,64] (the forward's operands and dL/dy);
  *   states from the forward above; ds_out float32 [B,H,64,64] or NULL (zero).  Outputs float32
  *   [B,T,H,64]: dr, dw, dk, dv, da, db (all required; dr, dw, dk, da, db are zeroed on the stream
  *   and accumulated, so they must not alias each other or an input); ds_in float32 [B,H,64,64] or
  *   NULL.  Dense batches only (no cu_seqlens).  Same status codes as the other entry points; the
  *   library allocates nothing. */
-RWKV7_API rwkv7_status rwkv7_wkv_prefill_save_bf16(int B, int T, int H, int N, const uint16_t *r,
+RWKV7_API rwkv7_status rwkv7_wkv_prefill_save_bf16(int path, int B, int T, int H, int N, const uint16_t *r,
                                                    const uint16_t *w, const uint16_t *k, const uint16_t *v,
                                                    const uint16_t *a, const uint16_t *b, const float *s_in,
                                                    uint16_t *y, float *s_out, float *states,

@@ -89,7 +89,7 @@ def load_library() -> ctypes.CDLL:
         ("rwkv7_wkv_decode_fused_bf16", [ci, ci, ci] + [vp] * 6 + [vp, vp, vp]),
         ("rwkv7_wkv_prefill_ext_bf16", [ci, ci, ci, ci, ci] + [vp] * 6 + [ctypes.POINTER(Options), vp, vp, vp, vp]),
         ("rwkv7_wkv_decode_ext_bf16", [ci, ci, ci] + [vp] * 6 + [ctypes.POINTER(Options), vp, vp, vp]),
-        ("rwkv7_wkv_prefill_save_bf16", [ci, ci, ci, ci] + [vp] * 6 + [vp, vp, vp, vp, vp]),
+        ("rwkv7_wkv_prefill_save_bf16", [ci, ci, ci, ci, ci] + [vp] * 6 + [vp, vp, vp, vp, vp]),
         ("rwkv7_wkv_backward_bf16", [ci, ci, ci, ci] + [vp] * 6 + [vp, vp, vp] + [vp] * 7 + [vp]),
     ):
         fn = getattr(lib, name)
@@ -271,17 +271,18 @@ def n_checkpoints(T: int) -> int:
     return (int(T) + 63) // 64
 
 
-def rwkv7_wkv_prefill_save_bf16(r, w, k, v, a, b, s_in, y, s_out, states, stream=None) -> None:
-    """bf16 prefill (sequential scan) that also writes ``states`` float32 ``[B, H, ceil(T/64), 64, 64]``,
-    the state before every 64th token, for ``rwkv7_wkv_backward_bf16``."""
+def rwkv7_wkv_prefill_save_bf16(r, w, k, v, a, b, s_in, y, s_out, states, stream=None, *,
+                                path: int = RWKV7_PATH_AUTO) -> None:
+    """bf16 prefill that also writes ``states`` float32 ``[B, H, ceil(T/64), 64, 64]``, the state before
+    every 64th token, for ``rwkv7_wkv_backward_bf16``."""
     B, T, H, N = r.shape
     for nm, t in (("r", r), ("w", w), ("k", k), ("v", v), ("a", a), ("b", b), ("y", y)):
         _check(t, nm, torch.bfloat16, (B, T, H, N))
     _check(s_in, "s_in", torch.float32, (B, H, N, N), allow_none=True)
     _check(s_out, "s_out", torch.float32, (B, H, N, N))
     _check(states, "states", torch.float32, (B, H, n_checkpoints(T), N, N))
-    _call("rwkv7_wkv_prefill_save_bf16", B, T, H, N, *[_ptr(t) for t in (r, w, k, v, a, b, s_in, y, s_out, states)],
-          _stream(stream))
+    _call("rwkv7_wkv_prefill_save_bf16", int(path), B, T, H, N,
+          *[_ptr(t) for t in (r, w, k, v, a, b, s_in, y, s_out, states)], _stream(stream))
 
 
 def rwkv7_wkv_backward_bf16(r, w, k, v, a, b, states, dy, ds_out, dr, dw, dk, dv, da, db, ds_in,
@@ -377,13 +378,13 @@ def decode_ext_(r, w, k, v, a, b, state, y=None, *, model_native=False, k_k=None
     return y
 
 
-def prefill_save(r, w, k, v, a, b, s_in=None, *, stream=None):
+def prefill_save(r, w, k, v, a, b, s_in=None, *, path: int = RWKV7_PATH_AUTO, stream=None):
     """Allocate and run the checkpointing prefill; returns ``(y, s_out, states)``."""
     B, T, H, N = r.shape
     y = torch.empty_like(r)
     s_out = torch.empty((B, H, N, N), dtype=torch.float32, device=r.device)
     states = torch.empty((B, H, n_checkpoints(T), N, N), dtype=torch.float32, device=r.device)
-    rwkv7_wkv_prefill_save_bf16(r, w, k, v, a, b, s_in, y, s_out, states, stream=stream)
+    rwkv7_wkv_prefill_save_bf16(r, w, k, v, a, b, s_in, y, s_out, states, stream=stream, path=path)
     return y, s_out, states
 
 

@@ -60,11 +60,12 @@ cudaError_t launch_chunk(const uint16_t *r, const uint16_t *w, const uint16_t *k
 // unused; key scale k_k [H,64] float32 or nullptr for ones) and the GroupNorm epilogue on y (ln_w,
 // ln_b [H,64] float32 or nullptr for ones / zeros).  schedule: 0 = chosen from the shape, 1 = one
 // CTA per (b, h), 2 = chunks of every pair spread over all SMs (cudaErrorInvalidValue when the
-// shape does not allow it).
+// shape does not allow it).  states: nullptr, or [B,H,ceil(T/64),64,64] float32 receiving the state
+// before every chunk (dense T only).
 cudaError_t launch_chunk_ext(const uint16_t *r, const uint16_t *w, const uint16_t *k, const uint16_t *v,
                              const uint16_t *a, const uint16_t *b, bool model_native, const float *k_k,
                              bool group_norm, const float *ln_w, const float *ln_b, const float *s_in, uint16_t *y,
                              float *s_out, const int32_t *cu_seqlens, int B, int T, long long total_T, int H,
-                             int schedule, int *err_word, cudaStream_t stream);
+                             int schedule, float *states, int *err_word, cudaStream_t stream);
 
 }  // namespace rwkv7

@@ -172,7 +172,7 @@ rwkv7_status rwkv7_wkv_prefill_ext_bf16(int path, int B, int T, int H, int N, co
   const long long total = static_cast<long long>(B) * T;
   if (use_chunk(path, T))
     return from_cuda(launch_chunk_ext(r, w, k, v, a, b, native, k_k, ln, ln_w, ln_b, s_in, y, s_out, nullptr, B, T,
-                                      total, H, schedule, error_word_ptr(), cs));
+                                      total, H, schedule, nullptr, error_word_ptr(), cs));
   return from_cuda(
       launch_scan_ext(r, w, k, v, a, b, native, k_k, ln, ln_w, ln_b, s_in, y, s_out, nullptr, B, T, total, H, cs));
 }
@@ -208,15 +208,20 @@ rwkv7_status rwkv7_wkv_decode_fused_bf16(int B, int H, int N, const uint16_t *r,
   return rwkv7_wkv_decode_ext_bf16(B, H, N, r, xw, k, v, xa, nullptr, &opt, s_inout, y, stream);
 }
 
-rwkv7_status rwkv7_wkv_prefill_save_bf16(int B, int T, int H, int N, const uint16_t *r, const uint16_t *w,
-                                         const uint16_t *k, const uint16_t *v, const uint16_t *a, const uint16_t *b,
-                                         const float *s_in, uint16_t *y, float *s_out, float *states,
-                                         rwkv7_stream_t stream) {
+rwkv7_status rwkv7_wkv_prefill_save_bf16(int path, int B, int T, int H, int N, const uint16_t *r,
+                                         const uint16_t *w, const uint16_t *k, const uint16_t *v, const uint16_t *a,
+                                         const uint16_t *b, const float *s_in, uint16_t *y, float *s_out,
+                                         float *states, rwkv7_stream_t stream) {
+  if (path != RWKV7_PATH_AUTO && path != RWKV7_PATH_SCAN && path != RWKV7_PATH_CHUNK) return RWKV7_ERR_INVALID;
   const rwkv7_status st = check_prefill(B, T, H, N, r, w, k, v, a, b, s_in, y, s_out);
   if (st != RWKV7_OK) return st;
   if (T > 0 && states == nullptr) return RWKV7_ERR_INVALID;
   if (!aligned16(states)) return RWKV7_ERR_ALIGN;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if (use_chunk(path, T))
+    return from_cuda(launch_chunk_ext(r, w, k, v, a, b, false, nullptr, false, nullptr, nullptr, s_in, y, s_out,
+                                      nullptr, B, T, static_cast<long long>(B) * T, H, 0, states, error_word_ptr(),
+                                      cs));
   return from_cuda(launch_scan_save(r, w, k, v, a, b, s_in, y, s_out, states, B, T, H, cs));
 }
 

@@ -114,6 +114,7 @@ struct Maps {
   // task-parallel schedule: the state a chunk starts from, float32 rows of 64 (box {32, 64},
   // 128-byte swizzle): s_in (or a zero block), and s_out, where every chunk leaves its end state
   CUtensorMap s_in, s_out;
+  CUtensorMap states;  // task-parallel checkpoints: [B*H*nck*64, 64] float32, same box
 };
 
 struct Args {
@@ -132,6 +133,8 @@ struct Args {
   unsigned long long *flags;  // [BH]: (epoch << 32) | chunks of the pair whose end state is in s_out
   unsigned epoch;             // unique per launch: flags of other launches never match
   int s_in_zero;              // the s_in map covers one zero block (row 0 for every pair)
+  float *states;              // nullptr, or [B, H, nck, 64, 64]: the state before every chunk (dense T)
+  int nck;                    // chunks per sequence, ceil(T / 64)
 };
 
 // One unit of work: chunk c of the (b, h) pair bh.
@@ -662,6 +665,11 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
         const int row = static_cast<int>(pt.bh * kN);
         tc::tma_store_2d(&maps.s_out, sB4S, 0, row);
         tc::tma_store_2d(&maps.s_out, sB4S + 64 * 128, 32, row);
+        if (A.states != nullptr && pt.c + 1 < A.nck) {
+          const int crow = static_cast<int>((pt.bh * A.nck + pt.c + 1) * kN);
+          tc::tma_store_2d(&maps.states, sB4S, 0, crow);
+          tc::tma_store_2d(&maps.states, sB4S + 64 * 128, 32, crow);
+        }
         tc::bulk_commit_group();
         tc::bulk_wait_all();
         tc::fence_proxy_async_global();
@@ -849,6 +857,12 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
     const int j0 = 4 * cq, t0 = 4 * tg;
     const uint32_t lane_base = static_cast<uint32_t>(32 * q) << 16;
 
+    if (kTask && A.states != nullptr) {
+      // checkpoint 0 of every pair is its start state
+      for (long long bh = blockIdx.x; bh < A.BH; bh += gridDim.x)
+        for (int e = tid; e < kN * kN; e += kComputeThreads)
+          A.states[bh * A.nck * (kN * kN) + e] = A.s_in ? A.s_in[bh * (kN * kN) + e] : 0.f;
+    }
     if (kTask && A.cu_seqlens != nullptr) {
       // empty sequences of a ragged batch have no task: their end state is the start state
       for (long long bh = blockIdx.x; bh < A.BH; bh += gridDim.x) {
@@ -868,6 +882,11 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
         v[vrow(x)] = A.s_in ? A.s_in[pair * (kN * kN) + static_cast<long long>(32 * ch + x) * kN + j] : 0.f;
       tc::tmem_st32(tmem + lane_base + TM_S + 32 * ch, v);
       store_state_rows_tf32(sB4S, j, ch, v);
+      if (A.states != nullptr) {
+        float *ck = A.states + pair * A.nck * (kN * kN) + static_cast<long long>(32 * ch) * kN + j;
+#pragma unroll
+        for (int x = 0; x < 32; ++x) ck[x * kN] = v[vrow(x)];
+      }
       tc::tmem_st_wait();
     }
     // Wait for the control warp (one thread polls, bounded); false once the CTA aborts.  Thread 0
@@ -966,6 +985,11 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
         for (int x = 0; x < 32; ++x) sv[x] = fmaf(gc_done, sv[x], v[x]);
         tc::tmem_st32(tmem + lane_base + TM_S + 32 * hh, sv);
         store_state_rows_tf32(sB4S, j, hh, sv);
+        if (A.states != nullptr && pt.c + 1 < A.nck) {
+          float *ck = A.states + (pt.bh * A.nck + pt.c + 1) * (kN * kN) + static_cast<long long>(32 * hh) * kN + j;
+#pragma unroll
+          for (int x = 0; x < 32; ++x) ck[x * kN] = sv[vrow(x)];
+        }
       } else {
         // S_C[i][j] = Gamma_C[j] S0[i][j] + X[j][i], rows i = 32 hh + x, in place in B4S (float32),
         // from where the control lane stores it to s_out by TMA
@@ -1386,8 +1410,9 @@ cudaError_t launch_chunk_ext(const uint16_t *r, const uint16_t *w, const uint16_
                              const uint16_t *a, const uint16_t *b, bool model_native, const float *k_k,
                              bool group_norm, const float *ln_w, const float *ln_b, const float *s_in, uint16_t *y,
                              float *s_out, const int32_t *cu_seqlens, int B, int T, long long total_T, int H,
-                             int schedule, int *err_word, cudaStream_t stream) {
+                             int schedule, float *states, int *err_word, cudaStream_t stream) {
   using namespace chunk;
+  if (states != nullptr && cu_seqlens != nullptr) return cudaErrorInvalidValue;
   if (total_T > 0x7fffffffLL || H > 0xffff || B > 65535) return cudaErrorInvalidValue;
   Maps maps;
   const void *ops[6] = {r, w, k, a, model_native ? nullptr : b, v};  // model-native: the b slot is never loaded
@@ -1402,7 +1427,9 @@ cudaError_t launch_chunk_ext(const uint16_t *r, const uint16_t *w, const uint16_
   // total_T, so rows of any length are covered; tasks past a sequence's end are skipped)
   const long long rows = (cu_seqlens == nullptr ? static_cast<long long>(T) : total_T) + C - 1;
   const long long ntasks = (rows / C) * BH;
-  Args args{y, s_in, s_out, cu_seqlens, T, total_T, H, err_word, k_k, ln_w, ln_b, ntasks, BH, nullptr, 0, 0};
+  const int nck = (T + C - 1) / C;
+  Args args{y, s_in, s_out, cu_seqlens, T, total_T, H, err_word, k_k, ln_w, ln_b, ntasks, BH, nullptr, 0, 0,
+            states, nck};
   // The task-parallel schedule pays when one CTA per pair would leave many SMs idle: measured on B200,
   // 48 and 96 pairs ran 1.2x and 1.1x faster, 1 and 2 pairs 1.6x; at 128 pairs and above the pair
   // schedule was as fast or faster.
@@ -1420,7 +1447,9 @@ cudaError_t launch_chunk_ext(const uint16_t *r, const uint16_t *w, const uint16_
     args.epoch = epoch;
     args.s_in_zero = s_in == nullptr ? 1 : 0;
     if (!make_state_map(&maps.s_in, s_in ? static_cast<const void *>(s_in) : ds.zeros, s_in ? BH * kN : kN) ||
-        !make_state_map(&maps.s_out, s_out, BH * kN))
+        !make_state_map(&maps.s_out, s_out, BH * kN) ||
+        !make_state_map(&maps.states, states ? static_cast<const void *>(states) : s_out,
+                        states ? BH * nck * kN : BH * kN))
       return cudaErrorInvalidValue;
   }
   if (model_native && group_norm) return launch_variant<true, true>(maps, args, B, H, task, grid_tasks, stream);
@@ -1434,7 +1463,7 @@ cudaError_t launch_chunk(const uint16_t *r, const uint16_t *w, const uint16_t *k
                          const int32_t *cu_seqlens, int B, int T, long long total_T, int H, int *err_word,
                          cudaStream_t stream) {
   return launch_chunk_ext(r, w, k, v, a, b, false, nullptr, false, nullptr, nullptr, s_in, y, s_out, cu_seqlens, B,
-                          T, total_T, H, 0, err_word, stream);
+                          T, total_T, H, 0, nullptr, err_word, stream);
 }
 
 }  // namespace rwkv7

@@ -6,7 +6,10 @@ float32 accumulation error over the sequence rather than an output rounding: max
 max|oracle|, per output, <= TOL_BWD.  It is stated here from the arithmetic: every gradient is a
 sum over later tokens of float32 products (relative rounding 2^-24 per operation), with the
 recomputed states carrying the same float32 error as the forward scan, which meets 1e-4 on fp32
-operands; 1e-3 leaves an order of magnitude for the longer sums.
+operands; 1e-3 leaves an order of magnitude for the longer sums.  That bar holds for checkpoints
+saved by the sequential scan; checkpoints saved by the chunked (tensor-core) forward carry its
+state error (tf32 products, within the 5e-3 bf16 bar of the forward), which the gradients inherit,
+so those are held to 5e-3.
 """
 
 import numpy as np
@@ -32,12 +35,12 @@ def _cuda():
     assert rk.rwkv7_get_last_error() == 0
 
 
-def _check(d, gr, with_s0=True, with_ds=True, tol=TOL_BWD):
+def _check(d, gr, with_s0=True, with_ds=True, tol=TOL_BWD, path=rk.RWKV7_PATH_SCAN):
     s0 = d["s0"] if with_s0 else None
     ds = gr["ds_out"] if with_ds else None
     go = oracle.wkv7_backward(*oracle_ops(d), s0, gr["dy_f32"], ds)
     dv = to_dev(d)
-    y, s_out, states = rk.prefill_save(*[dv[n] for n in OPS], dv["s0"] if with_s0 else None)
+    y, s_out, states = rk.prefill_save(*[dv[n] for n in OPS], dv["s0"] if with_s0 else None, path=path)
     g = rk.backward(*[dv[n] for n in OPS], states, gr["dy"].cuda(), ds.cuda() if ds is not None else None)
     torch.cuda.synchronize()
     errs = {n: rel_err(g[i], go[i]) for i, n in enumerate(GRADS + ("ds_in",))}
@@ -66,18 +69,31 @@ def test_backward_decay_regimes(z_mean):
     _check(d, gr)
 
 
-def test_saved_states_match_the_oracle_states():
-    # states[b, h, c] is the state before token 64 c: the oracle's end state after 64 c tokens
+# the chunked forward picks its schedule from the shape: 6 pairs run task-parallel, 120 pairs one
+# CTA per pair (fewer than 3/4 of the SMs would be left idle)
+@pytest.mark.parametrize("path,B,H,tol", [(rk.RWKV7_PATH_SCAN, 2, 3, 1e-4), (rk.RWKV7_PATH_CHUNK, 2, 3, 5e-3),
+                                          (rk.RWKV7_PATH_CHUNK, 2, 60, 5e-3)], ids=["scan", "chunk-tasks", "chunk-pair"])
+def test_saved_states_match_the_oracle_states(path, B, H, tol):
+    # states[b, h, c] is the state before token 64 c: the oracle's end state after 64 c tokens; the
+    # forward's own outputs are unchanged by saving
     T = 200
-    d = wi.draw(1, T, 2, seed=840, s0_std=0.1)
+    d = wi.draw(B, T, H, seed=840, s0_std=0.1)
     dv = to_dev(d)
-    _, _, states = rk.prefill_save(*[dv[n] for n in OPS], dv["s0"])
+    y, s_out, states = rk.prefill_save(*[dv[n] for n in OPS], dv["s0"], path=path)
+    y2, s2 = rk.prefill(*[dv[n] for n in OPS], dv["s0"], path=path)
     torch.cuda.synchronize()
+    assert torch.equal(y, y2) and torch.equal(s_out, s2)
     assert torch.equal(states[:, :, 0].cpu(), d["s0"])
     for c in range(1, rk.n_checkpoints(T)):
         sub = [x[:, :64 * c] for x in oracle_ops(d)]
         _, so = oracle.wkv7(*sub, d["s0"])
-        assert rel_err(states[:, :, c], so) <= 1e-4
+        assert rel_err(states[:, :, c], so) <= tol
+
+
+def test_backward_from_chunked_checkpoints():
+    d = wi.draw(2, 300, 3, seed=845, s0_std=0.1)
+    gr = wi.draw_grads(2, 300, 3, seed=846)
+    _check(d, gr, tol=5e-3, path=rk.RWKV7_PATH_CHUNK)
 
 
 def test_empty_sequence_passes_the_state_gradient():
@@ -97,7 +113,7 @@ def test_sampled_pairs_at_the_d768_shape():
     d = wi.draw(B, T, H, seed=860, s0_std=0.1)
     gr = wi.draw_grads(B, T, H, seed=861)
     dv = to_dev(d)
-    _, _, states = rk.prefill_save(*[dv[n] for n in OPS], dv["s0"])
+    _, _, states = rk.prefill_save(*[dv[n] for n in OPS], dv["s0"], path=rk.RWKV7_PATH_SCAN)
     g = rk.backward(*[dv[n] for n in OPS], states, gr["dy"].cuda(), gr["ds_out"].cuda())
     torch.cuda.synchronize()
     for (b, h) in ((0, 0), (5, 11)):

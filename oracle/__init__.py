@@ -230,3 +230,20 @@ def wkv7_backward(r, w, k, v, a, b, s_in, dy, ds_out=None, *, nthreads: Optional
     if st != 0:
         raise RuntimeError(f"oracle backward failed ({st})")
     return tuple(outs) + (ds_in,)
+
+
+def round_bf16(x) -> np.ndarray:
+    """Round float64 values to the nearest bfloat16 value, ties to even (8 significant bits), as float64.
+    For values in bfloat16's normal range (the reduced-precision decode state); zero stays zero."""
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)  # x = m * 2^e with 0.5 <= |m| < 1
+    return np.ldexp(np.rint(m * 256.0), e - 8)  # np.rint: round half to even
+
+
+def decode_step_bf16_state(r, w, k, v, a, b, s):
+    """One decode step with a bfloat16 state: the recurrence in float64 (``wkv7`` with T = 1) from the
+    state values ``s`` ``[B, H, N, N]``, then the new state rounded to bfloat16.  Token operands
+    ``[B, H, N]``.  Returns ``(y, s_new)`` as float64."""
+    ops = [_as_np(x, np.float64)[:, None] for x in (r, w, k, v, a, b)]
+    y, s_new = wkv7(*ops, _as_np(s, np.float64), precision="f64")
+    return y[:, 0], round_bf16(s_new)

@@ -255,22 +255,24 @@ def run_reference(args):
 
 # ---- our arm ------------------------------------------------------------------------------------------
 
-def bench_decode(lib7, dev, steps_target: int = 1024, layers: int = 24):
-    """Decode steps/s at B=256, H=16, rotating over `layers` distinct states."""
+def bench_decode(lib7, dev, steps_target: int = 1024, layers: int = 24, bf16_state: bool = False):
+    """Decode steps/s at B=256, H=16, rotating over `layers` distinct states (bf16_state: the
+    reduced-precision variant whose state is stored as bfloat16)."""
     case = wi.CASES["decode_l24_d1024_b256_1024steps"]
     B, H = case.B, case.H
     ntok = 8
     d = wi.draw(B, ntok, H, seed=case.seed, dtype="bf16")
     toks = [{n: d[n][:, t].contiguous().to(dev) for n in OPS} for t in range(ntok)]
-    states = torch.zeros(layers, B, H, N, N, device=dev)
+    states = torch.zeros(layers, B, H, N, N, device=dev, dtype=torch.bfloat16 if bf16_state else torch.float32)
     ys = [torch.empty(B, H, N, dtype=torch.bfloat16, device=dev) for _ in range(layers)]
     per_graph = layers * 4
+    step_fn = lib7.rwkv7_wkv_decode_bf16_bf16state if bf16_state else lib7.rwkv7_wkv_decode_bf16
 
     def one_pass(start):
         for i in range(per_graph):
             L = (start + i) % layers
             tk = toks[(start + i) % ntok]
-            lib7.rwkv7_wkv_decode_bf16(*[tk[n] for n in OPS], states[L], ys[L])
+            step_fn(*[tk[n] for n in OPS], states[L], ys[L])
 
     s = torch.cuda.Stream(device=dev)
     s.wait_stream(torch.cuda.current_stream())
@@ -293,9 +295,10 @@ def bench_decode(lib7, dev, steps_target: int = 1024, layers: int = 24):
     ms = e0.elapsed_time(e1)
     nsteps = reps * per_graph
     step_s = ms / 1e3 / nsteps
-    byts = decode_bytes(B, H)
+    byts = decode_bytes(B, H) - (B * H * 2 * N * N * 2 if bf16_state else 0)
     return {"workload": "decode_l24_d1024_b256", "B": B, "H": H, "steps": nsteps, "layer_states": layers,
-            "state_bytes_total": layers * B * H * N * N * 4, "steps_per_s": 1.0 / step_s,
+            "state_dtype": "bf16" if bf16_state else "f32",
+            "state_bytes_total": layers * B * H * N * N * (2 if bf16_state else 4), "steps_per_s": 1.0 / step_s,
             "tokens_per_s": B / step_s, "us_per_step": step_s * 1e6, "bytes_per_step": byts,
             "achieved_gbs": byts / step_s / 1e9, "launches": nsteps}
 
@@ -532,6 +535,11 @@ def run_ours(args):
         decode = bench_decode(lib7, dev, steps_target=args.decode_steps, layers=args.decode_layers)
         decode["frac"] = decode["achieved_gbs"] / peaks["hbm_gbs"]
         assert lib7.rwkv7_get_last_error() == 0
+        d16 = bench_decode(lib7, dev, steps_target=args.decode_steps, layers=args.decode_layers, bf16_state=True)
+        d16["frac"] = d16["achieved_gbs"] / peaks["hbm_gbs"]
+        assert lib7.rwkv7_get_last_error() == 0
+        decode["bf16_state"] = {k: d16[k] for k in ("state_dtype", "steps_per_s", "tokens_per_s", "us_per_step",
+                                                    "bytes_per_step", "achieved_gbs", "frac")}
 
     native = None
     if not args.no_native and args.path == "auto":

@@ -203,6 +203,20 @@ RWKV7_API rwkv7_status rwkv7_wkv_decode_ext_bf16(int B, int H, int N, const uint
                                                  const uint16_t *b, const rwkv7_options *opt, float *s_inout,
                                                  uint16_t *y, rwkv7_stream_t stream);
 
+/* ---- reduced-precision decode state ------------------------------------------------------
+ *
+ * The decode step with the state kept in HBM as bfloat16 [B, H, 64, 64] (s_inout: bf16 bit patterns,
+ * updated in place): each step widens it to float32, applies the update above in float32, writes y,
+ * and rounds the new state to nearest-even bf16.  Half the state traffic of rwkv7_wkv_decode_bf16.
+ * The pages keep the state in fp32 because w can be very close to 1 (RWKV-LM README copy,
+ * oa0.com/c/1004164); with a bf16 state every step adds up to 2^-8 relative rounding to it, so
+ * long decodes drift from the float32-state result: an opt-in for memory-bound serving, not the
+ * default.  Other arguments, errors and ownership as for rwkv7_wkv_decode_bf16. */
+RWKV7_API rwkv7_status rwkv7_wkv_decode_bf16_bf16state(int B, int H, int N, const uint16_t *r, const uint16_t *w,
+                                                       const uint16_t *k, const uint16_t *v, const uint16_t *a,
+                                                       const uint16_t *b, uint16_t *s_inout, uint16_t *y,
+                                                       rwkv7_stream_t stream);
+
 /* ---- training: forward with checkpoints, and the backward ----------------------------------
  *
  * The gradients of a loss L with respect to the operands and the initial state, given dL/dy

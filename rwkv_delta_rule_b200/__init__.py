@@ -28,7 +28,7 @@ __all__ = [
     "rwkv7_wkv_decode", "rwkv7_wkv_decode_bf16", "rwkv7_wkv_prefill_fused_bf16", "rwkv7_wkv_decode_fused_bf16",
     "rwkv7_wkv_prefill_ext_bf16", "rwkv7_wkv_decode_ext_bf16", "Options",
     "rwkv7_status_string", "rwkv7_get_last_error", "rwkv7_version",
-    "rwkv7_wkv_prefill_save_bf16", "rwkv7_wkv_backward_bf16",
+    "rwkv7_wkv_prefill_save_bf16", "rwkv7_wkv_backward_bf16", "rwkv7_wkv_decode_bf16_bf16state",
     "prefill", "decode_", "prefill_model_native", "decode_model_native_", "prefill_ext", "decode_ext_",
     "prefill_save", "backward", "EXPORTED_SYMBOLS",
 ]
@@ -42,7 +42,7 @@ EXPORTED_SYMBOLS = (
     "rwkv7_wkv_prefill", "rwkv7_wkv_prefill_bf16", "rwkv7_wkv_prefill_bf16_path", "rwkv7_wkv_prefill_varlen_bf16",
     "rwkv7_wkv_decode", "rwkv7_wkv_decode_bf16", "rwkv7_wkv_prefill_fused_bf16", "rwkv7_wkv_decode_fused_bf16",
     "rwkv7_wkv_prefill_ext_bf16", "rwkv7_wkv_decode_ext_bf16",
-    "rwkv7_wkv_prefill_save_bf16", "rwkv7_wkv_backward_bf16",
+    "rwkv7_wkv_prefill_save_bf16", "rwkv7_wkv_backward_bf16", "rwkv7_wkv_decode_bf16_bf16state",
     "rwkv7_status_string", "rwkv7_get_last_error", "rwkv7_version",
 )
 
@@ -91,6 +91,7 @@ def load_library() -> ctypes.CDLL:
         ("rwkv7_wkv_decode_ext_bf16", [ci, ci, ci] + [vp] * 6 + [ctypes.POINTER(Options), vp, vp, vp]),
         ("rwkv7_wkv_prefill_save_bf16", [ci, ci, ci, ci, ci] + [vp] * 6 + [vp, vp, vp, vp, vp]),
         ("rwkv7_wkv_backward_bf16", [ci, ci, ci, ci] + [vp] * 6 + [vp, vp, vp] + [vp] * 7 + [vp]),
+        ("rwkv7_wkv_decode_bf16_bf16state", [ci, ci, ci] + [vp] * 6 + [vp, vp, vp]),
     ):
         fn = getattr(lib, name)
         fn.argtypes = args
@@ -264,6 +265,16 @@ def rwkv7_wkv_decode_ext_bf16(r, w, k, v, a, b, s_inout, y, *, model_native=Fals
     opt = _options(model_native, k_k, group_norm, ln_w, ln_b, H, N)
     _call("rwkv7_wkv_decode_ext_bf16", B, H, N, *[_ptr(t) for t in (r, w, k, v, a, None if model_native else b)],
           ctypes.byref(opt), _ptr(s_inout), _ptr(y), _stream(stream))
+
+
+def rwkv7_wkv_decode_bf16_bf16state(r, w, k, v, a, b, s_inout, y, stream=None) -> None:
+    """One decode step with the state stored as bfloat16 ``[B, H, 64, 64]`` (updated in place)."""
+    B, H, N = r.shape
+    for nm, t in (("r", r), ("w", w), ("k", k), ("v", v), ("a", a), ("b", b), ("y", y)):
+        _check(t, nm, torch.bfloat16, (B, H, N))
+    _check(s_inout, "s_inout", torch.bfloat16, (B, H, N, N))
+    _call("rwkv7_wkv_decode_bf16_bf16state", B, H, N, *[_ptr(t) for t in (r, w, k, v, a, b, s_inout, y)],
+          _stream(stream))
 
 
 def n_checkpoints(T: int) -> int:

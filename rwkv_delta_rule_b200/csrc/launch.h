@@ -41,6 +41,12 @@ template <typename TIn>
 cudaError_t launch_decode(const TIn *r, const TIn *w, const TIn *k, const TIn *v, const TIn *a, const TIn *b,
                           float *s, TIn *y, int B, int H, cudaStream_t stream);
 
+// The bf16 step with the state stored as bf16 [B,H,64,64] (widened to float32 for the update, rounded
+// to nearest-even on store).
+cudaError_t launch_decode_bf16state(const uint16_t *r, const uint16_t *w, const uint16_t *k, const uint16_t *v,
+                                    const uint16_t *a, const uint16_t *b, uint16_t *s, uint16_t *y, int B, int H,
+                                    cudaStream_t stream);
+
 // The bf16 step with the optional parts: model-native inputs (w, a slots hold x_w, x_a; b unused;
 // key scale k_k [H,64] float32 or nullptr for ones) and the GroupNorm epilogue on y (ln_w, ln_b
 // [H,64] float32 or nullptr for ones / zeros).

@@ -208,6 +208,16 @@ rwkv7_status rwkv7_wkv_decode_fused_bf16(int B, int H, int N, const uint16_t *r,
   return rwkv7_wkv_decode_ext_bf16(B, H, N, r, xw, k, v, xa, nullptr, &opt, s_inout, y, stream);
 }
 
+rwkv7_status rwkv7_wkv_decode_bf16_bf16state(int B, int H, int N, const uint16_t *r, const uint16_t *w,
+                                             const uint16_t *k, const uint16_t *v, const uint16_t *a,
+                                             const uint16_t *b, uint16_t *s_inout, uint16_t *y,
+                                             rwkv7_stream_t stream) {
+  if (N != kN) return RWKV7_ERR_UNSUPPORTED;
+  if (B <= 0 || H <= 0 || !none_null(r, w, k, v, a, b, s_inout, y)) return RWKV7_ERR_INVALID;
+  if (!all_aligned(r, w, k, v, a, b, s_inout, y)) return RWKV7_ERR_ALIGN;
+  return from_cuda(launch_decode_bf16state(r, w, k, v, a, b, s_inout, y, B, H, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 rwkv7_status rwkv7_wkv_prefill_save_bf16(int path, int B, int T, int H, int N, const uint16_t *r,
                                          const uint16_t *w, const uint16_t *k, const uint16_t *v, const uint16_t *a,
                                          const uint16_t *b, const float *s_in, uint16_t *y, float *s_out,

@@ -12,6 +12,11 @@
 // and a warp covers two whole 256-byte rows per load.  The row sums S a and
 // S r are finished with four xor-shuffles inside each 16-lane half-warp.
 //
+// The reduced-precision variant keeps the state in HBM as bfloat16 (8 KiB per head instead of 16):
+// it is widened to float32 on load, updated in float32, and rounded to nearest-even bf16 on store.
+// The pages keep the state in fp32 (RWKV-LM README copy, oa0.com/c/1004164), so this is an
+// opt-in trade of state precision for half the decode traffic, not the default.
+//
 // The fused variant takes model-native inputs (decay pre-activation x_w in place of w, the key k,
 // the learning-rate pre-activation x_a in place of a, and the per-channel key scale k_k) and forms
 // w, a = -kk and b = kk * sigmoid(x_a) in-kernel; the key norm is one more 16-lane reduction.
@@ -20,9 +25,9 @@
 
 namespace rwkv7 {
 
-template <typename TIn> struct DecodeArgs {
+template <typename TIn, typename TS = float> struct DecodeArgs {
   const TIn *r, *w, *k, *v, *a, *b;  // fused: w = x_w, a = x_a, b unused
-  float *s;
+  TS *s;
   TIn *y;
   const float *k_k;  // fused: [H, 64] key scale, nullptr = ones
   int H;
@@ -31,9 +36,23 @@ template <typename TIn> struct DecodeArgs {
 
 __device__ __forceinline__ float4 ld_state(const float *p) { return *reinterpret_cast<const float4 *>(p); }
 __device__ __forceinline__ void st_state(float *p, float4 x) { *reinterpret_cast<float4 *>(p) = x; }
+// bf16 state: four elements in 8 bytes
+__device__ __forceinline__ float4 ld_state(const uint16_t *p) {
+  const uint2 u = *reinterpret_cast<const uint2 *>(p);
+  return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u), __uint_as_float(u.y << 16),
+                     __uint_as_float(u.y & 0xffff0000u));
+}
+__device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;\n" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+__device__ __forceinline__ void st_state(uint16_t *p, float4 x) {
+  *reinterpret_cast<uint2 *>(p) = make_uint2(bf16x2_rn(x.x, x.y), bf16x2_rn(x.z, x.w));
+}
 
-template <typename TIn, bool kFused, bool kLN>
-__global__ void __launch_bounds__(256) wkv7_decode_kernel(DecodeArgs<TIn> A) {
+template <typename TIn, bool kFused, bool kLN, typename TS = float>
+__global__ void __launch_bounds__(256) wkv7_decode_kernel(DecodeArgs<TIn, TS> A) {
   const long long pair = blockIdx.x;  // b * H + h
   const int tid = threadIdx.x;
   // fused: the decay and the learning rate of each of the 64 channels, computed once per CTA (the 16
@@ -46,7 +65,7 @@ __global__ void __launch_bounds__(256) wkv7_decode_kernel(DecodeArgs<TIn> A) {
   }
   const int c4 = tid & 15;   // column chunk: columns 4*c4 .. 4*c4+3
   const int rg = tid >> 4;   // rows rg + 16*m
-  float *S = A.s + pair * (kN * kN);
+  TS *S = A.s + pair * (kN * kN);
 
   float4 st[4];
 #pragma unroll
@@ -182,6 +201,82 @@ cudaError_t launch_decode_ext(const uint16_t *r, const uint16_t *w, const uint16
   else if (model_native) wkv7_decode_kernel<uint16_t, true, false><<<g, 256, 0, stream>>>(A);
   else if (group_norm) wkv7_decode_kernel<uint16_t, false, true><<<g, 256, 0, stream>>>(A);
   else wkv7_decode_kernel<uint16_t, false, false><<<g, 256, 0, stream>>>(A);
+  return cudaGetLastError();
+}
+
+// The bf16-state step: one CTA of 128 threads per (b, h); thread t holds columns 8*(t%8) .. +7 of
+// rows t/8 + 16*m (m = 0..3), so each state load and store is 16 bytes (8 bf16) as in the float32
+// kernel, and the row sums are three xor-shuffles inside 8 lanes.
+__device__ __forceinline__ void unpack8(uint4 u, float (&o)[8]) {
+  o[0] = __uint_as_float(u.x << 16);
+  o[1] = __uint_as_float(u.x & 0xffff0000u);
+  o[2] = __uint_as_float(u.y << 16);
+  o[3] = __uint_as_float(u.y & 0xffff0000u);
+  o[4] = __uint_as_float(u.z << 16);
+  o[5] = __uint_as_float(u.z & 0xffff0000u);
+  o[6] = __uint_as_float(u.w << 16);
+  o[7] = __uint_as_float(u.w & 0xffff0000u);
+}
+
+__global__ void __launch_bounds__(128) wkv7_decode_bf16state_kernel(DecodeArgs<uint16_t, uint16_t> A) {
+  const long long pair = blockIdx.x;
+  const int tid = threadIdx.x;
+  const int c8 = tid & 7, rg = tid >> 3;
+  uint16_t *S = A.s + pair * (kN * kN);
+  uint4 raw[4];
+#pragma unroll
+  for (int m = 0; m < 4; ++m) raw[m] = *reinterpret_cast<const uint4 *>(S + (rg + 16 * m) * kN + 8 * c8);
+  const long long vb = pair * kN;
+  float ww[8], kk[8], aa[8], bb[8], rr[8];
+  unpack8(*reinterpret_cast<const uint4 *>(A.w + vb + 8 * c8), ww);
+  unpack8(*reinterpret_cast<const uint4 *>(A.k + vb + 8 * c8), kk);
+  unpack8(*reinterpret_cast<const uint4 *>(A.a + vb + 8 * c8), aa);
+  unpack8(*reinterpret_cast<const uint4 *>(A.b + vb + 8 * c8), bb);
+  unpack8(*reinterpret_cast<const uint4 *>(A.r + vb + 8 * c8), rr);
+  float st[4][8], sa[4], yv[4], vv[4];
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    unpack8(raw[m], st[m]);
+    float p = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) p = fmaf(st[m][e], aa[e], p);
+    sa[m] = p;
+    vv[m] = bf16_bits_to_float(A.v[vb + rg + 16 * m]);
+  }
+#pragma unroll
+  for (int off = 4; off >= 1; off >>= 1)
+#pragma unroll
+    for (int m = 0; m < 4; ++m) sa[m] += __shfl_xor_sync(0xffffffffu, sa[m], off);
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    float p = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      st[m][e] = fmaf(st[m][e], ww[e], fmaf(sa[m], bb[e], vv[m] * kk[e]));
+      p = fmaf(st[m][e], rr[e], p);
+    }
+    yv[m] = p;
+    *reinterpret_cast<uint4 *>(S + (rg + 16 * m) * kN + 8 * c8) =
+        make_uint4(bf16x2_rn(st[m][0], st[m][1]), bf16x2_rn(st[m][2], st[m][3]), bf16x2_rn(st[m][4], st[m][5]),
+                   bf16x2_rn(st[m][6], st[m][7]));
+  }
+#pragma unroll
+  for (int off = 4; off >= 1; off >>= 1)
+#pragma unroll
+    for (int m = 0; m < 4; ++m) yv[m] += __shfl_xor_sync(0xffffffffu, yv[m], off);
+  if (c8 == 0) {
+#pragma unroll
+    for (int m = 0; m < 4; ++m) Elem<uint16_t>::store(A.y + vb + rg + 16 * m, yv[m]);
+  }
+}
+
+cudaError_t launch_decode_bf16state(const uint16_t *r, const uint16_t *w, const uint16_t *k, const uint16_t *v,
+                                    const uint16_t *a, const uint16_t *b, uint16_t *s, uint16_t *y, int B, int H,
+                                    cudaStream_t stream) {
+  DecodeArgs<uint16_t, uint16_t> A{r, w, k, v, a, b, s, y, nullptr, H, nullptr, nullptr};
+  const long long pairs = static_cast<long long>(B) * H;
+  if (pairs > 0x7fffffffLL) return cudaErrorInvalidValue;
+  wkv7_decode_bf16state_kernel<<<static_cast<unsigned>(pairs), 128, 0, stream>>>(A);
   return cudaGetLastError();
 }
 

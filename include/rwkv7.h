@@ -207,7 +207,8 @@ RWKV7_API rwkv7_status rwkv7_wkv_decode_ext_bf16(int B, int H, int N, const uint
  *
  * The decode step with the state kept in HBM as bfloat16 [B, H, 64, 64] (s_inout: bf16 bit patterns,
  * updated in place): each step widens it to float32, applies the update above in float32, writes y,
- * and rounds the new state to nearest-even bf16.  Half the state traffic of rwkv7_wkv_decode_bf16.
+ * and rounds the new state to nearest-even bf16.  Half the state traffic of rwkv7_wkv_decode_bf16
+ * (quantised states are explored in the RWKV-8 preview, trdm.cn/news/547794).
  * The pages keep the state in fp32 because w can be very close to 1 (RWKV-LM README copy,
  * oa0.com/c/1004164); with a bf16 state every step adds up to 2^-8 relative rounding to it, so
  * long decodes drift from the float32-state result: an opt-in for memory-bound serving, not the

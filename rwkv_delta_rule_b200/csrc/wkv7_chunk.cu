@@ -604,11 +604,12 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
   uint64_t *bar_m3 = bars + 4;     // c -> w: MMA3 done
   uint64_t *bar_b2 = bars + 5;     // w -> c: B2, A2 and the D2 initial value written
   uint64_t *bar_m2 = bars + 6;     // c -> c: MMA2 done
-  uint64_t *bar_st = bars + 7;     // w -> c: D4 read out (and, one pair per CTA, the state S0^T in B4S)
+  uint64_t *bar_st = bars + 7;     // w -> c: D4 read out and D2 set up (one pair per CTA: the state S0^T in B4S)
   uint64_t *bar_m4 = bars + 8;     // c -> w: MMA4 done
   uint64_t *bar_sin = bars + 9;    // task-parallel: the start state landed in B4S (tx bytes)
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_MISC + 80);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 84);
+  uint64_t *bar_sout = bars + 10;  // task-parallel: w -> c, the end state is in B4S (one arrival per hi-lane warp)
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_MISC + 88);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 92);
   float *GCs = reinterpret_cast<float *>(smem + OFF_MISC + MISC_GC);  // [2][64]
   float *pre4 = reinterpret_cast<float *>(smem + OFF_PRE);
   float *kkw = reinterpret_cast<float *>(smem + OFF_KX);        // [64] key scale of the head being prepared
@@ -628,7 +629,7 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
   constexpr int kCtrlWarp = kComputeThreads / 32;
 
   if (tid == 0) {
-    for (int i = 0; i < 10; ++i) tc::mbar_init(bars + i, i == 3 ? 2 : 1);  // b3: both compute groups
+    for (int i = 0; i < 11; ++i) tc::mbar_init(bars + i, i == 3 ? 2 : i == 10 ? 4 : 1);  // b3: both compute groups
     tc::fence_mbar_init();
     *abort_flag = 0;
     task_slot[0].n = task_slot[1].n = -1;
@@ -656,8 +657,8 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
       }
       // parity of the last issued phase of each barrier, or -1 when nothing was issued
       int last_tma = -1, last_m1 = -1, last_m3 = -1, last_m2 = -1, last_m4 = -1, last_sin = -1;
-      // Stores the end state of a finished task, which the compute warps left in B4S before arriving
-      // on bar_st (this lane's wait on it acquired their writes), to s_out by TMA; once the store has
+      // Stores the end state of a finished task, which the hi-lane warps left in B4S before arriving
+      // on bar_sout (this lane's wait on it acquired their writes), to s_out by TMA; once the store has
       // completed, raises the pair's flag (async-proxy fence, GPU-scope fence, then the flag word).
       // B4S is free again when this returns.  Done here, where the lane idles until the window ends.
       auto publish = [&](const Task &pt) {
@@ -765,9 +766,12 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
         }
         if (kTask) {
           // the start state, into B4S once the previous read-out is done with it
-          // the previous task's end state out of B4S, then (if already there) this task's start state in
-          if (!wait_or_abort(bar_st, ph, abort_flag)) { fail(); break; }
-          if (it > 0) publish(pt);
+          // the previous task's end state out of B4S (as soon as its read-out has written it), then (if
+          // already there) this task's start state in
+          if (it > 0) {
+            if (!wait_or_abort(bar_sout, (it - 1) & 1, abort_flag)) { fail(); break; }
+            publish(pt);
+          }
           state_issued = false;
           if (t.c == 0 || chain_ready(A.flags + t.bh, A.epoch, t.c)) load_state(t, ph);
         }
@@ -834,7 +838,7 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
         }
       }
       // the last task's flag, once the compute warps' final read-out has stored its end state
-      if (kTask && nit > 0 && !*abort_flag && wait_or_abort(bar_st, nit & 1, abort_flag)) publish(pt);
+      if (kTask && nit > 0 && !*abort_flag && wait_or_abort(bar_sout, (nit - 1) & 1, abort_flag)) publish(pt);
       // every copy and MMA issued here lands before the CTA exits (bounded; phases that
       // already completed return at once)
       if (last_tma >= 0) (void)tc::mbar_wait_bounded(bar_tma, last_tma, kMaxPolls);
@@ -892,7 +896,7 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
     // Wait for the control warp (one thread polls, bounded); false once the CTA aborts.  Thread 0
     // publishes the decision in a slot chosen by the call parity before the barrier, so every compute
     // thread reads the same value (a slot is rewritten only two calls later, after all have read it).
-    volatile int *decision = reinterpret_cast<volatile int *>(smem + OFF_MISC + 88);  // [2]
+    volatile int *decision = reinterpret_cast<volatile int *>(smem + OFF_MISC + 96);  // [2]
     uint32_t ncalls = 0;
     auto wait_ctrl = [&](uint64_t *bar, uint32_t parity) -> bool {
       const uint32_t slot = ncalls++ & 1u;
@@ -907,7 +911,7 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
       return decision[slot] != 0;
     };
     // The same for warps 4-7 alone (thread 128 polls; slots of their own).
-    volatile int *decision_hi = reinterpret_cast<volatile int *>(smem + OFF_MISC + 96);  // [2]
+    volatile int *decision_hi = reinterpret_cast<volatile int *>(smem + OFF_MISC + 104);  // [2]
     uint32_t ncalls_hi = 0;
     auto wait_group_hi = [&](uint64_t *bar, uint32_t parity) -> bool {
       const uint32_t slot = ncalls_hi++ & 1u;
@@ -934,7 +938,8 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
     // S_C^T = diag(Gamma_C) S0^T + X (lanes 64..127); each warp takes the column half ch.  D4 column
     // vr(i) holds value channel i.  One pair per CTA: the new state goes to TMEM and, as tf32, to B4S
     // for the next MMA4.  Task-parallel: S0 is the float32 copy in B4S and the new state replaces it
-    // there; after the next bar_st arrival the control lane stores it to s_out and raises the flag.
+    // there; on the hi-lane warps' bar_sout arrival the control lane stores it to s_out and raises the
+    // flag.
     float gc_done = 1.f;  // Gamma_C[j] of the chunk whose MMA4 is in flight (hi lanes)
     auto readout = [&](const Task &pt, uint32_t par) {
       const int hh = ch;
@@ -1000,6 +1005,8 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
         for (int x = 0; x < 32; ++x) s0[x] = *reinterpret_cast<const float *>(cp.p[x & 7] + x * 128);
 #pragma unroll
         for (int x = 0; x < 32; ++x) *reinterpret_cast<float *>(cp.p[x & 7] + x * 128) = fmaf(gc_done, s0[x], v[x]);
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(bar_sout);
       }
     };
 
@@ -1262,11 +1269,6 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
     if (have_prev && ok && wait_ctrl(bar_m4, (it - 1) & 1)) {
       tc::tc_fence_after();
       readout(pt, (it - 1) & 1);
-      if (kTask) {
-        // the last task's end state is stored: hand the flag to the control lane
-        compute_sync();
-        if (tid == 0) tc::mbar_arrive(bar_st);
-      }
     }
     if (!kTask && hi_lanes) {
       const long long pair = static_cast<long long>(blockIdx.y) * A.H + blockIdx.x;

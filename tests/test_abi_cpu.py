@@ -98,6 +98,26 @@ def test_varlen_rejects(cdll):
     assert cdll.rwkv7_wkv_prefill_varlen_bf16(0, 2, 10, 8, 1, 32, FAKE, *base) == 5
 
 
+def test_training_and_bf16_state_entry_points_reject(cdll):
+    ops = [FAKE] * 6
+    # rwkv7_wkv_prefill_save_bf16(path, B, T, H, N, ops, s_in, y, s_out, states, stream)
+    assert cdll.rwkv7_wkv_prefill_save_bf16(0, 1, 4, 1, 32, *ops, None, FAKE, FAKE, FAKE, None) == 5
+    assert cdll.rwkv7_wkv_prefill_save_bf16(0, 1, 4, 1, 64, *ops, None, FAKE, FAKE, None, None) == 1
+    assert cdll.rwkv7_wkv_prefill_save_bf16(0, 1, 4, 1, 64, *ops, None, FAKE, FAKE, MIS, None) == 2
+    assert cdll.rwkv7_wkv_prefill_save_bf16(5, 1, 4, 1, 64, *ops, None, FAKE, FAKE, FAKE, None) == 1
+    # rwkv7_wkv_backward_bf16(B, T, H, N, ops, states, dy, ds_out, dr dw dk dv da db, ds_in, stream)
+    grads = [FAKE] * 6
+    assert cdll.rwkv7_wkv_backward_bf16(1, 4, 1, 16, *ops, FAKE, FAKE, None, *grads, None, None) == 5
+    assert cdll.rwkv7_wkv_backward_bf16(0, 4, 1, 64, *ops, FAKE, FAKE, None, *grads, None, None) == 1
+    assert cdll.rwkv7_wkv_backward_bf16(1, 4, 1, 64, *ops, None, FAKE, None, *grads, None, None) == 1
+    assert cdll.rwkv7_wkv_backward_bf16(1, 4, 1, 64, *ops, FAKE, FAKE, None, *grads[:5], None, None, None) == 1
+    assert cdll.rwkv7_wkv_backward_bf16(1, 4, 1, 64, *ops, FAKE, FAKE, MIS, *grads, None, None) == 2
+    # rwkv7_wkv_decode_bf16_bf16state(B, H, N, ops, s_inout, y, stream)
+    assert cdll.rwkv7_wkv_decode_bf16_bf16state(1, 1, 64, *ops, None, FAKE, None) == 1
+    assert cdll.rwkv7_wkv_decode_bf16_bf16state(1, 1, 64, *ops, MIS, FAKE, None) == 2
+    assert cdll.rwkv7_wkv_decode_bf16_bf16state(1, 1, 48, *ops, FAKE, FAKE, None) == 5
+
+
 def test_binding_rejects_cpu_tensors():
     import torch
 

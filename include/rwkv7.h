@@ -179,7 +179,8 @@ RWKV7_API rwkv7_status rwkv7_wkv_decode_fused_bf16(int B, int H, int N, const ui
  *                         takes its start state from s_out, where the previous chunk of the same
  *                         (b, h) left it (flags in library-owned device memory order the two).
  *                         Needs B*H <= 65536 (else RWKV7_ERR_CUDA).  Up to 4 such launches may
- *                         run at once on a device.
+ *                         run at once on a device; the launch can be captured in a CUDA graph
+ *                         and replayed (every launch leaves the flags zeroed unless it fails).
  */
 typedef struct rwkv7_options {
   int model_native;

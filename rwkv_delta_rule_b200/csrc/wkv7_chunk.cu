@@ -143,6 +143,7 @@ struct Task {
   long long bh;    // b * H + h
   long long tok0;  // token row of the chunk's first token in the [tokens, H, 64] operands
   int c, h, Lc;    // chunk of the sequence, head, tokens in the chunk (1..64)
+  bool last;       // the sequence's last chunk
 };
 
 // Fills t with chunk c of pair bh (task index n); false for a chunk past the end of its sequence.
@@ -165,6 +166,7 @@ __device__ __forceinline__ bool task_set(const Args &A, long long n, int c, long
   t.h = h;
   t.tok0 = sb.start + static_cast<long long>(c) * C;
   t.Lc = min(C, sb.len - c * C);
+  t.last = static_cast<long long>(c + 1) * C >= sb.len;
   return true;
 }
 // One pair per CTA: its chunks in order.
@@ -674,8 +676,12 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
         tc::bulk_commit_group();
         tc::bulk_wait_all();
         tc::fence_proxy_async_global();
-        const unsigned long long val = (static_cast<unsigned long long>(A.epoch) << 32) |
-                                       static_cast<unsigned>(pt.c + 1);
+        // a sequence's last chunk has no successor, and every chunk of the pair has read the flag by
+        // now: it goes back to zero, so every launch leaves the flags as it found them (a CUDA graph
+        // replays a launch with the same epoch)
+        const unsigned long long val = pt.last ? 0ull
+                                               : ((static_cast<unsigned long long>(A.epoch) << 32) |
+                                                  static_cast<unsigned>(pt.c + 1));
         asm volatile("fence.acq_rel.gpu;\n\tst.relaxed.gpu.global.u64 [%0], %1;\n" ::"l"(A.flags + pt.bh), "l"(val)
                      : "memory");
       };

@@ -121,3 +121,60 @@ def test_schedule_value_is_checked():
     dv = to_dev(d)
     with pytest.raises(rk.Rwkv7Error):
         rk.prefill_ext(*[dv[n] for n in OPS], None, path=rk.RWKV7_PATH_CHUNK, schedule=3)
+
+
+def test_graph_replays_start_from_fresh_flags():
+    # a captured launch replays with the same epoch: each replay must still order its own chunks
+    B, T, H = 2, 300, 3
+    static = {n: torch.empty((B, T, H, 64), dtype=torch.bfloat16, device="cuda") for n in OPS}
+    s0 = torch.empty((B, H, 64, 64), device="cuda")
+    y = torch.empty((B, T, H, 64), dtype=torch.bfloat16, device="cuda")
+    s_out = torch.empty_like(s0)
+
+    def run():
+        rk.rwkv7_wkv_prefill_ext_bf16(rk.RWKV7_PATH_CHUNK, *[static[n] for n in OPS], s0, y, s_out,
+                                      schedule=rk.RWKV7_SCHED_TASKS)
+
+    d = wi.draw(B, T, H, seed=780, s0_std=0.1)
+    for n in OPS:
+        static[n].copy_(d[n])
+    s0.copy_(d["s0"])
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        run()
+    torch.cuda.current_stream().wait_stream(side)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        run()
+    for seed in (781, 782, 783):
+        d = wi.draw(B, T, H, seed=seed, s0_std=0.1)
+        for n in OPS:
+            static[n].copy_(d[n])
+        s0.copy_(d["s0"])
+        g.replay()
+        torch.cuda.synchronize()
+        yo, so = oracle.wkv7(*oracle_ops(d), d["s0"])
+        assert rel_err(y, yo) <= TOL_BF16, seed
+        assert rel_err(s_out, so) <= TOL_BF16, seed
+
+
+def test_concurrent_launches_on_separate_streams():
+    # launches running at once take different flag slots
+    runs = []
+    for i, seed in enumerate((790, 791, 792)):
+        d = wi.draw(2, 260, 3, seed=seed, s0_std=0.1)
+        dv = to_dev(d)
+        y = torch.empty_like(dv["r"])
+        s_out = torch.empty_like(dv["s0"])
+        runs.append((d, dv, y, s_out, torch.cuda.Stream()))
+    torch.cuda.synchronize()
+    for d, dv, y, s_out, st in runs:
+        with torch.cuda.stream(st):
+            rk.rwkv7_wkv_prefill_ext_bf16(rk.RWKV7_PATH_CHUNK, *[dv[n] for n in OPS], dv["s0"], y, s_out,
+                                          schedule=rk.RWKV7_SCHED_TASKS)
+    torch.cuda.synchronize()
+    for d, dv, y, s_out, st in runs:
+        yo, so = oracle.wkv7(*oracle_ops(d), d["s0"])
+        assert rel_err(y, yo) <= TOL_BF16
+        assert rel_err(s_out, so) <= TOL_BF16

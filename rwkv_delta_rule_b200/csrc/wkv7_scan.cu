@@ -6,13 +6,13 @@
 //
 // Rows of S are independent of each other: row i needs only its own values,
 // v_t[i] and the shared vectors r, w, k, a, b.  So a (b, h) pair is split
-// into 64 / ROWS row groups, one CTA each, and every row is spread over a quad
-// of 4 lanes that hold 16 columns each.  The two per-token dot products (S a
-// and S r) are finished with two xor-shuffles inside the quad.
+// into 64 / ROWS row groups, one CTA each, and every row is spread over
+// LANES lanes (8 in the 16-row variants: 8 columns each).  The two per-token
+// dot products (S a and S r) are finished with xor-shuffles inside those lanes.
 //
-// Column ownership inside a quad: lane q holds the 4-column chunks starting
-// at 16*m + 4*q (m = 0..3), so one vector read by a quad touches 4 adjacent
-// chunks of shared memory and 8 quads read the same addresses (broadcast).
+// Column ownership: lane q holds the 4-column chunks starting at 4*q + 4*LANES*m,
+// so the lanes of a row read adjacent chunks of shared memory and the rows of a
+// warp read the same addresses (broadcast).
 //
 // Per-token operands are staged into shared memory in tiles of TT tokens
 // with cp.async, double-buffered, and y is staged per tile and written back
@@ -20,7 +20,7 @@
 //
 // The fused variant takes model-native inputs (x_w in place of w, x_a in place of a, no b, and the
 // per-channel key scale k_k) and forms w, a = -kk and b = kk * sigmoid(x_a) per token in registers;
-// the key norm is two more xor-shuffles inside the quad, which holds all 64 columns of a row.
+// the key norm is one more reduction over the row's lanes, which hold all 64 columns of the row.
 //
 // The group-norm variant (x070 ln_x on y) runs one CTA of 256 threads per (b, h) (ROWS = 64), so
 // every token's 64 channels of y meet in one tile of shared memory; one warp per token normalises
@@ -30,8 +30,13 @@
 
 namespace rwkv7 {
 
-template <typename TIn, int ROWS> struct ScanCfg {
-  static constexpr int kThreads = ROWS * 4;
+// Lanes per state row in the 16-row variants (the 64-row group-norm variant keeps 4).  Measured on
+// B200 at B8 T4096 H12 (bf16 / float32 / model-native operands): 4 lanes 2.11 / 2.34 / 4.15 ms,
+// 8 lanes 1.53 / 1.98 / 3.21 ms, 16 lanes 1.70 / 1.90 / 3.30 ms.
+constexpr int kScanLanes = 8;
+
+template <typename TIn, int ROWS, int LANES = 4> struct ScanCfg {
+  static constexpr int kThreads = ROWS * LANES;
   static constexpr int kTT = sizeof(TIn) == 2 ? 32 : 16;  // tokens per tile (24+ KB per buffer)
   static constexpr int kVecElems = 5 * kN;                 // r, w, k, a, b
   static constexpr int kTokElems = kVecElems + ROWS;       // + this CTA's slice of v
@@ -59,10 +64,10 @@ template <typename TIn> struct ScanArgs {
   float *states;  // nullptr, or [B, H, ceil(T / 64), 64, 64]: the state before every 64th token (dense T)
 };
 
-template <typename TIn, int ROWS, bool kFused>
+template <typename TIn, int ROWS, bool kFused, int LANES>
 __device__ __forceinline__ void scan_load_tile(const ScanArgs<TIn> &A, TIn *buf, long long tok0, int ntok, int h,
                                                int row0) {
-  using C = ScanCfg<TIn, ROWS>;
+  using C = ScanCfg<TIn, ROWS, LANES>;
   const int total = ntok * C::kChunksTok;
   for (int c = threadIdx.x; c < total; c += C::kThreads) {
     const int tt = c / C::kChunksTok, cc = c - tt * C::kChunksTok;
@@ -80,10 +85,15 @@ __device__ __forceinline__ void scan_load_tile(const ScanArgs<TIn> &A, TIn *buf,
   }
 }
 
-template <typename TIn, int ROWS, bool kFused, bool kLN>
-__global__ void __launch_bounds__(ScanCfg<TIn, ROWS>::kThreads) wkv7_scan_kernel(ScanArgs<TIn> A) {
+// LANES lanes share a state row: lane q holds the 4-column chunks starting at 4 q + 4 LANES m
+// (m = 0 .. 16 / LANES - 1), CPL = 64 / LANES columns in all.
+template <typename TIn, int ROWS, bool kFused, bool kLN, int LANES = 4>
+__global__ void __launch_bounds__(ScanCfg<TIn, ROWS, LANES>::kThreads) wkv7_scan_kernel(ScanArgs<TIn> A) {
   static_assert(!kLN || ROWS == kN, "the group-norm epilogue needs all 64 rows in one CTA");
-  using C = ScanCfg<TIn, ROWS>;
+  static_assert(LANES == 4 || LANES == 8 || LANES == 16, "4, 8 or 16 lanes per row");
+  using C = ScanCfg<TIn, ROWS, LANES>;
+  constexpr int CPL = kN / LANES;  // columns per lane
+  constexpr int NM = CPL / 4;      // 4-column chunks per lane
   constexpr int kSplits = kN / ROWS;
   extern __shared__ __align__(16) uint8_t smem_raw[];
   TIn *bufs = reinterpret_cast<TIn *>(smem_raw);
@@ -96,27 +106,27 @@ __global__ void __launch_bounds__(ScanCfg<TIn, ROWS>::kThreads) wkv7_scan_kernel
   if (sb.len < 0) return;
 
   const int tid = threadIdx.x;
-  const int rloc = tid >> 2, q = tid & 3;
+  const int rloc = tid / LANES, q = tid % LANES;
   const int row = row0 + rloc;
   const long long sbase = (static_cast<long long>(bidx) * A.H + h) * (kN * kN) + static_cast<long long>(row) * kN;
 
-  float s[16];
+  float s[CPL];
 #pragma unroll
-  for (int m = 0; m < 4; ++m) {
+  for (int m = 0; m < NM; ++m) {
     float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (A.s_in != nullptr) x = *reinterpret_cast<const float4 *>(A.s_in + sbase + 16 * m + 4 * q);
+    if (A.s_in != nullptr) x = *reinterpret_cast<const float4 *>(A.s_in + sbase + 4 * LANES * m + 4 * q);
     s[4 * m + 0] = x.x; s[4 * m + 1] = x.y; s[4 * m + 2] = x.z; s[4 * m + 3] = x.w;
   }
 
-  float kkr[16];  // fused: key scale of this thread's 16 columns
+  float kkr[CPL];  // fused: key scale of this thread's columns
 #pragma unroll
-  for (int m = 0; m < 4; ++m)
+  for (int m = 0; m < NM; ++m)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) kkr[4 * m + e] = (kFused && A.k_k) ? A.k_k[h * kN + 16 * m + 4 * q + e] : 1.f;
+    for (int e = 0; e < 4; ++e) kkr[4 * m + e] = (kFused && A.k_k) ? A.k_k[h * kN + 4 * LANES * m + 4 * q + e] : 1.f;
 
   const int ntiles = (sb.len + C::kTT - 1) / C::kTT;
   if (ntiles > 0) {
-    scan_load_tile<TIn, ROWS, kFused>(A, bufs, sb.start, min(C::kTT, sb.len), h, row0);
+    scan_load_tile<TIn, ROWS, kFused, LANES>(A, bufs, sb.start, min(C::kTT, sb.len), h, row0);
     cp_async_commit();
   }
   for (int tile = 0; tile < ntiles; ++tile) {
@@ -124,7 +134,7 @@ __global__ void __launch_bounds__(ScanCfg<TIn, ROWS>::kThreads) wkv7_scan_kernel
     const int ntok = min(C::kTT, sb.len - t0);
     if (tile + 1 < ntiles) {
       const int t1 = t0 + C::kTT;
-      scan_load_tile<TIn, ROWS, kFused>(A, bufs + ((tile + 1) & 1) * C::kBufElems, sb.start + t1,
+      scan_load_tile<TIn, ROWS, kFused, LANES>(A, bufs + ((tile + 1) & 1) * C::kBufElems, sb.start + t1,
                                         min(C::kTT, sb.len - t1), h, row0);
       cp_async_commit();
       cp_async_wait<1>();
@@ -137,10 +147,10 @@ __global__ void __launch_bounds__(ScanCfg<TIn, ROWS>::kThreads) wkv7_scan_kernel
 #pragma unroll 2
     for (int tt = 0; tt < ntok; ++tt) {
       const TIn *tok = buf + tt * C::kTokElems;
-      float rr[16], ww[16], kk[16], aa[16], bb[16];
+      float rr[CPL], ww[CPL], kk[CPL], aa[CPL], bb[CPL];
 #pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const int col = 16 * m + 4 * q;
+      for (int m = 0; m < NM; ++m) {
+        const int col = 4 * LANES * m + 4 * q;
         Elem<TIn>::load4(tok + 0 * kN + col, rr + 4 * m);
         Elem<TIn>::load4(tok + 1 * kN + col, ww + 4 * m);
         Elem<TIn>::load4(tok + 2 * kN + col, kk + 4 * m);
@@ -154,20 +164,20 @@ __global__ void __launch_bounds__(ScanCfg<TIn, ROWS>::kThreads) wkv7_scan_kernel
         float *ck = A.states + ((static_cast<long long>(bidx) * A.H + h) * nck + ((t0 + tt) >> 6)) * (kN * kN) +
                     static_cast<long long>(row) * kN;
 #pragma unroll
-        for (int m = 0; m < 4; ++m)
-          *reinterpret_cast<float4 *>(ck + 16 * m + 4 * q) =
+        for (int m = 0; m < NM; ++m)
+          *reinterpret_cast<float4 *>(ck + 4 * LANES * m + 4 * q) =
               make_float4(s[4 * m + 0], s[4 * m + 1], s[4 * m + 2], s[4 * m + 3]);
       }
       if (kFused) {
-        // x070 prologue: kk = normalise(k * k_k) over the quad's 64 columns, a = -kk, b = kk * rate
+        // x070 prologue: kk = normalise(k * k_k) over the row's 64 columns, a = -kk, b = kk * rate
         float ss = 0.f;
 #pragma unroll
-        for (int c = 0; c < 16; ++c) ss = fmaf(kk[c] * kkr[c], kk[c] * kkr[c], ss);
-        ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-        ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+        for (int c = 0; c < CPL; ++c) ss = fmaf(kk[c] * kkr[c], kk[c] * kkr[c], ss);
+#pragma unroll
+        for (int off = 1; off < LANES; off <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
         const float inv = x070_inv_norm(ss);
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
+        for (int c = 0; c < CPL; ++c) {
           const float kkv = kk[c] * kkr[c] * inv;
           bb[c] = kkv * x070_sigmoid(aa[c]);
           aa[c] = -kkv;
@@ -175,35 +185,35 @@ __global__ void __launch_bounds__(ScanCfg<TIn, ROWS>::kThreads) wkv7_scan_kernel
         }
       }
 
-      // sa = S a (state before this token), four partial sums then the quad
+      // sa = S a (state before this token), four partial sums, then the row's lanes
       float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
 #pragma unroll
-      for (int c = 0; c < 16; c += 4) {
+      for (int c = 0; c < CPL; c += 4) {
         p0 = fmaf(s[c + 0], aa[c + 0], p0);
         p1 = fmaf(s[c + 1], aa[c + 1], p1);
         p2 = fmaf(s[c + 2], aa[c + 2], p2);
         p3 = fmaf(s[c + 3], aa[c + 3], p3);
       }
       float sa = (p0 + p1) + (p2 + p3);
-      sa += __shfl_xor_sync(0xffffffffu, sa, 1);
-      sa += __shfl_xor_sync(0xffffffffu, sa, 2);
+#pragma unroll
+      for (int off = 1; off < LANES; off <<= 1) sa += __shfl_xor_sync(0xffffffffu, sa, off);
 
       // S = S diag(w) + sa b^T + v k^T
 #pragma unroll
-      for (int c = 0; c < 16; ++c) s[c] = fmaf(s[c], ww[c], fmaf(sa, bb[c], vi * kk[c]));
+      for (int c = 0; c < CPL; ++c) s[c] = fmaf(s[c], ww[c], fmaf(sa, bb[c], vi * kk[c]));
 
       // y = S r (updated state)
       p0 = p1 = p2 = p3 = 0.f;
 #pragma unroll
-      for (int c = 0; c < 16; c += 4) {
+      for (int c = 0; c < CPL; c += 4) {
         p0 = fmaf(s[c + 0], rr[c + 0], p0);
         p1 = fmaf(s[c + 1], rr[c + 1], p1);
         p2 = fmaf(s[c + 2], rr[c + 2], p2);
         p3 = fmaf(s[c + 3], rr[c + 3], p3);
       }
       float y = (p0 + p1) + (p2 + p3);
-      y += __shfl_xor_sync(0xffffffffu, y, 1);
-      y += __shfl_xor_sync(0xffffffffu, y, 2);
+#pragma unroll
+      for (int off = 1; off < LANES; off <<= 1) y += __shfl_xor_sync(0xffffffffu, y, off);
       if (q == 0) ys[tt * ROWS + rloc] = y;
     }
     __syncthreads();
@@ -233,15 +243,15 @@ __global__ void __launch_bounds__(ScanCfg<TIn, ROWS>::kThreads) wkv7_scan_kernel
   }
 
 #pragma unroll
-  for (int m = 0; m < 4; ++m)
-    *reinterpret_cast<float4 *>(A.s_out + sbase + 16 * m + 4 * q) =
+  for (int m = 0; m < NM; ++m)
+    *reinterpret_cast<float4 *>(A.s_out + sbase + 4 * LANES * m + 4 * q) =
         make_float4(s[4 * m + 0], s[4 * m + 1], s[4 * m + 2], s[4 * m + 3]);
 }
 
-template <typename TIn, int ROWS, bool kFused = false, bool kLN = false>
+template <typename TIn, int ROWS, bool kFused = false, bool kLN = false, int LANES = kScanLanes>
 static cudaError_t launch_scan_rows(const ScanArgs<TIn> &A, int B, cudaStream_t stream) {
-  using C = ScanCfg<TIn, ROWS>;
-  auto kern = wkv7_scan_kernel<TIn, ROWS, kFused, kLN>;
+  using C = ScanCfg<TIn, ROWS, LANES>;
+  auto kern = wkv7_scan_kernel<TIn, ROWS, kFused, kLN, LANES>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(C::kSmemBytes));
   if (e != cudaSuccess) return e;
@@ -272,9 +282,9 @@ cudaError_t launch_scan_ext(const uint16_t *r, const uint16_t *w, const uint16_t
                             float *s_out, const int32_t *cu_seqlens, int B, int T, long long total_T, int H,
                             cudaStream_t stream) {
   ScanArgs<uint16_t> A{r, w, k, v, a, b, s_in, y, s_out, cu_seqlens, T, total_T, H, k_k, ln_w, ln_b, nullptr};
-  if (model_native && group_norm) return launch_scan_rows<uint16_t, 64, true, true>(A, B, stream);
+  if (model_native && group_norm) return launch_scan_rows<uint16_t, 64, true, true, 4>(A, B, stream);
   if (model_native) return launch_scan_rows<uint16_t, 16, true, false>(A, B, stream);
-  if (group_norm) return launch_scan_rows<uint16_t, 64, false, true>(A, B, stream);
+  if (group_norm) return launch_scan_rows<uint16_t, 64, false, true, 4>(A, B, stream);
   return launch_scan_rows<uint16_t, 16, false, false>(A, B, stream);
 }
 

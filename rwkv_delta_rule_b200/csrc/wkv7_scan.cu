@@ -7,7 +7,7 @@
 // Rows of S are independent of each other: row i needs only its own values,
 // v_t[i] and the shared vectors r, w, k, a, b.  So a (b, h) pair is split
 // into 64 / ROWS row groups, one CTA each, and every row is spread over
-// LANES lanes (8 in the 16-row variants: 8 columns each).  The two per-token
+// LANES lanes (8: 8 columns each).  The two per-token
 // dot products (S a and S r) are finished with xor-shuffles inside those lanes.
 //
 // Column ownership: lane q holds the 4-column chunks starting at 4*q + 4*LANES*m,
@@ -30,7 +30,8 @@
 
 namespace rwkv7 {
 
-// Lanes per state row in the 16-row variants (the 64-row group-norm variant keeps 4).  Measured on
+// Lanes per state row (every variant: the per-row arithmetic, and so the state, is then the same with
+// and without the group-norm epilogue, whose variant holds all 64 rows in one CTA).  Measured on
 // B200 at B8 T4096 H12 (bf16 / float32 / model-native operands): 4 lanes 2.11 / 2.34 / 4.15 ms,
 // 8 lanes 1.53 / 1.98 / 3.21 ms, 16 lanes 1.70 / 1.90 / 3.30 ms.
 constexpr int kScanLanes = 8;
@@ -282,9 +283,9 @@ cudaError_t launch_scan_ext(const uint16_t *r, const uint16_t *w, const uint16_t
                             float *s_out, const int32_t *cu_seqlens, int B, int T, long long total_T, int H,
                             cudaStream_t stream) {
   ScanArgs<uint16_t> A{r, w, k, v, a, b, s_in, y, s_out, cu_seqlens, T, total_T, H, k_k, ln_w, ln_b, nullptr};
-  if (model_native && group_norm) return launch_scan_rows<uint16_t, 64, true, true, 4>(A, B, stream);
+  if (model_native && group_norm) return launch_scan_rows<uint16_t, 64, true, true>(A, B, stream);
   if (model_native) return launch_scan_rows<uint16_t, 16, true, false>(A, B, stream);
-  if (group_norm) return launch_scan_rows<uint16_t, 64, false, true, 4>(A, B, stream);
+  if (group_norm) return launch_scan_rows<uint16_t, 64, false, true>(A, B, stream);
   return launch_scan_rows<uint16_t, 16, false, false>(A, B, stream);
 }
 

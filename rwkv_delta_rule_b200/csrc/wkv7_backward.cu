@@ -14,8 +14,9 @@
 // of S only meet the shared vectors.  A (b, h) pair is split into 4 row groups of 16 rows, one CTA
 // of 128 threads each; every row is spread over 8 lanes holding 8 columns.  Row sums (sa, g, dv)
 // are three xor-shuffles inside the 8 lanes; the column sums (dr, dk, db, dw, da: sums over rows)
-// are two xor-shuffles over the 4 rows of a warp, then the 4 warps' partials in shared memory, then
-// float32 atomics across the 4 row groups (the caller zeroes those outputs first).
+// go through shared memory: every thread stores its 5 x 8 partial products, then 80 threads each
+// sum one 4-column group over the 16 rows (float4 loads), then float32 atomics across the 4 row
+// groups (the caller zeroes those outputs first).
 //
 // The states S before every token are recomputed from the checkpoints the forward saved (the state
 // before every 64th token): per 64-token chunk, walked from the last, a forward pass from the
@@ -40,7 +41,7 @@ enum { V_R = 0, V_W = 1, V_K = 2, V_A = 3, V_B = 4, V_V = 5, V_DY = 6 };
 
 constexpr size_t kSmemSubck = sizeof(float) * kSubs * kRows * kN;   // 32 KB
 constexpr size_t kSmemStage = sizeof(uint16_t) * 2 * kStageElems;   // 14 KB
-constexpr size_t kSmemPart = sizeof(float) * 2 * 4 * 5 * kN;         // 10 KB
+constexpr size_t kSmemPart = sizeof(float) * kRows * 5 * kN;         // 20 KB: [row][5][64] partials
 constexpr size_t kSmemBytes = kSmemSubck + kSmemStage + kSmemPart;
 
 struct Args {
@@ -136,7 +137,7 @@ __global__ void __launch_bounds__(kThreads) wkv7_backward_kernel(const Args A) {
   const int h = blockIdx.x / kSplits;
   const int row0 = (blockIdx.x - h * kSplits) * kRows;
   const int bidx = blockIdx.y;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x;
   const int rl = tid >> 3, c0 = 8 * (tid & 7);
   const int row = row0 + rl;  // state row (value channel) of this thread
   const int T = A.T;
@@ -145,7 +146,6 @@ __global__ void __launch_bounds__(kThreads) wkv7_backward_kernel(const Args A) {
   const int nck = (T + kChunk - 1) / kChunk;
   const int nsub_last = nck > 0 ? (T - (nck - 1) * kChunk + kSub - 1) / kSub : 0;
   const int nvisits = nck > 0 ? 2 * nsub_last + 2 * kSubs * (nck - 1) : 0;
-  float *grads[5] = {A.dr, A.dk, A.db, A.dw, A.da};
 
   float G[8];  // dL/dS for this thread's columns of its row
 #pragma unroll
@@ -154,7 +154,6 @@ __global__ void __launch_bounds__(kThreads) wkv7_backward_kernel(const Args A) {
 #pragma unroll
   for (int e = 0; e < 8; ++e) S[e] = 0.f;
 
-  int pbuf = 0;
   if (nvisits > 0) {
     const Visit v0 = visit_at(0, nck, nsub_last);
     const int t0 = v0.c * kChunk + v0.s * kSub;
@@ -234,34 +233,35 @@ __global__ void __launch_bounds__(kThreads) wkv7_backward_kernel(const Args A) {
           p[4][e] = St[u][e] * g;
           G[e] = fmaf(G[e], w8[e], g * a8[e]);
         }
-        // sums over the warp's 4 rows (lane bits 3, 4)
-#pragma unroll
-        for (int q = 0; q < 5; ++q)
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            p[q][e] += __shfl_xor_sync(0xffffffffu, p[q][e], 8);
-            p[q][e] += __shfl_xor_sync(0xffffffffu, p[q][e], 16);
-          }
+        // column sums: every thread's partials to shared memory, then one 4-column group over the
+        // 16 rows per thread (80 of them), then the 4 row groups through float32 atomics
         const long long tok = tok_base + t0 + u;
-        float *pw = part + pbuf * (4 * 5 * kN);
-        if (lane < 8) {
 #pragma unroll
-          for (int q = 0; q < 5; ++q) {
-            float *dst = pw + (warp * 5 + q) * kN + c0;
-            *reinterpret_cast<float4 *>(dst) = make_float4(p[q][0], p[q][1], p[q][2], p[q][3]);
-            *reinterpret_cast<float4 *>(dst + 4) = make_float4(p[q][4], p[q][5], p[q][6], p[q][7]);
-          }
+        for (int q = 0; q < 5; ++q) {
+          float *dst = part + (rl * 5 + q) * kN + c0;
+          *reinterpret_cast<float4 *>(dst) = make_float4(p[q][0], p[q][1], p[q][2], p[q][3]);
+          *reinterpret_cast<float4 *>(dst + 4) = make_float4(p[q][4], p[q][5], p[q][6], p[q][7]);
         }
         if ((tid & 7) == 0) A.dv[(tok * A.H + h) * kN + row] = dv;
         __syncthreads();
-        // the 4 warps' partials, then the 4 row groups through float32 atomics
-        for (int idx = tid; idx < 5 * kN; idx += kThreads) {
-          const int q = idx >> 6, col = idx & 63;
-          const float sum = (pw[(0 * 5 + q) * kN + col] + pw[(1 * 5 + q) * kN + col]) +
-                            (pw[(2 * 5 + q) * kN + col] + pw[(3 * 5 + q) * kN + col]);
-          atomicAdd(grads[q] + (tok * A.H + h) * kN + col, sum);
+        if (tid < 5 * kN / 4) {
+          const int q = tid >> 4, c4 = (tid & 15) * 4;
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int rr = 0; rr < kRows; ++rr) {
+            const float4 x = *reinterpret_cast<const float4 *>(part + (rr * 5 + q) * kN + c4);
+            acc.x += x.x;
+            acc.y += x.y;
+            acc.z += x.z;
+            acc.w += x.w;
+          }
+          float *g = (q == 0 ? A.dr : q == 1 ? A.dk : q == 2 ? A.db : q == 3 ? A.dw : A.da) + (tok * A.H + h) * kN + c4;
+          atomicAdd(g + 0, acc.x);
+          atomicAdd(g + 1, acc.y);
+          atomicAdd(g + 2, acc.z);
+          atomicAdd(g + 3, acc.w);
         }
-        pbuf ^= 1;
+        __syncthreads();  // the partials are rewritten by the next token
       }
     }
     // every thread is done with this staging buffer before the next visit refills it

@@ -230,12 +230,9 @@ __device__ __forceinline__ uint32_t mnmaj_bf16(uint32_t krows, uint32_t k, uint3
 // channels 4l + e (l = 0..7) of V, then write 8 rows with distinct (row % 8), i.e. 8 distinct bank
 // groups of the 128-byte swizzle.  Only the order of D4's columns changes; the read-out undoes it.
 __host__ __device__ constexpr int vrow(int i) { return (i & 32) | ((i & 3) << 3) | ((i >> 2) & 7); }
-// The row order in use: vrow when the state lives in TMEM (one pair per CTA); the natural order in the
-// task-parallel schedule, where the state arrives by TMA as rows of s_out.
-template <bool kTask>
-__host__ __device__ constexpr int vr(int i) {
-  return kTask ? i : vrow(i);
-}
+// In the task-parallel schedule the state arrives in B4S by TMA in this row order too: its tensor map
+// views each 64 x 64 state as (key, l, e, half, pair) with strides (1, 4, 1, 32, 64) rows, so the box
+// lands channel 32 half + 4 l + e in row 32 half + 8 e + l.
 
 // One column k = j of 32 consecutive rows row0 .. row0+31 (row0 a multiple of
 // 8) of a K-major 32-bit operand whose K-atoms hold `rows` rows: row row0 + x
@@ -434,7 +431,7 @@ __device__ __forceinline__ void invert_unit_lower(const float *Ls, float *Ts, fl
 // operand.  Each thread covers 4 channels x 8 tokens; tokens at or past Lcn act as w = 1, b = k =
 // v = 0.  Gamma_t is formed as pre4[g] times the running product inside the group, exactly as the
 // operand construction of R~ and A~ forms it.  Warps 4-7 synchronise among themselves.
-template <bool kFused, bool kTask>
+template <bool kFused>
 __device__ __forceinline__ void prep_next(const uint8_t *smem, uint8_t *sA1, uint8_t *sB1, uint8_t *sB4Vn, float *pre4,
                                           float *GCn, float *wtot, const float *kkw, float *invn, int tid4, int Lcn) {
   const int lane = tid4 & 31, wq = tid4 >> 5;
@@ -550,7 +547,7 @@ __device__ __forceinline__ void prep_next(const uint8_t *smem, uint8_t *sA1, uin
     st_tf32x4(b1r + tc::sw128(t, chunk), bb[0] * ig[0], bb[1] * ig[1], bb[2] * ig[2], bb[3] * ig[3]);
     st_tf32x4(b1r + tc::sw128(64 + t, chunk), kk[0] * ig[0], kk[1] * ig[1], kk[2] * ig[2], kk[3] * ig[3]);
   }
-  // V^T (row = vr(value channel), K = token); bf16 values are exact in tf32
+  // V^T (row = vrow(value channel), K = token); bf16 values are exact in tf32
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     float vv[4][4];
@@ -565,7 +562,7 @@ __device__ __forceinline__ void prep_next(const uint8_t *smem, uint8_t *sA1, uin
     }
 #pragma unroll
     for (int e = 0; e < 4; ++e)
-      *reinterpret_cast<uint4 *>(sB4Vn + kmaj_tf32(64, vr<kTask>(j0 + e), tb + 4 * h)) =
+      *reinterpret_cast<uint4 *>(sB4Vn + kmaj_tf32(64, vrow(j0 + e), tb + 4 * h)) =
           make_uint4(__float_as_uint(vv[0][e]), __float_as_uint(vv[1][e]), __float_as_uint(vv[2][e]),
                      __float_as_uint(vv[3][e]));
   }
@@ -665,13 +662,13 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
       // B4S is free again when this returns.  Done here, where the lane idles until the window ends.
       auto publish = [&](const Task &pt) {
         tc::fence_proxy_async_smem();
-        const int row = static_cast<int>(pt.bh * kN);
-        tc::tma_store_2d(&maps.s_out, sB4S, 0, row);
-        tc::tma_store_2d(&maps.s_out, sB4S + 64 * 128, 32, row);
+        const int blk = static_cast<int>(pt.bh);
+        tc::tma_store_5d(&maps.s_out, sB4S, 0, 0, 0, 0, blk);
+        tc::tma_store_5d(&maps.s_out, sB4S + 64 * 128, 32, 0, 0, 0, blk);
         if (A.states != nullptr && pt.c + 1 < A.nck) {
-          const int crow = static_cast<int>((pt.bh * A.nck + pt.c + 1) * kN);
-          tc::tma_store_2d(&maps.states, sB4S, 0, crow);
-          tc::tma_store_2d(&maps.states, sB4S + 64 * 128, 32, crow);
+          const int cblk = static_cast<int>(pt.bh * A.nck + pt.c + 1);
+          tc::tma_store_5d(&maps.states, sB4S, 0, 0, 0, 0, cblk);
+          tc::tma_store_5d(&maps.states, sB4S + 64 * 128, 32, 0, 0, 0, cblk);
         }
         tc::bulk_commit_group();
         tc::bulk_wait_all();
@@ -690,10 +687,10 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
       bool state_issued = false;
       auto load_state = [&](const Task &t, uint32_t ph) {
         const CUtensorMap *sm = t.c > 0 ? &maps.s_out : &maps.s_in;
-        const int row = (t.c == 0 && A.s_in_zero) ? 0 : static_cast<int>(t.bh * kN);
+        const int blk = (t.c == 0 && A.s_in_zero) ? 0 : static_cast<int>(t.bh);
         tc::mbar_arrive_expect_tx(bar_sin, kN * kN * 4);
-        tc::tma_load_2d(sB4S, sm, bar_sin, 0, row);
-        tc::tma_load_2d(sB4S + 64 * 128, sm, bar_sin, 32, row);
+        tc::tma_load_5d(sB4S, sm, bar_sin, 0, 0, 0, 0, blk);
+        tc::tma_load_5d(sB4S + 64 * 128, sm, bar_sin, 32, 0, 0, 0, blk);
         state_issued = true;
         last_sin = static_cast<int>(ph);
       };
@@ -942,7 +939,7 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
     bool ok = true;
     // Read-out of a finished chunk: y rows (lanes 0..63) and the state update
     // S_C^T = diag(Gamma_C) S0^T + X (lanes 64..127); each warp takes the column half ch.  D4 column
-    // vr(i) holds value channel i.  One pair per CTA: the new state goes to TMEM and, as tf32, to B4S
+    // vrow(i) holds value channel i.  One pair per CTA: the new state goes to TMEM and, as tf32, to B4S
     // for the next MMA4.  Task-parallel: S0 is the float32 copy in B4S and the new state replaces it
     // there; on the hi-lane warps' bar_sout arrival the control lane stores it to s_out and raises the
     // flag.
@@ -973,8 +970,8 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
           const float rs = rsqrtf(var + kLnEps);
 #pragma unroll
           for (int x = 0; x < 32; ++x) {
-            const int cidx2 = 32 * hh + x;  // value channel of logical position x (D4 column vr(x))
-            v[vr<kTask>(x)] = fmaf((v[vr<kTask>(x)] - mean) * rs, lp[cidx2], lp[64 + cidx2]);
+            const int cidx2 = 32 * hh + x;  // value channel of logical position x (D4 column vrow(x))
+            v[vrow(x)] = fmaf((v[vrow(x)] - mean) * rs, lp[cidx2], lp[64 + cidx2]);
           }
         }
         if (tl < pt.Lc) {
@@ -982,10 +979,10 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
 #pragma unroll
           for (int cc = 0; cc < 4; ++cc) {
             uint4 w4;
-            w4.x = pack_bf16x2(v[vr<kTask>(8 * cc + 0)], v[vr<kTask>(8 * cc + 1)]);
-            w4.y = pack_bf16x2(v[vr<kTask>(8 * cc + 2)], v[vr<kTask>(8 * cc + 3)]);
-            w4.z = pack_bf16x2(v[vr<kTask>(8 * cc + 4)], v[vr<kTask>(8 * cc + 5)]);
-            w4.w = pack_bf16x2(v[vr<kTask>(8 * cc + 6)], v[vr<kTask>(8 * cc + 7)]);
+            w4.x = pack_bf16x2(v[vrow(8 * cc + 0)], v[vrow(8 * cc + 1)]);
+            w4.y = pack_bf16x2(v[vrow(8 * cc + 2)], v[vrow(8 * cc + 3)]);
+            w4.z = pack_bf16x2(v[vrow(8 * cc + 4)], v[vrow(8 * cc + 5)]);
+            w4.w = pack_bf16x2(v[vrow(8 * cc + 6)], v[vrow(8 * cc + 7)]);
             *reinterpret_cast<uint4 *>(dst + 8 * cc) = w4;
           }
         }
@@ -1002,8 +999,9 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
           for (int x = 0; x < 32; ++x) ck[x * kN] = sv[vrow(x)];
         }
       } else {
-        // S_C[i][j] = Gamma_C[j] S0[i][j] + X[j][i], rows i = 32 hh + x, in place in B4S (float32),
-        // from where the control lane stores it to s_out by TMA
+        // S_C[i][j] = Gamma_C[j] S0[i][j] + X[j][i] for the channels i held in B4S rows 32 hh + x (vrow
+        // order, which is also D4's column order), in place in B4S (float32), from where the control
+        // lane stores it to s_out by TMA
         // (all 32 loads first: stores through these pointers would otherwise order every later load)
         const ColPtrs cp = col_ptrs(sB4S, 64, 32 * hh, j);
         float s0[32];
@@ -1026,7 +1024,7 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
         if (t0.n >= 0) {
           load_head(t0.h, 0, tid - 128);
           group_sync_hi();
-          prep_next<kFused, kTask>(smem, sA1, sB1, sB4V, pre4, GCs, wtot, kkw, invn, tid - 128, t0.Lc);
+          prep_next<kFused>(smem, sA1, sB1, sB4V, pre4, GCs, wtot, kkw, invn, tid - 128, t0.Lc);
         }
       }
       compute_sync();
@@ -1039,7 +1037,7 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
         load_head(have ? t.h : 0, 1, tid - 128);
       }
       if (have && warp >= 4 && wait_group_hi(bar_tma, 0))
-        prep_next<kFused, kTask>(smem, sA1, sB1, sB4V, pre4, GCs, wtot, kkw, invn, tid - 128, t.Lc);
+        prep_next<kFused>(smem, sA1, sB1, sB4V, pre4, GCs, wtot, kkw, invn, tid - 128, t.Lc);
       compute_sync();
     }
 
@@ -1227,14 +1225,14 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
             if (nt.n >= 0) {
               load_head(nt.h, (it + 1) & 1, tid - 128);
               group_sync_hi();
-              prep_next<kFused, kTask>(smem, sA1, sB1, sB4V + ((it + 1) & 1) * 16384, pre4,
+              prep_next<kFused>(smem, sA1, sB1, sB4V + ((it + 1) & 1) * 16384, pre4,
                                        GCs + ((it + 1) & 1) * 64, wtot, kkw, invn, tid - 128, nt.Lc);
             }
           }
         } else {
           Task nt = t;
           if (pair_next(A, nt) && wait_group_hi(bar_tma, (it + 1) & 1))
-            prep_next<kFused, kTask>(smem, sA1, sB1, sB4V + ((it + 1) & 1) * 16384, pre4, GCs + ((it + 1) & 1) * 64,
+            prep_next<kFused>(smem, sA1, sB1, sB4V + ((it + 1) & 1) * 16384, pre4, GCs + ((it + 1) & 1) * 64,
                                      wtot, kkw, invn, tid - 128, nt.Lc);
         }
       }
@@ -1325,14 +1323,18 @@ static bool make_map(CUtensorMap *map, const void *base, long long tokens, int H
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-static bool make_state_map(CUtensorMap *map, const void *base, long long rows) {
+// A run of `blocks` float32 64 x 64 states as the 5-D tensor (key, l, e, half, block) over rows
+// 32 half + 4 l + e: one box of 32 keys x all 64 rows lands row 32 half + 4 l + e in shared-memory row
+// 32 half + 8 e + l (vrow), the chain operand's row order.
+static bool make_state_map(CUtensorMap *map, const void *base, long long blocks) {
   PFN_encodeTiled enc = get_encode();
   if (enc == nullptr) return false;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kN), static_cast<cuuint64_t>(rows)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kN) * 4};
-  const cuuint32_t box[2] = {32, static_cast<cuuint32_t>(kN)};
-  const cuuint32_t estr[2] = {1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void *>(base), dims, strides, box, estr,
+  const cuuint64_t row = static_cast<cuuint64_t>(kN) * 4;  // bytes per state row
+  const cuuint64_t dims[5] = {static_cast<cuuint64_t>(kN), 8, 4, 2, static_cast<cuuint64_t>(blocks)};
+  const cuuint64_t strides[4] = {4 * row, row, 32 * row, 64 * row};
+  const cuuint32_t box[5] = {32, 8, 4, 2, 1};
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 5, const_cast<void *>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -1454,10 +1456,9 @@ cudaError_t launch_chunk_ext(const uint16_t *r, const uint16_t *w, const uint16_
     args.flags = ds.flags + static_cast<long long>(epoch % kFlagSlots) * kMaxChainPairs;
     args.epoch = epoch;
     args.s_in_zero = s_in == nullptr ? 1 : 0;
-    if (!make_state_map(&maps.s_in, s_in ? static_cast<const void *>(s_in) : ds.zeros, s_in ? BH * kN : kN) ||
-        !make_state_map(&maps.s_out, s_out, BH * kN) ||
-        !make_state_map(&maps.states, states ? static_cast<const void *>(states) : s_out,
-                        states ? BH * nck * kN : BH * kN))
+    if (!make_state_map(&maps.s_in, s_in ? static_cast<const void *>(s_in) : ds.zeros, s_in ? BH : 1) ||
+        !make_state_map(&maps.s_out, s_out, BH) ||
+        !make_state_map(&maps.states, states ? static_cast<const void *>(states) : s_out, states ? BH * nck : BH))
       return cudaErrorInvalidValue;
   }
   if (model_native && group_norm) return launch_variant<true, true>(maps, args, B, H, task, grid_tasks, stream);

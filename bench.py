@@ -64,7 +64,7 @@ def load_peaks():
 # L2) scaled by B to the B=8 workload; the
 # figure holds only for the kernel source it was taken on (sha256 prefix of wkv7_chunk.cu), and the
 # line reports null for any other build.  The capture is summarised under profiles/.
-MEASURED_TRAFFIC = {"source_sha256": "79a597c6bb94c6e7", "bytes_per_token_head": (151927808 + 14160896) / (4 * 4096 * 12)}
+MEASURED_TRAFFIC = {"source_sha256": "e56f7e438c3e1b20", "bytes_per_token_head": (151925760 + 14336768) / (4 * 4096 * 12)}
 
 
 def measured_traffic(B, T, H, path):

@@ -81,6 +81,13 @@ __device__ __forceinline__ void warp_mean_var64(float x0, float x1, float &mean,
 }
 
 // ---- cp.async (16-byte, L2-only) ---------------------------------------------
+// Programmatic dependent launch.  pdl_wait: the grid launched before this one in the stream (if
+// this launch allowed overlap with it) has completed and its memory is visible; a no-op otherwise.
+// pdl_trigger: the next grid in the stream may start launching once every CTA of this grid has
+// called it or exited (it still waits in its own pdl_wait before touching memory).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

@@ -55,6 +55,10 @@ template <typename TIn, bool kFused, bool kLN, typename TS = float>
 __global__ void __launch_bounds__(256) wkv7_decode_kernel(DecodeArgs<TIn, TS> A) {
   const long long pair = blockIdx.x;  // b * H + h
   const int tid = threadIdx.x;
+  // the step before may still be finishing (its launch allowed this grid to start early): every CTA
+  // of this grid has started once all have passed the trigger, and none reads memory before the wait
+  pdl_trigger();
+  pdl_wait();
   // fused: the decay and the learning rate of each of the 64 channels, computed once per CTA (the 16
   // row groups share them) by threads 0..63 while the state loads are in flight
   __shared__ float s_w[kFused ? kN : 1], s_rate[kFused ? kN : 1];
@@ -179,14 +183,33 @@ __global__ void __launch_bounds__(256) wkv7_decode_kernel(DecodeArgs<TIn, TS> A)
   }
 }
 
+// Launches a decode step allowing programmatic overlap with the grid before it in the stream: its CTAs
+// may be placed while that grid drains, and wait (pdl_wait) before reading the state it wrote.
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_overlapped(void (*kernel)(KArgs...), unsigned grid, unsigned block, cudaStream_t stream,
+                                     Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
 template <typename TIn>
 cudaError_t launch_decode(const TIn *r, const TIn *w, const TIn *k, const TIn *v, const TIn *a, const TIn *b,
                           float *s, TIn *y, int B, int H, cudaStream_t stream) {
   DecodeArgs<TIn> A{r, w, k, v, a, b, s, y, nullptr, H, nullptr, nullptr};
   const long long pairs = static_cast<long long>(B) * H;
   if (pairs > 0x7fffffffLL) return cudaErrorInvalidValue;
-  wkv7_decode_kernel<TIn, false, false><<<static_cast<unsigned>(pairs), 256, 0, stream>>>(A);
-  return cudaGetLastError();
+  return launch_overlapped(wkv7_decode_kernel<TIn, false, false>, static_cast<unsigned>(pairs), 256, stream, A);
 }
 
 cudaError_t launch_decode_ext(const uint16_t *r, const uint16_t *w, const uint16_t *k, const uint16_t *v,
@@ -197,11 +220,10 @@ cudaError_t launch_decode_ext(const uint16_t *r, const uint16_t *w, const uint16
   const long long pairs = static_cast<long long>(B) * H;
   if (pairs > 0x7fffffffLL) return cudaErrorInvalidValue;
   const unsigned g = static_cast<unsigned>(pairs);
-  if (model_native && group_norm) wkv7_decode_kernel<uint16_t, true, true><<<g, 256, 0, stream>>>(A);
-  else if (model_native) wkv7_decode_kernel<uint16_t, true, false><<<g, 256, 0, stream>>>(A);
-  else if (group_norm) wkv7_decode_kernel<uint16_t, false, true><<<g, 256, 0, stream>>>(A);
-  else wkv7_decode_kernel<uint16_t, false, false><<<g, 256, 0, stream>>>(A);
-  return cudaGetLastError();
+  if (model_native && group_norm) return launch_overlapped(wkv7_decode_kernel<uint16_t, true, true>, g, 256, stream, A);
+  if (model_native) return launch_overlapped(wkv7_decode_kernel<uint16_t, true, false>, g, 256, stream, A);
+  if (group_norm) return launch_overlapped(wkv7_decode_kernel<uint16_t, false, true>, g, 256, stream, A);
+  return launch_overlapped(wkv7_decode_kernel<uint16_t, false, false>, g, 256, stream, A);
 }
 
 // The bf16-state step: one CTA of 128 threads per (b, h); thread t holds columns 8*(t%8) .. +7 of
@@ -219,6 +241,8 @@ __device__ __forceinline__ void unpack8(uint4 u, float (&o)[8]) {
 }
 
 __global__ void __launch_bounds__(128) wkv7_decode_bf16state_kernel(DecodeArgs<uint16_t, uint16_t> A) {
+  pdl_trigger();
+  pdl_wait();
   const long long pair = blockIdx.x;
   const int tid = threadIdx.x;
   const int c8 = tid & 7, rg = tid >> 3;
@@ -276,8 +300,7 @@ cudaError_t launch_decode_bf16state(const uint16_t *r, const uint16_t *w, const 
   DecodeArgs<uint16_t, uint16_t> A{r, w, k, v, a, b, s, y, nullptr, H, nullptr, nullptr};
   const long long pairs = static_cast<long long>(B) * H;
   if (pairs > 0x7fffffffLL) return cudaErrorInvalidValue;
-  wkv7_decode_bf16state_kernel<<<static_cast<unsigned>(pairs), 128, 0, stream>>>(A);
-  return cudaGetLastError();
+  return launch_overlapped(wkv7_decode_bf16state_kernel, static_cast<unsigned>(pairs), 128, stream, A);
 }
 
 template cudaError_t launch_decode<float>(const float *, const float *, const float *, const float *, const float *,

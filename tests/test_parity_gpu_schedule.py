@@ -4,7 +4,8 @@ float64 oracle, through the C ABI's option entry point.
 
 Shapes cover fewer pairs than SMs, more pairs than SMs (several tasks per CTA, and CTAs whose next
 chunk is held by another CTA in the same round), ragged last chunks, one-chunk sequences, a zero and
-a given initial state, in-place state, and the model-native / GroupNorm variants.
+a given initial state, in-place state, the model-native / GroupNorm variants, and the automatic
+choice with more pairs than SMs (a partial last wave).
 """
 
 import numpy as np
@@ -76,6 +77,7 @@ def test_many_pairs_sampled():
     d = wi.draw(B, T, H, seed=740, s0_std=0.1)
     y2, s2 = _run(d, rk.RWKV7_SCHED_TASKS)
     y1, s1 = _run(d, rk.RWKV7_SCHED_PAIR)
+    y0, s0 = _run(d, rk.RWKV7_SCHED_AUTO)
     rng = np.random.default_rng(741)
     for _ in range(4):
         b, h = int(rng.integers(B)), int(rng.integers(H))
@@ -85,6 +87,8 @@ def test_many_pairs_sampled():
         assert rel_err(s2[b:b + 1, h:h + 1], so) <= TOL_BF16
     assert rel_err(y2, y1.float().cpu().numpy()) <= 1e-2
     assert rel_err(s2, s1.cpu().numpy()) <= 1e-2
+    assert rel_err(y0, y1.float().cpu().numpy()) <= 1e-2
+    assert rel_err(s0, s1.cpu().numpy()) <= 1e-2
 
 
 @pytest.mark.parametrize("sched", SCHEDS)
@@ -114,6 +118,33 @@ def test_repeated_launches_reuse_flag_slots():
     torch.cuda.synchronize()
     assert rel_err(y, yo) <= TOL_BF16
     assert rel_err(s, so) <= TOL_BF16
+
+
+@pytest.mark.parametrize("B,T,H", [(2, 200, 80), (1, 130, 300)])
+def test_auto_with_a_partial_last_wave(B, T, H):
+    # more pairs than SMs (160 and 300 pairs on 148 SMs): the automatic choice, against the oracle and
+    # against the explicit one-CTA-per-pair schedule
+    d = wi.draw(B, T, H, seed=790 + H, s0_std=0.1)
+    yo, so = oracle.wkv7(*oracle_ops(d), d["s0"])
+    y, s = _run(d, rk.RWKV7_SCHED_AUTO)
+    assert rel_err(y, yo) <= TOL_BF16
+    assert rel_err(s, so) <= TOL_BF16
+    yp, sp = _run(d, rk.RWKV7_SCHED_PAIR)
+    assert rel_err(y, yp.float().cpu().numpy()) <= 1e-2
+    assert rel_err(s, sp.cpu().numpy()) <= 1e-2
+
+
+def test_auto_with_a_partial_last_wave_saves_every_checkpoint():
+    B, T, H = 2, 200, 80
+    d = wi.draw(B, T, H, seed=795, s0_std=0.1)
+    dv = to_dev(d)
+    y, s_out, states = rk.prefill_save(*[dv[n] for n in OPS], dv["s0"], path=rk.RWKV7_PATH_CHUNK)
+    torch.cuda.synchronize()
+    assert torch.equal(states[:, :, 0].cpu(), d["s0"])
+    for c in range(1, rk.n_checkpoints(T)):
+        sub = [x[:, :64 * c] for x in oracle_ops(d)]
+        _, so = oracle.wkv7(*sub, d["s0"])
+        assert rel_err(states[:, :, c], so) <= TOL_BF16
 
 
 def test_schedule_value_is_checked():

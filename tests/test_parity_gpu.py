@@ -191,6 +191,31 @@ def test_full_prefill_d768_b8_t4096():
 
 
 @pytest.mark.slow
+@pytest.mark.parametrize("path", [rk.RWKV7_PATH_CHUNK, rk.RWKV7_PATH_SCAN])
+def test_full_size_pure_accumulation_every_pair(path):
+    # w = 1, a = b = 0 at the D768 B8 T4096 H12 shape and launch configuration: the recurrence reduces to
+    # S_t = S0 + sum_{tau <= t} v_tau k_tau^T, a closed form checked on EVERY (b, h): the end state in
+    # full, y at sampled tokens (float64 matmuls of the same bf16 values)
+    case = wi.CASES["prefill_d768_b8_t4096"]
+    d = wi.draw_case(case)
+    dd = to_dev(d)
+    dd["w"] = torch.ones_like(dd["w"])
+    dd["a"] = torch.zeros_like(dd["a"])
+    dd["b"] = torch.zeros_like(dd["b"])
+    y, s = gpu_prefill(dd, dd["s0"], path)
+    v = d["v"].double().numpy().transpose(0, 2, 3, 1)  # [B, H, 64 (i), T]
+    k = d["k"].double().numpy().transpose(0, 2, 1, 3)  # [B, H, T, 64 (j)]
+    r = d["r"].double().numpy()                          # [B, T, H, 64]
+    s0 = d["s0"].double().numpy()
+    assert rel_err(s, s0 + np.matmul(v, k)) <= TOL_F32
+    yc = y.float().cpu().numpy()
+    for t in (0, 63, 64, 1000, case.T - 1):
+        st = s0 + np.matmul(v[..., :t + 1], k[:, :, :t + 1])
+        yo = np.einsum("bhij,bhj->bhi", st, r[:, t])
+        assert rel_err(yc[:, t], yo) <= TOL_BF16, t
+
+
+@pytest.mark.slow
 def test_full_prefill_d2048_chained():
     case = wi.CASES["prefill_d2048_b16_t8192_chained"]
     d = wi.draw_case(case)

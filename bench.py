@@ -10,9 +10,11 @@ flush is needed between steps.
 
 One JSON line is printed by rank 0:
   value      prefill tokens/s over all ranks (device time, CUDA events, max over ranks)
-  e2e        the same metric through the C-ABI call with host buffers: pinned
-             host -> device copies of the operands and initial state, the call,
-             and device -> host copies of y and the final state, all timed
+  e2e        the same metric through the C-ABI call with host buffers
+             (rwkv7_wkv_prefill_host_bf16): pinned host -> device copies of the
+             operands and initial state, the prefill, and device -> host copies of
+             y and the final state, in batch slices whose copies overlap the
+             compute of other slices; all timed
   roofline   the prefill kernel's algorithmic HBM bytes / its average launch time
   decode     wkv7s decode steps/s at the L24-D1024 shape (B=256, H=16), rotating
              over 24 layer states (1.6 GB) so the state cannot stay in L2
@@ -495,13 +497,14 @@ def run_ours(args):
         h2d = sum(t.numel() * t.element_size() for t in host.values()) + host_s0.numel() * 4
         d2h = host_y.numel() * host_y.element_size() + host_s.numel() * 4
 
+        staging = {**dd, "s_in": s0, "y": y, "s_out": s_out}
+
         def e2e_step():
-            for n in OPS:
-                dd[n].copy_(host[n], non_blocking=True)
-            s0.copy_(host_s0, non_blocking=True)
-            step()
-            host_y.copy_(y, non_blocking=True)
-            host_s.copy_(s_out, non_blocking=True)
+            # one C-ABI call: per batch slice, pinned host -> device copies of the operands and the
+            # initial state, the prefill, and device -> host copies of y and the final state, the
+            # copies of one slice overlapping the compute and copies of others
+            lib7.rwkv7_wkv_prefill_host_bf16(path, *[host[n] for n in OPS], host_s0, host_y, host_s, staging,
+                                             slices=args.e2e_slices, stream=stream)
 
         for _ in range(2):
             e2e_step()
@@ -519,7 +522,7 @@ def run_ours(args):
         e2e_ms = max_over_ranks(a0.elapsed_time(a1), world)
         e2e_value = tokens_per_step * k_e2e / (e2e_ms / 1e3)
         e2e = {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "steps": k_e2e}
+               "steps": k_e2e, "call": "rwkv7_wkv_prefill_host_bf16", "slices": args.e2e_slices or "auto"}
 
     peaks, peak_kind = load_peaks()
     algo = prefill_bytes(B, T, H)
@@ -603,6 +606,8 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=1024)
     ap.add_argument("--decode-layers", type=int, default=24, help="distinct decode states rotated over")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-slices", type=int, default=0,
+                    help="batch slices of the host-buffer call in the e2e leg (0: chosen by the library)")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--ref-tokens", type=int, default=4096)

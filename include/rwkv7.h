@@ -191,6 +191,28 @@ typedef struct rwkv7_options {
   int chunk_schedule;
 } rwkv7_options;
 
+/* ---- prefill from and to host memory ------------------------------------------------------
+ *
+ * The bf16 prefill of rwkv7_wkv_prefill_bf16_path for operands that live in host memory: r, w, k,
+ * v, a, b ([B,T,H,64] bf16), s_in ([B,H,64,64] float32, NULL = zero state), y and s_out are HOST
+ * pointers; dev_r .. dev_b, dev_s_in, dev_y, dev_s_out are DEVICE buffers of the same shapes that
+ * the call uses as staging (dev_s_in may be NULL when s_in is).  The batch is cut into `slices`
+ * runs of whole rows b (0 = chosen by the call, at most B); per slice the call copies the slice's
+ * operands (and initial state) host -> device, runs the prefill on it once they have landed, and
+ * copies its y and final state device -> host, on two internal streams ordered after `stream`, so
+ * the copies of one slice overlap the compute and the copies of others.  On return the work is
+ * queued; `stream` waits for all of it (synchronise `stream` before reading y / s_out).  For the
+ * copies to overlap, the host buffers must be page-locked (cudaHostAlloc / cudaHostRegister);
+ * pageable buffers give the same results without overlap.  Every pointer must be 16-byte aligned.
+ * Errors as for the device entry point; a failure leaves the outputs undefined. */
+RWKV7_API rwkv7_status rwkv7_wkv_prefill_host_bf16(int path, int B, int T, int H, int N, const uint16_t *r,
+                                                   const uint16_t *w, const uint16_t *k, const uint16_t *v,
+                                                   const uint16_t *a, const uint16_t *b, const float *s_in,
+                                                   uint16_t *y, float *s_out, uint16_t *dev_r, uint16_t *dev_w,
+                                                   uint16_t *dev_k, uint16_t *dev_v, uint16_t *dev_a,
+                                                   uint16_t *dev_b, float *dev_s_in, uint16_t *dev_y,
+                                                   float *dev_s_out, int slices, rwkv7_stream_t stream);
+
 /* bf16 prefill with options (NULL = none); other arguments as for rwkv7_wkv_prefill_bf16_path. */
 RWKV7_API rwkv7_status rwkv7_wkv_prefill_ext_bf16(int path, int B, int T, int H, int N, const uint16_t *r,
                                                   const uint16_t *w, const uint16_t *k, const uint16_t *v,

@@ -29,7 +29,7 @@ __all__ = [
     "rwkv7_wkv_prefill_ext_bf16", "rwkv7_wkv_decode_ext_bf16", "Options",
     "rwkv7_status_string", "rwkv7_get_last_error", "rwkv7_version",
     "rwkv7_wkv_prefill_save_bf16", "rwkv7_wkv_backward_bf16", "rwkv7_wkv_decode_bf16_bf16state",
-    "prefill", "decode_", "prefill_model_native", "decode_model_native_", "prefill_ext", "decode_ext_",
+    "rwkv7_wkv_prefill_host_bf16", "prefill", "decode_", "prefill_model_native", "decode_model_native_", "prefill_ext", "decode_ext_",
     "prefill_save", "backward", "EXPORTED_SYMBOLS",
 ]
 
@@ -43,7 +43,7 @@ EXPORTED_SYMBOLS = (
     "rwkv7_wkv_decode", "rwkv7_wkv_decode_bf16", "rwkv7_wkv_prefill_fused_bf16", "rwkv7_wkv_decode_fused_bf16",
     "rwkv7_wkv_prefill_ext_bf16", "rwkv7_wkv_decode_ext_bf16",
     "rwkv7_wkv_prefill_save_bf16", "rwkv7_wkv_backward_bf16", "rwkv7_wkv_decode_bf16_bf16state",
-    "rwkv7_status_string", "rwkv7_get_last_error", "rwkv7_version",
+    "rwkv7_wkv_prefill_host_bf16", "rwkv7_status_string", "rwkv7_get_last_error", "rwkv7_version",
 )
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -92,6 +92,8 @@ def load_library() -> ctypes.CDLL:
         ("rwkv7_wkv_prefill_save_bf16", [ci, ci, ci, ci, ci] + [vp] * 6 + [vp, vp, vp, vp, vp]),
         ("rwkv7_wkv_backward_bf16", [ci, ci, ci, ci] + [vp] * 6 + [vp, vp, vp] + [vp] * 7 + [vp]),
         ("rwkv7_wkv_decode_bf16_bf16state", [ci, ci, ci] + [vp] * 6 + [vp, vp, vp]),
+        ("rwkv7_wkv_prefill_host_bf16", [ci, ci, ci, ci, ci] + [vp] * 6 + [vp, vp, vp] + [vp] * 6 + [vp, vp, vp]
+         + [ci, vp]),
     ):
         fn = getattr(lib, name)
         fn.argtypes = args
@@ -118,6 +120,15 @@ def _stream(stream) -> Optional[int]:
     if isinstance(stream, torch.cuda.Stream):
         return stream.cuda_stream
     return int(stream)
+
+
+def _check_host(t: torch.Tensor, name: str, dtype: torch.dtype, shape):
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if t.is_cuda:
+        raise ValueError(f"{name} must be a host (CPU) tensor")
+    if t.dtype != dtype or not t.is_contiguous() or tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must be a contiguous {dtype} tensor of shape {tuple(shape)}")
 
 
 def _check(t: Optional[torch.Tensor], name: str, dtype: torch.dtype, shape=None, allow_none=False):
@@ -169,6 +180,26 @@ def rwkv7_wkv_prefill_bf16_path(path, r, w, k, v, a, b, s_in, y, s_out, stream=N
     """bfloat16 prefill with an explicit kernel (RWKV7_PATH_SCAN or RWKV7_PATH_CHUNK)."""
     _prefill_common("rwkv7_wkv_prefill_bf16_path", torch.bfloat16, r, w, k, v, a, b, s_in, y, s_out, stream,
                     path=path)
+
+
+def rwkv7_wkv_prefill_host_bf16(path, r, w, k, v, a, b, s_in, y, s_out, dev, slices=0, stream=None) -> None:
+    """bfloat16 prefill from and to host memory: r .. b, s_in (or None), y and s_out are CPU tensors
+    (page-locked for the copies to overlap); ``dev`` maps "r", "w", "k", "v", "a", "b", "s_in" (when
+    s_in is given), "y", "s_out" to CUDA staging tensors of the same shapes.  The call queues the
+    sliced copies and launches on ``stream``; synchronise it before reading y / s_out."""
+    B, T, H, N = r.shape
+    for nm, t in (("r", r), ("w", w), ("k", k), ("v", v), ("a", a), ("b", b), ("y", y)):
+        _check_host(t, nm, torch.bfloat16, (B, T, H, N))
+        _check(dev[nm], "dev " + nm, torch.bfloat16, (B, T, H, N))
+    _check_host(s_out, "s_out", torch.float32, (B, H, N, N))
+    _check(dev["s_out"], "dev s_out", torch.float32, (B, H, N, N))
+    if s_in is not None:
+        _check_host(s_in, "s_in", torch.float32, (B, H, N, N))
+        _check(dev["s_in"], "dev s_in", torch.float32, (B, H, N, N))
+    dsi = dev["s_in"] if s_in is not None else None
+    _call("rwkv7_wkv_prefill_host_bf16", int(path), B, T, H, N, *[_ptr(t) for t in (r, w, k, v, a, b, s_in, y, s_out)],
+          *[_ptr(dev[n]) for n in ("r", "w", "k", "v", "a", "b")], _ptr(dsi), _ptr(dev["y"]), _ptr(dev["s_out"]),
+          int(slices), _stream(stream))
 
 
 def rwkv7_wkv_prefill_varlen_bf16(path, cu_seqlens, max_T, r, w, k, v, a, b, s_in, y, s_out, stream=None) -> None:

@@ -116,6 +116,77 @@ rwkv7_status rwkv7_wkv_prefill_bf16(int B, int T, int H, int N, const uint16_t *
   return rwkv7_wkv_prefill_bf16_path(RWKV7_PATH_AUTO, B, T, H, N, r, w, k, v, a, b, s_in, y, s_out, stream);
 }
 
+rwkv7_status rwkv7_wkv_prefill_host_bf16(int path, int B, int T, int H, int N, const uint16_t *r, const uint16_t *w,
+                                         const uint16_t *k, const uint16_t *v, const uint16_t *a, const uint16_t *b,
+                                         const float *s_in, uint16_t *y, float *s_out, uint16_t *dev_r,
+                                         uint16_t *dev_w, uint16_t *dev_k, uint16_t *dev_v, uint16_t *dev_a,
+                                         uint16_t *dev_b, float *dev_s_in, uint16_t *dev_y, float *dev_s_out,
+                                         int slices, rwkv7_stream_t stream) {
+  if (path != RWKV7_PATH_AUTO && path != RWKV7_PATH_SCAN && path != RWKV7_PATH_CHUNK) return RWKV7_ERR_INVALID;
+  rwkv7_status st = check_prefill(B, T, H, N, r, w, k, v, a, b, s_in, y, s_out);
+  if (st != RWKV7_OK) return st;
+  st = check_prefill(B, T, H, N, dev_r, dev_w, dev_k, dev_v, dev_a, dev_b, dev_s_in, dev_y, dev_s_out);
+  if (st != RWKV7_OK) return st;
+  if (slices < 0 || (s_in != nullptr && dev_s_in == nullptr)) return RWKV7_ERR_INVALID;
+  // default: 4 slices (B200 over PCIe, B8 T4096 H12: 4.79 / 5.07 / 5.17 / 5.09 / 5.10 M tokens/s end
+  // to end with 1 / 2 / 4 / 8 / 16 slices; the host -> device copies bound it)
+  const int ns = slices == 0 ? (B < 4 ? B : 4) : (slices < B ? slices : B);
+  const bool chunk = use_chunk(path, T);
+  cudaStream_t user = reinterpret_cast<cudaStream_t>(stream);
+  const uint16_t *hops[6] = {r, w, k, v, a, b};
+  uint16_t *dops[6] = {dev_r, dev_w, dev_k, dev_v, dev_a, dev_b};
+  const long long row_elems = static_cast<long long>(T) * H * kN;  // operand elements per batch row
+  const long long row_state = static_cast<long long>(H) * kN * kN;  // state elements per batch row
+  // host -> device copies on `stream`; the prefill on `ks`; device -> host copies on `os`
+  cudaStream_t ks = nullptr, os = nullptr;
+  cudaEvent_t ev_in = nullptr, ev_k = nullptr, ev_done = nullptr;
+  cudaError_t e = cudaStreamCreateWithFlags(&ks, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&os, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_done, cudaEventDisableTiming);
+  for (int i = 0; i < ns && e == cudaSuccess; ++i) {
+    const int b0 = static_cast<int>(static_cast<long long>(B) * i / ns);
+    const int b1 = static_cast<int>(static_cast<long long>(B) * (i + 1) / ns);
+    const int nb = b1 - b0;
+    const size_t op_bytes = static_cast<size_t>(nb * row_elems) * sizeof(uint16_t);
+    const size_t st_bytes = static_cast<size_t>(nb * row_state) * sizeof(float);
+    const long long oo = b0 * row_elems, so = b0 * row_state;
+    // one event pair per slice, released by the runtime once the work that records them is done
+    e = cudaEventCreateWithFlags(&ev_in, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_k, cudaEventDisableTiming);
+    for (int q = 0; q < 6 && e == cudaSuccess && op_bytes > 0; ++q)
+      e = cudaMemcpyAsync(dops[q] + oo, hops[q] + oo, op_bytes, cudaMemcpyHostToDevice, user);
+    if (e == cudaSuccess && s_in != nullptr)
+      e = cudaMemcpyAsync(dev_s_in + so, s_in + so, st_bytes, cudaMemcpyHostToDevice, user);
+    if (e == cudaSuccess) e = cudaEventRecord(ev_in, user);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(ks, ev_in, 0);
+    if (e == cudaSuccess) {
+      const uint16_t *dr = dev_r + oo, *dw = dev_w + oo, *dk = dev_k + oo, *dv = dev_v + oo, *da = dev_a + oo,
+                     *db = dev_b + oo;
+      const float *dsi = s_in != nullptr ? dev_s_in + so : nullptr;
+      const long long total = static_cast<long long>(nb) * T;
+      e = chunk ? launch_chunk(dr, dw, dk, dv, da, db, dsi, dev_y + oo, dev_s_out + so, nullptr, nb, T, total, H,
+                               error_word_ptr(), ks)
+                : launch_scan<uint16_t>(dr, dw, dk, dv, da, db, dsi, dev_y + oo, dev_s_out + so, nullptr, nb, T, total,
+                                        H, ks);
+    }
+    if (e == cudaSuccess) e = cudaEventRecord(ev_k, ks);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(os, ev_k, 0);
+    if (e == cudaSuccess && op_bytes > 0)
+      e = cudaMemcpyAsync(y + oo, dev_y + oo, op_bytes, cudaMemcpyDeviceToHost, os);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(s_out + so, dev_s_out + so, st_bytes, cudaMemcpyDeviceToHost, os);
+    if (ev_in != nullptr) cudaEventDestroy(ev_in);
+    if (ev_k != nullptr) cudaEventDestroy(ev_k);
+    ev_in = ev_k = nullptr;
+  }
+  // `stream` waits for the last device -> host copy (the copies on `os` run in order)
+  if (e == cudaSuccess) e = cudaEventRecord(ev_done, os);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(user, ev_done, 0);
+  if (ev_done != nullptr) cudaEventDestroy(ev_done);
+  if (ks != nullptr) cudaStreamDestroy(ks);
+  if (os != nullptr) cudaStreamDestroy(os);
+  return from_cuda(e);
+}
+
 rwkv7_status rwkv7_wkv_prefill_varlen_bf16(int path, int B, int total_T, int max_T, int H, int N,
                                            const int32_t *cu_seqlens, const uint16_t *r, const uint16_t *w,
                                            const uint16_t *k, const uint16_t *v, const uint16_t *a,

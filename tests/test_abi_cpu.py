@@ -118,6 +118,23 @@ def test_training_and_bf16_state_entry_points_reject(cdll):
     assert cdll.rwkv7_wkv_decode_bf16_bf16state(1, 1, 48, *ops, FAKE, FAKE, None) == 5
 
 
+def test_host_prefill_rejects(cdll):
+    ops = [FAKE] * 6
+    # rwkv7_wkv_prefill_host_bf16(path, B, T, H, N, host ops, s_in, y, s_out, dev ops, dev s_in, dev y,
+    #                             dev s_out, slices, stream)
+    def call(path=0, N=64, host=FAKE, dev=FAKE, s_in=None, dev_s_in=None, slices=0):
+        return cdll.rwkv7_wkv_prefill_host_bf16(path, 2, 4, 1, N, *([host] * 6), s_in, host, host, *([dev] * 6),
+                                                dev_s_in, dev, dev, slices, None)
+    assert call(path=9) == 1
+    assert call(N=32) == 5
+    assert call(host=None) == 1
+    assert call(dev=None) == 1
+    assert call(host=MIS) == 2
+    assert call(dev=MIS) == 2
+    assert call(s_in=FAKE, dev_s_in=None) == 1  # an initial state needs its staging buffer
+    assert call(slices=-1) == 1
+
+
 def test_binding_rejects_cpu_tensors():
     import torch
 

@@ -27,11 +27,14 @@
  *   patterns (uint16_t); the others use float32.
  *
  * Ownership and execution:
- *   - Every pointer is a device pointer owned by the caller; the library
- *     allocates nothing per call and keeps no pointer after returning.
+ *   - Every pointer is a device pointer owned by the caller (except the host
+ *     buffers of rwkv7_wkv_prefill_host_bf16); the library allocates no memory
+ *     per call and keeps no pointer after returning.
  *   - Calls only enqueue work on `stream` (NULL = the legacy default stream)
  *     and return; they never synchronise, so they can be captured into a CUDA
- *     graph.  Results are ready once the stream reaches that point.
+ *     graph.  Results are ready once the stream reaches that point.  (The
+ *     host-buffer prefill also uses two streams of its own, ordered after
+ *     `stream` and joined back into it.)
  *   - s_in may be NULL (zero initial state) and may equal s_out (in place).
  *     y must not overlap any other argument.
  *   - Every pointer must be 16-byte aligned.

@@ -467,8 +467,7 @@ def run_ours(args):
     # per-launch durations over the timed region, on the launching stream
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     e_start, e_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(local, os.path.join(ROOT, "gpurun_out", "clocks_bench.csv")
-                          if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else None)
+    clocks = ClockSampler(local, args.clocks_csv)
     with clocks:
         barrier(world)
         torch.cuda.synchronize()
@@ -606,6 +605,7 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=1024)
     ap.add_argument("--decode-layers", type=int, default=24, help="distinct decode states rotated over")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--clocks-csv", default=None, help="also write the raw nvidia-smi clock samples here")
     ap.add_argument("--e2e-slices", type=int, default=0,
                     help="batch slices of the host-buffer call in the e2e leg (0: chosen by the library)")
     ap.add_argument("--no-cpu", action="store_true")

@@ -75,3 +75,20 @@ def test_host_prefill_empty_sequence_copies_the_state():
     y, s = _host_call(e, rk.RWKV7_PATH_AUTO, slices=2)
     assert torch.equal(s, d["s0"])
     assert y.numel() == 0
+
+
+@pytest.mark.slow
+def test_host_prefill_at_the_d768_shape_equals_the_device_call():
+    # the bench's end-to-end call (B8 T4096 H12, default slices): the same kernels on batch slices,
+    # so every element equals the device-buffer call's (a pair's arithmetic does not depend on the
+    # other pairs of its launch), and sampled pairs match the oracle
+    case = wi.CASES["prefill_d768_b8_t4096"]
+    d = wi.draw_case(case)
+    y, s = _host_call(d, rk.RWKV7_PATH_AUTO)
+    yd, sd = _device_call(d, rk.RWKV7_PATH_AUTO)
+    assert torch.equal(y, yd) and torch.equal(s, sd)
+    for b, h in ((0, 0), (7, 11)):
+        sub = [x[b:b + 1, :, h:h + 1] for x in oracle_ops(d)]
+        yo, so = oracle.wkv7(*sub, d["s0"][b:b + 1, h:h + 1])
+        assert rel_err(y[b:b + 1, :, h:h + 1], yo) <= TOL_BF16
+        assert rel_err(s[b:b + 1, h:h + 1], so) <= TOL_BF16

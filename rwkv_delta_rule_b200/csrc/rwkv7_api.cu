@@ -1,7 +1,9 @@
 // rwkv7_api.cu -- the extern "C" entry points declared in include/rwkv7.h:
 // host-side argument checks, kernel choice and launches.  Nothing here
-// allocates, synchronises or touches the data; every step of the computation
-// runs in the kernels.
+// allocates memory or synchronises; apart from the host-buffer prefill, which
+// queues copies between the caller's host and device buffers around the
+// launches, nothing here touches the data: every step of the computation runs
+// in the kernels.
 #include "../../include/rwkv7.h"
 #include "common.cuh"
 #include "launch.h"
@@ -12,7 +14,7 @@ __device__ int g_error_word = 0;
 
 namespace {
 
-constexpr int kVersion = 100;  // 0.1.0
+constexpr int kVersion = 200;  // 0.2.0: adds the host-buffer prefill
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 

@@ -18,6 +18,11 @@ The start state of every chunk comes from a forward pass that keeps the chunk-bo
 the checkpointing forward does).  Eleven dense products per chunk, each of the shapes the forward
 kernel already runs on the tensor cores.  Not built as a kernel yet: the training backward runs the
 sequential form.
+
+The second part fixes the operand precision of those products for such a kernel, by emulating the
+rounding of each product's operands (tf32 or bf16) on bf16 inputs: every product in bf16 misses the
+5e-3 bar; the inverse's adjoint (dTinv, both dLab products) and dD2 in bf16 with the rest, and the
+recomputed forward products, in tf32 stay within 2.5e-3.
 """
 
 import numpy as np
@@ -27,48 +32,52 @@ import oracle
 from test_chunk_algebra import C, blocked_unit_lower_inverse
 
 
-def chunk_forward_parts(rr, ww, kk, vv, aa, bb, ST):
+def exact(name, a, b):
+    return a @ b
+
+
+def chunk_forward_parts(rr, ww, kk, vv, aa, bb, ST, mm=exact):
     """The forward chunk of ``chunked_head`` (padded C x N operands, ST = S0^T), keeping every
-    intermediate the backward needs."""
+    intermediate the backward needs.  ``mm(name, a, b)`` forms each matrix product."""
     N = rr.shape[1]
     G = np.cumprod(ww, axis=0)
     Gx = np.vstack([np.ones((1, N)), G[:-1]])
     GC = G[-1]
     At, Rt, Bh, Kh = aa * Gx, rr * G, bb / G, kk / G
     Lm, Rm = np.vstack([Rt, At]), np.vstack([Bh, Kh])
-    D1 = Lm @ Rm.T
+    D1 = mm("MMA1", Lm, Rm.T)
     strict = np.tril(np.ones((C, C)), -1)
     incl = np.tril(np.ones((C, C)), 0)
     Mrb, Mrk = D1[:C, :C] * incl, D1[:C, C:] * incl
     Lab, Lak = D1[C:, :C] * strict, D1[C:, C:] * strict
     Tinv = blocked_unit_lower_inverse(Lab)
     Z = np.hstack([At, Lak])
-    WU = Tinv @ Z
+    WU = mm("MMA3", Tinv, Z)
     Bbar, Kbar = bb * (GC / G), kk * (GC / G)
     init = np.vstack([np.hstack([Rt, Mrk]), np.hstack([np.zeros((N, N)), Kbar.T])])
     P = np.vstack([Mrb, Bbar.T])
-    D2 = init + P @ WU
+    D2 = init + mm("MMA2", P, WU)
     X = np.vstack([ST, vv])
-    D4 = D2 @ X
+    D4 = mm("MMA4", D2, X)
     return dict(G=G, Gx=Gx, GC=GC, At=At, Rt=Rt, Bh=Bh, Kh=Kh, Lm=Lm, Rm=Rm, Tinv=Tinv, Z=Z, WU=WU, P=P,
                 D2=D2, X=X, D4=D4, strict=strict, incl=incl)
 
 
-def chunk_backward(f, rr, ww, kk, vv, aa, bb, ST, dY, dSTn):
+def chunk_backward(f, rr, ww, kk, vv, aa, bb, ST, dY, dSTn, mm=exact):
     """Adjoints of one chunk: given dY (C x N) and dSTn (adjoint of S_C^T), returns
     (dr, dw, dk, dv, da, db) (C x N each) and the adjoint of S0^T."""
     N = rr.shape[1]
     G, Gx, GC = f["G"], f["Gx"], f["GC"]
     # chain: D4 = D2 X, S_C^T = diag(GC) S0^T + D4[C:], Y = D4[:C]
     dD4 = np.vstack([dY, dSTn])
-    dX = f["D2"].T @ dD4
-    dD2 = dD4 @ f["X"].T
+    dX = mm("dX", f["D2"].T, dD4)
+    dD2 = mm("dD2", dD4, f["X"].T)
     dST = GC[:, None] * dSTn + dX[:N]
     dvv = dX[N:]
     dGC = np.sum(dSTn * ST, axis=1)
     # transition: D2 = init + P WU
-    dP = dD2 @ f["WU"].T
-    dWU = f["P"].T @ dD2
+    dP = mm("dP", dD2, f["WU"].T)
+    dWU = mm("dWU", f["P"].T, dD2)
     dRt = dD2[:C, :N].copy()
     dMrk = dD2[:C, N:].copy()
     dKbar = dD2[C:, N:].T.copy()
@@ -76,15 +85,15 @@ def chunk_backward(f, rr, ww, kk, vv, aa, bb, ST, dY, dSTn):
     dBbar = dP[C:].T
     # WY form: WU = Tinv Z, Tinv = (I - Lab)^-1
     Tinv = f["Tinv"]
-    dTinv = dWU @ f["Z"].T
-    dZ = Tinv.T @ dWU
+    dTinv = mm("dTinv", dWU, f["Z"].T)
+    dZ = mm("dZ", Tinv.T, dWU)
     dAt = dZ[:, :N].copy()
     dLak = dZ[:, N:]
-    dLab = Tinv.T @ dTinv @ Tinv.T
+    dLab = mm("dLab2", mm("dLab1", Tinv.T, dTinv), Tinv.T)
     # products: D1 = Lm Rm^T, masked
     dD1 = np.block([[dMrb * f["incl"], dMrk * f["incl"]], [dLab * f["strict"], dLak * f["strict"]]])
-    dLm = dD1 @ f["Rm"]
-    dRm = dD1.T @ f["Lm"]
+    dLm = mm("dLm", dD1, f["Rm"])
+    dRm = mm("dRm", dD1.T, f["Lm"])
     dRt += dLm[:C]
     dAt += dLm[C:]
     dBh, dKh = dRm[:C], dRm[C:]
@@ -101,7 +110,7 @@ def chunk_backward(f, rr, ww, kk, vv, aa, bb, ST, dY, dSTn):
     return (drr, dww, dkk, dvv, daa, dbb), dST
 
 
-def chunked_backward_head(r, w, k, v, a, b, s0, dy, ds_out):
+def chunked_backward_head(r, w, k, v, a, b, s0, dy, ds_out, mm=exact):
     """r..b, dy: [T, N]; s0, ds_out: [N, N].  Returns (dr, dw, dk, dv, da, db, ds_in)."""
     T, N = r.shape
     pad = lambda x, c0, Lc, fill=0.0: np.concatenate([x[c0:c0 + Lc], np.full((C - Lc, N), fill)], 0)
@@ -113,7 +122,7 @@ def chunked_backward_head(r, w, k, v, a, b, s0, dy, ds_out):
         ops = [pad(x, c0, Lc) for x in (r, w, k, v, a, b)]
         ops[1] = pad(w, c0, Lc, 1.0)
         starts.append(ST)
-        f = chunk_forward_parts(ops[0], ops[1], ops[2], ops[3], ops[4], ops[5], ST)
+        f = chunk_forward_parts(ops[0], ops[1], ops[2], ops[3], ops[4], ops[5], ST, mm)
         ST = f["GC"][:, None] * ST + f["D4"][C:]
     grads = [np.zeros((T, N)) for _ in range(6)]
     dSTn = ds_out.T.copy()
@@ -121,8 +130,8 @@ def chunked_backward_head(r, w, k, v, a, b, s0, dy, ds_out):
         Lc = min(C, T - c0)
         rr, kk, vv, aa, bb = (pad(x, c0, Lc) for x in (r, k, v, a, b))
         ww = pad(w, c0, Lc, 1.0)
-        f = chunk_forward_parts(rr, ww, kk, vv, aa, bb, ST0)
-        g, dSTn = chunk_backward(f, rr, ww, kk, vv, aa, bb, ST0, pad(dy, c0, Lc), dSTn)
+        f = chunk_forward_parts(rr, ww, kk, vv, aa, bb, ST0, mm)
+        g, dSTn = chunk_backward(f, rr, ww, kk, vv, aa, bb, ST0, pad(dy, c0, Lc), dSTn, mm)
         for i in range(6):
             grads[i][c0:c0 + Lc] = g[i][:Lc]
     return tuple(grads) + (dSTn.T,)
@@ -153,3 +162,47 @@ def test_chunked_backward_matches_the_backward_oracle(T):
         scale = np.abs(ref[i]).max()
         np.testing.assert_allclose(got[i], ref[i][0, :, 0], atol=1e-9 * scale, err_msg=n)
     np.testing.assert_allclose(got[6], ref[6][0, 0], atol=1e-9 * np.abs(ref[6]).max(), err_msg="ds_in")
+
+
+# ---- operand precision of the products (plan for a tensor-core backward) ----------------------------
+
+def round_operand(x, fmt):
+    """Round to tf32 (10 explicit mantissa bits) or bf16 (7), to nearest even, via float32."""
+    if fmt == "f64":
+        return x
+    u = np.asarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    drop = 13 if fmt == "tf32" else 16
+    u = (u + ((1 << (drop - 1)) - 1) + ((u >> drop) & 1)) >> drop << drop
+    return u.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def rounding_mm(plan):
+    return lambda name, a, b: round_operand(a, plan[name]) @ round_operand(b, plan[name])
+
+
+BWD = ("dX", "dD2", "dP", "dWU", "dTinv", "dZ", "dLab1", "dLab2", "dLm", "dRm")
+
+
+def _worst_rel_err(plan, T=256, seeds=(1, 2)):
+    worst = 0.0
+    for seed in seeds:
+        r, w, k, v, a, b, s0, dy, ds_out = _inputs(T, seed)
+        r, w, k, v, a, b, dy = (round_operand(x, "bf16") for x in (r, w, k, v, a, b, dy))  # bf16 operands
+        ref = oracle.wkv7_backward(*[x[None, :, None] for x in (r, w, k, v, a, b)], s0[None, None],
+                                   dy[None, :, None], ds_out[None, None])
+        got = chunked_backward_head(r, w, k, v, a, b, s0, dy, ds_out, rounding_mm(plan))
+        for i in range(7):
+            rr = ref[i][0, :, 0] if i < 6 else ref[6][0, 0]
+            worst = max(worst, float(np.abs(got[i] - rr).max() / np.abs(rr).max()))
+    return worst
+
+
+def test_product_precision_plan():
+    # the forward products recomputed at tf32; of the backward's, the inverse's adjoint (dTinv and
+    # both dLab products) and dD2 in bf16, the rest in tf32: within the 5e-3 bar of bf16 operands with
+    # margin, while every product in bf16 is not (the column-sum products dLm, dRm need tf32)
+    fwd = {"MMA1": "tf32", "MMA3": "tf32", "MMA2": "tf32", "MMA4": "tf32"}
+    plan = dict(fwd, **{n: "tf32" for n in BWD})
+    plan.update({n: "bf16" for n in ("dTinv", "dLab1", "dLab2", "dD2")})
+    assert _worst_rel_err(plan) <= 2.5e-3
+    assert _worst_rel_err(dict(fwd, **{n: "bf16" for n in BWD})) > 5e-3

@@ -1,6 +1,8 @@
 """Pins of the float64 backward oracle (``oracle.wkv7_backward``) against things it does not share:
-central finite differences of the forward oracle, torch autograd of an independent token loop, and
-closed forms of the special case w = 1, a = 0 (where the state is a plain prefix sum).
+central finite differences of the forward oracle, torch autograd of an independent token loop,
+closed forms of the special case w = 1, a = 0 (where the state is a plain prefix sum), and the
+forward oracle run on the reversed sequence with a and b swapped (the adjoint state's recurrence),
+which gives dv and ds_in.
 
 The scalar differentiated everywhere is L = sum <dy, y> + <ds_out, s_out>.
 """
@@ -124,3 +126,27 @@ def test_empty_sequence_passes_the_state_gradient_through():
     g = oracle.wkv7_backward(*[x[n] for n in NAMES], s0, dy, ds)
     assert all(a.size == 0 for a in g[:6])
     assert np.array_equal(g[6], ds)
+
+
+@pytest.mark.parametrize("T", [1, 5, 70])
+def test_adjoint_state_is_the_forward_recurrence_reversed(T):
+    # G_t = dL/dS_t obeys G_{t-1} = G_t (diag(w_t) + a_t b_t^T)^T + dy_{t-1} r_{t-1}^T from
+    # G_{T-1} = ds_out + dy_{T-1} r_{T-1}^T: the forward recurrence in reverse time with a and b
+    # swapped, v := dy and k := r.  Run by the FORWARD oracle with r := k, its outputs are G_t k_t =
+    # dv_t and its end state (after one more step with token 0's transition and no injection) is
+    # ds_in: two backward outputs from the forward oracle alone.
+    x, s0, dy, ds = _draw(2, T, 3, 8, seed=40 + T)
+    g = oracle.wkv7_backward(*[x[n] for n in NAMES], s0, dy, ds)
+    B, _, H, N = dy.shape
+    rev = {n: np.zeros((B, T + 1, H, N)) for n in NAMES}
+    rev["w"][:, 0] = 1.0                           # step 0: only the injection dy_{T-1} r_{T-1}^T
+    rev["w"][:, 1:] = x["w"][:, ::-1]              # step tau >= 1: transition of token T - tau
+    rev["a"][:, 1:] = x["b"][:, ::-1]
+    rev["b"][:, 1:] = x["a"][:, ::-1]
+    rev["v"][:, :T] = dy[:, ::-1]                  # step tau < T: injection of token T - 1 - tau
+    rev["k"][:, :T] = x["r"][:, ::-1]
+    rev["r"][:, :T] = x["k"][:, ::-1]              # read-out G_t k_t
+    y, s = oracle.wkv7(*[rev[n] for n in NAMES], ds, precision="f64")
+    scale = np.abs(g[3]).max()
+    np.testing.assert_allclose(y[:, :T][:, ::-1], g[3], atol=1e-12 * scale)   # dv
+    np.testing.assert_allclose(s, g[6], atol=1e-12 * np.abs(g[6]).max())      # ds_in

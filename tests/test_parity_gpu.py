@@ -143,6 +143,49 @@ def test_decode_steps_equal_oracle(dtype):
     assert rel_err(st, so) <= tol
 
 
+@pytest.mark.parametrize("bf16_state", [False, True])
+def test_decode_steps_in_a_cuda_graph(bf16_state):
+    # back-to-back steps on ONE state, captured in a CUDA graph and replayed: each step's launch may
+    # overlap the previous step's last wave (programmatic dependent launch) and must still read the
+    # state that step wrote
+    B, H, T = 4, 6, 24
+    d = wi.draw(B, T, H, seed=14, s0_std=0.1)
+    ops = [n + "_f32" for n in OPS]
+    steps = {n: torch.stack([d[n][:, t].contiguous() for t in range(T)]).cuda() for n in OPS}  # [T, B, H, 64]
+    ys = torch.empty((T, B, H, 64), dtype=torch.bfloat16, device="cuda")
+    st = (d["s0"].to(torch.bfloat16) if bf16_state else d["s0"]).cuda()
+    st0 = st.clone()
+    step = rk.rwkv7_wkv_decode_bf16_bf16state if bf16_state else rk.rwkv7_wkv_decode_bf16
+
+    def run():
+        for t in range(T):
+            step(*[steps[n][t] for n in OPS], st, ys[t])
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        run()  # warm-up outside the capture
+    torch.cuda.current_stream().wait_stream(side)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        run()
+    st.copy_(st0)
+    g.replay()
+    torch.cuda.synchronize()
+    if bf16_state:
+        s_or = oracle.round_bf16(d["s0"].numpy())
+        yo = []
+        for t in range(T):
+            y1, s_or = oracle.decode_step_bf16_state(*[d[n][:, t] for n in ops], s_or)
+            yo.append(y1)
+        assert rel_err(ys.transpose(0, 1), np.stack(yo, 1)) <= TOL_BF16
+        assert rel_err(st.float(), s_or) <= 2.0 ** -7
+    else:
+        yo, so = oracle.wkv7(*oracle_ops(d), d["s0"])
+        assert rel_err(ys.transpose(0, 1), yo) <= TOL_BF16
+        assert rel_err(st, so) <= TOL_BF16
+
+
 @pytest.mark.parametrize("path", PATHS)
 def test_varlen_small(path):
     lens = torch.tensor([1, 0, 33, 64, 65, 7, 200])

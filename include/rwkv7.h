@@ -217,6 +217,41 @@ RWKV7_API rwkv7_status rwkv7_wkv_prefill_host_bf16(int path, int B, int T, int H
                                                    uint16_t *dev_b, float *dev_s_in, uint16_t *dev_y,
                                                    float *dev_s_out, int slices, rwkv7_stream_t stream);
 
+/* ---- prefill from and to host memory, allocating nothing ----------------------------------
+ *
+ * The pages have no counterpart of this call: it exists for callers that hold their data in host
+ * memory and cannot allocate device memory.  Examples: a plain C program or a binding from another
+ * language that reaches the GPU only through this library and does not link the CUDA runtime, so it
+ * has no way to create device buffers; a process whose device memory is handed out by an allocator
+ * it does not control; a serving loop that must not call cudaMalloc / cudaFree, which can
+ * synchronise the whole device.  rwkv7_wkv_prefill_host_bf16 needs device staging buffers from its
+ * caller; this call instead stages through one array of RWKV7_NOALLOC_STAGING_BYTES in the
+ * library's static device memory (every GPU that loads the library holds it until the process
+ * exits) and allocates nothing: no cudaMalloc, no cudaFree, no stream or event.
+ *
+ * r, w, k, v, a, b ([B,T,H,64] bf16), s_in ([B,H,64,64] float32, NULL = zero state), y and s_out are
+ * HOST pointers, 16-byte aligned.  On `stream` the call copies the operands (and s_in) into the
+ * array, runs the prefill that `path` selects (as rwkv7_wkv_prefill_bf16_path), and copies y and the
+ * final state back; synchronise `stream` before reading y / s_out.  Page-locked host buffers make
+ * the copies asynchronous; pageable ones give the same results.
+ *   Size limit: with P = B*T*H*64*2 bytes (one operand) and Q = B*H*64*64*4 bytes (one state), each
+ *   rounded up to a multiple of 256, the call needs 7*P + Q bytes (7*P + 2*Q when s_in is given).
+ *   A call that needs more than RWKV7_NOALLOC_STAGING_BYTES returns RWKV7_ERR_INVALID and enqueues
+ *   nothing.
+ *   Shared array: every call uses the same array, which keeps the previous call's contents (nothing
+ *   in it has to start at zero: each call writes every byte it reads).  Calls whose work overlaps
+ *   on the GPU (other streams, other host threads) race on it; calls on one stream are ordered.
+ *   Set-up: the first call on a device looks up the array's device address (cudaGetSymbolAddress,
+ *   with that device current) and caches it; make that first call before any stream capture.
+ * Other errors as for rwkv7_wkv_prefill_host_bf16. */
+#define RWKV7_NOALLOC_STAGING_BYTES (32u * 1024u * 1024u)
+RWKV7_API rwkv7_status rwkv7_wkv_prefill_host_noalloc_bf16(int path, int B, int T, int H, int N,
+                                                           const uint16_t *r, const uint16_t *w,
+                                                           const uint16_t *k, const uint16_t *v,
+                                                           const uint16_t *a, const uint16_t *b,
+                                                           const float *s_in, uint16_t *y, float *s_out,
+                                                           rwkv7_stream_t stream);
+
 /* bf16 prefill with options (NULL = none); other arguments as for rwkv7_wkv_prefill_bf16_path. */
 RWKV7_API rwkv7_status rwkv7_wkv_prefill_ext_bf16(int path, int B, int T, int H, int N, const uint16_t *r,
                                                   const uint16_t *w, const uint16_t *k, const uint16_t *v,

@@ -29,7 +29,7 @@ __all__ = [
     "rwkv7_wkv_prefill_ext_bf16", "rwkv7_wkv_decode_ext_bf16", "Options",
     "rwkv7_status_string", "rwkv7_get_last_error", "rwkv7_version",
     "rwkv7_wkv_prefill_save_bf16", "rwkv7_wkv_backward_bf16", "rwkv7_wkv_decode_bf16_bf16state",
-    "rwkv7_wkv_prefill_host_bf16", "prefill", "decode_", "prefill_model_native", "decode_model_native_", "prefill_ext", "decode_ext_",
+    "rwkv7_wkv_prefill_host_bf16", "rwkv7_wkv_prefill_host_noalloc_bf16", "NOALLOC_STAGING_BYTES", "prefill", "decode_", "prefill_model_native", "decode_model_native_", "prefill_ext", "decode_ext_",
     "prefill_save", "backward", "EXPORTED_SYMBOLS",
 ]
 
@@ -44,7 +44,10 @@ EXPORTED_SYMBOLS = (
     "rwkv7_wkv_prefill_ext_bf16", "rwkv7_wkv_decode_ext_bf16",
     "rwkv7_wkv_prefill_save_bf16", "rwkv7_wkv_backward_bf16", "rwkv7_wkv_decode_bf16_bf16state",
     "rwkv7_wkv_prefill_host_bf16", "rwkv7_status_string", "rwkv7_get_last_error", "rwkv7_version",
+    "rwkv7_wkv_prefill_host_noalloc_bf16",
 )
+# RWKV7_NOALLOC_STAGING_BYTES of include/rwkv7.h: the staging limit of rwkv7_wkv_prefill_host_noalloc_bf16
+NOALLOC_STAGING_BYTES = 32 * 1024 * 1024
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _lib: Optional[ctypes.CDLL] = None
@@ -94,6 +97,7 @@ def load_library() -> ctypes.CDLL:
         ("rwkv7_wkv_decode_bf16_bf16state", [ci, ci, ci] + [vp] * 6 + [vp, vp, vp]),
         ("rwkv7_wkv_prefill_host_bf16", [ci, ci, ci, ci, ci] + [vp] * 6 + [vp, vp, vp] + [vp] * 6 + [vp, vp, vp]
          + [ci, vp]),
+        ("rwkv7_wkv_prefill_host_noalloc_bf16", [ci] + pre),
     ):
         fn = getattr(lib, name)
         fn.argtypes = args
@@ -200,6 +204,21 @@ def rwkv7_wkv_prefill_host_bf16(path, r, w, k, v, a, b, s_in, y, s_out, dev, sli
     _call("rwkv7_wkv_prefill_host_bf16", int(path), B, T, H, N, *[_ptr(t) for t in (r, w, k, v, a, b, s_in, y, s_out)],
           *[_ptr(dev[n]) for n in ("r", "w", "k", "v", "a", "b")], _ptr(dsi), _ptr(dev["y"]), _ptr(dev["s_out"]),
           int(slices), _stream(stream))
+
+
+def rwkv7_wkv_prefill_host_noalloc_bf16(path, r, w, k, v, a, b, s_in, y, s_out, stream=None) -> None:
+    """bfloat16 prefill from and to host memory that allocates nothing: r .. b, s_in (or None), y and
+    s_out are CPU tensors, staged through the library's static device array (at most
+    ``NOALLOC_STAGING_BYTES`` per call).  For callers that cannot allocate device memory.  Queued on
+    ``stream``; synchronise it before reading y / s_out."""
+    B, T, H, N = r.shape
+    for nm, t in (("r", r), ("w", w), ("k", k), ("v", v), ("a", a), ("b", b), ("y", y)):
+        _check_host(t, nm, torch.bfloat16, (B, T, H, N))
+    _check_host(s_out, "s_out", torch.float32, (B, H, N, N))
+    if s_in is not None:
+        _check_host(s_in, "s_in", torch.float32, (B, H, N, N))
+    _call("rwkv7_wkv_prefill_host_noalloc_bf16", int(path), B, T, H, N,
+          *[_ptr(t) for t in (r, w, k, v, a, b, s_in, y, s_out)], _stream(stream))
 
 
 def rwkv7_wkv_prefill_varlen_bf16(path, cu_seqlens, max_T, r, w, k, v, a, b, s_in, y, s_out, stream=None) -> None:

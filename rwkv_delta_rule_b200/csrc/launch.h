@@ -6,6 +6,11 @@
 
 namespace rwkv7 {
 
+// The library's device error word on the current device (looked up once per device), and the
+// kernel choice of the bf16 prefill entry points for a path value and the longest sequence.
+int *device_error_word();
+bool prefill_uses_chunk(int path, long long max_T);
+
 // Sequential scan over [B,T,H,64] (cu_seqlens == nullptr) or a packed ragged
 // batch (cu_seqlens = device offsets, total_T tokens).  TIn: float or
 // uint16_t (bfloat16 bits).

@@ -60,6 +60,10 @@ rwkv7_status check_prefill(int B, long long tokens, int H, int N, const TIn *r, 
 }
 
 }  // namespace
+
+int *device_error_word() { return error_word_ptr(); }
+bool prefill_uses_chunk(int path, long long max_T) { return use_chunk(path, max_T); }
+
 }  // namespace rwkv7
 
 using namespace rwkv7;

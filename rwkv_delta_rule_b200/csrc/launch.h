@@ -60,6 +60,14 @@ cudaError_t launch_decode_ext(const uint16_t *r, const uint16_t *w, const uint16
                               bool group_norm, const float *ln_w, const float *ln_b, float *s, uint16_t *y, int B,
                               int H, cudaStream_t stream);
 
+// The chunked prefill as a warp-specialised pipeline (one persistent CTA per SM walking its (b, h)
+// pairs' chunks with three chunks in flight); same arguments as launch_chunk_ext without the schedule.
+cudaError_t launch_chunk_pipe(const uint16_t *r, const uint16_t *w, const uint16_t *k, const uint16_t *v,
+                              const uint16_t *a, const uint16_t *b, bool model_native, const float *k_k,
+                              bool group_norm, const float *ln_w, const float *ln_b, const float *s_in, uint16_t *y,
+                              float *s_out, const int32_t *cu_seqlens, int B, int T, long long total_T, int H,
+                              float *states, int *err_word, cudaStream_t stream);
+
 // Chunked tensor-core prefill (bfloat16 operands), same layouts as
 // launch_scan.  err_word: device word that bounded waits report into.
 cudaError_t launch_chunk(const uint16_t *r, const uint16_t *w, const uint16_t *k, const uint16_t *v,

@@ -240,7 +240,7 @@ rwkv7_status rwkv7_wkv_prefill_ext_bf16(int path, int B, int T, int H, int N, co
   const float *k_k = native ? opt->k_k : nullptr;
   const float *ln_w = ln ? opt->ln_w : nullptr, *ln_b = ln ? opt->ln_b : nullptr;
   const int schedule = opt != nullptr ? opt->chunk_schedule : 0;
-  if (schedule < 0 || schedule > 2) return RWKV7_ERR_INVALID;
+  if (schedule < 0 || schedule > 3) return RWKV7_ERR_INVALID;
   // model-native calls have no b: the shared checks see a in its place
   const rwkv7_status st = check_prefill(B, T, H, N, r, w, k, v, a, native ? a : b, s_in, y, s_out);
   if (st != RWKV7_OK) return st;

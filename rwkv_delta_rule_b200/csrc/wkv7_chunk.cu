@@ -1422,6 +1422,9 @@ cudaError_t launch_chunk_ext(const uint16_t *r, const uint16_t *w, const uint16_
                              float *s_out, const int32_t *cu_seqlens, int B, int T, long long total_T, int H,
                              int schedule, float *states, int *err_word, cudaStream_t stream) {
   using namespace chunk;
+  if (schedule == 3)
+    return launch_chunk_pipe(r, w, k, v, a, b, model_native, k_k, group_norm, ln_w, ln_b, s_in, y, s_out, cu_seqlens,
+                             B, T, total_T, H, states, err_word, stream);
   if (states != nullptr && cu_seqlens != nullptr) return cudaErrorInvalidValue;
   if (total_T > 0x7fffffffLL || H > 0xffff || B > 65535) return cudaErrorInvalidValue;
   Maps maps;

@@ -75,14 +75,22 @@ typedef enum rwkv7_status {
   RWKV7_ERR_ALIGN = 2,
   RWKV7_ERR_CUDA = 3,
   RWKV7_ERR_TIMEOUT = 4,
-  RWKV7_ERR_UNSUPPORTED = 5
+  RWKV7_ERR_UNSUPPORTED = 5,
+  RWKV7_ERR_DOMAIN = 6
 } rwkv7_status;
 
 /* Prefill kernels: AUTO picks by T and dtype (bf16 with T >= 128 -> CHUNK,
  * otherwise SCAN); SCAN is the sequential kernel (state in registers); CHUNK
- * is the chunked tensor-core kernel (bf16 only).  CHUNK requires every decay
- * w >= 0.27 (it divides by products of up to 64 decays in float32); the
- * model's decay exp(-e^-0.5 sigmoid(x)) always lies in [0.5452, 1). */
+ * is the chunked tensor-core kernel (bf16 only).
+ * Decay domain of CHUNK: the chunked form divides by the product of up to 64
+ * consecutive decays.  Its schedules 0-2 (see rwkv7_options.chunk_schedule)
+ * need that product to stay >= 2^-100 in every channel of every 64-token
+ * chunk (true whenever every w >= 0.34; the model's decay
+ * exp(-e^-0.5 sigmoid(x)) always lies in [0.5452, 1)); a chunk outside it is
+ * detected on the device and reported by rwkv7_get_last_error() as
+ * RWKV7_ERR_DOMAIN, and that call's y and s_out are not valid.  Schedule 3 and
+ * SCAN are exact for every w in [0, 1] (schedule 3 runs such a chunk token by
+ * token in float32). */
 typedef enum rwkv7_prefill_path {
   RWKV7_PATH_AUTO = 0,
   RWKV7_PATH_SCAN = 1,
@@ -184,6 +192,10 @@ RWKV7_API rwkv7_status rwkv7_wkv_decode_fused_bf16(int B, int H, int N, const ui
  *                         Needs B*H <= 65536 (else RWKV7_ERR_CUDA).  Up to 4 such launches may
  *                         run at once on a device; the launch can be captured in a CUDA graph
  *                         and replayed (every launch leaves the flags zeroed unless it fails).
+ *                     3 = a warp-specialised pipeline: one persistent CTA per SM walks its (b, h)
+ *                         pairs' chunks with three chunks in flight (operand preparation, masks
+ *                         and inverse, state chain on separate warps); exact for every decay in
+ *                         [0, 1] (see the decay domain above).  Needs H <= 65535.
  */
 typedef struct rwkv7_options {
   int model_native;
@@ -316,8 +328,9 @@ RWKV7_API rwkv7_status rwkv7_wkv_backward_bf16(int B, int T, int H, int N, const
 /* Static English description of a status code (never NULL). */
 RWKV7_API const char *rwkv7_status_string(rwkv7_status status);
 
-/* Reads and clears the device error word of the current device (RWKV7_OK or
- * RWKV7_ERR_TIMEOUT), and reports a pending CUDA error as RWKV7_ERR_CUDA.
+/* Reads and clears the device error word of the current device (RWKV7_OK,
+ * RWKV7_ERR_TIMEOUT or RWKV7_ERR_DOMAIN: the first error recorded since the
+ * last call), and reports a pending CUDA error as RWKV7_ERR_CUDA.
  * Synchronises the current device. */
 RWKV7_API rwkv7_status rwkv7_get_last_error(void);
 

@@ -23,7 +23,7 @@ import torch
 
 __all__ = [
     "RWKV7_PATH_AUTO", "RWKV7_PATH_SCAN", "RWKV7_PATH_CHUNK", "RWKV7_SCHED_AUTO", "RWKV7_SCHED_PAIR",
-    "RWKV7_SCHED_TASKS", "Rwkv7Error", "library_path", "load_library",
+    "RWKV7_SCHED_TASKS", "RWKV7_SCHED_PIPE", "Rwkv7Error", "library_path", "load_library",
     "rwkv7_wkv_prefill", "rwkv7_wkv_prefill_bf16", "rwkv7_wkv_prefill_bf16_path", "rwkv7_wkv_prefill_varlen_bf16",
     "rwkv7_wkv_decode", "rwkv7_wkv_decode_bf16", "rwkv7_wkv_prefill_fused_bf16", "rwkv7_wkv_decode_fused_bf16",
     "rwkv7_wkv_prefill_ext_bf16", "rwkv7_wkv_decode_ext_bf16", "Options",
@@ -35,7 +35,7 @@ __all__ = [
 
 RWKV7_PATH_AUTO, RWKV7_PATH_SCAN, RWKV7_PATH_CHUNK = 0, 1, 2
 # chunk-path schedules (rwkv7_options.chunk_schedule)
-RWKV7_SCHED_AUTO, RWKV7_SCHED_PAIR, RWKV7_SCHED_TASKS = 0, 1, 2
+RWKV7_SCHED_AUTO, RWKV7_SCHED_PAIR, RWKV7_SCHED_TASKS, RWKV7_SCHED_PIPE = 0, 1, 2, 3
 N_HEAD = 64
 
 EXPORTED_SYMBOLS = (

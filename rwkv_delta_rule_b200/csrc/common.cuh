@@ -12,7 +12,9 @@ constexpr int kN = 64;  // head size; the pages fix it at 64 (compile-time -D_N_
 // Device error word: kernels that give up on a bounded wait store a nonzero
 // code through the pointer they are given (the library's word, defined in
 // rwkv7_api.cu); the host reads and clears it in rwkv7_get_last_error().
-enum DeviceError : int { kDevErrNone = 0, kDevErrTimeout = 1 };
+// kDevErrDomain: a chunked-prefill kernel met a chunk whose decay product lies outside what it can
+// factorise (its results for that call are not valid).
+enum DeviceError : int { kDevErrNone = 0, kDevErrTimeout = 1, kDevErrDomain = 2 };
 
 __device__ __forceinline__ void report_device_error(int *word, int code) {
   if (word != nullptr) atomicCAS(word, 0, code);

@@ -78,6 +78,7 @@ const char *rwkv7_status_string(rwkv7_status status) {
     case RWKV7_ERR_CUDA: return "CUDA error";
     case RWKV7_ERR_TIMEOUT: return "device wait timed out";
     case RWKV7_ERR_UNSUPPORTED: return "unsupported size (head size must be 64)";
+    case RWKV7_ERR_DOMAIN: return "decay product of a chunk outside the chunked kernel's range (outputs invalid)";
   }
   return "unknown status";
 }
@@ -91,7 +92,8 @@ rwkv7_status rwkv7_get_last_error(void) {
   if (cudaMemcpyFromSymbol(&word, g_error_word, sizeof(int)) != cudaSuccess) return RWKV7_ERR_CUDA;
   if (word != 0 && cudaMemcpyToSymbol(g_error_word, &zero, sizeof(int)) != cudaSuccess) return RWKV7_ERR_CUDA;
   if (cudaGetLastError() != cudaSuccess) return RWKV7_ERR_CUDA;
-  return word == kDevErrNone ? RWKV7_OK : RWKV7_ERR_TIMEOUT;
+  if (word == kDevErrNone) return RWKV7_OK;
+  return word == kDevErrDomain ? RWKV7_ERR_DOMAIN : RWKV7_ERR_TIMEOUT;
 }
 
 rwkv7_status rwkv7_wkv_prefill(int B, int T, int H, int N, const float *r, const float *w, const float *k,

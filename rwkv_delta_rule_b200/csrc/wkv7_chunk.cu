@@ -433,7 +433,8 @@ __device__ __forceinline__ void invert_unit_lower(const float *Ls, float *Ts, fl
 // operand construction of R~ and A~ forms it.  Warps 4-7 synchronise among themselves.
 template <bool kFused>
 __device__ __forceinline__ void prep_next(const uint8_t *smem, uint8_t *sA1, uint8_t *sB1, uint8_t *sB4Vn, float *pre4,
-                                          float *GCn, float *wtot, const float *kkw, float *invn, int tid4, int Lcn) {
+                                          float *GCn, float *wtot, const float *kkw, float *invn, int tid4, int Lcn,
+                                          int *err) {
   const int lane = tid4 & 31, wq = tid4 >> 5;
   const int cq = tid4 & 15, to = tid4 >> 4;  // channel quad; token octet (2 per warp)
   const int j0 = 4 * cq, tb = 8 * to;
@@ -514,6 +515,11 @@ __device__ __forceinline__ void prep_next(const uint8_t *smem, uint8_t *sA1, uin
   *reinterpret_cast<float4 *>(pre4 + (2 * to) * 64 + j0) = make_float4(p0[0], p0[1], p0[2], p0[3]);
   *reinterpret_cast<float4 *>(pre4 + (2 * to + 1) * 64 + j0) = make_float4(p1[0], p1[1], p1[2], p1[3]);
   if (to == 0) *reinterpret_cast<float4 *>(GCn + j0) = make_float4(gc[0], gc[1], gc[2], gc[3]);
+  // B^ and K^ divide by the decay products of the chunk: below 2^-100 (or not a number) the factors
+  // leave float32's range and the chunk's results are not valid; the call reports it
+  if (to == 0 && !(gc[0] >= 7.8886090522101181e-31f && gc[1] >= 7.8886090522101181e-31f &&
+                   gc[2] >= 7.8886090522101181e-31f && gc[3] >= 7.8886090522101181e-31f))
+    report_device_error(err, kDevErrDomain);
   // [B^; K^] rows (K-major tf32; K = channel), and Gamma_t itself (float32) where the operand
   // construction will put R~ = r Gamma_t: it reads Gamma_t there and overwrites it in place
   uint8_t *b1r = sB1 + (j0 >> 5) * (128 * 128);
@@ -1024,7 +1030,7 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
         if (t0.n >= 0) {
           load_head(t0.h, 0, tid - 128);
           group_sync_hi();
-          prep_next<kFused>(smem, sA1, sB1, sB4V, pre4, GCs, wtot, kkw, invn, tid - 128, t0.Lc);
+          prep_next<kFused>(smem, sA1, sB1, sB4V, pre4, GCs, wtot, kkw, invn, tid - 128, t0.Lc, A.err);
         }
       }
       compute_sync();
@@ -1037,7 +1043,7 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
         load_head(have ? t.h : 0, 1, tid - 128);
       }
       if (have && warp >= 4 && wait_group_hi(bar_tma, 0))
-        prep_next<kFused>(smem, sA1, sB1, sB4V, pre4, GCs, wtot, kkw, invn, tid - 128, t.Lc);
+        prep_next<kFused>(smem, sA1, sB1, sB4V, pre4, GCs, wtot, kkw, invn, tid - 128, t.Lc, A.err);
       compute_sync();
     }
 
@@ -1226,14 +1232,14 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
               load_head(nt.h, (it + 1) & 1, tid - 128);
               group_sync_hi();
               prep_next<kFused>(smem, sA1, sB1, sB4V + ((it + 1) & 1) * 16384, pre4,
-                                       GCs + ((it + 1) & 1) * 64, wtot, kkw, invn, tid - 128, nt.Lc);
+                                       GCs + ((it + 1) & 1) * 64, wtot, kkw, invn, tid - 128, nt.Lc, A.err);
             }
           }
         } else {
           Task nt = t;
           if (pair_next(A, nt) && wait_group_hi(bar_tma, (it + 1) & 1))
             prep_next<kFused>(smem, sA1, sB1, sB4V + ((it + 1) & 1) * 16384, pre4, GCs + ((it + 1) & 1) * 64,
-                                     wtot, kkw, invn, tid - 128, nt.Lc);
+                                     wtot, kkw, invn, tid - 128, nt.Lc, A.err);
         }
       }
       if (!(ok = wait_ctrl(bar_m3, ph))) break;

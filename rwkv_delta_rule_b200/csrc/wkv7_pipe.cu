@@ -270,6 +270,20 @@ __device__ __forceinline__ void unpack8(const uint4 &u, float (&v)[8]) {
   v[6] = __uint_as_float(u.w << 16);
   v[7] = __uint_as_float(u.w & 0xffff0000u);
 }
+// 16 floats -> 8 bf16 pairs as the register image of 8 TMEM columns
+__device__ __forceinline__ void pack16(const float (&v)[16], float (&p)[8]) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) p[i] = __uint_as_float(pack_bf16x2(v[2 * i], v[2 * i + 1]));
+}
+// the 16-byte bf16 chunk of v[8h .. 8h + 7]
+__device__ __forceinline__ uint4 pack_half(const float (&v)[16], int h) {
+  return make_uint4(pack_bf16x2(v[8 * h], v[8 * h + 1]), pack_bf16x2(v[8 * h + 2], v[8 * h + 3]),
+                    pack_bf16x2(v[8 * h + 4], v[8 * h + 5]), pack_bf16x2(v[8 * h + 6], v[8 * h + 7]));
+}
+__device__ __forceinline__ void keep16(float (&v)[16], int col0, int lim) {
+#pragma unroll
+  for (int x = 0; x < 16; ++x) v[x] = col0 + x <= lim ? v[x] : 0.f;
+}
 // keep v[x] where col0 + x <= lim (causal mask); zero the rest
 __device__ __forceinline__ void keep8(float (&v)[8], int col0, int lim) {
 #pragma unroll
@@ -315,9 +329,9 @@ struct Group {
   volatile int *slot;
   uint32_t calls;
 };
-__device__ __noinline__ bool gwait(Group &g, const Ctl &ctl, uint64_t *b0, uint32_t p0, uint64_t *b1 = nullptr,
-                                   uint32_t p1 = 0, uint64_t *b2 = nullptr, uint32_t p2 = 0,
-                                   uint64_t *b3 = nullptr, uint32_t p3 = 0) {
+__device__ __forceinline__ bool gwait(Group &g, const Ctl &ctl, uint64_t *b0, uint32_t p0, uint64_t *b1 = nullptr,
+                                      uint32_t p1 = 0, uint64_t *b2 = nullptr, uint32_t p2 = 0,
+                                      uint64_t *b3 = nullptr, uint32_t p3 = 0) {
   const uint32_t s = g.calls++ & 1u;
   if (g.leader) {
     bool ok = wait_or_abort(b0, p0, ctl.abort);
@@ -350,17 +364,33 @@ __device__ __forceinline__ void block16_store_bf16(uint8_t *op, int row0, int co
   }
 }
 // The four 16x16 diagonal blocks D_s = (I - L_ss)^-1 by forward substitution, into Ts (float32), run
-// by two warps: lanes 0-15 of warp w solve block 2w, lanes 16-31 block 2w + 1, one column per lane
-// (x_r = [r == c] + sum_{q<r} L_rq x_q, pushed column by column so a step's updates are independent).
+// by two warps: lanes 0-15 of warp w solve block 2w, lanes 16-31 block 2w + 1, one column c per lane:
+// x_r = [r == c] + sum_{q<r} L_rq x_q, row by row, each row of L read with 16-byte loads as it is
+// needed (the sum split over two accumulators to halve the dependent chain).
 __device__ __forceinline__ void invert_diagonal(const float *Ls, float *Ts, int w, int lane) {
   const int blk = 2 * w + (lane >> 4), base = 16 * blk, cix = lane & 15;
   float x[16];
+  x[0] = cix == 0 ? 1.f : 0.f;
 #pragma unroll
-  for (int r = 0; r < 16; ++r) x[r] = (r == cix) ? 1.f : 0.f;
+  for (int r = 1; r < 16; ++r) {
+    const float *row = Ls + (base + r) * LDL + base;
+    float acc0 = (r == cix) ? 1.f : 0.f, acc1 = 0.f;
 #pragma unroll
-  for (int q = 0; q < 15; ++q) {
+    for (int q4 = 0; q4 < (r + 3) / 4; ++q4) {
+      const float4 u = *reinterpret_cast<const float4 *>(row + 4 * q4);
+      const float uu[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-    for (int r = q + 1; r < 16; ++r) x[r] = fmaf(Ls[(base + r) * LDL + base + q], x[q], x[r]);
+      for (int e = 0; e < 4; ++e) {
+        const int q = 4 * q4 + e;
+        if (q < r) {
+          if (q & 1)
+            acc1 = fmaf(uu[e], x[q], acc1);
+          else
+            acc0 = fmaf(uu[e], x[q], acc0);
+        }
+      }
+    }
+    x[r] = acc0 + acc1;
   }
   float *D = ts_block(Ts, blk, blk);
 #pragma unroll
@@ -579,10 +609,8 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_pipe_kernel(const __grid_con
 
   if (warp == W_MMA) {
     // ===== MMA issue ==================================================================================
-    // Per chunk n, in this order: MMA1 of chunk n + 1 (its preparation finishes early in the mask stage
-    // of chunk n), MMA3, MMA2 + MMA4a and MMA4b of chunk n.  MMAs of one thread run in issue order, so
-    // an MMA may read what an earlier one wrote with no wait in between, and overwrite what an earlier
-    // one read (MMA1 of chunk n + 1 reuses the X slot of chunk n - 1, whose MMA4b came before).
+    // MMAs of one thread run in issue order, so an MMA may read what an earlier one wrote with no wait
+    // in between, and overwrite what an earlier one read.
     if (lane == 0) {
       long long total = 0;
       {
@@ -608,66 +636,87 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_pipe_kernel(const __grid_con
         }
         tc::mma_commit(bar(B_M1));
       };
-      long long n = 0;
-      bool ok = total > 0;
-      if (ok && (ok = wait_or_abort(bar(B_AB_FULL), 0, abort_flag))) {
-        tc::tc_fence_after();
-        mma1(0);
-      }
-      for (; ok && n < total; ++n) {
-        const uint32_t sl = static_cast<uint32_t>(n & 1);
-        // MMA1 of chunk n + 1 and MMA3 of chunk n (D3 = [A~^T; Lak^T] Tinv^T, into the D4 slot of chunk n,
-        // once chunk n - 2 is read out), in the order their inputs arrive
-        {
-          bool need1 = n + 1 < total, need3 = true;
-          const uint32_t p1 = static_cast<uint32_t>((n + 1) & 1), pe = static_cast<uint32_t>(((n >> 1) + 1) & 1);
-          const uint64_t t0 = tc::globaltimer_ns();
-          while (need1 || need3) {
-            if (need3 && tc::mbar_test_wait(bar(B_B3), sl) &&
-                (n < 2 || tc::mbar_test_wait(bar(B_D4_EMPTY + sl), pe))) {
-              tc::tc_fence_after();
+      // The next chunk of each MMA kind; each is issued as soon as its inputs are there, the later
+      // stages first.  MMA1 of chunk c reuses the X slot of chunk c - 2 (its MMA4b must have been
+      // issued), MMA3 of chunk c the D4 slot of chunk c - 2 (read out) and B2 of chunk c - 1 (MMA2 of
+      // chunk c - 1 issued before it).
+      long long i1 = 0, i3 = 0, i2 = 0, i4 = 0;
+      bool ok = true;
+      uint64_t t_idle = 0;
+      while (i4 < total) {
+        if (i4 < i2 && tc::mbar_test_wait(bar(B_S_FULL), static_cast<uint32_t>(i4 & 1))) {
+          // MMA4b (tf32, A from TMEM): D4 += [Q; E] S0^T
+          tc::tc_fence_after();
+          const uint32_t sl = static_cast<uint32_t>(i4 & 1);
 #pragma unroll
-              for (int ks = 0; ks < 4; ++ks)
-                tc::mma_ss(0, tmem + TM_D4 + 64 * sl, dA3 + ((ks * 2048) >> 4), dB3 + ((ks * 32) >> 4), id3, ks > 0);
-              tc::mma_commit(bar(B_M3));
-              need3 = false;
-            } else if (need1 && tc::mbar_test_wait(bar(B_AB_FULL), p1)) {
-              tc::tc_fence_after();
-              mma1(n + 1);
-              need1 = false;
-            } else {
-              (void)tc::mbar_try_wait_hint(need1 ? bar(B_AB_FULL) : bar(B_B3), need1 ? p1 : sl, 200);
-              if (*abort_flag || tc::globaltimer_ns() - t0 > kWaitLimitNs) {
-                ok = false;
-                break;
-              }
-            }
+          for (int ks = 0; ks < 8; ++ks) {
+            const uint32_t off = (ks >> 2) * (64 * 128) + (ks & 3) * 32;
+            tc::mma_ts_tf32(tmem + TM_D4 + 64 * sl, tmem + TM_X + 128 * sl + 8 * ks, dS + (off >> 4), id4, 1);
           }
-          if (!ok) break;
-        }
-        // MMA2 (bf16, A from TMEM): D2 += [Mrb; B-^T] [W~ U~]; MMA4a (tf32): D4 = [P; F] V
-        if (!(ok = wait_or_abort(bar(B_B2), sl, abort_flag))) break;
-        if (!(ok = wait_or_abort(bar(B_VT_FULL), sl, abort_flag))) break;
-        tc::tc_fence_after();
+          tc::mma_commit(bar(B_M4 + sl));
+          ++i4;
+          t_idle = 0;
+        } else if (i2 < i3 && tc::mbar_test_wait(bar(B_B2), static_cast<uint32_t>(i2 & 1)) &&
+                   tc::mbar_test_wait(bar(B_VT_FULL), static_cast<uint32_t>(i2 & 1))) {
+          // MMA2 (bf16, A from TMEM): D2 += [Mrb; B-^T] [W~ U~]; MMA4a (tf32): D4 = [P; F] V
+          tc::tc_fence_after();
+          const uint32_t sl = static_cast<uint32_t>(i2 & 1);
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-          tc::mma_ts_bf16(tmem + TM_X + 128 * sl, tmem + TM_A2 + 32 * sl + 8 * ks, dB2 + ((ks * 32) >> 4), id2, 1);
-        tc::mma_commit(bar(B_M2));
+          for (int ks = 0; ks < 4; ++ks)
+            tc::mma_ts_bf16(tmem + TM_X + 128 * sl, tmem + TM_A2 + 32 * sl + 8 * ks, dB2 + ((ks * 32) >> 4), id2, 1);
+          tc::mma_commit(bar(B_M2));
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint32_t off = (ks >> 2) * (64 * 128) + (ks & 3) * 32;
-          tc::mma_ts_tf32(tmem + TM_D4 + 64 * sl, tmem + TM_X + 128 * sl + 64 + 8 * ks, dVT + (off >> 4), id4, ks > 0);
-        }
-        tc::mma_commit(bar(B_M4A));
-        // MMA4b (tf32, A from TMEM): D4 += [Q; E] S0^T, once the state is in B4S
-        if (!(ok = wait_or_abort(bar(B_S_FULL), sl, abort_flag))) break;
-        tc::tc_fence_after();
+          for (int ks = 0; ks < 8; ++ks) {
+            const uint32_t off = (ks >> 2) * (64 * 128) + (ks & 3) * 32;
+            tc::mma_ts_tf32(tmem + TM_D4 + 64 * sl, tmem + TM_X + 128 * sl + 64 + 8 * ks, dVT + (off >> 4), id4,
+                            ks > 0);
+          }
+          tc::mma_commit(bar(B_M4A));
+          ++i2;
+          t_idle = 0;
+        } else if (i3 < i1 && i3 <= i2 && tc::mbar_test_wait(bar(B_B3), static_cast<uint32_t>(i3 & 1)) &&
+                   (i3 < 2 || tc::mbar_test_wait(bar(B_D4_EMPTY + (i3 & 1)), static_cast<uint32_t>(((i3 >> 1) + 1) & 1)))) {
+          // MMA3 (bf16): D3 = [A~^T; Lak^T] Tinv^T, into the D4 slot of the chunk
+          tc::tc_fence_after();
+          const uint32_t sl = static_cast<uint32_t>(i3 & 1);
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint32_t off = (ks >> 2) * (64 * 128) + (ks & 3) * 32;
-          tc::mma_ts_tf32(tmem + TM_D4 + 64 * sl, tmem + TM_X + 128 * sl + 8 * ks, dS + (off >> 4), id4, 1);
+          for (int ks = 0; ks < 4; ++ks)
+            tc::mma_ss(0, tmem + TM_D4 + 64 * sl, dA3 + ((ks * 2048) >> 4), dB3 + ((ks * 32) >> 4), id3, ks > 0);
+          tc::mma_commit(bar(B_M3));
+          ++i3;
+          t_idle = 0;
+        } else if (i1 < total && i1 <= i4 + 1 && tc::mbar_test_wait(bar(B_AB_FULL), static_cast<uint32_t>(i1 & 1))) {
+          tc::tc_fence_after();
+          mma1(i1);
+          ++i1;
+          t_idle = 0;
+        } else {
+          // nothing ready: sleep on the barrier the pipeline most likely waits for (up to 0.5 us; it wakes
+          // when that barrier completes), bounded in time
+          uint64_t *wb;
+          uint32_t wp;
+          if (i4 < i2) {
+            wb = bar(B_S_FULL);
+            wp = static_cast<uint32_t>(i4 & 1);
+          } else if (i2 < i3) {
+            wb = bar(B_B2);
+            wp = static_cast<uint32_t>(i2 & 1);
+          } else if (i3 < i1) {
+            wb = bar(B_B3);
+            wp = static_cast<uint32_t>(i3 & 1);
+          } else {
+            wb = bar(B_AB_FULL);
+            wp = static_cast<uint32_t>(i1 & 1);
+          }
+          (void)tc::mbar_try_wait_hint(wb, wp, 500);
+          const uint64_t now = tc::globaltimer_ns();
+          if (t_idle == 0) {
+            t_idle = now;
+          } else if (*abort_flag || now - t_idle > kWaitLimitNs) {
+            ok = false;
+            break;
+          }
         }
-        tc::mma_commit(bar(B_M4 + sl));
       }
       if (!ok) fail(ctl);
       // every MMA issued here completes before the CTA exits (a commit tracks all earlier MMAs of the
@@ -928,37 +977,39 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_pipe_kernel(const __grid_con
       if (q >= 2) {
         // A~ row t (A1) -> the A~^T block of A3 (bf16; MMA3 of the previous chunk is done with A3)
 #pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
-          float v[8];
-          tc::tmem_ld8(A1 + 8 * c, v);
-          *reinterpret_cast<uint4 *>(sA3 + tc::sw128(t, c)) = pack8(v);
+        for (int c = 0; c < 4; ++c) {
+          float v[16];
+          tc::tmem_ld16(A1 + 16 * c, v);
+          *reinterpret_cast<uint4 *>(sA3 + tc::sw128(t, 2 * c)) = pack_half(v, 0);
+          *reinterpret_cast<uint4 *>(sA3 + tc::sw128(t, 2 * c + 1)) = pack_half(v, 1);
         }
         tc::tc_fence_before();
         if (lane == 0) tc::mbar_arrive(bar(B_A1_EMPTY));
         __syncwarp();
         // rows of Lab (strictly lower, m < t) -> Ls
 #pragma unroll 1
-        for (int c = 0; c < 4 * (dh + 1); ++c) {
-          float v[8];
-          tc::tmem_ld8(X + 8 * c, v);
-          keep8(v, 8 * c, t - 1);
-          float *row = Ls + t * LDL + 8 * c;
-          *reinterpret_cast<float4 *>(row) = make_float4(v[0], v[1], v[2], v[3]);
-          *reinterpret_cast<float4 *>(row + 4) = make_float4(v[4], v[5], v[6], v[7]);
+        for (int c = 0; c < 2 * (dh + 1); ++c) {
+          float v[16];
+          tc::tmem_ld16(X + 16 * c, v);
+          keep16(v, 16 * c, t - 1);
+          float *row = Ls + t * LDL + 16 * c;
+#pragma unroll
+          for (int x = 0; x < 16; x += 4) *reinterpret_cast<float4 *>(row + x) = make_float4(v[x], v[x + 1], v[x + 2], v[x + 3]);
         }
         nbar_arrive(NB_LS, 128);
         // rows of Lak (strictly lower) -> the Lak^T block of A3
 #pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
-          float v[8];
-          if (c < 4 * (dh + 1)) {
-            tc::tmem_ld8(X + 64 + 8 * c, v);
-            keep8(v, 8 * c, t - 1);
+        for (int c = 0; c < 4; ++c) {
+          float v[16];
+          if (c < 2 * (dh + 1)) {
+            tc::tmem_ld16(X + 64 + 16 * c, v);
+            keep16(v, 16 * c, t - 1);
           } else {
 #pragma unroll
-            for (int x = 0; x < 8; ++x) v[x] = 0.f;
+            for (int x = 0; x < 16; ++x) v[x] = 0.f;
           }
-          *reinterpret_cast<uint4 *>(sA3 + 64 * 128 + tc::sw128(t, c)) = pack8(v);
+          *reinterpret_cast<uint4 *>(sA3 + 64 * 128 + tc::sw128(t, 2 * c)) = pack_half(v, 0);
+          *reinterpret_cast<uint4 *>(sA3 + 64 * 128 + tc::sw128(t, 2 * c + 1)) = pack_half(v, 1);
         }
         // the D2 set-up of lanes 64..127 (Lab and Lak have been read): E-part = 0, F-part = K-^T[j][m] =
         // Gamma_C[j] K^[m][j] (column j of the B1 slot's K^ rows); A2's lower half B-^T[j][m] =
@@ -967,53 +1018,53 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_pipe_kernel(const __grid_con
         const uint8_t *colb = b1 + (t >> 5) * (128 * 128) + (t & 3) * 4;
         const uint32_t cchunk = (t & 31) >> 2;
 #pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
-          float kv[8], bv[8], z[8];
+        for (int c = 0; c < 4; ++c) {
+          float kv[16], bv[16], z[16], bp[8];
 #pragma unroll
-          for (int x = 0; x < 8; ++x) {
-            const uint32_t sw = (cchunk ^ x) << 4;  // row 8c + x (and 64 + 8c + x) has (row & 7) == x
-            kv[x] = gcj * *reinterpret_cast<const float *>(colb + (64 + 8 * c + x) * 128 + sw);
-            bv[x] = gcj * *reinterpret_cast<const float *>(colb + (8 * c + x) * 128 + sw);
+          for (int x = 0; x < 16; ++x) {
+            const uint32_t sw = (cchunk ^ (x & 7)) << 4;  // row 16c + x (and 64 + 16c + x) has (row & 7) == x & 7
+            kv[x] = gcj * *reinterpret_cast<const float *>(colb + (64 + 16 * c + x) * 128 + sw);
+            bv[x] = gcj * *reinterpret_cast<const float *>(colb + (16 * c + x) * 128 + sw);
             z[x] = 0.f;
           }
-          tc::tmem_st8(X + 64 + 8 * c, kv);
-          tc::tmem_st8(X + 8 * c, z);
-          const uint4 bp = pack8(bv);
-          tc::tmem_st4u(A2 + 4 * c, bp.x, bp.y, bp.z, bp.w);
+          tc::tmem_st16(X + 64 + 16 * c, kv);
+          tc::tmem_st16(X + 16 * c, z);
+          pack16(bv, bp);
+          tc::tmem_st8(A2 + 8 * c, bp);
         }
         tc::tmem_st_wait();
       } else {
         // rows of Mrb (inclusive, m <= t) -> A2 upper half; R~ row t (A1) over them: the Q-part of D2
 #pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
-          float v[8];
-          if (c < 4 * (dh + 1)) {
-            tc::tmem_ld8(X + 8 * c, v);
-            keep8(v, 8 * c, t);
+        for (int c = 0; c < 4; ++c) {
+          float v[16], bp[8];
+          if (c < 2 * (dh + 1)) {
+            tc::tmem_ld16(X + 16 * c, v);
+            keep16(v, 16 * c, t);
           } else {
 #pragma unroll
-            for (int x = 0; x < 8; ++x) v[x] = 0.f;
+            for (int x = 0; x < 16; ++x) v[x] = 0.f;
           }
-          const uint4 bp = pack8(v);
-          tc::tmem_st4u(A2 + 4 * c, bp.x, bp.y, bp.z, bp.w);
-          tc::tmem_ld8(A1 + 8 * c, v);
-          tc::tmem_st8(X + 8 * c, v);
+          pack16(v, bp);
+          tc::tmem_st8(A2 + 8 * c, bp);
+          tc::tmem_ld16(A1 + 16 * c, v);
+          tc::tmem_st16(X + 16 * c, v);
         }
         tc::tc_fence_before();
         if (lane == 0) tc::mbar_arrive(bar(B_A1_EMPTY));
         __syncwarp();
         // rows of Mrk (inclusive) masked in place: the P-part
 #pragma unroll 1
-        for (int c = 4 * dh; c < 8; ++c) {
-          float v[8];
-          if (c < 4 * (dh + 1)) {
-            tc::tmem_ld8(X + 64 + 8 * c, v);
-            keep8(v, 8 * c, t);
+        for (int c = 2 * dh; c < 4; ++c) {
+          float v[16];
+          if (c < 2 * (dh + 1)) {
+            tc::tmem_ld16(X + 64 + 16 * c, v);
+            keep16(v, 16 * c, t);
           } else {
 #pragma unroll
-            for (int x = 0; x < 8; ++x) v[x] = 0.f;
+            for (int x = 0; x < 16; ++x) v[x] = 0.f;
           }
-          tc::tmem_st8(X + 64 + 8 * c, v);
+          tc::tmem_st16(X + 64 + 16 * c, v);
         }
         tc::tmem_st_wait();
         // the diagonal blocks of the inverse, once Lab is in Ls
@@ -1037,10 +1088,11 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_pipe_kernel(const __grid_con
       {
         const uint32_t nrow = 32 * q + lane;
 #pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
-          float v[8];
-          tc::tmem_ld8(tmem + TM_D4 + 64 * sl + lane_base + 8 * c, v);
-          *reinterpret_cast<uint4 *>(sB2 + tc::sw128(nrow, c)) = pack8(v);
+        for (int c = 0; c < 4; ++c) {
+          float v[16];
+          tc::tmem_ld16(tmem + TM_D4 + 64 * sl + lane_base + 16 * c, v);
+          *reinterpret_cast<uint4 *>(sB2 + tc::sw128(nrow, 2 * c)) = pack_half(v, 0);
+          *reinterpret_cast<uint4 *>(sB2 + tc::sw128(nrow, 2 * c + 1)) = pack_half(v, 1);
         }
       }
       tc::fence_proxy_async_smem();

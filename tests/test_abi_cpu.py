@@ -51,6 +51,7 @@ def test_library_needs_no_shared_cuda_runtime():
 def test_status_strings(cdll):
     assert lib7.rwkv7_status_string(0) == "ok"
     assert "64" in lib7.rwkv7_status_string(5)
+    assert "range" in lib7.rwkv7_status_string(6)
     assert lib7.rwkv7_status_string(99) == "unknown status"
     assert lib7.rwkv7_version() >= 100
 

@@ -1,0 +1,122 @@
+"""GPU parity of the prefill across the decay domain [0, 1] against the float64 oracle.
+
+The chunked form divides by the product of up to 64 consecutive decays.  The model's decays lie in
+[0.5452, 1) (RWKV-7 G0 7.2B walkthrough, lshu.cn/news/198401, section 7.1), but the recurrence takes any
+w in [0, 1], so the kernels are checked on decays the model never produces:
+  * w ~ U(0.27, 0.55): every chunked schedule stays inside its factorised range and matches the oracle;
+  * w ~ U(0.02, 0.27), w = 0 in places, and a long sequence with a stretch of fast decays: the
+    pipelined schedule (which runs an out-of-range chunk token by token) and the sequential scan match
+    the oracle, and the other chunked schedules report RWKV7_ERR_DOMAIN instead of returning silently;
+  * w = 1 everywhere (no decay at all).
+Bars as for every bf16 parity test: max|gpu - oracle| / max|oracle| <= 5e-3 for y and the end state.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import rwkv_delta_rule_b200 as rk
+import wkv7_inputs as wi
+from helpers import OPS, TOL_BF16, need_cuda, oracle_ops, rel_err, to_dev
+
+pytestmark = pytest.mark.gpu
+
+ERR_DOMAIN = 6
+
+
+@pytest.fixture(autouse=True)
+def _cuda():
+    need_cuda()
+    rk.load_library()
+    assert rk.rwkv7_get_last_error() == 0
+    yield
+
+
+def _draw(B, T, H, seed, wfun):
+    """The config generator's inputs with the decay replaced by wfun(generator, shape), rounded to bf16."""
+    d = wi.draw(B, T, H, seed=seed, s0_std=0.1)
+    g = torch.Generator().manual_seed(seed + 1)
+    w = wfun(g, d["w"].shape).to(torch.bfloat16)
+    d["w"], d["w_f32"] = w, w.float()
+    return d
+
+
+def _uniform(lo, hi):
+    return lambda g, shape: lo + (hi - lo) * torch.rand(shape, generator=g)
+
+
+def _chunk(d, sched, path=rk.RWKV7_PATH_CHUNK):
+    dv = to_dev(d)
+    y, s = rk.prefill_ext(*[dv[n] for n in OPS], dv["s0"], path=path, schedule=sched)
+    torch.cuda.synchronize()
+    return y, s, rk.rwkv7_get_last_error()
+
+
+@pytest.mark.parametrize("sched", [rk.RWKV7_SCHED_PAIR, rk.RWKV7_SCHED_TASKS, rk.RWKV7_SCHED_PIPE])
+@pytest.mark.parametrize("B,T,H", [(1, 300, 2), (2, 1000, 3)])
+def test_moderate_decay_every_chunk_schedule(B, T, H, sched):
+    d = _draw(B, T, H, 900 + T, _uniform(0.27, 0.55))
+    yo, so = oracle.wkv7(*oracle_ops(d), d["s0"])
+    y, s, st = _chunk(d, sched)
+    assert st == 0
+    assert rel_err(y, yo) <= TOL_BF16
+    assert rel_err(s, so) <= TOL_BF16
+
+
+@pytest.mark.parametrize("B,T,H", [(1, 300, 2), (2, 130, 3)])
+def test_fast_decay(B, T, H):
+    d = _draw(B, T, H, 910 + T, _uniform(0.02, 0.27))
+    yo, so = oracle.wkv7(*oracle_ops(d), d["s0"])
+    y, s, st = _chunk(d, rk.RWKV7_SCHED_PIPE)
+    assert st == 0
+    assert rel_err(y, yo) <= TOL_BF16
+    assert rel_err(s, so) <= TOL_BF16
+    y, s, st = _chunk(d, rk.RWKV7_SCHED_AUTO, path=rk.RWKV7_PATH_SCAN)
+    assert st == 0
+    assert rel_err(y, yo) <= TOL_BF16
+    assert rel_err(s, so) <= TOL_BF16
+    # the other chunked schedules cannot factorise these chunks: they say so
+    for sched in (rk.RWKV7_SCHED_PAIR, rk.RWKV7_SCHED_TASKS):
+        _, _, st = _chunk(d, sched)
+        assert st == ERR_DOMAIN, sched
+
+
+def test_zero_decay_in_places():
+    def wfun(g, shape):
+        w = 0.55 + 0.45 * torch.rand(shape, generator=g)
+        return torch.where(torch.rand(shape, generator=g) < 0.01, torch.zeros(shape), w)
+
+    d = _draw(1, 257, 2, 920, wfun)
+    yo, so = oracle.wkv7(*oracle_ops(d), d["s0"])
+    y, s, st = _chunk(d, rk.RWKV7_SCHED_PIPE)
+    assert st == 0
+    assert rel_err(y, yo) <= TOL_BF16
+    assert rel_err(s, so) <= TOL_BF16
+
+
+def test_long_sequence_with_a_stretch_of_fast_decay():
+    # T = 4096: model decays, except tokens 700..1400 (chunks 10..21) with w ~ U(0.02, 0.27)
+    def wfun(g, shape):
+        w = 0.5452 + 0.4548 * torch.rand(shape, generator=g)
+        w[:, 700:1400] = 0.02 + 0.25 * torch.rand(w[:, 700:1400].shape, generator=g)
+        return w
+
+    d = _draw(1, 4096, 2, 930, wfun)
+    yo, so = oracle.wkv7(*oracle_ops(d), d["s0"])
+    y, s, st = _chunk(d, rk.RWKV7_SCHED_PIPE)
+    assert st == 0
+    assert rel_err(y, yo) <= TOL_BF16
+    assert rel_err(s, so) <= TOL_BF16
+    _, _, st = _chunk(d, rk.RWKV7_SCHED_AUTO)
+    assert st == ERR_DOMAIN
+
+
+@pytest.mark.parametrize("sched", [rk.RWKV7_SCHED_AUTO, rk.RWKV7_SCHED_PIPE])
+def test_no_decay(sched):
+    d = _draw(2, 200, 2, 940, lambda g, shape: torch.ones(shape))
+    yo, so = oracle.wkv7(*oracle_ops(d), d["s0"])
+    y, s, st = _chunk(d, sched)
+    assert st == 0
+    assert rel_err(y, yo) <= TOL_BF16
+    assert rel_err(s, so) <= TOL_BF16

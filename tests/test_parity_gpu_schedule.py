@@ -1,6 +1,7 @@
-"""GPU parity of the chunked prefill under both schedules of its work -- one CTA per (b, h), and every
-chunk a task spread over all SMs with the state handed between CTAs through s_out -- against the
-float64 oracle, through the C ABI's option entry point.
+"""GPU parity of the chunked prefill under its three schedules of work -- one CTA per (b, h); every chunk
+a task spread over all SMs with the state handed between CTAs through s_out; and the warp-specialised
+pipeline (one persistent CTA per SM, three chunks in flight) -- against the float64 oracle, through the
+C ABI's option entry point.
 
 Shapes cover fewer pairs than SMs, more pairs than SMs (several tasks per CTA, and CTAs whose next
 chunk is held by another CTA in the same round), ragged last chunks, one-chunk sequences, a zero and
@@ -19,7 +20,8 @@ from helpers import OPS, TOL_BF16, need_cuda, oracle_ops, rel_err, to_dev
 
 pytestmark = pytest.mark.gpu
 
-SCHEDS = [pytest.param(rk.RWKV7_SCHED_PAIR, id="pair"), pytest.param(rk.RWKV7_SCHED_TASKS, id="tasks")]
+SCHEDS = [pytest.param(rk.RWKV7_SCHED_PAIR, id="pair"), pytest.param(rk.RWKV7_SCHED_TASKS, id="tasks"),
+          pytest.param(rk.RWKV7_SCHED_PIPE, id="pipe")]
 
 
 @pytest.fixture(autouse=True)
@@ -78,6 +80,7 @@ def test_many_pairs_sampled():
     y2, s2 = _run(d, rk.RWKV7_SCHED_TASKS)
     y1, s1 = _run(d, rk.RWKV7_SCHED_PAIR)
     y0, s0 = _run(d, rk.RWKV7_SCHED_AUTO)
+    y3, s3 = _run(d, rk.RWKV7_SCHED_PIPE)
     rng = np.random.default_rng(741)
     for _ in range(4):
         b, h = int(rng.integers(B)), int(rng.integers(H))
@@ -89,6 +92,14 @@ def test_many_pairs_sampled():
     assert rel_err(s2, s1.cpu().numpy()) <= 1e-2
     assert rel_err(y0, y1.float().cpu().numpy()) <= 1e-2
     assert rel_err(s0, s1.cpu().numpy()) <= 1e-2
+    assert rel_err(y3, y1.float().cpu().numpy()) <= 1e-2
+    assert rel_err(s3, s1.cpu().numpy()) <= 1e-2
+    for _ in range(4):
+        b, h = int(rng.integers(B)), int(rng.integers(H))
+        sub = {n: d[n + "_f32"][b:b + 1, :, h:h + 1] for n in OPS}
+        yo, so = oracle.wkv7(*[sub[n] for n in OPS], d["s0"][b:b + 1, h:h + 1])
+        assert rel_err(y3[b:b + 1, :, h:h + 1], yo) <= TOL_BF16
+        assert rel_err(s3[b:b + 1, h:h + 1], so) <= TOL_BF16
 
 
 @pytest.mark.parametrize("sched", SCHEDS)
@@ -151,7 +162,7 @@ def test_schedule_value_is_checked():
     d = wi.draw(1, 64, 1, seed=770)
     dv = to_dev(d)
     with pytest.raises(rk.Rwkv7Error):
-        rk.prefill_ext(*[dv[n] for n in OPS], None, path=rk.RWKV7_PATH_CHUNK, schedule=3)
+        rk.prefill_ext(*[dv[n] for n in OPS], None, path=rk.RWKV7_PATH_CHUNK, schedule=4)
 
 
 def test_graph_replays_start_from_fresh_flags():

@@ -45,9 +45,12 @@
  *   B, H <= 0, T < 0, a NULL required pointer -> RWKV7_ERR_INVALID
  *   a pointer that is not 16-byte aligned     -> RWKV7_ERR_ALIGN
  *   a failed launch                           -> RWKV7_ERR_CUDA
- * Kernels that wait on an mbarrier give up after a bounded number of polls,
- * record the fact in a device error word and return; rwkv7_get_last_error()
- * reads and clears that word (it synchronises the current device).
+ * Kernels that wait on an mbarrier or on another CTA give up after a bounded
+ * number of polls, record the fact in a device error word and return;
+ * rwkv7_get_last_error() reads and clears that word (it synchronises the
+ * current device).  After a timeout it also resets the chunked kernel's chain
+ * flags, so replays of a captured launch are valid again only once it has
+ * been called.
  * No C++ exception crosses this interface.
  */
 #ifndef RWKV7_H
@@ -105,7 +108,9 @@ RWKV7_API rwkv7_status rwkv7_wkv_prefill(int B, int T, int H, int N, const float
                                const float *k, const float *v, const float *a, const float *b,
                                const float *s_in, float *y, float *s_out, rwkv7_stream_t stream);
 
-/* Same, bfloat16 operands and y (bit patterns), float32 state. */
+/* Same, bfloat16 operands and y (bit patterns), float32 state.  The kernel is
+ * chosen as for RWKV7_PATH_AUTO, so the decay domain of CHUNK above applies
+ * from T >= 128 (a violation is reported as RWKV7_ERR_DOMAIN). */
 RWKV7_API rwkv7_status rwkv7_wkv_prefill_bf16(int B, int T, int H, int N, const uint16_t *r,
                                     const uint16_t *w, const uint16_t *k, const uint16_t *v,
                                     const uint16_t *a, const uint16_t *b, const float *s_in,
@@ -119,7 +124,10 @@ RWKV7_API rwkv7_status rwkv7_wkv_prefill_bf16_path(int path, int B, int T, int H
                                          const uint16_t *a, const uint16_t *b, const float *s_in,
                                          uint16_t *y, float *s_out, rwkv7_stream_t stream);
 
-/* Ragged batch in packed layout: B sequences, row b owns the tokens
+/* Ragged batch in packed layout (the long-context workload at the 7.2B width
+ * with per-row lengths, as a serving batch of unequal prompts; the pages'
+ * GPT mode, RWKV-7 G0 7.2B walkthrough, lshu.cn/news/198401, section 3.2, runs
+ * each row as its own sequence): B sequences, row b owns the tokens
  * cu_seqlens[b] .. cu_seqlens[b+1]-1 of the [total_T, H, N] operands.
  * cu_seqlens is a DEVICE array of B+1 non-decreasing int32 offsets with
  * cu_seqlens[0] = 0 and cu_seqlens[B] = total_T (not checked on the host,
@@ -190,8 +198,12 @@ RWKV7_API rwkv7_status rwkv7_wkv_decode_fused_bf16(int B, int H, int N, const ui
  *                         takes its start state from s_out, where the previous chunk of the same
  *                         (b, h) left it (flags in library-owned device memory order the two).
  *                         Needs B*H <= 65536 (else RWKV7_ERR_CUDA).  Up to 4 such launches may
- *                         run at once on a device; the launch can be captured in a CUDA graph
- *                         and replayed (every launch leaves the flags zeroed unless it fails).
+ *                         run at once on a device: successive launches take 4 flag slots in
+ *                         turn.  A launch captured in a CUDA graph keeps the slot of its capture
+ *                         for every replay, so graphs replayed at the same time must have been
+ *                         captured into different slots (captures that are not 4 launches apart);
+ *                         every launch leaves the flags zeroed unless it times out (see Errors).
+ *                         Choice 0 never takes this schedule while `stream` is capturing.
  *                     3 = a warp-specialised pipeline: one persistent CTA per SM walks its (b, h)
  *                         pairs' chunks with three chunks in flight (operand preparation, masks
  *                         and inverse, state chain on separate warps); exact for every decay in
@@ -208,6 +220,9 @@ typedef struct rwkv7_options {
 
 /* ---- prefill from and to host memory ------------------------------------------------------
  *
+ * The pages run the model from host-side code (the RWKV-LM README copy, oa0.com/c/1004164, and the
+ * walkthrough's GPT / RNN modes, lshu.cn/news/198401, section 3.2) but give no call of this kind; it
+ * is the end-to-end form of the prefill for a caller whose tokens and state live in host memory.
  * The bf16 prefill of rwkv7_wkv_prefill_bf16_path for operands that live in host memory: r, w, k,
  * v, a, b ([B,T,H,64] bf16), s_in ([B,H,64,64] float32, NULL = zero state), y and s_out are HOST
  * pointers; dev_r .. dev_b, dev_s_in, dev_y, dev_s_out are DEVICE buffers of the same shapes that
@@ -322,6 +337,18 @@ RWKV7_API rwkv7_status rwkv7_wkv_backward_bf16(int B, int T, int H, int N, const
                                                const uint16_t *b, const float *states, const uint16_t *dy,
                                                const float *ds_out, float *dr, float *dw, float *dk, float *dv,
                                                float *da, float *db, float *ds_in, rwkv7_stream_t stream);
+
+/* ---- test hook ------------------------------------------------------------------------------
+ *
+ * For tests of the failure path only (the pages have no counterpart): sets, for every later launch
+ * of the chunked kernel in this process, the bound of each device wait to `max_polls` polls (0 =
+ * the production bound, about 2^22) and, in the task-parallel schedule, names a (b, h) pair
+ * `skip_publish_pair` = b*H + h whose first chunk never raises its chain flag (-1 = none), so that
+ * the wait of its second chunk runs out.  Such a launch returns with RWKV7_ERR_TIMEOUT recorded
+ * (rwkv7_get_last_error) and its y and s_out are not valid.  Not thread-safe with concurrent
+ * launches; call rwkv7_test_set_wait_hooks(0, -1) to restore production behaviour.  Always
+ * returns RWKV7_OK. */
+RWKV7_API rwkv7_status rwkv7_test_set_wait_hooks(unsigned max_polls, long long skip_publish_pair);
 
 /* ---- status ---------------------------------------------------------------- */
 

@@ -27,7 +27,7 @@ __all__ = [
     "rwkv7_wkv_prefill", "rwkv7_wkv_prefill_bf16", "rwkv7_wkv_prefill_bf16_path", "rwkv7_wkv_prefill_varlen_bf16",
     "rwkv7_wkv_decode", "rwkv7_wkv_decode_bf16", "rwkv7_wkv_prefill_fused_bf16", "rwkv7_wkv_decode_fused_bf16",
     "rwkv7_wkv_prefill_ext_bf16", "rwkv7_wkv_decode_ext_bf16", "Options",
-    "rwkv7_status_string", "rwkv7_get_last_error", "rwkv7_version",
+    "rwkv7_status_string", "rwkv7_get_last_error", "rwkv7_version", "rwkv7_test_set_wait_hooks",
     "rwkv7_wkv_prefill_save_bf16", "rwkv7_wkv_backward_bf16", "rwkv7_wkv_decode_bf16_bf16state",
     "rwkv7_wkv_prefill_host_bf16", "rwkv7_wkv_prefill_host_noalloc_bf16", "NOALLOC_STAGING_BYTES", "prefill", "decode_", "prefill_model_native", "decode_model_native_", "prefill_ext", "decode_ext_",
     "prefill_save", "backward", "EXPORTED_SYMBOLS",
@@ -44,7 +44,7 @@ EXPORTED_SYMBOLS = (
     "rwkv7_wkv_prefill_ext_bf16", "rwkv7_wkv_decode_ext_bf16",
     "rwkv7_wkv_prefill_save_bf16", "rwkv7_wkv_backward_bf16", "rwkv7_wkv_decode_bf16_bf16state",
     "rwkv7_wkv_prefill_host_bf16", "rwkv7_status_string", "rwkv7_get_last_error", "rwkv7_version",
-    "rwkv7_wkv_prefill_host_noalloc_bf16",
+    "rwkv7_wkv_prefill_host_noalloc_bf16", "rwkv7_test_set_wait_hooks",
 )
 # RWKV7_NOALLOC_STAGING_BYTES of include/rwkv7.h: the staging limit of rwkv7_wkv_prefill_host_noalloc_bf16
 NOALLOC_STAGING_BYTES = 32 * 1024 * 1024
@@ -108,6 +108,8 @@ def load_library() -> ctypes.CDLL:
     lib.rwkv7_get_last_error.restype = ci
     lib.rwkv7_version.argtypes = []
     lib.rwkv7_version.restype = ci
+    lib.rwkv7_test_set_wait_hooks.argtypes = [ctypes.c_uint, ctypes.c_longlong]
+    lib.rwkv7_test_set_wait_hooks.restype = ci
     _lib = lib
     return lib
 
@@ -372,6 +374,13 @@ def rwkv7_get_last_error() -> int:
 
 def rwkv7_version() -> int:
     return int(load_library().rwkv7_version())
+
+
+def rwkv7_test_set_wait_hooks(max_polls: int = 0, skip_publish_pair: int = -1) -> None:
+    """Test hook of the failure path: bound every device wait of later chunked launches to
+    ``max_polls`` polls (0 = production bound) and keep the chain flag of pair ``skip_publish_pair``'s
+    first chunk down in the task-parallel schedule (-1 = none).  ``(0, -1)`` restores the defaults."""
+    _call("rwkv7_test_set_wait_hooks", int(max_polls), int(skip_publish_pair))
 
 
 # ---- conveniences: allocate outputs with torch, then call the entry points ------------------------

@@ -11,6 +11,13 @@ namespace rwkv7 {
 int *device_error_word();
 bool prefill_uses_chunk(int path, long long max_T);
 
+// Test hooks of the chunked prefill (process-wide): the bound of every device wait (0 = the
+// production bound) and a (b, h) pair whose first chunk never raises its flag in the task-parallel
+// schedule (-1 = none), so its successor's bounded wait runs out.
+void set_chunk_test_hooks(uint32_t max_polls, long long skip_publish_pair);
+// Zeroes the task-parallel schedule's flag words on the current device (synchronous).
+cudaError_t clear_chain_flags();
+
 // Sequential scan over [B,T,H,64] (cu_seqlens == nullptr) or a packed ragged
 // batch (cu_seqlens = device offsets, total_T tokens).  TIn: float or
 // uint16_t (bfloat16 bits).

@@ -4,6 +4,8 @@
 // queues copies between the caller's host and device buffers around the
 // launches, nothing here touches the data: every step of the computation runs
 // in the kernels.
+#include <mutex>
+
 #include "../../include/rwkv7.h"
 #include "common.cuh"
 #include "launch.h"
@@ -23,15 +25,19 @@ template <typename... P> bool none_null(const P *...ps) { return ((ps != nullptr
 
 rwkv7_status from_cuda(cudaError_t e) { return e == cudaSuccess ? RWKV7_OK : RWKV7_ERR_CUDA; }
 
-// Device address of the error word on the current device (looked up once per device).
+// Device address of the error word on the current device (looked up once per device; the cache is
+// shared by host threads, so it is read and filled under a lock).
 int *error_word_ptr() {
   static int *cache[64] = {};
+  static std::mutex mu;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
-  if (dev >= 0 && dev < 64 && cache[dev] != nullptr) return cache[dev];
+  const bool cached = dev >= 0 && dev < 64;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cached && cache[dev] != nullptr) return cache[dev];
   void *p = nullptr;
   if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess) return nullptr;
-  if (dev >= 0 && dev < 64) cache[dev] = static_cast<int *>(p);
+  if (cached) cache[dev] = static_cast<int *>(p);
   return static_cast<int *>(p);
 }
 
@@ -93,7 +99,16 @@ rwkv7_status rwkv7_get_last_error(void) {
   if (word != 0 && cudaMemcpyToSymbol(g_error_word, &zero, sizeof(int)) != cudaSuccess) return RWKV7_ERR_CUDA;
   if (cudaGetLastError() != cudaSuccess) return RWKV7_ERR_CUDA;
   if (word == kDevErrNone) return RWKV7_OK;
-  return word == kDevErrDomain ? RWKV7_ERR_DOMAIN : RWKV7_ERR_TIMEOUT;
+  if (word == kDevErrDomain) return RWKV7_ERR_DOMAIN;
+  // A launch that gave up may have left chain flags raised (a later replay of a captured launch has
+  // the same epoch and would take them for its own): zero them all before anything runs again.
+  if (clear_chain_flags() != cudaSuccess) return RWKV7_ERR_CUDA;
+  return RWKV7_ERR_TIMEOUT;
+}
+
+rwkv7_status rwkv7_test_set_wait_hooks(unsigned max_polls, long long skip_publish_pair) {
+  set_chunk_test_hooks(max_polls, skip_publish_pair);
+  return RWKV7_OK;
 }
 
 rwkv7_status rwkv7_wkv_prefill(int B, int T, int H, int N, const float *r, const float *w, const float *k,

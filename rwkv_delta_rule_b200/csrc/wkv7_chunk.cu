@@ -100,9 +100,10 @@ __device__ __forceinline__ void compute_sync() { asm volatile("bar.sync 1, 256;\
 __device__ __forceinline__ void group_sync_lo() { asm volatile("bar.sync 2, 128;\n" ::: "memory"); }
 __device__ __forceinline__ void group_sync_hi() { asm volatile("bar.sync 3, 128;\n" ::: "memory"); }
 
-// Bounded mbarrier wait that also gives up once the CTA is aborting.
-__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
-  for (uint32_t i = 0; i < kMaxPolls; ++i) {
+// Bounded mbarrier wait (at most `limit` polls) that also gives up once the CTA is aborting.
+__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                              uint32_t limit) {
+  for (uint32_t i = 0; i < limit; ++i) {
     if (tc::mbar_try_wait(bar, parity)) return true;
     if ((i & 255u) == 255u && *abort_flag) return false;
   }
@@ -135,6 +136,8 @@ struct Args {
   int s_in_zero;              // the s_in map covers one zero block (row 0 for every pair)
   float *states;              // nullptr, or [B, H, nck, 64, 64]: the state before every chunk (dense T)
   int nck;                    // chunks per sequence, ceil(T / 64)
+  uint32_t max_polls;         // bound of every wait (kMaxPolls unless a test lowers it)
+  long long skip_publish;     // test hook: this pair's first chunk never raises its flag (-1: none)
 };
 
 // One unit of work: chunk c of the (b, h) pair bh.
@@ -205,8 +208,8 @@ __device__ __forceinline__ bool chain_ready(const unsigned long long *flag, unsi
   return false;
 }
 __device__ __forceinline__ bool wait_chain(const unsigned long long *flag, unsigned epoch, int c,
-                                           volatile int *abort_flag) {
-  for (uint32_t i = 0; i < kMaxPolls; ++i) {
+                                           volatile int *abort_flag, uint32_t limit) {
+  for (uint32_t i = 0; i < limit; ++i) {
     if (chain_ready(flag, epoch, c)) return true;
     if ((i & 63u) == 63u && *abort_flag) return false;
     __nanosleep(64);
@@ -685,8 +688,12 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
         const unsigned long long val = pt.last ? 0ull
                                                : ((static_cast<unsigned long long>(A.epoch) << 32) |
                                                   static_cast<unsigned>(pt.c + 1));
-        asm volatile("fence.acq_rel.gpu;\n\tst.relaxed.gpu.global.u64 [%0], %1;\n" ::"l"(A.flags + pt.bh), "l"(val)
-                     : "memory");
+        // (test hook: the named pair's first chunk keeps its flag down, so its successor's bounded wait
+        // runs out)
+        if (pt.bh != A.skip_publish || pt.c != 0)
+          asm volatile("fence.acq_rel.gpu;\n\tst.relaxed.gpu.global.u64 [%0], %1;\n" ::"l"(A.flags + pt.bh),
+                       "l"(val)
+                       : "memory");
       };
       // The start state of task t into B4S (s_in for a first chunk, else s_out once the flag is up).
       // Looked for without blocking after bar_st and after MMA3; waited for before MMA4.
@@ -742,7 +749,7 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
       for (uint32_t it = 0; have; ++it) {
         const uint32_t ph = it & 1;
         // MMA1 (tf32): D1 = [R~; A~] [B^; K^]^T, once the operands are in place
-        if (!wait_or_abort(bar_p1, ph, abort_flag)) { fail(); break; }
+        if (!wait_or_abort(bar_p1, ph, abort_flag, A.max_polls)) { fail(); break; }
         tc::tc_fence_after();
         {
           constexpr uint32_t idesc = tc::instr_desc(tc::kFmtTF32, 128, 128, false, false);
@@ -778,14 +785,14 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
           // the previous task's end state out of B4S (as soon as its read-out has written it), then (if
           // already there) this task's start state in
           if (it > 0) {
-            if (!wait_or_abort(bar_sout, (it - 1) & 1, abort_flag)) { fail(); break; }
+            if (!wait_or_abort(bar_sout, (it - 1) & 1, abort_flag, A.max_polls)) { fail(); break; }
             publish(pt);
           }
           state_issued = false;
           if (t.c == 0 || chain_ready(A.flags + t.bh, A.epoch, t.c)) load_state(t, ph);
         }
         // MMA3 (bf16): D3 = [A~^T; Lak^T] Tinv^T
-        if (!wait_or_abort(bar_b3, ph, abort_flag)) { fail(); break; }
+        if (!wait_or_abort(bar_b3, ph, abort_flag, A.max_polls)) { fail(); break; }
         tc::tc_fence_after();
         {
           constexpr uint32_t idesc = tc::instr_desc(tc::kFmtBF16, 128, 64, true, false);
@@ -799,7 +806,7 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
         }
         if (kTask && !state_issued && chain_ready(A.flags + t.bh, A.epoch, t.c)) load_state(t, ph);
         // MMA2 (bf16, A from TMEM): D2 += [Mrb; B-^T] [W~ U~]
-        if (!wait_or_abort(bar_b2, ph, abort_flag)) { fail(); break; }
+        if (!wait_or_abort(bar_b2, ph, abort_flag, A.max_polls)) { fail(); break; }
         tc::tc_fence_after();
         {
           constexpr uint32_t idesc = tc::instr_desc(tc::kFmtBF16, 128, 128, false, false);
@@ -814,10 +821,10 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
         // MMA2's accumulator as its A operand with no wait in between: MMAs issued by one thread
         // execute in issue order.
         if (kTask && !state_issued) {
-          if (!wait_chain(A.flags + t.bh, A.epoch, t.c, abort_flag)) { fail(); break; }
+          if (!wait_chain(A.flags + t.bh, A.epoch, t.c, abort_flag, A.max_polls)) { fail(); break; }
           load_state(t, ph);
         }
-        if (!wait_or_abort(kTask ? bar_sin : bar_st, ph, abort_flag)) { fail(); break; }
+        if (!wait_or_abort(kTask ? bar_sin : bar_st, ph, abort_flag, A.max_polls)) { fail(); break; }
         tc::tc_fence_after();
         {
           constexpr uint32_t idesc = tc::instr_desc(tc::kFmtTF32, 128, 64, false, false);
@@ -847,9 +854,11 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
         }
       }
       // the last task's flag, once the compute warps' final read-out has stored its end state
-      if (kTask && nit > 0 && !*abort_flag && wait_or_abort(bar_sout, (nit - 1) & 1, abort_flag)) publish(pt);
-      // every copy and MMA issued here lands before the CTA exits (bounded; phases that
-      // already completed return at once)
+      if (kTask && nit > 0 && !*abort_flag && wait_or_abort(bar_sout, (nit - 1) & 1, abort_flag, A.max_polls))
+        publish(pt);
+      // every copy and MMA issued here lands before the CTA exits (bounded, always by the production
+      // bound: a copy still in flight must not outlive the CTA; phases that already completed return
+      // at once)
       if (last_tma >= 0) (void)tc::mbar_wait_bounded(bar_tma, last_tma, kMaxPolls);
       if (last_sin >= 0) (void)tc::mbar_wait_bounded(bar_sin, last_sin, kMaxPolls);
       if (last_m1 >= 0) (void)tc::mbar_wait_bounded(bar_m1, last_m1, kMaxPolls);
@@ -910,7 +919,7 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
     auto wait_ctrl = [&](uint64_t *bar, uint32_t parity) -> bool {
       const uint32_t slot = ncalls++ & 1u;
       if (tid == 0) {
-        if (!wait_or_abort(bar, parity, abort_flag)) {
+        if (!wait_or_abort(bar, parity, abort_flag, A.max_polls)) {
           *abort_flag = 1;
           report_device_error(A.err, kDevErrTimeout);
         }
@@ -925,7 +934,7 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
     auto wait_group_hi = [&](uint64_t *bar, uint32_t parity) -> bool {
       const uint32_t slot = ncalls_hi++ & 1u;
       if (tid == 128) {
-        if (!wait_or_abort(bar, parity, abort_flag)) {
+        if (!wait_or_abort(bar, parity, abort_flag, A.max_polls)) {
           *abort_flag = 1;
           report_device_error(A.err, kDevErrTimeout);
         }
@@ -1302,17 +1311,16 @@ typedef CUresult (*PFN_encodeTiled)(CUtensorMap *, CUtensorMapDataType, cuuint32
                                     const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
                                     CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// The driver's tensor-map encoder, looked up once (a function-local static: thread-safe initialisation).
 static PFN_encodeTiled get_encode() {
-  static PFN_encodeTiled fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
+  static const PFN_encodeTiled fn = []() -> PFN_encodeTiled {
     void *p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_encodeTiled>(p);
-  }
+      return reinterpret_cast<PFN_encodeTiled>(p);
+    return nullptr;
+  }();
   return fn;
 }
 
@@ -1379,6 +1387,11 @@ static bool device_scratch(DeviceScratch &ds) {
   ds = c;
   return true;
 }
+
+// Test hooks (process-wide; the defaults are the production values): the bound of every wait, and a
+// pair whose first chunk never raises its flag in the task-parallel schedule.
+static std::atomic<uint32_t> g_hook_max_polls{kMaxPolls};
+static std::atomic<long long> g_hook_skip_publish{-1};
 
 // A fresh epoch per launch (never 0, so zeroed flags match no launch).
 static unsigned next_epoch() {
@@ -1448,15 +1461,21 @@ cudaError_t launch_chunk_ext(const uint16_t *r, const uint16_t *w, const uint16_
   const long long ntasks = (rows / C) * BH;
   const int nck = (T + C - 1) / C;
   Args args{y, s_in, s_out, cu_seqlens, T, total_T, H, err_word, k_k, ln_w, ln_b, ntasks, BH, nullptr, 0, 0,
-            states, nck};
+            states, nck, g_hook_max_polls.load(), -1};
   // The task-parallel schedule pays when one CTA per pair would leave many SMs idle: measured on B200,
   // 48 and 96 pairs ran 1.2x and 1.1x faster, 1 and 2 pairs 1.6x; at 128 pairs and above the pair
   // schedule was as fast or faster.
   DeviceScratch ds;
   bool task = false;
   int grid_tasks = 0;
+  // Under stream capture the automatic choice keeps to one CTA per pair: a captured launch keeps the
+  // flag slot and epoch of its capture for every replay, so two replays running at once could share
+  // a slot; the task-parallel schedule stays available there on explicit request.
+  cudaStreamCaptureStatus capture = cudaStreamCaptureStatusNone;
+  if (schedule == 0 && cudaStreamIsCapturing(stream, &capture) != cudaSuccess) return cudaErrorInvalidValue;
   if (schedule != 1 && ntasks > 0 && ntasks < (1LL << 31) && BH <= kMaxChainPairs && device_scratch(ds)) {
-    task = schedule == 2 || 4 * BH <= 3 * static_cast<long long>(ds.sms);
+    task = schedule == 2 ||
+           (capture == cudaStreamCaptureStatusNone && 4 * BH <= 3 * static_cast<long long>(ds.sms));
     grid_tasks = static_cast<int>(ntasks < ds.sms ? ntasks : ds.sms);
   }
   if (schedule == 2 && !task) return cudaErrorInvalidValue;
@@ -1464,6 +1483,7 @@ cudaError_t launch_chunk_ext(const uint16_t *r, const uint16_t *w, const uint16_
     const unsigned epoch = next_epoch();
     args.flags = ds.flags + static_cast<long long>(epoch % kFlagSlots) * kMaxChainPairs;
     args.epoch = epoch;
+    args.skip_publish = g_hook_skip_publish.load();
     args.s_in_zero = s_in == nullptr ? 1 : 0;
     if (!make_state_map(&maps.s_in, s_in ? static_cast<const void *>(s_in) : ds.zeros, s_in ? BH : 1) ||
         !make_state_map(&maps.s_out, s_out, BH) ||
@@ -1474,6 +1494,17 @@ cudaError_t launch_chunk_ext(const uint16_t *r, const uint16_t *w, const uint16_
   if (model_native) return launch_variant<true, false>(maps, args, B, H, task, grid_tasks, stream);
   if (group_norm) return launch_variant<false, true>(maps, args, B, H, task, grid_tasks, stream);
   return launch_variant<false, false>(maps, args, B, H, task, grid_tasks, stream);
+}
+
+void set_chunk_test_hooks(uint32_t max_polls, long long skip_publish_pair) {
+  chunk::g_hook_max_polls.store(max_polls == 0 ? chunk::kMaxPolls : max_polls);
+  chunk::g_hook_skip_publish.store(skip_publish_pair);
+}
+
+cudaError_t clear_chain_flags() {
+  chunk::DeviceScratch ds;
+  if (!chunk::device_scratch(ds)) return cudaErrorInvalidValue;
+  return cudaMemset(ds.flags, 0, sizeof(unsigned long long) * chunk::kFlagSlots * chunk::kMaxChainPairs);
 }
 
 cudaError_t launch_chunk(const uint16_t *r, const uint16_t *w, const uint16_t *k, const uint16_t *v,

@@ -21,7 +21,7 @@ def test_reference_arm_prints_one_contract_line():
                 "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
         assert key in d, key
     assert d["value"] > 0 and d["unit"] == "tokens/s" and d["higher_is_better"] is True
-    assert d["config"]["workload"] == "prefill_d768_b8_t4096"
+    assert d["config"]["workload"] == "prefill_d4096_b4_t16384"
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}

@@ -24,6 +24,12 @@ All arithmetic above is float32; the operands are then rounded to the storage
 dtype (round-to-nearest-even for bf16).  The returned float32 copies hold the
 *rounded* values, so the oracle sees exactly the bytes the GPU sees.
 
+``device``: the draws above can also run on a CUDA device (a generator of that
+device, same seed, same order).  The distributions are the same but the random
+stream is the device's, so the values differ from a CPU draw of the same seed;
+the benchmark draws its full-size workloads this way (seconds instead of
+minutes), every parity test draws on the CPU.
+
 The configurations are the pages' model widths with head size 64:
 0.1B D768 (H=12), 1.5B D2048 (H=32), L24-D1024 (H=16), 7.2B-scale D4096 (H=64).
 """
@@ -74,27 +80,30 @@ def storage_dtype(name: str) -> torch.dtype:
 
 
 def draw(B: int, T: int, H: int, N: int = N_HEAD, *, seed: int, dtype: str = "bf16",
-         z_mean: float = 0.0, s0_std: Optional[float] = None) -> Dict[str, torch.Tensor]:
+         z_mean: float = 0.0, s0_std: Optional[float] = None, device=None,
+         f32_copies: bool = True) -> Dict[str, torch.Tensor]:
     """Draw one workload.
 
     Returns a dict with
-      ``r, w, k, v, a, b``: storage-dtype tensors ``[B, T, H, N]`` (contiguous, CPU);
-      ``<name>_f32``: the same values as float32;
+      ``r, w, k, v, a, b``: storage-dtype tensors ``[B, T, H, N]`` (contiguous, on ``device``,
+      the CPU by default);
+      ``<name>_f32``: the same values as float32 (omitted when ``f32_copies`` is False);
       ``s0``: float32 ``[B, H, N, N]`` or ``None`` for a zero state.
     """
-    g = torch.Generator(device="cpu")
+    dev = torch.device("cpu" if device is None else device)
+    g = torch.Generator(device=dev)
     g.manual_seed(int(seed))
     shp = (B, T, H, N)
     f32 = torch.float32
-    r = torch.randn(shp, generator=g, dtype=f32)
-    z = torch.randn(shp, generator=g, dtype=f32) + float(z_mean)
-    kh = torch.randn(shp, generator=g, dtype=f32)
-    s = torch.rand(shp, generator=g, dtype=f32) + 0.5
-    v = torch.randn(shp, generator=g, dtype=f32)
-    alpha = torch.rand(shp, generator=g, dtype=f32)
+    r = torch.randn(shp, generator=g, dtype=f32, device=dev)
+    z = torch.randn(shp, generator=g, dtype=f32, device=dev) + float(z_mean)
+    kh = torch.randn(shp, generator=g, dtype=f32, device=dev)
+    s = torch.rand(shp, generator=g, dtype=f32, device=dev) + 0.5
+    v = torch.randn(shp, generator=g, dtype=f32, device=dev)
+    alpha = torch.rand(shp, generator=g, dtype=f32, device=dev)
     s0 = None
     if s0_std is not None:
-        s0 = torch.randn((B, H, N, N), generator=g, dtype=f32) * float(s0_std)
+        s0 = torch.randn((B, H, N, N), generator=g, dtype=f32, device=dev) * float(s0_std)
 
     kh = kh / kh.norm(dim=-1, keepdim=True)
     k = kh * s
@@ -108,34 +117,37 @@ def draw(B: int, T: int, H: int, N: int = N_HEAD, *, seed: int, dtype: str = "bf
     for nm, x in (("r", r), ("w", w), ("k", k), ("v", v), ("a", a), ("b", b)):
         xs = x.to(sd).contiguous()
         out[nm] = xs
-        out[nm + "_f32"] = xs.to(f32) if sd != f32 else xs
+        if f32_copies:
+            out[nm + "_f32"] = xs.to(f32) if sd != f32 else xs
     out["s0"] = s0
     return out
 
 
 def draw_model_native(B: int, T: int, H: int, N: int = N_HEAD, *, seed: int, z_mean: float = 0.0,
-                      s0_std: Optional[float] = None) -> Dict[str, torch.Tensor]:
+                      s0_std: Optional[float] = None, device=None) -> Dict[str, torch.Tensor]:
     """Draw model-native inputs for the fused operand prologue (no prologue arithmetic here).
 
     Returns bf16 ``[B, T, H, N]`` tensors ``r`` ~ N(0,1), ``xw`` (decay pre-activation) ~
     N(z_mean, 1), ``k`` = unit vector per (b, t, h) times U(0.5, 1.5) per channel, ``v`` ~ N(0,1)
     and ``xa`` (in-context learning-rate pre-activation) ~ N(0,1); ``<name>_f32`` copies; ``k_k``:
-    float32 ``[H, N]`` ~ U(0.5, 1.5); ``s0``: float32 ``[B, H, N, N]`` or None.
+    float32 ``[H, N]`` ~ U(0.5, 1.5); ``s0``: float32 ``[B, H, N, N]`` or None.  ``device`` as in
+    :func:`draw`.
     """
-    g = torch.Generator(device="cpu")
+    dev = torch.device("cpu" if device is None else device)
+    g = torch.Generator(device=dev)
     g.manual_seed(int(seed))
     shp = (B, T, H, N)
     f32 = torch.float32
-    r = torch.randn(shp, generator=g, dtype=f32)
-    xw = torch.randn(shp, generator=g, dtype=f32) + float(z_mean)
-    kh = torch.randn(shp, generator=g, dtype=f32)
-    s = torch.rand(shp, generator=g, dtype=f32) + 0.5
-    v = torch.randn(shp, generator=g, dtype=f32)
-    xa = torch.randn(shp, generator=g, dtype=f32)
-    k_k = torch.rand((H, N), generator=g, dtype=f32) + 0.5
+    r = torch.randn(shp, generator=g, dtype=f32, device=dev)
+    xw = torch.randn(shp, generator=g, dtype=f32, device=dev) + float(z_mean)
+    kh = torch.randn(shp, generator=g, dtype=f32, device=dev)
+    s = torch.rand(shp, generator=g, dtype=f32, device=dev) + 0.5
+    v = torch.randn(shp, generator=g, dtype=f32, device=dev)
+    xa = torch.randn(shp, generator=g, dtype=f32, device=dev)
+    k_k = torch.rand((H, N), generator=g, dtype=f32, device=dev) + 0.5
     s0 = None
     if s0_std is not None:
-        s0 = torch.randn((B, H, N, N), generator=g, dtype=f32) * float(s0_std)
+        s0 = torch.randn((B, H, N, N), generator=g, dtype=f32, device=dev) * float(s0_std)
     k = kh / kh.norm(dim=-1, keepdim=True) * s
     out: Dict[str, torch.Tensor] = {}
     for nm, x in (("r", r), ("xw", xw), ("k", k), ("v", v), ("xa", xa)):
@@ -191,19 +203,23 @@ def cu_seqlens(lengths: torch.Tensor) -> torch.Tensor:
 
 
 def draw_packed(lengths: torch.Tensor, H: int, N: int = N_HEAD, *, seed: int, dtype: str = "bf16",
-                z_mean: float = 0.0, s0_std: Optional[float] = None) -> Dict[str, torch.Tensor]:
+                z_mean: float = 0.0, s0_std: Optional[float] = None, device=None,
+                f32_copies: bool = True) -> Dict[str, torch.Tensor]:
     """Draw a ragged batch in packed layout ``[sum(T_b), H, N]``.
 
     Same recipe as :func:`draw` with B = 1 and T = sum(T_b); row b owns tokens
     ``cu_seqlens[b] .. cu_seqlens[b+1]-1``.  ``s0`` is ``[len(lengths), H, N, N]``.
     """
     total = int(lengths.sum())
-    d = draw(1, total, H, N, seed=seed, dtype=dtype, z_mean=z_mean, s0_std=None)
+    d = draw(1, total, H, N, seed=seed, dtype=dtype, z_mean=z_mean, s0_std=None, device=device,
+             f32_copies=f32_copies)
     out = {key: (val[0] if val is not None else None) for key, val in d.items()}
     if s0_std is not None:
-        g = torch.Generator(device="cpu")
+        dev = torch.device("cpu" if device is None else device)
+        g = torch.Generator(device=dev)
         g.manual_seed(int(seed) + 7919)
-        out["s0"] = torch.randn((lengths.numel(), H, N, N), generator=g, dtype=torch.float32) * float(s0_std)
+        out["s0"] = torch.randn((lengths.numel(), H, N, N), generator=g, dtype=torch.float32,
+                                device=dev) * float(s0_std)
     else:
         out["s0"] = None
     out["cu_seqlens"] = cu_seqlens(lengths)

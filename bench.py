@@ -77,7 +77,7 @@ def load_peaks():
 # operands, larger than L2) forced to that schedule, scaled by the token-heads of a launch; the figure
 # holds only for the kernel source it was taken on (sha256 prefix of wkv7_chunk.cu), and the line
 # reports null for any other build.  The capture is summarised under profiles/.
-MEASURED_TRAFFIC = {"source_sha256": None, "bytes_per_token_head": None}
+MEASURED_TRAFFIC = {"source_sha256": "c06158a488ffaa82", "bytes_per_token_head": (805509888 + 125476608) / (16384 * 64)}
 
 
 def measured_traffic(B, T, H, schedule):
@@ -376,9 +376,8 @@ def bench_chained(lib7, dev, steps, peaks):
     st = lib7.rwkv7_get_last_error()
     byts = prefill_bytes(B * half, H, B, state_in=False) + prefill_bytes(B * half, H, B, state_in=True)
     out = {"B": B, "T": case.T, "H": H, "calls_per_step": 2, "step_ms": ms, "tokens_per_s": B * case.T / (ms / 1e3),
-           "status": st, "roofline": hbm_roofline(byts, ms / 2, peaks, note="per call: half the step's bytes "
+           "status": st, "roofline": hbm_roofline(byts / 2, ms / 2, peaks, note="per call: half the step's bytes "
                                                    "over half the step time")}
-    out["roofline"]["algorithmic_bytes_per_launch"] = byts / 2
     del parts, y, s_mid, s_out
     free_device()
     return out

@@ -4,7 +4,8 @@
   bounded to a few thousand polls and one (b, h) pair's first chunk keeps its chain flag down in the
   task-parallel schedule, so the next chunk of that pair waits on a flag that nothing raises.  The
   launch must return, rwkv7_get_last_error() must report RWKV7_ERR_TIMEOUT once (and then OK), and
-  the launches after it, on every flag slot, must match the float64 oracle again.
+  the launches after it, on every flag slot, must match the float64 oracle again.  With a bound of 32
+  polls, ordinary waits give up early on both schedules: the launch must still return cleanly.
 * Guard bands: y and s_out sit inside larger buffers filled with a canary bit pattern.  After ragged
   batches (empty rows, rows of 1, 63, 65, 70 and 130 tokens, rows whose offsets leave [0, total_T],
   tokens that belong to no row) and dense calls with ragged tail chunks, every byte outside what the
@@ -83,6 +84,36 @@ def test_chain_wait_runs_out_reports_timeout_and_recovers():
         assert rk.rwkv7_get_last_error() == 0, i
         assert rel_err(y, yo) <= TOL_BF16, i
         assert rel_err(s_out, so) <= TOL_BF16, i
+
+
+@pytest.mark.parametrize("sched", [rk.RWKV7_SCHED_PAIR, rk.RWKV7_SCHED_TASKS])
+def test_waits_that_give_up_early_abort_cleanly(sched):
+    """With every wait bounded to 32 polls, ordinary waits (MMA completions, tile loads) give up before
+    the hardware is done: whichever wait runs out first, the CTA must abort, drain what it issued and
+    return; the call reports OK or TIMEOUT, and the next launch with the production bound is exact."""
+    B, T, H = 2, 640, 3
+    d = wi.draw(B, T, H, seed=4244, s0_std=0.1)
+    yo, so = oracle.wkv7(*oracle_ops(d), d["s0"])
+    dv = to_dev(d)
+    y = torch.empty(B, T, H, N, dtype=torch.bfloat16, device="cuda")
+    s_out = torch.empty(B, H, N, N, device="cuda")
+    rk.rwkv7_test_set_wait_hooks(32, -1)
+    t0 = time.monotonic()
+    try:
+        rk.rwkv7_wkv_prefill_ext_bf16(rk.RWKV7_PATH_CHUNK, *[dv[n] for n in OPS], dv["s0"], y, s_out,
+                                      schedule=sched)
+        torch.cuda.synchronize()
+        elapsed = time.monotonic() - t0
+        st = rk.rwkv7_get_last_error()
+    finally:
+        rk.rwkv7_test_set_wait_hooks(0, -1)
+    assert st in (0, ERR_TIMEOUT), rk.rwkv7_status_string(st)
+    assert elapsed < 30.0
+    assert rk.rwkv7_get_last_error() == 0
+    rk.rwkv7_wkv_prefill_ext_bf16(rk.RWKV7_PATH_CHUNK, *[dv[n] for n in OPS], dv["s0"], y, s_out, schedule=sched)
+    torch.cuda.synchronize()
+    assert rk.rwkv7_get_last_error() == 0
+    assert rel_err(y, yo) <= TOL_BF16 and rel_err(s_out, so) <= TOL_BF16
 
 
 def test_hook_defaults_leave_every_schedule_exact():

@@ -56,6 +56,22 @@ def test_prefill_model_native_without_key_scale_and_state(path):
     assert rel_err(s, so) <= TOL_BF16
 
 
+@pytest.mark.parametrize("sched", [rk.RWKV7_SCHED_PAIR, rk.RWKV7_SCHED_TASKS, rk.RWKV7_SCHED_PIPE],
+                         ids=["pair", "tasks", "pipe"])
+@pytest.mark.parametrize("T", [64, 65, 200, 1000])
+def test_prefill_model_native_every_schedule(T, sched):
+    """Every chunked schedule with model-native inputs, across one chunk, ragged tails and many chunks
+    (the decays and learning rates are formed ahead of the chunk that uses them)."""
+    d = wi.draw_model_native(2, T, 3, seed=420 + T, s0_std=0.1)
+    yo, so = _oracle(d, d["k_k"], d["s0"])
+    dev = {n: d[n].cuda() for n in NATIVE}
+    y, s = rk.prefill_ext(dev["r"], dev["xw"], dev["k"], dev["v"], dev["xa"], None, d["s0"].cuda(),
+                          path=rk.RWKV7_PATH_CHUNK, model_native=True, k_k=d["k_k"].cuda(), schedule=sched)
+    torch.cuda.synchronize()
+    assert rel_err(y, yo) <= TOL_BF16
+    assert rel_err(s, so) <= TOL_BF16
+
+
 @pytest.mark.parametrize("z_mean", [-3.0, 3.0])
 def test_prefill_model_native_decay_regimes(z_mean):
     d = wi.draw_model_native(2, 320, 2, seed=410, z_mean=z_mean, s0_std=0.1)

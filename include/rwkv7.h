@@ -48,9 +48,9 @@
  * Kernels that wait on an mbarrier or on another CTA give up after a bounded
  * number of polls, record the fact in a device error word and return;
  * rwkv7_get_last_error() reads and clears that word (it synchronises the
- * current device).  After a timeout it also resets the chunked kernel's chain
- * flags, so replays of a captured launch are valid again only once it has
- * been called.
+ * current device).  When the word holds an error it also resets the chunked
+ * kernel's chain flags, so after a timeout, replays of a captured launch are
+ * valid again only once it has been called.
  * No C++ exception crosses this interface.
  */
 #ifndef RWKV7_H
@@ -350,7 +350,12 @@ RWKV7_API rwkv7_status rwkv7_wkv_backward_bf16(int B, int T, int H, int N, const
  * returns RWKV7_OK. */
 RWKV7_API rwkv7_status rwkv7_test_set_wait_hooks(unsigned max_polls, long long skip_publish_pair);
 
-/* ---- status ---------------------------------------------------------------- */
+/* ---- status ----------------------------------------------------------------
+ * Library plumbing with no counterpart on the pages: how a caller learns that a call was refused
+ * (the return codes above) or that a kernel gave up or met inputs outside its range (the device
+ * error word below).  RWKV7_ERR_DOMAIN follows from the pages' own fp32 note on w (RWKV-LM README
+ * copy, oa0.com/c/1004164): the chunked form divides by decay products, which only float32 range
+ * limits. */
 
 /* Static English description of a status code (never NULL). */
 RWKV7_API const char *rwkv7_status_string(rwkv7_status status);
@@ -358,7 +363,8 @@ RWKV7_API const char *rwkv7_status_string(rwkv7_status status);
 /* Reads and clears the device error word of the current device (RWKV7_OK,
  * RWKV7_ERR_TIMEOUT or RWKV7_ERR_DOMAIN: the first error recorded since the
  * last call), and reports a pending CUDA error as RWKV7_ERR_CUDA.
- * Synchronises the current device. */
+ * Synchronises the current device.  When it reports an error it also zeroes the
+ * chunked kernel's chain flags (see chunk_schedule 2). */
 RWKV7_API rwkv7_status rwkv7_get_last_error(void);
 
 /* Library version as major*10000 + minor*100 + patch. */

@@ -99,11 +99,11 @@ rwkv7_status rwkv7_get_last_error(void) {
   if (word != 0 && cudaMemcpyToSymbol(g_error_word, &zero, sizeof(int)) != cudaSuccess) return RWKV7_ERR_CUDA;
   if (cudaGetLastError() != cudaSuccess) return RWKV7_ERR_CUDA;
   if (word == kDevErrNone) return RWKV7_OK;
-  if (word == kDevErrDomain) return RWKV7_ERR_DOMAIN;
   // A launch that gave up may have left chain flags raised (a later replay of a captured launch has
-  // the same epoch and would take them for its own): zero them all before anything runs again.
+  // the same epoch and would take them for its own), and the word keeps only the first error of a
+  // sequence of launches: after any recorded error, zero all flags before anything runs again.
   if (clear_chain_flags() != cudaSuccess) return RWKV7_ERR_CUDA;
-  return RWKV7_ERR_TIMEOUT;
+  return word == kDevErrDomain ? RWKV7_ERR_DOMAIN : RWKV7_ERR_TIMEOUT;
 }
 
 rwkv7_status rwkv7_test_set_wait_hooks(unsigned max_polls, long long skip_publish_pair) {

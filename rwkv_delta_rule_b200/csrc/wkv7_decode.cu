@@ -52,25 +52,18 @@ __device__ __forceinline__ void st_state(uint16_t *p, float4 x) {
 }
 
 template <typename TIn, bool kFused, bool kLN, typename TS = float>
-__global__ void __launch_bounds__(256) wkv7_decode_kernel(DecodeArgs<TIn, TS> A) {
+__global__ void __launch_bounds__(256, 5) wkv7_decode_kernel(DecodeArgs<TIn, TS> A) {
   const long long pair = blockIdx.x;  // b * H + h
   const int tid = threadIdx.x;
   // the step before may still be finishing (its launch allowed this grid to start early): every CTA
   // of this grid has started once all have passed the trigger, and none reads memory before the wait
   pdl_trigger();
   pdl_wait();
-  // fused: the decay and the learning rate of each of the 64 channels, computed once per CTA (the 16
-  // row groups share them) by threads 0..63 while the state loads are in flight
-  __shared__ float s_w[kFused ? kN : 1], s_rate[kFused ? kN : 1];
-  if (kFused && tid < kN) {
-    const long long vbase = pair * kN;
-    s_w[tid] = x070_decay(Elem<TIn>::load(A.w + vbase + tid));
-    s_rate[tid] = x070_sigmoid(Elem<TIn>::load(A.a + vbase + tid));
-  }
   const int c4 = tid & 15;   // column chunk: columns 4*c4 .. 4*c4+3
   const int rg = tid >> 4;   // rows rg + 16*m
   TS *S = A.s + pair * (kN * kN);
 
+  // the state loads go out first, so everything below overlaps them
   float4 st[4];
 #pragma unroll
   for (int m = 0; m < 4; ++m) st[m] = ld_state(S + (rg + 16 * m) * kN + 4 * c4);
@@ -78,11 +71,9 @@ __global__ void __launch_bounds__(256) wkv7_decode_kernel(DecodeArgs<TIn, TS> A)
   const long long vb = pair * kN;
   float ww[4], kk[4], aa[4], bb[4], rr[4], vv[4];
   Elem<TIn>::load4(A.k + vb + 4 * c4, kk);
-  if (!kFused) {
-    Elem<TIn>::load4(A.w + vb + 4 * c4, ww);
-    Elem<TIn>::load4(A.a + vb + 4 * c4, aa);
-    Elem<TIn>::load4(A.b + vb + 4 * c4, bb);
-  }
+  Elem<TIn>::load4(A.w + vb + 4 * c4, ww);  // fused: x_w
+  Elem<TIn>::load4(A.a + vb + 4 * c4, aa);  // fused: x_a
+  if (!kFused) Elem<TIn>::load4(A.b + vb + 4 * c4, bb);
   Elem<TIn>::load4(A.r + vb + 4 * c4, rr);
   float sa[4];
   if (kFused) {
@@ -112,12 +103,26 @@ __global__ void __launch_bounds__(256) wkv7_decode_kernel(DecodeArgs<TIn, TS> A)
     const float inv = x070_inv_norm(ss);
 #pragma unroll
     for (int m = 0; m < 4; ++m) sa[m] *= -inv;
-    __syncthreads();  // s_w / s_rate
+    // the decays and learning rates of this thread's 4 channels: lanes l and l ^ 16 hold the same
+    // channels, so each forms two of each (lane bit 4 picks which two) and they swap the rest
+    const bool upper = (tid & 16) != 0;
+    float dw[2], dr[2];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      bb[e] = kx[e] * inv * s_rate[4 * c4 + e];
-      ww[e] = s_w[4 * c4 + e];
+    for (int e = 0; e < 2; ++e) {
+      dw[e] = x070_decay(upper ? ww[2 + e] : ww[e]);
+      dr[e] = x070_sigmoid(upper ? aa[2 + e] : aa[e]);
     }
+    float rate[4];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const float ow = __shfl_xor_sync(0xffffffffu, dw[e], 16), orr = __shfl_xor_sync(0xffffffffu, dr[e], 16);
+      ww[e] = upper ? ow : dw[e];
+      ww[2 + e] = upper ? dw[e] : ow;
+      rate[e] = upper ? orr : dr[e];
+      rate[2 + e] = upper ? dr[e] : orr;
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) bb[e] = kx[e] * inv * rate[e];
   } else {
 #pragma unroll
     for (int m = 0; m < 4; ++m) {

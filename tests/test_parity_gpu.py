@@ -299,12 +299,18 @@ def test_full_decode_l24_d1024_equals_prefill():
 
 @pytest.mark.slow
 def test_full_prefill_d4096_b4_t16384_and_ragged():
+    # the headline workload in the launch configuration the bench times (AUTO: one CTA per pair at 256
+    # pairs): 12 sampled pairs against the oracle, and every element against the sequential scan, an
+    # independent kernel (the chunked form's inverse and decay algebra on every pair)
     case = wi.CASES["prefill_d4096_b4_t16384"]
     d = wi.draw_case(case)
     dd = to_dev(d)
     y, s = gpu_prefill(dd, None)
-    check_pairs(d, None, y.cpu(), s.cpu(), sampled_pairs(case.B, case.H, 3, 4), TOL_BF16)
-    del dd, y, s, d
+    check_pairs(d, None, y.cpu(), s.cpu(), sampled_pairs(case.B, case.H, 12, 4), TOL_BF16)
+    ys, ss = gpu_prefill(dd, None, rk.RWKV7_PATH_SCAN)
+    assert rel_err(y, ys.float().cpu().numpy()) <= TOL_BF16_PAIR
+    assert rel_err(s, ss.cpu().numpy()) <= TOL_BF16
+    del dd, y, s, d, ys, ss
     lens = wi.ragged_lengths(case.B, 1024, 16384, seed=case.seed + 1)
     d = wi.draw_packed(lens, case.H, seed=case.seed + 2, z_mean=case.z_mean)
     dd = to_dev(d)
@@ -323,3 +329,27 @@ def test_full_prefill_d4096_b4_t16384_and_ragged():
             yo, so = oracle.wkv7(*ops, None)
             assert rel_err(y[lo:hi, h:h + 1][None], yo) <= TOL_BF16, (b, h)
             assert rel_err(s[b:b + 1, h:h + 1], so) <= TOL_BF16, (b, h)
+
+
+@pytest.mark.slow
+def test_full_size_headline_pure_accumulation_every_pair():
+    # w = 1, a = b = 0 at the headline shape (B4 T16384 H64) and launch configuration: the end state of
+    # EVERY (b, h) equals sum_t v_t k_t^T (zero initial state), and y at sampled tokens equals the
+    # closed form (float64 matmuls of the same bf16 values)
+    case = wi.CASES["prefill_d4096_b4_t16384"]
+    d = wi.draw_case(case)
+    dd = to_dev(d)
+    dd["w"] = torch.ones_like(dd["w"])
+    dd["a"] = torch.zeros_like(dd["a"])
+    dd["b"] = torch.zeros_like(dd["b"])
+    y, s = gpu_prefill(dd, None)
+    del dd
+    v = d["v"].double().numpy().transpose(0, 2, 3, 1)  # [B, H, 64 (i), T]
+    k = d["k"].double().numpy().transpose(0, 2, 1, 3)  # [B, H, T, 64 (j)]
+    r = d["r"].double().numpy()                          # [B, T, H, 64]
+    assert rel_err(s, np.matmul(v, k)) <= TOL_F32
+    yc = y.float().cpu().numpy()
+    for t in (0, 63, 64, 8191, case.T - 1):
+        st = np.matmul(v[..., :t + 1], k[:, :, :t + 1])
+        yo = np.einsum("bhij,bhj->bhi", st, r[:, t])
+        assert rel_err(yc[:, t], yo) <= TOL_BF16, t

@@ -30,8 +30,18 @@
 namespace rwkv7 {
 namespace bwd {
 
-constexpr int kRows = 16;                 // state rows per CTA (4 CTAs per (b, h))
-constexpr int kThreads = kRows * 8;       // 8 lanes per row: 128 threads, 4 warps of 4 rows
+// A thread layout: 16 state rows per CTA (4 CTAs per (b, h)), kLanes lanes per row, each holding
+// 64 / kLanes columns: 128 threads at 8 lanes, 256 at 16 (twice the warps for the same rows, to hide
+// the latency of the per-token chain).
+template <int kLanes> struct Layout {
+  static constexpr int kRows = 16;
+  static constexpr int kCols = kN / kLanes;              // 8 or 4
+  static constexpr int kThreads = kRows * kLanes;        // 128 or 256
+};
+#ifndef RWKV7_BWD_LANES
+#define RWKV7_BWD_LANES 16
+#endif
+constexpr int kBwdLanes = RWKV7_BWD_LANES;  // the layout the library launches
 constexpr int kSub = 8;                   // tokens per sub-block
 constexpr int kChunk = 64;                // tokens per saved state
 constexpr int kSubs = kChunk / kSub;      // sub-blocks per chunk
@@ -39,10 +49,10 @@ constexpr int kTokVec = 7;                // staged per token: r, w, k, a, b, v,
 constexpr int kStageElems = kSub * kTokVec * kN;
 enum { V_R = 0, V_W = 1, V_K = 2, V_A = 3, V_B = 4, V_V = 5, V_DY = 6 };
 
-constexpr size_t kSmemSubck = sizeof(float) * kSubs * kRows * kN;   // 32 KB
+template <int kLanes> __host__ __device__ constexpr size_t smem_subck() { return sizeof(float) * kSubs * Layout<kLanes>::kRows * kN; }
 constexpr size_t kSmemStage = sizeof(uint16_t) * 2 * kStageElems;   // 14 KB
-constexpr size_t kSmemPart = sizeof(float) * kRows * 5 * kN;         // 20 KB: [row][5][64] partials
-constexpr size_t kSmemBytes = kSmemSubck + kSmemStage + kSmemPart;
+template <int kLanes> __host__ __device__ constexpr size_t smem_part() { return sizeof(float) * Layout<kLanes>::kRows * 5 * kN; }
+template <int kLanes> __host__ __device__ constexpr size_t smem_bytes() { return smem_subck<kLanes>() + kSmemStage + smem_part<kLanes>(); }
 
 struct Args {
   const uint16_t *r, *w, *k, *v, *a, *b, *dy;
@@ -76,6 +86,7 @@ __device__ __forceinline__ Visit visit_at(int kk, int nck, int nsub_last) {
   return v;
 }
 
+template <int kThreads>
 __device__ __forceinline__ void stage_visit(const Args &A, uint16_t *buf, long long tok0, int ntok, int h) {
   const int total = ntok * kTokVec * 8;  // 16-byte pieces
   for (int c = threadIdx.x; c < total; c += kThreads) {
@@ -92,53 +103,64 @@ __device__ __forceinline__ void stage_visit(const Args &A, uint16_t *buf, long l
   }
 }
 
-__device__ __forceinline__ void ld8(const uint16_t *p, float (&o)[8]) {
-  const uint4 u = *reinterpret_cast<const uint4 *>(p);
-  o[0] = __uint_as_float(u.x << 16);
-  o[1] = __uint_as_float(u.x & 0xffff0000u);
-  o[2] = __uint_as_float(u.y << 16);
-  o[3] = __uint_as_float(u.y & 0xffff0000u);
-  o[4] = __uint_as_float(u.z << 16);
-  o[5] = __uint_as_float(u.z & 0xffff0000u);
-  o[6] = __uint_as_float(u.w << 16);
-  o[7] = __uint_as_float(u.w & 0xffff0000u);
+// kC consecutive bf16 values (kC = 8: one 16-byte load, 4: one 8-byte load) as floats
+template <int kC> __device__ __forceinline__ void ldc(const uint16_t *p, float (&o)[kC]) {
+  if constexpr (kC == 8) {
+    const uint4 u = *reinterpret_cast<const uint4 *>(p);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      o[2 * i] = __uint_as_float(w[i] << 16);
+      o[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+  } else {
+    static_assert(kC == 4, "4 or 8 columns per thread");
+    const uint2 u = *reinterpret_cast<const uint2 *>(p);
+    o[0] = __uint_as_float(u.x << 16);
+    o[1] = __uint_as_float(u.x & 0xffff0000u);
+    o[2] = __uint_as_float(u.y << 16);
+    o[3] = __uint_as_float(u.y & 0xffff0000u);
+  }
 }
 
-__device__ __forceinline__ float rowsum8(float x) {
-  x += __shfl_xor_sync(0xffffffffu, x, 1);
-  x += __shfl_xor_sync(0xffffffffu, x, 2);
-  x += __shfl_xor_sync(0xffffffffu, x, 4);
+// sum over the kLanes lanes that hold one row
+template <int kLanes> __device__ __forceinline__ float rowsum(float x) {
+#pragma unroll
+  for (int off = 1; off < kLanes; off <<= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
   return x;
 }
 
-// One forward token on this thread's 8 columns (c0 ..) of row `row`: S <- S diag(w) + (S a) b^T + v k^T.
-__device__ __forceinline__ void fwd_token(float (&S)[8], const uint16_t *tk, int c0, int row) {
-  float w8[8], k8[8], a8[8], b8[8];
-  ld8(tk + V_W * kN + c0, w8);
-  ld8(tk + V_K * kN + c0, k8);
-  ld8(tk + V_A * kN + c0, a8);
-  ld8(tk + V_B * kN + c0, b8);
+// One forward token on this thread's columns (c0 ..) of row `row`: S <- S diag(w) + (S a) b^T + v k^T.
+template <int kLanes, int kC>
+__device__ __forceinline__ void fwd_token(float (&S)[kC], const uint16_t *tk, int c0, int row) {
+  float w8[kC], k8[kC], a8[kC], b8[kC];
+  ldc<kC>(tk + V_W * kN + c0, w8);
+  ldc<kC>(tk + V_K * kN + c0, k8);
+  ldc<kC>(tk + V_A * kN + c0, a8);
+  ldc<kC>(tk + V_B * kN + c0, b8);
   const float vi = bf16_bits_to_float(tk[V_V * kN + row]);
   float sa = 0.f;
 #pragma unroll
-  for (int e = 0; e < 8; ++e) sa = fmaf(S[e], a8[e], sa);
-  sa = rowsum8(sa);
+  for (int e = 0; e < kC; ++e) sa = fmaf(S[e], a8[e], sa);
+  sa = rowsum<kLanes>(sa);
 #pragma unroll
-  for (int e = 0; e < 8; ++e) S[e] = fmaf(S[e], w8[e], fmaf(sa, b8[e], vi * k8[e]));
+  for (int e = 0; e < kC; ++e) S[e] = fmaf(S[e], w8[e], fmaf(sa, b8[e], vi * k8[e]));
 }
 
-__global__ void __launch_bounds__(kThreads) wkv7_backward_kernel(const Args A) {
+template <int kLanes>
+__global__ void __launch_bounds__(Layout<kLanes>::kThreads) wkv7_backward_kernel(const Args A) {
+  constexpr int kRows = Layout<kLanes>::kRows, kC = Layout<kLanes>::kCols, kThreads = Layout<kLanes>::kThreads;
   extern __shared__ __align__(16) uint8_t smem_raw[];
   float *subck = reinterpret_cast<float *>(smem_raw);
-  uint16_t *stage = reinterpret_cast<uint16_t *>(smem_raw + kSmemSubck);
-  float *part = reinterpret_cast<float *>(smem_raw + kSmemSubck + kSmemStage);
+  uint16_t *stage = reinterpret_cast<uint16_t *>(smem_raw + smem_subck<kLanes>());
+  float *part = reinterpret_cast<float *>(smem_raw + smem_subck<kLanes>() + kSmemStage);
 
   constexpr int kSplits = kN / kRows;
   const int h = blockIdx.x / kSplits;
   const int row0 = (blockIdx.x - h * kSplits) * kRows;
   const int bidx = blockIdx.y;
   const int tid = threadIdx.x;
-  const int rl = tid >> 3, c0 = 8 * (tid & 7);
+  const int rl = tid / kLanes, c0 = kC * (tid % kLanes);
   const int row = row0 + rl;  // state row (value channel) of this thread
   const int T = A.T;
   const long long pair = static_cast<long long>(bidx) * A.H + h;
@@ -147,17 +169,17 @@ __global__ void __launch_bounds__(kThreads) wkv7_backward_kernel(const Args A) {
   const int nsub_last = nck > 0 ? (T - (nck - 1) * kChunk + kSub - 1) / kSub : 0;
   const int nvisits = nck > 0 ? 2 * nsub_last + 2 * kSubs * (nck - 1) : 0;
 
-  float G[8];  // dL/dS for this thread's columns of its row
+  float G[kC];  // dL/dS for this thread's columns of its row
 #pragma unroll
-  for (int e = 0; e < 8; ++e) G[e] = A.ds_out ? A.ds_out[pair * (kN * kN) + row * kN + c0 + e] : 0.f;
-  float S[8];  // running state of the forward passes
+  for (int e = 0; e < kC; ++e) G[e] = A.ds_out ? A.ds_out[pair * (kN * kN) + row * kN + c0 + e] : 0.f;
+  float S[kC];  // running state of the forward passes
 #pragma unroll
-  for (int e = 0; e < 8; ++e) S[e] = 0.f;
+  for (int e = 0; e < kC; ++e) S[e] = 0.f;
 
   if (nvisits > 0) {
     const Visit v0 = visit_at(0, nck, nsub_last);
     const int t0 = v0.c * kChunk + v0.s * kSub;
-    stage_visit(A, stage, tok_base + t0, min(kSub, T - t0), h);
+    stage_visit<kThreads>(A, stage, tok_base + t0, min(kSub, T - t0), h);
     cp_async_commit();
   }
   for (int kk = 0; kk < nvisits; ++kk) {
@@ -165,7 +187,7 @@ __global__ void __launch_bounds__(kThreads) wkv7_backward_kernel(const Args A) {
     if (kk + 1 < nvisits) {
       const Visit vn = visit_at(kk + 1, nck, nsub_last);
       const int tn = vn.c * kChunk + vn.s * kSub;
-      stage_visit(A, stage + ((kk + 1) & 1) * kStageElems, tok_base + tn, min(kSub, T - tn), h);
+      stage_visit<kThreads>(A, stage + ((kk + 1) & 1) * kStageElems, tok_base + tn, min(kSub, T - tn), h);
       cp_async_commit();
       cp_async_wait<1>();
     } else {
@@ -182,41 +204,41 @@ __global__ void __launch_bounds__(kThreads) wkv7_backward_kernel(const Args A) {
       if (vis.s == 0) {
         const float *ck = A.states + (pair * nck + vis.c) * (kN * kN) + row * kN + c0;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) S[e] = ck[e];
+        for (int e = 0; e < kC; ++e) S[e] = ck[e];
       }
 #pragma unroll
-      for (int e = 0; e < 8; ++e) sck[e] = S[e];
-      for (int u = 0; u < Ls; ++u) fwd_token(S, buf + u * kTokVec * kN, c0, row);
+      for (int e = 0; e < kC; ++e) sck[e] = S[e];
+      for (int u = 0; u < Ls; ++u) fwd_token<kLanes, kC>(S, buf + u * kTokVec * kN, c0, row);
     } else {
       // this sub-block's states: St[u] before token t0 + u, St[u + 1] after it
-      float St[kSub + 1][8];
+      float St[kSub + 1][kC];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) St[0][e] = sck[e];
+      for (int e = 0; e < kC; ++e) St[0][e] = sck[e];
 #pragma unroll
       for (int u = 0; u < kSub; ++u) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) St[u + 1][e] = St[u][e];
-        if (u < Ls) fwd_token(St[u + 1], buf + u * kTokVec * kN, c0, row);
+        for (int e = 0; e < kC; ++e) St[u + 1][e] = St[u][e];
+        if (u < Ls) fwd_token<kLanes, kC>(St[u + 1], buf + u * kTokVec * kN, c0, row);
       }
 #pragma unroll
       for (int u = kSub - 1; u >= 0; --u) {
         if (u >= Ls) continue;  // uniform across the CTA
         const uint16_t *tk = buf + u * kTokVec * kN;
-        float r8[8], w8[8], k8[8], a8[8], b8[8];
-        ld8(tk + V_R * kN + c0, r8);
-        ld8(tk + V_W * kN + c0, w8);
-        ld8(tk + V_K * kN + c0, k8);
-        ld8(tk + V_A * kN + c0, a8);
-        ld8(tk + V_B * kN + c0, b8);
+        float r8[kC], w8[kC], k8[kC], a8[kC], b8[kC];
+        ldc<kC>(tk + V_R * kN + c0, r8);
+        ldc<kC>(tk + V_W * kN + c0, w8);
+        ldc<kC>(tk + V_K * kN + c0, k8);
+        ldc<kC>(tk + V_A * kN + c0, a8);
+        ldc<kC>(tk + V_B * kN + c0, b8);
         const float vi = bf16_bits_to_float(tk[V_V * kN + row]);
         const float dyi = bf16_bits_to_float(tk[V_DY * kN + row]);
         // y_t = S' r_t
 #pragma unroll
-        for (int e = 0; e < 8; ++e) G[e] = fmaf(dyi, r8[e], G[e]);
-        float p[5][8];  // column partials: dr, dk, db, dw, da
+        for (int e = 0; e < kC; ++e) G[e] = fmaf(dyi, r8[e], G[e]);
+        float p[5][kC];  // column partials: dr, dk, db, dw, da
         float dv = 0.f, sa = 0.f, g = 0.f;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
+        for (int e = 0; e < kC; ++e) {
           p[0][e] = St[u + 1][e] * dyi;
           dv = fmaf(G[e], k8[e], dv);
           p[1][e] = G[e] * vi;
@@ -224,25 +246,26 @@ __global__ void __launch_bounds__(kThreads) wkv7_backward_kernel(const Args A) {
           g = fmaf(G[e], b8[e], g);
           p[3][e] = G[e] * St[u][e];
         }
-        dv = rowsum8(dv);
-        sa = rowsum8(sa);
-        g = rowsum8(g);
+        dv = rowsum<kLanes>(dv);
+        sa = rowsum<kLanes>(sa);
+        g = rowsum<kLanes>(g);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
+        for (int e = 0; e < kC; ++e) {
           p[2][e] = G[e] * sa;
           p[4][e] = St[u][e] * g;
           G[e] = fmaf(G[e], w8[e], g * a8[e]);
         }
         // column sums: every thread's partials to shared memory, then one 4-column group over the
-        // 16 rows per thread (80 of them), then the 4 row groups through float32 atomics
+        // CTA's rows per thread (80 of them), then the row groups through float32 atomics
         const long long tok = tok_base + t0 + u;
 #pragma unroll
         for (int q = 0; q < 5; ++q) {
           float *dst = part + (rl * 5 + q) * kN + c0;
-          *reinterpret_cast<float4 *>(dst) = make_float4(p[q][0], p[q][1], p[q][2], p[q][3]);
-          *reinterpret_cast<float4 *>(dst + 4) = make_float4(p[q][4], p[q][5], p[q][6], p[q][7]);
+#pragma unroll
+          for (int x = 0; x < kC; x += 4)
+            *reinterpret_cast<float4 *>(dst + x) = make_float4(p[q][x], p[q][x + 1], p[q][x + 2], p[q][x + 3]);
         }
-        if ((tid & 7) == 0) A.dv[(tok * A.H + h) * kN + row] = dv;
+        if (tid % kLanes == 0) A.dv[(tok * A.H + h) * kN + row] = dv;
         __syncthreads();
         if (tid < 5 * kN / 4) {
           const int q = tid >> 4, c4 = (tid & 15) * 4;
@@ -269,7 +292,7 @@ __global__ void __launch_bounds__(kThreads) wkv7_backward_kernel(const Args A) {
   }
   if (A.ds_in != nullptr)
 #pragma unroll
-    for (int e = 0; e < 8; ++e) A.ds_in[pair * (kN * kN) + row * kN + c0 + e] = G[e];
+    for (int e = 0; e < kC; ++e) A.ds_in[pair * (kN * kN) + row * kN + c0 + e] = G[e];
 }
 
 }  // namespace bwd
@@ -280,11 +303,13 @@ cudaError_t launch_backward(const uint16_t *r, const uint16_t *w, const uint16_t
                             float *ds_in, int B, int T, int H, cudaStream_t stream) {
   using namespace bwd;
   Args A{r, w, k, v, a, b, dy, states, ds_out, dr, dw, dk, dv, da, db, ds_in, T, H};
-  cudaError_t e = cudaFuncSetAttribute(wkv7_backward_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(kSmemBytes));
+  constexpr int kLanes = kBwdLanes;
+  using L = Layout<kLanes>;
+  cudaError_t e = cudaFuncSetAttribute(wkv7_backward_kernel<kLanes>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem_bytes<kLanes>()));
   if (e != cudaSuccess) return e;
-  dim3 grid(H * (kN / kRows), B);
-  wkv7_backward_kernel<<<grid, kThreads, kSmemBytes, stream>>>(A);
+  dim3 grid(H * (kN / L::kRows), B);
+  wkv7_backward_kernel<kLanes><<<grid, L::kThreads, smem_bytes<kLanes>(), stream>>>(A);
   return cudaGetLastError();
 }
 

@@ -86,14 +86,14 @@ typedef enum rwkv7_status {
  * otherwise SCAN); SCAN is the sequential kernel (state in registers); CHUNK
  * is the chunked tensor-core kernel (bf16 only).
  * Decay domain of CHUNK: the chunked form divides by the product of up to 64
- * consecutive decays.  Its schedules 0-2 (see rwkv7_options.chunk_schedule)
- * need that product to stay >= 2^-100 in every channel of every 64-token
- * chunk (true whenever every w >= 0.34; the model's decay
- * exp(-e^-0.5 sigmoid(x)) always lies in [0.5452, 1)); a chunk outside it is
- * detected on the device and reported by rwkv7_get_last_error() as
- * RWKV7_ERR_DOMAIN, and that call's y and s_out are not valid.  Schedule 3 and
- * SCAN are exact for every w in [0, 1] (schedule 3 runs such a chunk token by
- * token in float32). */
+ * consecutive decays, so it factorises a 64-token chunk only while that
+ * product stays >= 2^-100 in every channel (true whenever every w >= 0.34; the
+ * model's decay exp(-e^-0.5 sigmoid(x)) always lies in [0.5452, 1)).  A chunk
+ * outside that range (w near 0, or exactly 0) is detected on the device and run
+ * token by token in float32 instead, on every schedule, so CHUNK, AUTO and SCAN
+ * are exact for every w in [0, 1].  (With model-native inputs the decay cannot
+ * leave the range; there such a chunk would be reported by
+ * rwkv7_get_last_error() as RWKV7_ERR_DOMAIN.) */
 typedef enum rwkv7_prefill_path {
   RWKV7_PATH_AUTO = 0,
   RWKV7_PATH_SCAN = 1,
@@ -109,8 +109,8 @@ RWKV7_API rwkv7_status rwkv7_wkv_prefill(int B, int T, int H, int N, const float
                                const float *s_in, float *y, float *s_out, rwkv7_stream_t stream);
 
 /* Same, bfloat16 operands and y (bit patterns), float32 state.  The kernel is
- * chosen as for RWKV7_PATH_AUTO, so the decay domain of CHUNK above applies
- * from T >= 128 (a violation is reported as RWKV7_ERR_DOMAIN). */
+ * chosen as for RWKV7_PATH_AUTO (see the decay domain above: exact for every
+ * w in [0, 1]). */
 RWKV7_API rwkv7_status rwkv7_wkv_prefill_bf16(int B, int T, int H, int N, const uint16_t *r,
                                     const uint16_t *w, const uint16_t *k, const uint16_t *v,
                                     const uint16_t *a, const uint16_t *b, const float *s_in,
@@ -206,8 +206,9 @@ RWKV7_API rwkv7_status rwkv7_wkv_decode_fused_bf16(int B, int H, int N, const ui
  *                         Choice 0 never takes this schedule while `stream` is capturing.
  *                     3 = a warp-specialised pipeline: one persistent CTA per SM walks its (b, h)
  *                         pairs' chunks with three chunks in flight (operand preparation, masks
- *                         and inverse, state chain on separate warps); exact for every decay in
- *                         [0, 1] (see the decay domain above).  Needs H <= 65535.
+ *                         and inverse, state chain on separate warps).  Needs H <= 65535.
+ *                     Every schedule is exact for every decay in [0, 1] (see the decay domain
+ *                     above).
  */
 typedef struct rwkv7_options {
   int model_native;

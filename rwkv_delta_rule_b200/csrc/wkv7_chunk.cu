@@ -138,6 +138,9 @@ struct Args {
   int nck;                    // chunks per sequence, ceil(T / 64)
   uint32_t max_polls;         // bound of every wait (kMaxPolls unless a test lowers it)
   long long skip_publish;     // test hook: this pair's first chunk never raises its flag (-1: none)
+  // the operands [tokens, H, 64] (bf16), read directly by the token-by-token path of a chunk outside
+  // the factorised range
+  const uint16_t *r, *w, *k, *v, *a, *b;
 };
 
 // One unit of work: chunk c of the (b, h) pair bh.
@@ -437,7 +440,7 @@ __device__ __forceinline__ void invert_unit_lower(const float *Ls, float *Ts, fl
 template <bool kFused>
 __device__ __forceinline__ void prep_next(const uint8_t *smem, uint8_t *sA1, uint8_t *sB1, uint8_t *sB4Vn, float *pre4,
                                           float *GCn, float *wtot, const float *kkw, float *invn, int tid4, int Lcn,
-                                          int *err) {
+                                          int *err, volatile int *dflag) {
   const int lane = tid4 & 31, wq = tid4 >> 5;
   const int cq = tid4 & 15, to = tid4 >> 4;  // channel quad; token octet (2 per warp)
   const int j0 = 4 * cq, tb = 8 * to;
@@ -493,6 +496,7 @@ __device__ __forceinline__ void prep_next(const uint8_t *smem, uint8_t *sA1, uin
   if (lane >= 16)
     *reinterpret_cast<float4 *>(wtot + wq * 64 + j0) =
         make_float4(exo[0] * oct[0], exo[1] * oct[1], exo[2] * oct[2], exo[3] * oct[3]);
+  if (tid4 == 0) *dflag = 0;
   group_sync_hi();
   float p0[4], p1[4], gc[4];
 #pragma unroll
@@ -519,10 +523,16 @@ __device__ __forceinline__ void prep_next(const uint8_t *smem, uint8_t *sA1, uin
   *reinterpret_cast<float4 *>(pre4 + (2 * to + 1) * 64 + j0) = make_float4(p1[0], p1[1], p1[2], p1[3]);
   if (to == 0) *reinterpret_cast<float4 *>(GCn + j0) = make_float4(gc[0], gc[1], gc[2], gc[3]);
   // B^ and K^ divide by the decay products of the chunk: below 2^-100 (or not a number) the factors
-  // leave float32's range and the chunk's results are not valid; the call reports it
+  // leave float32's range and the chunk's tensor-core results are not valid.  With bf16 operands the
+  // chunk is flagged and its read-out runs its tokens one by one instead; model-native inputs never
+  // get there (every decay is >= 0.5452), and would report it.
   if (to == 0 && !(gc[0] >= 7.8886090522101181e-31f && gc[1] >= 7.8886090522101181e-31f &&
-                   gc[2] >= 7.8886090522101181e-31f && gc[3] >= 7.8886090522101181e-31f))
-    report_device_error(err, kDevErrDomain);
+                   gc[2] >= 7.8886090522101181e-31f && gc[3] >= 7.8886090522101181e-31f)) {
+    if (kFused)
+      report_device_error(err, kDevErrDomain);
+    else
+      *dflag = 1;
+  }
   // [B^; K^] rows (K-major tf32; K = channel), and Gamma_t itself (float32) where the operand
   // construction will put R~ = r Gamma_t: it reads Gamma_t there and overwrites it in place
   uint8_t *b1r = sB1 + (j0 >> 5) * (128 * 128);
@@ -578,6 +588,111 @@ __device__ __forceinline__ void prep_next(const uint8_t *smem, uint8_t *sA1, uin
   tc::fence_proxy_async_smem();
 }
 
+// 16 consecutive bf16 values (32 bytes, 16-byte aligned) as floats
+__device__ __forceinline__ void ld16_bf16(const uint16_t *p, float (&o)[16]) {
+  const uint4 u0 = *reinterpret_cast<const uint4 *>(p), u1 = *reinterpret_cast<const uint4 *>(p + 8);
+  const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+  for (int x = 0; x < 8; ++x) {
+    o[2 * x] = __uint_as_float(w[x] << 16);
+    o[2 * x + 1] = __uint_as_float(w[x] & 0xffff0000u);
+  }
+}
+
+// The token-by-token path of a chunk whose decay products left the factorised range (bf16 operands),
+// run by the 256 compute threads in place of the chunk's read-out: the start state goes to Ls as
+// float32 (row i = value channel, column j), every token is applied in float32 in the pages' order
+// (sa = S a; S = S diag(w) + sa b^T + v k^T; y = S r), exact for every decay in [0, 1], and the end
+// state goes back where the read-out would have left it (one pair per CTA: TMEM, its tf32 copy in
+// B4S and the checkpoint; task-parallel: float32 in B4S).  Thread t owns row t / 4, columns
+// 16 (t % 4) .. + 15; row sums are two xor-shuffles inside the quad.
+template <bool kLN, bool kTask>
+__device__ __forceinline__ void chunk_by_tokens(const Args &A, const Task &pt, uint8_t *sB4S, float *Ls, float *ybuf,
+                                             const float *lnp, uint32_t tmem_s, int tid, bool hi_lanes, int j,
+                                             int hh, int lane) {
+  if (hi_lanes) {
+    if constexpr (!kTask) {
+      float sv[32];
+      tc::tmem_ld32(tmem_s + 32 * hh, sv);
+#pragma unroll
+      for (int x = 0; x < 32; ++x) Ls[(32 * hh + x) * LDL + j] = sv[vrow(x)];
+    } else {
+      const ColPtrs cp = col_ptrs(sB4S, 64, 32 * hh, j);
+#pragma unroll
+      for (int x = 0; x < 32; ++x)
+        Ls[(32 * hh + x) * LDL + j] = *reinterpret_cast<const float *>(cp.p[vrow(x) & 7] + vrow(x) * 128);
+    }
+  }
+  compute_sync();
+  const int i = tid >> 2, c0 = 16 * (tid & 3);
+  float S[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) S[e] = Ls[i * LDL + c0 + e];
+  for (int u = 0; u < pt.Lc; ++u) {
+    const long long base = ((pt.tok0 + u) * A.H + pt.h) * kN;
+    float w[16], k[16], a[16], b[16], r[16];
+    ld16_bf16(A.w + base + c0, w);
+    ld16_bf16(A.k + base + c0, k);
+    ld16_bf16(A.a + base + c0, a);
+    ld16_bf16(A.b + base + c0, b);
+    ld16_bf16(A.r + base + c0, r);
+    const float vi = bf16_bits_to_float(A.v[base + i]);
+    float sa = 0.f;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) sa = fmaf(S[e], a[e], sa);
+    sa += __shfl_xor_sync(0xffffffffu, sa, 1);
+    sa += __shfl_xor_sync(0xffffffffu, sa, 2);
+    float yv = 0.f;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      S[e] = fmaf(S[e], w[e], fmaf(sa, b[e], vi * k[e]));
+      yv = fmaf(S[e], r[e], yv);
+    }
+    yv += __shfl_xor_sync(0xffffffffu, yv, 1);
+    yv += __shfl_xor_sync(0xffffffffu, yv, 2);
+    if constexpr (!kLN) {
+      if ((tid & 3) == 0) A.y[base + i] = float_to_bf16_bits(yv);
+    } else {
+      // ln_x over the token's 64 outputs, by warp 0 (two channels per lane)
+      if ((tid & 3) == 0) ybuf[i] = yv;
+      compute_sync();
+      if (tid < 32) {
+        const float y0 = ybuf[tid], y1 = ybuf[tid + 32];
+        float mean, var;
+        warp_mean_var64(y0, y1, mean, var);
+        const float rs = rsqrtf(var + kLnEps);
+        A.y[base + tid] = float_to_bf16_bits(fmaf((y0 - mean) * rs, lnp[tid], lnp[64 + tid]));
+        A.y[base + tid + 32] = float_to_bf16_bits(fmaf((y1 - mean) * rs, lnp[tid + 32], lnp[96 + tid]));
+      }
+      compute_sync();
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 16; ++e) Ls[i * LDL + c0 + e] = S[e];
+  compute_sync();
+  if (hi_lanes) {
+    if constexpr (!kTask) {
+      float sv[32];
+#pragma unroll
+      for (int x = 0; x < 32; ++x) sv[vrow(x)] = Ls[(32 * hh + x) * LDL + j];
+      tc::tmem_st32(tmem_s + 32 * hh, sv);
+      store_state_rows_tf32(sB4S, j, hh, sv);
+      if (A.states != nullptr && pt.c + 1 < A.nck) {
+        float *ck = A.states + (pt.bh * A.nck + pt.c + 1) * (kN * kN) + static_cast<long long>(32 * hh) * kN + j;
+#pragma unroll
+        for (int x = 0; x < 32; ++x) ck[x * kN] = sv[vrow(x)];
+      }
+      tc::tmem_st_wait();
+    } else {
+      const ColPtrs cp = col_ptrs(sB4S, 64, 32 * hh, j);
+#pragma unroll
+      for (int x = 0; x < 32; ++x)
+        *reinterpret_cast<float *>(cp.p[vrow(x) & 7] + vrow(x) * 128) = Ls[(32 * hh + x) * LDL + j];
+    }
+  }
+  (void)lane;
+}
+
 // kFused: model-native inputs -- the w, a and b tiles hold x_w, x_a and nothing; w = decay(x_w),
 // a = -kk and b = kk * sigmoid(x_a) with kk = k * k_k / |k * k_k| are formed where the operands are
 // built (the decay-scan / [B^; K^] preparation and P1), and only five tiles are loaded per chunk.
@@ -616,6 +731,8 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
   uint64_t *bar_m4 = bars + 8;     // c -> w: MMA4 done
   uint64_t *bar_sin = bars + 9;    // task-parallel: the start state landed in B4S (tx bytes)
   uint64_t *bar_sout = bars + 10;  // task-parallel: w -> c, the end state is in B4S (one arrival per hi-lane warp)
+  // [2] by chunk parity: the preparation found the chunk's decay products outside the factorised range
+  volatile int *dflag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 192);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_MISC + 88);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 92);
   float *GCs = reinterpret_cast<float *>(smem + OFF_MISC + MISC_GC);  // [2][64]
@@ -961,6 +1078,16 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
     float gc_done = 1.f;  // Gamma_C[j] of the chunk whose MMA4 is in flight (hi lanes)
     auto readout = [&](const Task &pt, uint32_t par) {
       const int hh = ch;
+      if (!kFused && dflag[par] != 0) {
+        // the chunk left the factorised range: its tensor-core results are dropped
+        chunk_by_tokens<kLN, kTask>(A, pt, sB4S, Ls, Ts, lnw + par * 128, tmem + lane_base + TM_S, tid, hi_lanes, j,
+                                    hh, lane);
+        if (kTask && hi_lanes) {
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(bar_sout);
+        }
+        return;
+      }
       float v[32];
       tc::tmem_ld32(tmem + lane_base + TM_D4 + 32 * hh, v);
       if (!hi_lanes) {
@@ -1039,7 +1166,7 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
         if (t0.n >= 0) {
           load_head(t0.h, 0, tid - 128);
           group_sync_hi();
-          prep_next<kFused>(smem, sA1, sB1, sB4V, pre4, GCs, wtot, kkw, invn, tid - 128, t0.Lc, A.err);
+          prep_next<kFused>(smem, sA1, sB1, sB4V, pre4, GCs, wtot, kkw, invn, tid - 128, t0.Lc, A.err, dflag);
         }
       }
       compute_sync();
@@ -1052,7 +1179,7 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
         load_head(have ? t.h : 0, 1, tid - 128);
       }
       if (have && warp >= 4 && wait_group_hi(bar_tma, 0))
-        prep_next<kFused>(smem, sA1, sB1, sB4V, pre4, GCs, wtot, kkw, invn, tid - 128, t.Lc, A.err);
+        prep_next<kFused>(smem, sA1, sB1, sB4V, pre4, GCs, wtot, kkw, invn, tid - 128, t.Lc, A.err, dflag);
       compute_sync();
     }
 
@@ -1241,14 +1368,14 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
               load_head(nt.h, (it + 1) & 1, tid - 128);
               group_sync_hi();
               prep_next<kFused>(smem, sA1, sB1, sB4V + ((it + 1) & 1) * 16384, pre4,
-                                       GCs + ((it + 1) & 1) * 64, wtot, kkw, invn, tid - 128, nt.Lc, A.err);
+                                       GCs + ((it + 1) & 1) * 64, wtot, kkw, invn, tid - 128, nt.Lc, A.err, dflag + ((it + 1) & 1));
             }
           }
         } else {
           Task nt = t;
           if (pair_next(A, nt) && wait_group_hi(bar_tma, (it + 1) & 1))
             prep_next<kFused>(smem, sA1, sB1, sB4V + ((it + 1) & 1) * 16384, pre4, GCs + ((it + 1) & 1) * 64,
-                                     wtot, kkw, invn, tid - 128, nt.Lc, A.err);
+                                     wtot, kkw, invn, tid - 128, nt.Lc, A.err, dflag + ((it + 1) & 1));
         }
       }
       if (!(ok = wait_ctrl(bar_m3, ph))) break;
@@ -1461,7 +1588,7 @@ cudaError_t launch_chunk_ext(const uint16_t *r, const uint16_t *w, const uint16_
   const long long ntasks = (rows / C) * BH;
   const int nck = (T + C - 1) / C;
   Args args{y, s_in, s_out, cu_seqlens, T, total_T, H, err_word, k_k, ln_w, ln_b, ntasks, BH, nullptr, 0, 0,
-            states, nck, g_hook_max_polls.load(), -1};
+            states, nck, g_hook_max_polls.load(), -1, r, w, k, v, a, b};
   // The task-parallel schedule pays when one CTA per pair would leave many SMs idle: measured on B200,
   // 48 and 96 pairs ran 1.2x and 1.1x faster, 1 and 2 pairs 1.6x; at 128 pairs and above the pair
   // schedule was as fast or faster.

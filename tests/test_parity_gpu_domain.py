@@ -4,9 +4,10 @@ The chunked form divides by the product of up to 64 consecutive decays.  The mod
 [0.5452, 1) (RWKV-7 G0 7.2B walkthrough, lshu.cn/news/198401, section 7.1), but the recurrence takes any
 w in [0, 1], so the kernels are checked on decays the model never produces:
   * w ~ U(0.27, 0.55): every chunked schedule stays inside its factorised range and matches the oracle;
-  * w ~ U(0.02, 0.27), w = 0 in places, and a long sequence with a stretch of fast decays: the
-    pipelined schedule (which runs an out-of-range chunk token by token) and the sequential scan match
-    the oracle, and the other chunked schedules report RWKV7_ERR_DOMAIN instead of returning silently;
+  * w ~ U(0.02, 0.27), w = 0 in places, and a long sequence with a stretch of fast decays: every
+    chunked schedule runs a chunk outside its factorised range token by token in float32, so all of
+    them, AUTO and the sequential scan match the oracle (model-native inputs never leave the range;
+    they would report RWKV7_ERR_DOMAIN);
   * w = 1 everywhere (no decay at all).
 Bars as for every bf16 parity test: max|gpu - oracle| / max|oracle| <= 5e-3 for y and the end state.
 """
@@ -76,10 +77,12 @@ def test_fast_decay(B, T, H):
     assert st == 0
     assert rel_err(y, yo) <= TOL_BF16
     assert rel_err(s, so) <= TOL_BF16
-    # the other chunked schedules cannot factorise these chunks: they say so
-    for sched in (rk.RWKV7_SCHED_PAIR, rk.RWKV7_SCHED_TASKS):
-        _, _, st = _chunk(d, sched)
-        assert st == ERR_DOMAIN, sched
+    # the other chunked schedules cannot factorise these chunks either: they run them token by token
+    for sched in (rk.RWKV7_SCHED_AUTO, rk.RWKV7_SCHED_PAIR, rk.RWKV7_SCHED_TASKS):
+        y, s, st = _chunk(d, sched)
+        assert st == 0, sched
+        assert rel_err(y, yo) <= TOL_BF16, sched
+        assert rel_err(s, so) <= TOL_BF16, sched
 
 
 def test_zero_decay_in_places():
@@ -89,10 +92,11 @@ def test_zero_decay_in_places():
 
     d = _draw(1, 257, 2, 920, wfun)
     yo, so = oracle.wkv7(*oracle_ops(d), d["s0"])
-    y, s, st = _chunk(d, rk.RWKV7_SCHED_PIPE)
-    assert st == 0
-    assert rel_err(y, yo) <= TOL_BF16
-    assert rel_err(s, so) <= TOL_BF16
+    for sched in (rk.RWKV7_SCHED_PIPE, rk.RWKV7_SCHED_PAIR, rk.RWKV7_SCHED_TASKS):
+        y, s, st = _chunk(d, sched)
+        assert st == 0, sched
+        assert rel_err(y, yo) <= TOL_BF16, sched
+        assert rel_err(s, so) <= TOL_BF16, sched
 
 
 def test_long_sequence_with_a_stretch_of_fast_decay():
@@ -104,12 +108,46 @@ def test_long_sequence_with_a_stretch_of_fast_decay():
 
     d = _draw(1, 4096, 2, 930, wfun)
     yo, so = oracle.wkv7(*oracle_ops(d), d["s0"])
-    y, s, st = _chunk(d, rk.RWKV7_SCHED_PIPE)
-    assert st == 0
-    assert rel_err(y, yo) <= TOL_BF16
+    for sched in (rk.RWKV7_SCHED_PIPE, rk.RWKV7_SCHED_AUTO, rk.RWKV7_SCHED_PAIR, rk.RWKV7_SCHED_TASKS):
+        y, s, st = _chunk(d, sched)
+        assert st == 0, sched
+        assert rel_err(y, yo) <= TOL_BF16, sched
+        assert rel_err(s, so) <= TOL_BF16, sched
+
+
+@pytest.mark.parametrize("sched", [rk.RWKV7_SCHED_PAIR, rk.RWKV7_SCHED_TASKS])
+def test_fast_decay_with_options_and_checkpoints(sched):
+    # the token-by-token path with the GroupNorm epilogue, and the checkpointing forward's saved states
+    def wfun(g, shape):
+        w = 0.5452 + 0.4548 * torch.rand(shape, generator=g)
+        w[:, 64:192] = 0.02 + 0.25 * torch.rand(w[:, 64:192].shape, generator=g)
+        return w
+
+    d = _draw(2, 300, 3, 950, wfun)
+    yo, so = oracle.wkv7(*oracle_ops(d), d["s0"])
+    ln = wi.draw_group_norm(3, seed=951)
+    yn = oracle.group_norm_heads(yo, ln["ln_w"], ln["ln_b"])
+    dv = to_dev(d)
+    y, s = rk.prefill_ext(*[dv[n] for n in OPS], dv["s0"], path=rk.RWKV7_PATH_CHUNK, group_norm=True,
+                          ln_w=ln["ln_w"].cuda(), ln_b=ln["ln_b"].cuda(), schedule=sched)
+    torch.cuda.synchronize()
+    assert rk.rwkv7_get_last_error() == 0
+    assert rel_err(y, yn) <= TOL_BF16
     assert rel_err(s, so) <= TOL_BF16
-    _, _, st = _chunk(d, rk.RWKV7_SCHED_AUTO)
-    assert st == ERR_DOMAIN
+    if sched == rk.RWKV7_SCHED_PAIR:
+        return
+    # checkpoints: the state before every 64th token (the chunked forward saves them on the tasks schedule)
+    y2, s2, states = rk.prefill_save(*[dv[n] for n in OPS], dv["s0"], path=rk.RWKV7_PATH_CHUNK)
+    torch.cuda.synchronize()
+    assert rk.rwkv7_get_last_error() == 0
+    assert rel_err(y2, yo) <= TOL_BF16
+    for c in range(states.shape[2]):
+        t = 64 * c
+        if t == 0:
+            ref = d["s0"].numpy()
+        else:
+            _, ref = oracle.wkv7(*[d[n + "_f32"][:, :t] for n in OPS], d["s0"])
+        assert rel_err(states[:, :, c], ref) <= TOL_BF16, c
 
 
 @pytest.mark.parametrize("sched", [rk.RWKV7_SCHED_AUTO, rk.RWKV7_SCHED_PIPE])

@@ -51,7 +51,13 @@ enum { V_R = 0, V_W = 1, V_K = 2, V_A = 3, V_B = 4, V_V = 5, V_DY = 6 };
 
 template <int kLanes> __host__ __device__ constexpr size_t smem_subck() { return sizeof(float) * kSubs * Layout<kLanes>::kRows * kN; }
 constexpr size_t kSmemStage = sizeof(uint16_t) * 2 * kStageElems;   // 14 KB
-template <int kLanes> __host__ __device__ constexpr size_t smem_part() { return sizeof(float) * Layout<kLanes>::kRows * 5 * kN; }
+// the column partials of one token: [row][5][64] at 8 lanes; at 16 lanes the two rows a warp holds are
+// summed first ([row pair][5][64]) and the buffer is doubled, alternating by token
+template <int kLanes> __host__ __device__ constexpr int part_rows() { return kLanes == 16 ? Layout<kLanes>::kRows / 2 : Layout<kLanes>::kRows; }
+template <int kLanes> __host__ __device__ constexpr int part_bufs() { return kLanes == 16 ? 2 : 1; }
+template <int kLanes> __host__ __device__ constexpr size_t smem_part() {
+  return sizeof(float) * part_bufs<kLanes>() * part_rows<kLanes>() * 5 * kN;
+}
 template <int kLanes> __host__ __device__ constexpr size_t smem_bytes() { return smem_subck<kLanes>() + kSmemStage + smem_part<kLanes>(); }
 
 struct Args {
@@ -147,8 +153,9 @@ __device__ __forceinline__ void fwd_token(float (&S)[kC], const uint16_t *tk, in
   for (int e = 0; e < kC; ++e) S[e] = fmaf(S[e], w8[e], fmaf(sa, b8[e], vi * k8[e]));
 }
 
+// (3 CTAs per SM: a grid of 4 CTAs per (b, h) is all resident up to 111 pairs)
 template <int kLanes>
-__global__ void __launch_bounds__(Layout<kLanes>::kThreads) wkv7_backward_kernel(const Args A) {
+__global__ void __launch_bounds__(Layout<kLanes>::kThreads, 3) wkv7_backward_kernel(const Args A) {
   constexpr int kRows = Layout<kLanes>::kRows, kC = Layout<kLanes>::kCols, kThreads = Layout<kLanes>::kThreads;
   extern __shared__ __align__(16) uint8_t smem_raw[];
   float *subck = reinterpret_cast<float *>(smem_raw);
@@ -255,15 +262,30 @@ __global__ void __launch_bounds__(Layout<kLanes>::kThreads) wkv7_backward_kernel
           p[4][e] = St[u][e] * g;
           G[e] = fmaf(G[e], w8[e], g * a8[e]);
         }
-        // column sums: every thread's partials to shared memory, then one 4-column group over the
-        // CTA's rows per thread (80 of them), then the row groups through float32 atomics
+        // column sums: the partials to shared memory (at 16 lanes, the warp's two rows summed first, by
+        // an xor-shuffle over lane bit 4), then one 4-column group over the CTA's rows per thread (80 of
+        // them), then the row groups through float32 atomics
         const long long tok = tok_base + t0 + u;
+        constexpr int kPR = part_rows<kLanes>();
+        float *pbuf = part + (part_bufs<kLanes>() == 2 ? (u & 1) : 0) * (kPR * 5 * kN);
+        int prow = rl;
+        bool writes = true;
+        if constexpr (kLanes == 16) {
 #pragma unroll
-        for (int q = 0; q < 5; ++q) {
-          float *dst = part + (rl * 5 + q) * kN + c0;
+          for (int q = 0; q < 5; ++q)
 #pragma unroll
-          for (int x = 0; x < kC; x += 4)
-            *reinterpret_cast<float4 *>(dst + x) = make_float4(p[q][x], p[q][x + 1], p[q][x + 2], p[q][x + 3]);
+            for (int e = 0; e < kC; ++e) p[q][e] += __shfl_xor_sync(0xffffffffu, p[q][e], 16);
+          prow = rl >> 1;
+          writes = (tid & 16) == 0;
+        }
+        if (writes) {
+#pragma unroll
+          for (int q = 0; q < 5; ++q) {
+            float *dst = pbuf + (prow * 5 + q) * kN + c0;
+#pragma unroll
+            for (int x = 0; x < kC; x += 4)
+              *reinterpret_cast<float4 *>(dst + x) = make_float4(p[q][x], p[q][x + 1], p[q][x + 2], p[q][x + 3]);
+          }
         }
         if (tid % kLanes == 0) A.dv[(tok * A.H + h) * kN + row] = dv;
         __syncthreads();
@@ -271,8 +293,8 @@ __global__ void __launch_bounds__(Layout<kLanes>::kThreads) wkv7_backward_kernel
           const int q = tid >> 4, c4 = (tid & 15) * 4;
           float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-          for (int rr = 0; rr < kRows; ++rr) {
-            const float4 x = *reinterpret_cast<const float4 *>(part + (rr * 5 + q) * kN + c4);
+          for (int rr = 0; rr < kPR; ++rr) {
+            const float4 x = *reinterpret_cast<const float4 *>(pbuf + (rr * 5 + q) * kN + c4);
             acc.x += x.x;
             acc.y += x.y;
             acc.z += x.z;
@@ -284,7 +306,9 @@ __global__ void __launch_bounds__(Layout<kLanes>::kThreads) wkv7_backward_kernel
           atomicAdd(g + 2, acc.z);
           atomicAdd(g + 3, acc.w);
         }
-        __syncthreads();  // the partials are rewritten by the next token
+        // the partials are rewritten by the next token (one buffer) or by the token after it, which
+        // every thread reaches only through the next token's barrier (two buffers)
+        if constexpr (part_bufs<kLanes>() == 1) __syncthreads();
       }
     }
     // every thread is done with this staging buffer before the next visit refills it

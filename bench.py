@@ -108,6 +108,21 @@ def decode_bytes(B, H, elem=2, state_elem=4, n_ops=6):
     return B * H * (2 * N * N * state_elem + (n_ops + 1) * N * elem)
 
 
+# Prefill FLOPs per token-head of the chunked form at a fixed reference chunk C = 64 (so that the choice
+# of chunk size cannot move the figure): 2 (8 C N + 4 N^2 + C^2 / 6) = 99.7 kflop
+PREFILL_FLOP_PER_TOKEN_HEAD = 2 * (8 * 64 * N + 4 * N * N + 64 * 64 / 6)
+
+
+def tensor_view(tokens, H, ms, peaks):
+    """The same launch against the tensor-core bound: algorithmic FLOPs at C = 64 over the launch time,
+    against the measured dense bf16 peak (the products run in bf16 and tf32; tf32 has half that peak,
+    so this fraction is an upper bound of the tensor pipe's share)."""
+    flops = PREFILL_FLOP_PER_TOKEN_HEAD * tokens * H
+    tf = flops / (ms / 1e3) / 1e12
+    return {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": tf / peaks["bf16_tflops"], "flops_per_launch": flops}
+
+
 def hbm_roofline(byts, ms, peaks, **extra):
     achieved = byts / (ms / 1e3) / 1e9
     out = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -468,10 +483,14 @@ def bench_decode(lib7, dev, peaks, steps_target=1024, layers=24, bf16_state=Fals
     byts = decode_bytes(B, H, state_elem=2 if bf16_state else 4)
     del g, states, ys
     free_device()
-    return {"B": B, "H": H, "steps": nsteps, "layer_states": layers, "state_dtype": "bf16" if bf16_state else "f32",
-            "tokens": "fresh token every step (1024 distinct per graph)", "steps_per_s": 1.0 / step_s,
-            "tokens_per_s": B / step_s, "us_per_step": step_s * 1e6, "status": st,
-            "roofline": hbm_roofline(byts, step_s * 1e3, peaks)}
+    out = {"B": B, "H": H, "steps": nsteps, "layer_states": layers, "state_dtype": "bf16" if bf16_state else "f32",
+           "tokens": "fresh token every step (1024 distinct per graph)", "steps_per_s": 1.0 / step_s,
+           "tokens_per_s": B / step_s, "us_per_step": step_s * 1e6, "status": st,
+           "roofline": hbm_roofline(byts, step_s * 1e3, peaks)}
+    if layers == 1:
+        out["roofline"]["note"] = ("one state (64 MiB float32) stays in the 126 MB L2: an L2-assisted figure, "
+                                   "not an HBM one")
+    return out
 
 
 def bench_options(lib7, dev, steps, peaks, *, native, group_norm, decode=True, layers=24):
@@ -553,12 +572,13 @@ def bench_options(lib7, dev, steps, peaks, *, native, group_norm, decode=True, l
     return out
 
 
-def bench_backward(lib7, dev, steps=5):
+def bench_backward(lib7, dev, steps=5, T=None):
     """The training pair on the 0.1B prefill shape: the checkpointing forward (a saved state every 64
     tokens) and the backward (float32 gradients of r, w, k, v, a, b and the initial state).
     Reports ms per call and tokens/s; the backward is bound by its per-token CUDA-core work."""
     case = wi.CASES[SMALL]
-    B, T, H = case.B, case.T, case.H
+    B, H = case.B, case.H
+    T = T or case.T
     d = wi.draw(B, T, H, seed=case.seed, s0_std=case.s0_std, device=dev, f32_copies=False)
     gr = wi.draw_grads(B, T, H, seed=case.seed + 2)
     dd = {n: d[n] for n in OPS}
@@ -582,7 +602,7 @@ def bench_backward(lib7, dev, steps=5):
         ms = time_calls(fn, steps, stream, warmup=2)
         out[name] = {"ms": ms, "tokens_per_s": B * T / (ms / 1e3)}
     assert lib7.rwkv7_get_last_error() == 0
-    out["workload"] = SMALL
+    out["workload"] = SMALL if T == case.T else f"{SMALL} at T={T}"
     out["outputs"] = "float32 dr, dw, dk, dv, da, db [B,T,H,64] and ds_in; dy bf16, ds_out float32"
     del d, dd, y, s_out, states, g
     free_device()
@@ -693,7 +713,8 @@ def run_ours(args):
     roofline = hbm_roofline(algo, per_launch_ms, peaks, traffic=(args.traffic if args.traffic is not None
                                                                  else measured_traffic(B, T, H, args.schedule)),
                             peak_source=peak_kind, kernel="wkv7 chunked prefill (tcgen05)",
-                            peak_kind="burst copy bandwidth (kernel timed back to back, about 3 ms per launch)")
+                            peak_kind="burst copy bandwidth (kernel timed back to back, about 3 ms per launch)",
+                            tensor_view=tensor_view(B * T, H, per_launch_ms, peaks))
     del d, dd, y, s_out, s0
     free_device()
 
@@ -708,6 +729,7 @@ def run_ours(args):
             dec = bench_decode(lib7, dev, peaks, steps_target=args.decode_steps, layers=args.decode_layers)
             dec["bf16_state"] = bench_decode(lib7, dev, peaks, steps_target=args.decode_steps,
                                              layers=args.decode_layers, bf16_state=True)
+            dec["l2_assisted_single_state"] = bench_decode(lib7, dev, peaks, steps_target=args.decode_steps, layers=1)
             configs["decode_l24_d1024_b256_1024steps"] = dec
         configs[HEADLINE] = {"B": B, "T": T, "H": H, "launch_ms": per_launch_ms,
                              "tokens_per_s": B * T / (per_launch_ms / 1e3), "status": 0, "roofline": roofline,
@@ -726,7 +748,7 @@ def run_ours(args):
 
     train = None
     if not args.no_backward:
-        train = bench_backward(lib7, dev)
+        train = bench_backward(lib7, dev, T=args.train_seqlen or None)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -780,6 +802,7 @@ def main():
     ap.add_argument("--no-native", action="store_true",
                     help="skip the option entry points' lines (model-native inputs, GroupNorm epilogue)")
     ap.add_argument("--no-backward", action="store_true", help="skip the training (forward-save + backward) line")
+    ap.add_argument("--train-seqlen", type=int, default=0, help="override T of the training leg (profiling runs only)")
     ap.add_argument("--decode-steps", type=int, default=3072)
     ap.add_argument("--decode-layers", type=int, default=24, help="distinct decode states rotated over")
     ap.add_argument("--no-e2e", action="store_true")

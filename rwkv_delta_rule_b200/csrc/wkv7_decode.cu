@@ -68,6 +68,7 @@ __global__ void __launch_bounds__(256, 5) wkv7_decode_kernel(DecodeArgs<TIn, TS>
 #pragma unroll
   for (int m = 0; m < 4; ++m) st[m] = ld_state(S + (rg + 16 * m) * kN + 4 * c4);
 
+  // then every other load, before any arithmetic waits on one: a single memory round trip per CTA
   const long long vb = pair * kN;
   float ww[4], kk[4], aa[4], bb[4], rr[4], vv[4];
   Elem<TIn>::load4(A.k + vb + 4 * c4, kk);
@@ -75,15 +76,20 @@ __global__ void __launch_bounds__(256, 5) wkv7_decode_kernel(DecodeArgs<TIn, TS>
   Elem<TIn>::load4(A.a + vb + 4 * c4, aa);  // fused: x_a
   if (!kFused) Elem<TIn>::load4(A.b + vb + 4 * c4, bb);
   Elem<TIn>::load4(A.r + vb + 4 * c4, rr);
+#pragma unroll
+  for (int m = 0; m < 4; ++m) vv[m] = Elem<TIn>::load(A.v + vb + rg + 16 * m);
+  float4 ksc = make_float4(1.f, 1.f, 1.f, 1.f);  // fused: the key scale of this thread's channels
+  if (kFused && A.k_k != nullptr)
+    ksc = *reinterpret_cast<const float4 *>(A.k_k + static_cast<int>(pair % A.H) * kN + 4 * c4);
   float sa[4];
   if (kFused) {
     // x070 prologue: kk = normalise(k * k_k) over the 64 channels, a = -kk, b = kk * rate, decay from
     // x_w.  S a = -(S kx) / |kx| with kx = k * k_k: the row sums of S kx and |kx|^2 share the shuffles.
-    const int h = static_cast<int>(pair % A.H);
+    const float kscale[4] = {ksc.x, ksc.y, ksc.z, ksc.w};
     float kx[4], ss = 0.f;
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      kx[e] = A.k_k ? kk[e] * A.k_k[h * kN + 4 * c4 + e] : kk[e];
+      kx[e] = kk[e] * kscale[e];
       ss = fmaf(kx[e], kx[e], ss);
     }
 #pragma unroll
@@ -137,9 +143,6 @@ __global__ void __launch_bounds__(256, 5) wkv7_decode_kernel(DecodeArgs<TIn, TS>
 #pragma unroll
       for (int m = 0; m < 4; ++m) sa[m] += __shfl_xor_sync(0xffffffffu, sa[m], off);
   }
-#pragma unroll
-  for (int m = 0; m < 4; ++m) vv[m] = Elem<TIn>::load(A.v + vb + rg + 16 * m);
-
   float yv[4];
 #pragma unroll
   for (int m = 0; m < 4; ++m) {

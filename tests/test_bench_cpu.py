@@ -25,3 +25,43 @@ def test_reference_arm_prints_one_contract_line():
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def _bench():
+    if ROOT not in sys.path:
+        sys.path.insert(0, ROOT)
+    import bench
+
+    return bench
+
+
+def test_bench_algorithmic_bytes_and_flops():
+    # the roofline arithmetic against the workloads' own figures: 896 B per token-head for six bf16
+    # operands and y, 16 KiB per state, 33,664 B per decode head-step, 99.7 kflop per token-head at C = 64
+    b = _bench()
+    assert b.prefill_bytes(8 * 4096, 12, 8) == 7 * 8 * 4096 * 12 * 64 * 2 + 2 * 8 * 12 * 64 * 64 * 4 == 355467264
+    assert b.prefill_bytes(4 * 16384, 64, 4, state_in=False) == 7 * 4 * 16384 * 64 * 128 + 4 * 64 * 16384
+    assert b.prefill_bytes(64, 2, 1, elem=4, state_in=False) == 7 * 64 * 2 * 64 * 4 + 2 * 64 * 64 * 4
+    assert b.decode_bytes(256, 16) == 256 * 16 * 33664 == 137887744
+    assert b.decode_bytes(256, 16, state_elem=2) == 256 * 16 * (2 * 64 * 64 * 2 + 7 * 64 * 2)
+    assert b.decode_bytes(256, 16, n_ops=5) == 256 * 16 * (2 * 64 * 64 * 4 + 6 * 64 * 2)
+    assert abs(b.PREFILL_FLOP_PER_TOKEN_HEAD - 99669.33) < 0.01
+    peaks = {"hbm_gbs": 1000.0, "bf16_tflops": 1000.0}
+    r = b.hbm_roofline(2e9, 4.0, peaks)  # 2 GB in 4 ms = 500 GB/s
+    assert abs(r["achieved"] - 500.0) < 1e-9 and abs(r["frac"] - 0.5) < 1e-12 and r["unit"] == "GB/s"
+    t = b.tensor_view(1000, 10, 1.0, peaks)  # 1e4 token-heads x 99.7 kflop in 1 ms
+    assert abs(t["achieved"] - 1e4 * b.PREFILL_FLOP_PER_TOKEN_HEAD / 1e-3 / 1e12) < 1e-9
+    assert t["bound"] == "tensor" and abs(t["frac"] - t["achieved"] / 1000.0) < 1e-12
+
+
+def test_bench_clock_summary_flags_throttling():
+    b = _bench()
+    c = b.ClockSampler(0)
+    c.lines = ["0, 1965, 1965, 700, 0x0, Not Active, Not Active, Not Active, Not Active",
+               "0, 1900, 1965, 990, 0x4, Not Active, Not Active, Not Active, Active",
+               "0, 1500, 1965, 400, 0x20, Not Active, Active, Not Active, Not Active"]
+    s = c.summary()
+    assert s["sm_max_mhz"] == 1965.0 and s["samples"] == 3
+    assert s["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]
+    c.lines = []
+    assert c.summary()["reasons"] == ["unsampled"]

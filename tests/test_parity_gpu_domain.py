@@ -158,3 +158,28 @@ def test_no_decay(sched):
     assert st == 0
     assert rel_err(y, yo) <= TOL_BF16
     assert rel_err(s, so) <= TOL_BF16
+
+
+def test_fast_decay_checkpoints_one_cta_per_pair():
+    # 120 (b, h) pairs: AUTO takes one CTA per pair for the checkpointing forward; chunks 1..2 of every
+    # sequence run token by token, and the saved states and y match the oracle on sampled pairs
+    def wfun(g, shape):
+        w = 0.5452 + 0.4548 * torch.rand(shape, generator=g)
+        w[:, 64:192] = 0.02 + 0.25 * torch.rand(w[:, 64:192].shape, generator=g)
+        return w
+
+    B, T, H = 2, 260, 60
+    d = _draw(B, T, H, 960, wfun)
+    dv = to_dev(d)
+    y, s_out, states = rk.prefill_save(*[dv[n] for n in OPS], dv["s0"], path=rk.RWKV7_PATH_CHUNK)
+    torch.cuda.synchronize()
+    assert rk.rwkv7_get_last_error() == 0
+    for (b, h) in ((0, 0), (1, 59), (0, 31), (1, 7)):
+        ops = [d[n + "_f32"][b:b + 1, :, h:h + 1] for n in OPS]
+        s0 = d["s0"][b:b + 1, h:h + 1]
+        yo, so = oracle.wkv7(*ops, s0)
+        assert rel_err(y[b:b + 1, :, h:h + 1], yo) <= TOL_BF16, (b, h)
+        assert rel_err(s_out[b:b + 1, h:h + 1], so) <= TOL_BF16, (b, h)
+        for c in range(1, states.shape[2]):
+            _, ref = oracle.wkv7(*[x[:, :64 * c] for x in ops], s0)
+            assert rel_err(states[b:b + 1, h:h + 1, c], ref) <= TOL_BF16, (b, h, c)

@@ -718,11 +718,11 @@ def run_ours(args):
     del d, dd, y, s_out, s0
     free_device()
 
-    configs = None
+    per_workload = None
     schedules = None
     if not args.no_configs:
         K = args.config_steps
-        configs = {"prefill_f32_b1_t64_h2": bench_f32_small(lib7, dev, 200, peaks),
+        per_workload = {"prefill_f32_b1_t64_h2": bench_f32_small(lib7, dev, 200, peaks),
                    "prefill_d768_b8_t4096": bench_prefill(lib7, dev, SMALL, K, peaks),
                    "prefill_d2048_b16_t8192_chained": bench_chained(lib7, dev, K, peaks)}
         if not args.no_decode:
@@ -730,11 +730,11 @@ def run_ours(args):
             dec["bf16_state"] = bench_decode(lib7, dev, peaks, steps_target=args.decode_steps,
                                              layers=args.decode_layers, bf16_state=True)
             dec["l2_assisted_single_state"] = bench_decode(lib7, dev, peaks, steps_target=args.decode_steps, layers=1)
-            configs["decode_l24_d1024_b256_1024steps"] = dec
-        configs[HEADLINE] = {"B": B, "T": T, "H": H, "launch_ms": per_launch_ms,
+            per_workload["decode_l24_d1024_b256_1024steps"] = dec
+        per_workload[HEADLINE] = {"B": B, "T": T, "H": H, "launch_ms": per_launch_ms,
                              "tokens_per_s": B * T / (per_launch_ms / 1e3), "status": 0, "roofline": roofline,
                              "note": "the headline step"}
-        configs["prefill_d4096_b4_ragged"] = bench_ragged(lib7, dev, K, peaks)
+        per_workload["prefill_d4096_b4_ragged"] = bench_ragged(lib7, dev, K, peaks)
         schedules = {"pipelined (schedule 3)": {
             SMALL: bench_prefill(lib7, dev, SMALL, K, peaks, schedule=3),
             HEADLINE: bench_prefill(lib7, dev, HEADLINE, max(3, K // 2), peaks, schedule=3)}}
@@ -772,7 +772,7 @@ def run_ours(args):
         "gpu_launches": args.steps,
         "clocks": clocks.summary(),
         "cpu_baseline": cpu,
-        "configs": configs,
+        "configs": per_workload,
         "schedules": schedules,
         "options": native,
         "training": train,

@@ -235,7 +235,9 @@ typedef struct rwkv7_options {
  * queued; `stream` waits for all of it (synchronise `stream` before reading y / s_out).  For the
  * copies to overlap, the host buffers must be page-locked (cudaHostAlloc / cudaHostRegister);
  * pageable buffers give the same results without overlap.  Every pointer must be 16-byte aligned.
- * Not meant for CUDA graph capture (it creates and releases its streams per call).
+ * The two internal streams are created on a device's first call and kept until the process exits
+ * (calls on one device share them, so their work is ordered; each call creates and releases only a
+ * few events).  Not meant for CUDA graph capture: the work forks onto those streams.
  * Errors as for the device entry point; a failure leaves the outputs undefined. */
 RWKV7_API rwkv7_status rwkv7_wkv_prefill_host_bf16(int path, int B, int T, int H, int N, const uint16_t *r,
                                                    const uint16_t *w, const uint16_t *k, const uint16_t *v,

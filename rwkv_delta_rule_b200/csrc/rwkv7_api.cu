@@ -68,6 +68,31 @@ rwkv7_status check_prefill(int B, long long tokens, int H, int N, const TIn *r, 
 }  // namespace
 
 int *device_error_word() { return error_word_ptr(); }
+
+// The two internal streams of the host-buffer prefill on the current device (kernels; device -> host
+// copies), created on first use and kept for the life of the process, so a call does not pay for
+// creating and destroying streams.  Calls on one device share them: their work is ordered on them,
+// and each call's own order comes from its events.
+cudaError_t host_prefill_streams(cudaStream_t &ks, cudaStream_t &os) {
+  static cudaStream_t cache[64][2] = {};
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < 2; ++i)
+    if (cache[dev][i] == nullptr) {
+      e = cudaStreamCreateWithFlags(&cache[dev][i], cudaStreamNonBlocking);
+      if (e != cudaSuccess) {
+        cache[dev][i] = nullptr;
+        return e;
+      }
+    }
+  ks = cache[dev][0];
+  os = cache[dev][1];
+  return cudaSuccess;
+}
 bool prefill_uses_chunk(int path, long long max_T) { return use_chunk(path, max_T); }
 
 }  // namespace rwkv7
@@ -163,8 +188,7 @@ rwkv7_status rwkv7_wkv_prefill_host_bf16(int path, int B, int T, int H, int N, c
   // host -> device copies on `stream`; the prefill on `ks`; device -> host copies on `os`
   cudaStream_t ks = nullptr, os = nullptr;
   cudaEvent_t ev_in = nullptr, ev_k = nullptr, ev_done = nullptr;
-  cudaError_t e = cudaStreamCreateWithFlags(&ks, cudaStreamNonBlocking);
-  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&os, cudaStreamNonBlocking);
+  cudaError_t e = host_prefill_streams(ks, os);
   if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_done, cudaEventDisableTiming);
   for (int i = 0; i < ns && e == cudaSuccess; ++i) {
     const int b0 = static_cast<int>(static_cast<long long>(B) * i / ns);
@@ -205,8 +229,6 @@ rwkv7_status rwkv7_wkv_prefill_host_bf16(int path, int B, int T, int H, int N, c
   if (e == cudaSuccess) e = cudaEventRecord(ev_done, os);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(user, ev_done, 0);
   if (ev_done != nullptr) cudaEventDestroy(ev_done);
-  if (ks != nullptr) cudaStreamDestroy(ks);
-  if (os != nullptr) cudaStreamDestroy(os);
   return from_cuda(e);
 }
 

@@ -183,3 +183,37 @@ def test_fast_decay_checkpoints_one_cta_per_pair():
         for c in range(1, states.shape[2]):
             _, ref = oracle.wkv7(*[x[:, :64 * c] for x in ops], s0)
             assert rel_err(states[b:b + 1, h:h + 1, c], ref) <= TOL_BF16, (b, h, c)
+
+
+@pytest.mark.parametrize("H", [2, 60])  # 6 and 180 pairs: the task-parallel and the one-CTA-per-pair schedule
+def test_fast_decay_ragged_batch(H):
+    # packed rows of 70, 1, 200 and 130 tokens with a stretch of fast decay: the token-by-token path
+    # indexes the packed layout through each row's offsets
+    lengths = torch.tensor([70, 1, 200, 130])
+    cu = wi.cu_seqlens(lengths)
+    total = int(lengths.sum())
+
+    def wfun(g, shape):
+        w = 0.5452 + 0.4548 * torch.rand(shape, generator=g)
+        w[:, 60:180] = 0.02 + 0.25 * torch.rand(w[:, 60:180].shape, generator=g)
+        return w
+
+    d = _draw(1, total, H, 970 + H, wfun)
+    Bn = lengths.numel()
+    g = torch.Generator().manual_seed(971 + H)
+    s_in = (torch.randn((Bn, H, 64, 64), generator=g) * 0.1).contiguous()
+    ops = {n: d[n][0].cuda() for n in OPS}
+    y = torch.empty(total, H, 64, dtype=torch.bfloat16, device="cuda")
+    s_out = torch.empty(Bn, H, 64, 64, device="cuda")
+    rk.rwkv7_wkv_prefill_varlen_bf16(rk.RWKV7_PATH_CHUNK, cu.cuda(), int(lengths.max()), *[ops[n] for n in OPS],
+                                     s_in.cuda(), y, s_out)
+    torch.cuda.synchronize()
+    assert rk.rwkv7_get_last_error() == 0
+    heads = range(H) if H <= 2 else (0, H // 2, H - 1)
+    for b in range(Bn):
+        lo, hi = int(cu[b]), int(cu[b + 1])
+        for h in heads:
+            sl = [d[n + "_f32"][:, lo:hi, h:h + 1] for n in OPS]
+            yo, so = oracle.wkv7(*sl, s_in[b:b + 1, h:h + 1])
+            assert rel_err(y[lo:hi, h:h + 1][None], yo) <= TOL_BF16, (b, h)
+            assert rel_err(s_out[b:b + 1, h:h + 1], so) <= TOL_BF16, (b, h)

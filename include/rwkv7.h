@@ -82,7 +82,7 @@ typedef enum rwkv7_status {
   RWKV7_ERR_DOMAIN = 6
 } rwkv7_status;
 
-/* Prefill kernels: AUTO picks by T and dtype (bf16 with T >= 128 -> CHUNK,
+/* Prefill kernels: AUTO picks by T and dtype (bf16 with T >= 48 -> CHUNK,
  * otherwise SCAN); SCAN is the sequential kernel (state in registers); CHUNK
  * is the chunked tensor-core kernel (bf16 only).
  * Decay domain of CHUNK: the chunked form divides by the product of up to 64

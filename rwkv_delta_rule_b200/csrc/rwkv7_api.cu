@@ -41,10 +41,13 @@ int *error_word_ptr() {
   return static_cast<int *>(p);
 }
 
-// Kernel choice for bf16 prefill.  AUTO takes the chunked tensor-core kernel
-// once a sequence spans two chunks; shorter ones are latency-bound either way
-// and the sequential scan has no set-up cost.
-constexpr long long kChunkMinT = 128;
+// Kernel choice for bf16 prefill.  AUTO takes the chunked tensor-core kernel from
+// 48 tokens on.  Measured on B200 (scan / chunk, us per call): B1 H12 T32 15.8 / 16.3,
+// T64 20.9 / 21.0, T96 29.1 / 21.1; B8 H12 T32 15.7 / 16.4, T48 22.1 / 16.6, T64
+// 27.7 / 16.6; B64 H32 T32 181 / 164, T48 270 / 166, T64 355 / 167; B256 H16 T16
+// 189 / 317, T48 528 / 321, T127 1371 / 538.  Below that the sequential scan is as
+// fast or faster: its per-token chain is short and it has no set-up.
+constexpr long long kChunkMinT = 48;
 bool use_chunk(int path, long long max_T) {
   return path == RWKV7_PATH_CHUNK || (path == RWKV7_PATH_AUTO && max_T >= kChunkMinT);
 }

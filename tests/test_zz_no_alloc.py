@@ -47,7 +47,7 @@ def test_noalloc_host_prefill_matches_device_entry_point(pinned):
     need_cuda()
     cdll = lib7.load_library()
     calls = [
-        # chunked kernel (AUTO at T >= 128), initial state given, ragged last chunk
+        # chunked kernel (AUTO at T >= 48), initial state given, ragged last chunk
         dict(B=2, T=200, H=3, seed=71, s0_std=0.1, path=lib7.RWKV7_PATH_AUTO),
         # sequential kernel, zero initial state, a different layout of the shared array
         dict(B=3, T=70, H=2, seed=72, s0_std=None, path=lib7.RWKV7_PATH_SCAN),

@@ -431,6 +431,26 @@ __device__ __forceinline__ void invert_unit_lower(const float *Ls, float *Ts, fl
   group_sync_lo();
 }
 
+// Model-native inputs: the in-context learning rates sigmoid(x_a) of a chunk, by warps 0-3 (tid < 128)
+// once their inverse is done, as float32 [token][channel] over the raw x_a and b slots (the b slot is
+// not loaded for these inputs), where the preparation on warps 4-7 reads them.  Each thread converts
+// 4 channels x 8 tokens; all read before any is written (the float32 rows overlay the bf16 tile).
+__device__ __forceinline__ void rates_to_smem(uint8_t *smem, int tid) {
+  const int j0 = 4 * (tid & 15), tb = 8 * (tid >> 4);
+  float sg[8][4];
+#pragma unroll
+  for (int tt = 0; tt < 8; ++tt) {
+    raw4(smem, RAW_A, tb + tt, j0, sg[tt]);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) sg[tt][e] = x070_sigmoid(sg[tt][e]);
+  }
+  group_sync_lo();
+  float *rate = reinterpret_cast<float *>(smem + OFF_RAW + RAW_A * kTile);
+#pragma unroll
+  for (int tt = 0; tt < 8; ++tt)
+    *reinterpret_cast<float4 *>(rate + (tb + tt) * 64 + j0) = make_float4(sg[tt][0], sg[tt][1], sg[tt][2], sg[tt][3]);
+}
+
 // Work of warps 4-7 on the chunk after the current one, done while warps 0-3 invert (tid4 = tid -
 // 128): the decay scan (pre4[g][j] = product of w over the tokens before 4-token group g; GCn[j] =
 // product over the chunk), the MMA1 B operand [B^; K^] = [b; k] / Gamma_t (tf32) and the MMA4 V^T
@@ -440,7 +460,9 @@ __device__ __forceinline__ void invert_unit_lower(const float *Ls, float *Ts, fl
 template <bool kFused>
 __device__ __forceinline__ void prep_next(const uint8_t *smem, uint8_t *sA1, uint8_t *sB1, uint8_t *sB4Vn, float *pre4,
                                           float *GCn, float *wtot, const float *kkw, float *invn, int tid4, int Lcn,
-                                          int *err, volatile int *dflag) {
+                                          int *err, volatile int *dflag, uint64_t *bar_rate = nullptr,
+                                          uint32_t rate_parity = 0, volatile int *abort_flag = nullptr,
+                                          uint32_t max_polls = 0) {
   const int lane = tid4 & 31, wq = tid4 >> 5;
   const int cq = tid4 & 15, to = tid4 >> 4;  // channel quad; token octet (2 per warp)
   const int j0 = 4 * cq, tb = 8 * to;
@@ -533,6 +555,12 @@ __device__ __forceinline__ void prep_next(const uint8_t *smem, uint8_t *sA1, uin
     else
       *dflag = 1;
   }
+  // model-native inputs with the rates from warps 0-3: every thread waits for them (bounded; on
+  // expiry the CTA aborts and what follows is discarded)
+  if (kFused && bar_rate != nullptr && !wait_or_abort(bar_rate, rate_parity, abort_flag, max_polls)) {
+    *abort_flag = 1;
+    report_device_error(err, kDevErrTimeout);
+  }
   // [B^; K^] rows (K-major tf32; K = channel), and Gamma_t itself (float32) where the operand
   // construction will put R~ = r Gamma_t: it reads Gamma_t there and overwrites it in place
   uint8_t *b1r = sB1 + (j0 >> 5) * (128 * 128);
@@ -545,10 +573,21 @@ __device__ __forceinline__ void prep_next(const uint8_t *smem, uint8_t *sA1, uin
     if (t < Lcn) {
       raw4(smem, RAW_K, t, j0, kk);
       if (kFused) {
-        // b = kk * sigmoid(x_a), kk = k * k_k / |k * k_k| (the tile in the a slot holds x_a)
-        raw4(smem, RAW_A, t, j0, bb);
+        // b = kk * sigmoid(x_a), kk = k * k_k / |k * k_k| (the tile in the a slot holds x_a, or warps
+        // 0-3 have left the rates there as float32)
+        if (bar_rate != nullptr) {
+          const float4 u = *reinterpret_cast<const float4 *>(smem + OFF_RAW + RAW_A * kTile + (t * 64 + j0) * 4);
+          bb[0] = u.x;
+          bb[1] = u.y;
+          bb[2] = u.z;
+          bb[3] = u.w;
+        } else {
+          raw4(smem, RAW_A, t, j0, bb);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) bb[e] = kk[e] * kks[e] * inv[tt] * x070_sigmoid(bb[e]);
+          for (int e = 0; e < 4; ++e) bb[e] = x070_sigmoid(bb[e]);
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) bb[e] = kk[e] * kks[e] * inv[tt] * bb[e];
       } else {
         raw4(smem, RAW_B, t, j0, bb);
       }
@@ -731,6 +770,8 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
   uint64_t *bar_m4 = bars + 8;     // c -> w: MMA4 done
   uint64_t *bar_sin = bars + 9;    // task-parallel: the start state landed in B4S (tx bytes)
   uint64_t *bar_sout = bars + 10;  // task-parallel: w -> c, the end state is in B4S (one arrival per hi-lane warp)
+  // model-native inputs: warps 0-3 -> warps 4-7, the next chunk's rates are in shared memory
+  uint64_t *bar_rate = reinterpret_cast<uint64_t *>(smem + OFF_MISC + 200);
   // [2] by chunk parity: the preparation found the chunk's decay products outside the factorised range
   volatile int *dflag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 192);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_MISC + 88);
@@ -755,6 +796,7 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
 
   if (tid == 0) {
     for (int i = 0; i < 11; ++i) tc::mbar_init(bars + i, i == 3 ? 2 : i == 10 ? 4 : 1);  // b3: both compute groups
+    tc::mbar_init(bar_rate, 1);
     tc::fence_mbar_init();
     *abort_flag = 0;
     task_slot[0].n = task_slot[1].n = -1;
@@ -1060,6 +1102,23 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
       group_sync_hi();
       return decision_hi[slot] != 0;
     };
+    // The same for warps 0-3 alone (thread 0 polls; slots of their own).
+    volatile int *decision_lo = reinterpret_cast<volatile int *>(smem + OFF_MISC + 208);  // [2]
+    uint32_t ncalls_lo = 0;
+    auto wait_group_lo = [&](uint64_t *bar, uint32_t parity) -> bool {
+      const uint32_t slot = ncalls_lo++ & 1u;
+      if (tid == 0) {
+        if (!wait_or_abort(bar, parity, abort_flag, A.max_polls)) {
+          *abort_flag = 1;
+          report_device_error(A.err, kDevErrTimeout);
+        }
+        decision_lo[slot] = *abort_flag == 0 ? 1 : 0;
+      }
+      group_sync_lo();
+      return decision_lo[slot] != 0;
+    };
+    // model-native inputs: rate hand-offs from warps 0-3 to warps 4-7 so far (the parity of the next)
+    uint32_t nrate = 0;
     // The per-head parameters of a task, loaded by warps 4-7 (tid4 = tid - 128) before its
     // preparation: the key scale (model-native inputs) and ln_w, ln_b into buffer `par`.
     auto load_head = [&](int hd, uint32_t par, int tid4) {
@@ -1302,6 +1361,21 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
         // ---- P4: Tinv = (I - Lab)^-1 as the bf16 operand B3
         invert_unit_lower(Ls, Ts, Zs, sB3, warp, lane);
         if (tid == 0) tc::mbar_arrive(bar_b3);
+        if constexpr (kFused) {
+          // then the next task's rates, which warps 4-7 would otherwise form in their (longer) share
+          bool next = false;
+          if constexpr (kTask) {
+            next = wait_group_lo(bar_tma, (it + 1) & 1) && task_slot[(it + 1) & 1].n >= 0;
+          } else {
+            Task nt = t;
+            next = pair_next(A, nt) && wait_group_lo(bar_tma, (it + 1) & 1);
+          }
+          if (next) {
+            rates_to_smem(smem, tid);
+            group_sync_lo();
+            if (tid == 0) tc::mbar_arrive(bar_rate);
+          }
+        }
       } else {
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
@@ -1368,14 +1442,19 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
               load_head(nt.h, (it + 1) & 1, tid - 128);
               group_sync_hi();
               prep_next<kFused>(smem, sA1, sB1, sB4V + ((it + 1) & 1) * 16384, pre4,
-                                       GCs + ((it + 1) & 1) * 64, wtot, kkw, invn, tid - 128, nt.Lc, A.err, dflag + ((it + 1) & 1));
+                                       GCs + ((it + 1) & 1) * 64, wtot, kkw, invn, tid - 128, nt.Lc, A.err, dflag + ((it + 1) & 1),
+                                       kFused ? bar_rate : nullptr, nrate & 1u, abort_flag, A.max_polls);
+              nrate += kFused ? 1u : 0u;
             }
           }
         } else {
           Task nt = t;
-          if (pair_next(A, nt) && wait_group_hi(bar_tma, (it + 1) & 1))
+          if (pair_next(A, nt) && wait_group_hi(bar_tma, (it + 1) & 1)) {
             prep_next<kFused>(smem, sA1, sB1, sB4V + ((it + 1) & 1) * 16384, pre4, GCs + ((it + 1) & 1) * 64,
-                                     wtot, kkw, invn, tid - 128, nt.Lc, A.err, dflag + ((it + 1) & 1));
+                                     wtot, kkw, invn, tid - 128, nt.Lc, A.err, dflag + ((it + 1) & 1),
+                                     kFused ? bar_rate : nullptr, nrate & 1u, abort_flag, A.max_polls);
+            nrate += kFused ? 1u : 0u;
+          }
         }
       }
       if (!(ok = wait_ctrl(bar_m3, ph))) break;

@@ -431,12 +431,60 @@ __device__ __forceinline__ void invert_unit_lower(const float *Ls, float *Ts, fl
   group_sync_lo();
 }
 
-// Model-native inputs: the in-context learning rates sigmoid(x_a) of a chunk, by warps 0-3 (tid < 128)
-// once their inverse is done, as float32 [token][channel] over the raw x_a and b slots (the b slot is
-// not loaded for these inputs), where the preparation on warps 4-7 reads them.  Each thread converts
-// 4 channels x 8 tokens; all read before any is written (the float32 rows overlay the bf16 tile).
-__device__ __forceinline__ void rates_to_smem(uint8_t *smem, int tid) {
-  const int j0 = 4 * (tid & 15), tb = 8 * (tid >> 4);
+// 1 / |k * k_k| of the 8 tokens tb.. of a thread that holds channels j0..j0+3 (kks: their k_k); the 16
+// lanes of a half-warp hold the 64 channels of the same tokens.  Tokens at or past Lcn count as k = 0.
+__device__ __forceinline__ void key_inv_norms(const uint8_t *smem, const float (&kks)[4], int tb, int j0, int Lcn,
+                                              float (&inv)[8]) {
+#pragma unroll
+  for (int tt = 0; tt < 8; ++tt) {
+    float kv[4], ss = 0.f;
+    if (tb + tt < Lcn) {
+      raw4(smem, RAW_K, tb + tt, j0, kv);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) kv[e] = 0.f;
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) ss = fmaf(kv[e] * kks[e], kv[e] * kks[e], ss);
+#pragma unroll
+    for (int off = 8; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    inv[tt] = x070_inv_norm(ss);
+  }
+}
+
+// The MMA4 V^T operand of a chunk from its raw v tile (row = vrow(value channel), K = token; bf16
+// values are exact in tf32) for the 8 tokens tb.. and channels j0..j0+3 of a thread; tokens at or
+// past Lcn are zeros.  The caller fences for the async proxy.
+__device__ __forceinline__ void vt_rows(const uint8_t *smem, uint8_t *sB4Vn, int tb, int j0, int Lcn) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    float vv[4][4];
+#pragma unroll
+    for (int tt = 0; tt < 4; ++tt) {
+      if (tb + 4 * h + tt < Lcn) {
+        raw4(smem, RAW_V, tb + 4 * h + tt, j0, vv[tt]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) vv[tt][e] = 0.f;
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      *reinterpret_cast<uint4 *>(sB4Vn + kmaj_tf32(64, vrow(j0 + e), tb + 4 * h)) =
+          make_uint4(__float_as_uint(vv[0][e]), __float_as_uint(vv[1][e]), __float_as_uint(vv[2][e]),
+                     __float_as_uint(vv[3][e]));
+  }
+}
+
+// Model-native inputs: the part of the next chunk's preparation that warps 0-3 (tid < 128) take once
+// their inverse is done, in the layout warps 4-7 use (4 channels x 8 tokens per thread): the
+// in-context learning rates sigmoid(x_a) as float32 [token][channel] over the raw x_a and b slots (the
+// b slot is not loaded for these inputs; every thread reads its x_a values before the group writes
+// any), the per-token key norms into invn, and V^T.  kk_src: the head's k_k (null: ones).  Ends with
+// the group's barrier.
+__device__ __forceinline__ void prep_lo_fused(uint8_t *smem, uint8_t *sB4Vn, const float *kk_src, float *invn, int tid,
+                                              int Lcn) {
+  const int cq = tid & 15, j0 = 4 * cq, tb = 8 * (tid >> 4);
   float sg[8][4];
 #pragma unroll
   for (int tt = 0; tt < 8; ++tt) {
@@ -444,11 +492,20 @@ __device__ __forceinline__ void rates_to_smem(uint8_t *smem, int tid) {
 #pragma unroll
     for (int e = 0; e < 4; ++e) sg[tt][e] = x070_sigmoid(sg[tt][e]);
   }
+  float kks[4], inv[8];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) kks[e] = kk_src ? kk_src[j0 + e] : 1.f;
+  key_inv_norms(smem, kks, tb, j0, Lcn, inv);
+  vt_rows(smem, sB4Vn, tb, j0, Lcn);
   group_sync_lo();
   float *rate = reinterpret_cast<float *>(smem + OFF_RAW + RAW_A * kTile);
 #pragma unroll
-  for (int tt = 0; tt < 8; ++tt)
+  for (int tt = 0; tt < 8; ++tt) {
     *reinterpret_cast<float4 *>(rate + (tb + tt) * 64 + j0) = make_float4(sg[tt][0], sg[tt][1], sg[tt][2], sg[tt][3]);
+    if (cq == 0) invn[tb + tt] = inv[tt];
+  }
+  tc::fence_proxy_async_smem();
+  group_sync_lo();
 }
 
 // Work of warps 4-7 on the chunk after the current one, done while warps 0-3 invert (tid4 = tid -
@@ -480,26 +537,17 @@ __device__ __forceinline__ void prep_next(const uint8_t *smem, uint8_t *sA1, uin
       for (int e = 0; e < 4; ++e) G[tt][e] = 1.f;
     }
   }
+  // model-native inputs: with bar_rate, warps 0-3 form this chunk's rates, key norms and V^T
+  const bool lo_part = kFused && bar_rate != nullptr;
   float kks[4] = {1.f, 1.f, 1.f, 1.f}, inv[8];
   if (kFused) {
-    // 1 / |k * k_k| per token: the 16 lanes of a half-warp hold the 64 channels of its tokens
 #pragma unroll
     for (int e = 0; e < 4; ++e) kks[e] = kkw[j0 + e];
+    if (!lo_part) {
+      key_inv_norms(smem, kks, tb, j0, Lcn, inv);
 #pragma unroll
-    for (int tt = 0; tt < 8; ++tt) {
-      float kv[4], ss = 0.f;
-      if (tb + tt < Lcn) {
-        raw4(smem, RAW_K, tb + tt, j0, kv);
-      } else {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) kv[e] = 0.f;
-      }
-#pragma unroll
-      for (int e = 0; e < 4; ++e) ss = fmaf(kv[e] * kks[e], kv[e] * kks[e], ss);
-#pragma unroll
-      for (int off = 8; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-      inv[tt] = x070_inv_norm(ss);
-      if (cq == 0) invn[tb + tt] = inv[tt];
+      for (int tt = 0; tt < 8; ++tt)
+        if (cq == 0) invn[tb + tt] = inv[tt];
     }
   }
 #pragma unroll
@@ -557,9 +605,13 @@ __device__ __forceinline__ void prep_next(const uint8_t *smem, uint8_t *sA1, uin
   }
   // model-native inputs with the rates from warps 0-3: every thread waits for them (bounded; on
   // expiry the CTA aborts and what follows is discarded)
-  if (kFused && bar_rate != nullptr && !wait_or_abort(bar_rate, rate_parity, abort_flag, max_polls)) {
-    *abort_flag = 1;
-    report_device_error(err, kDevErrTimeout);
+  if (lo_part) {
+    if (!wait_or_abort(bar_rate, rate_parity, abort_flag, max_polls)) {
+      *abort_flag = 1;
+      report_device_error(err, kDevErrTimeout);
+    }
+#pragma unroll
+    for (int tt = 0; tt < 8; ++tt) inv[tt] = invn[tb + tt];
   }
   // [B^; K^] rows (K-major tf32; K = channel), and Gamma_t itself (float32) where the operand
   // construction will put R~ = r Gamma_t: it reads Gamma_t there and overwrites it in place
@@ -575,7 +627,7 @@ __device__ __forceinline__ void prep_next(const uint8_t *smem, uint8_t *sA1, uin
       if (kFused) {
         // b = kk * sigmoid(x_a), kk = k * k_k / |k * k_k| (the tile in the a slot holds x_a, or warps
         // 0-3 have left the rates there as float32)
-        if (bar_rate != nullptr) {
+        if (lo_part) {
           const float4 u = *reinterpret_cast<const float4 *>(smem + OFF_RAW + RAW_A * kTile + (t * 64 + j0) * 4);
           bb[0] = u.x;
           bb[1] = u.y;
@@ -605,25 +657,8 @@ __device__ __forceinline__ void prep_next(const uint8_t *smem, uint8_t *sA1, uin
     st_tf32x4(b1r + tc::sw128(t, chunk), bb[0] * ig[0], bb[1] * ig[1], bb[2] * ig[2], bb[3] * ig[3]);
     st_tf32x4(b1r + tc::sw128(64 + t, chunk), kk[0] * ig[0], kk[1] * ig[1], kk[2] * ig[2], kk[3] * ig[3]);
   }
-  // V^T (row = vrow(value channel), K = token); bf16 values are exact in tf32
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    float vv[4][4];
-#pragma unroll
-    for (int tt = 0; tt < 4; ++tt) {
-      if (tb + 4 * h + tt < Lcn) {
-        raw4(smem, RAW_V, tb + 4 * h + tt, j0, vv[tt]);
-      } else {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) vv[tt][e] = 0.f;
-      }
-    }
-#pragma unroll
-    for (int e = 0; e < 4; ++e)
-      *reinterpret_cast<uint4 *>(sB4Vn + kmaj_tf32(64, vrow(j0 + e), tb + 4 * h)) =
-          make_uint4(__float_as_uint(vv[0][e]), __float_as_uint(vv[1][e]), __float_as_uint(vv[2][e]),
-                     __float_as_uint(vv[3][e]));
-  }
+  // V^T (warps 0-3 build it with the rates)
+  if (!lo_part) vt_rows(smem, sB4Vn, tb, j0, Lcn);
   tc::fence_proxy_async_smem();
 }
 
@@ -1362,17 +1397,17 @@ __global__ void __launch_bounds__(kThreads, 1) wkv7_chunk_kernel(const __grid_co
         invert_unit_lower(Ls, Ts, Zs, sB3, warp, lane);
         if (tid == 0) tc::mbar_arrive(bar_b3);
         if constexpr (kFused) {
-          // then the next task's rates, which warps 4-7 would otherwise form in their (longer) share
+          // then the next task's rates, key norms and V^T, which warps 4-7 would otherwise form in their
+          // (longer) share
           bool next = false;
+          Task nt = t;
           if constexpr (kTask) {
-            next = wait_group_lo(bar_tma, (it + 1) & 1) && task_slot[(it + 1) & 1].n >= 0;
+            next = wait_group_lo(bar_tma, (it + 1) & 1) && (nt = task_slot[(it + 1) & 1], nt.n >= 0);
           } else {
-            Task nt = t;
             next = pair_next(A, nt) && wait_group_lo(bar_tma, (it + 1) & 1);
           }
           if (next) {
-            rates_to_smem(smem, tid);
-            group_sync_lo();
+            prep_lo_fused(smem, sB4V + ((it + 1) & 1) * 16384, A.k_k ? A.k_k + nt.h * kN : nullptr, invn, tid, nt.Lc);
             if (tid == 0) tc::mbar_arrive(bar_rate);
           }
         }

@@ -123,6 +123,17 @@ def tensor_view(tokens, H, ms, peaks):
             "frac": tf / peaks["bf16_tflops"], "flops_per_launch": flops}
 
 
+def training_bytes(B, T, H):
+    """Algorithmic HBM bytes of the training pair over B x T tokens and H heads: the checkpointing
+    forward reads 6 bf16 operands and the initial state and writes y, a state every 64 tokens and the
+    final state; the backward reads the 6 operands, dy, the saved states and ds_out and writes 6
+    float32 gradients and ds_in."""
+    th, pairs, nck = B * T * H, B * H, -(-T // 64)
+    fwd = th * 7 * N * 2 + pairs * (nck + 2) * N * N * 4
+    bwd = th * (7 * N * 2 + 6 * N * 4) + pairs * (nck + 2) * N * N * 4
+    return fwd, bwd
+
+
 def hbm_roofline(byts, ms, peaks, **extra):
     achieved = byts / (ms / 1e3) / 1e9
     out = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -572,10 +583,11 @@ def bench_options(lib7, dev, steps, peaks, *, native, group_norm, decode=True, l
     return out
 
 
-def bench_backward(lib7, dev, steps=5, T=None):
+def bench_backward(lib7, dev, peaks, steps=5, T=None):
     """The training pair on the 0.1B prefill shape: the checkpointing forward (a saved state every 64
     tokens) and the backward (float32 gradients of r, w, k, v, a, b and the initial state).
-    Reports ms per call and tokens/s; the backward is bound by its per-token CUDA-core work."""
+    Reports ms per call, tokens/s and each call's HBM roofline; the backward is bound by its per-token
+    CUDA-core work (its fraction of HBM shows how far from the memory bound that leaves it)."""
     case = wi.CASES[SMALL]
     B, H = case.B, case.H
     T = T or case.T
@@ -598,9 +610,10 @@ def bench_backward(lib7, dev, steps=5, T=None):
         lib7.rwkv7_wkv_backward_bf16(*[dd[n] for n in OPS], states, dy, ds, *g, ds_in, stream)
 
     out = {}
+    nbytes = dict(zip(("forward_save", "backward"), training_bytes(B, T, H)))
     for name, fn in (("forward_save", fwd), ("backward", bwd)):
         ms = time_calls(fn, steps, stream, warmup=2)
-        out[name] = {"ms": ms, "tokens_per_s": B * T / (ms / 1e3)}
+        out[name] = {"ms": ms, "tokens_per_s": B * T / (ms / 1e3), "roofline": hbm_roofline(nbytes[name], ms, peaks)}
     assert lib7.rwkv7_get_last_error() == 0
     out["workload"] = SMALL if T == case.T else f"{SMALL} at T={T}"
     out["outputs"] = "float32 dr, dw, dk, dv, da, db [B,T,H,64] and ds_in; dy bf16, ds_out float32"
@@ -748,7 +761,7 @@ def run_ours(args):
 
     train = None
     if not args.no_backward:
-        train = bench_backward(lib7, dev, T=args.train_seqlen or None)
+        train = bench_backward(lib7, dev, peaks, T=args.train_seqlen or None)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:

@@ -46,6 +46,12 @@ def test_bench_algorithmic_bytes_and_flops():
     assert b.decode_bytes(256, 16, state_elem=2) == 256 * 16 * (2 * 64 * 64 * 2 + 7 * 64 * 2)
     assert b.decode_bytes(256, 16, n_ops=5) == 256 * 16 * (2 * 64 * 64 * 4 + 6 * 64 * 2)
     assert abs(b.PREFILL_FLOP_PER_TOKEN_HEAD - 99669.33) < 0.01
+    # training pair at B8 T4096 H12: per token-head 7 bf16 vectors forward (6 operands + y) and 7 bf16
+    # + 6 float32 vectors backward; per pair 64 saved states plus two more (s_in/s_out, ds_out/ds_in)
+    fwd, bwd = b.training_bytes(8, 4096, 12)
+    assert fwd == 8 * 4096 * 12 * 896 + 96 * 66 * 16384
+    assert bwd == 8 * 4096 * 12 * (896 + 1536) + 96 * 66 * 16384
+    assert b.training_bytes(1, 65, 1) == (65 * 896 + 4 * 16384, 65 * 2432 + 4 * 16384)  # two chunks
     peaks = {"hbm_gbs": 1000.0, "bf16_tflops": 1000.0}
     r = b.hbm_roofline(2e9, 4.0, peaks)  # 2 GB in 4 ms = 500 GB/s
     assert abs(r["achieved"] - 500.0) < 1e-9 and abs(r["frac"] - 0.5) < 1e-12 and r["unit"] == "GB/s"

@@ -77,7 +77,7 @@ def load_peaks():
 # operands, larger than L2) forced to that schedule, scaled by the token-heads of a launch; the figure
 # holds only for the kernel source it was taken on (sha256 prefix of wkv7_chunk.cu), and the line
 # reports null for any other build.  The capture is summarised under profiles/.
-MEASURED_TRAFFIC = {"source_sha256": "70d8c2337de517f2", "bytes_per_token_head": (805687552 + 124459008) / (16384 * 64)}
+MEASURED_TRAFFIC = {"source_sha256": "ec571157ca8177a4", "bytes_per_token_head": (805728000 + 124227584) / (16384 * 64)}
 
 
 def measured_traffic(B, T, H, schedule):

@@ -116,6 +116,42 @@ def test_waits_that_give_up_early_abort_cleanly(sched):
     assert rel_err(y, yo) <= TOL_BF16 and rel_err(s_out, so) <= TOL_BF16
 
 
+@pytest.mark.parametrize("sched", [rk.RWKV7_SCHED_PAIR, rk.RWKV7_SCHED_TASKS])
+def test_model_native_waits_that_give_up_early_abort_cleanly(sched):
+    """The same with model-native inputs, where warps 0-3 hand the next chunk's rates, key norms and
+    V^T to warps 4-7 through a wait of its own: it too gives up, the CTA aborts and returns, and the
+    next launch is exact (against the float64 prologue and recurrence)."""
+    B, T, H = 2, 640, 3
+    d = wi.draw_model_native(B, T, H, seed=4245, s0_std=0.1)
+    names = ("r", "xw", "k", "v", "xa")
+    yo, so = oracle.wkv7_model_native(*[d[n + "_f32"] for n in names], d["k_k"], d["s0"])
+    dv = {n: d[n].cuda() for n in names}
+    kk, s0 = d["k_k"].cuda(), d["s0"].cuda()
+    y = torch.empty(B, T, H, N, dtype=torch.bfloat16, device="cuda")
+    s_out = torch.empty(B, H, N, N, device="cuda")
+
+    def call():
+        rk.rwkv7_wkv_prefill_ext_bf16(rk.RWKV7_PATH_CHUNK, dv["r"], dv["xw"], dv["k"], dv["v"], dv["xa"], None, s0,
+                                      y, s_out, model_native=True, k_k=kk, schedule=sched)
+
+    rk.rwkv7_test_set_wait_hooks(32, -1)
+    t0 = time.monotonic()
+    try:
+        call()
+        torch.cuda.synchronize()
+        elapsed = time.monotonic() - t0
+        st = rk.rwkv7_get_last_error()
+    finally:
+        rk.rwkv7_test_set_wait_hooks(0, -1)
+    assert st in (0, ERR_TIMEOUT), rk.rwkv7_status_string(st)
+    assert elapsed < 30.0
+    assert rk.rwkv7_get_last_error() == 0
+    call()
+    torch.cuda.synchronize()
+    assert rk.rwkv7_get_last_error() == 0
+    assert rel_err(y, yo) <= TOL_BF16 and rel_err(s_out, so) <= TOL_BF16
+
+
 def test_hook_defaults_leave_every_schedule_exact():
     """With the hooks at their defaults (and after being set and reset) nothing times out."""
     rk.rwkv7_test_set_wait_hooks(1 << 12, 0)

@@ -452,10 +452,12 @@ def decode_tokens(B, T, H, seed, dev, native=False):
     return toks, extra
 
 
-def bench_decode(lib7, dev, peaks, steps_target=1024, layers=24, bf16_state=False, toks=None):
+def bench_decode(lib7, dev, peaks, steps_target=1024, layers=24, bf16_state=False, toks=None, independent=False):
     """Decode steps/s at the L24-D1024 shape (B=256, H=16): every step reads a fresh token (1024 distinct
     tokens per CUDA graph of 1024 steps) and one of `layers` distinct states (1.6 GB in float32),
-    so neither the operands nor the state stay in L2.  `bf16_state`: the state stored as bfloat16."""
+    so neither the operands nor the state stay in L2.  `bf16_state`: the state stored as bfloat16.
+    `independent`: the steps set the `independent_state` option (each layer has its own state, so a
+    step's state loads may start before the step before it has finished)."""
     case = wi.CASES["decode_l24_d1024_b256_1024steps"]
     B, H, T = case.B, case.H, case.T
     if toks is None:
@@ -463,6 +465,11 @@ def bench_decode(lib7, dev, peaks, steps_target=1024, layers=24, bf16_state=Fals
     states = torch.zeros(layers, B, H, N, N, device=dev, dtype=torch.bfloat16 if bf16_state else torch.float32)
     ys = [torch.empty(B, H, N, dtype=torch.bfloat16, device=dev) for _ in range(layers)]
     step_fn = lib7.rwkv7_wkv_decode_bf16_bf16state if bf16_state else lib7.rwkv7_wkv_decode_bf16
+    if independent:
+        ext = lib7.rwkv7_wkv_decode_ext_bf16state if bf16_state else lib7.rwkv7_wkv_decode_ext_bf16
+
+        def step_fn(*args):
+            ext(*args, independent_state=True)
 
     def one_pass():
         for i in range(T):
@@ -495,6 +502,7 @@ def bench_decode(lib7, dev, peaks, steps_target=1024, layers=24, bf16_state=Fals
     del g, states, ys
     free_device()
     out = {"B": B, "H": H, "steps": nsteps, "layer_states": layers, "state_dtype": "bf16" if bf16_state else "f32",
+           "independent_state": bool(independent),
            "tokens": "fresh token every step (1024 distinct per graph)", "steps_per_s": 1.0 / step_s,
            "tokens_per_s": B / step_s, "us_per_step": step_s * 1e6, "status": st,
            "roofline": hbm_roofline(byts, step_s * 1e3, peaks)}
@@ -548,34 +556,40 @@ def bench_options(lib7, dev, steps, peaks, *, native, group_norm, decode=True, l
         states = torch.zeros(layers, Bd, Hd, N, N, device=dev)
         ys = [torch.empty(Bd, Hd, N, dtype=torch.bfloat16, device=dev) for _ in range(layers)]
 
-        def one_pass():
-            for i in range(Td):
-                src = {n: toks[n][i] for n in names}
-                lib7.rwkv7_wkv_decode_ext_bf16(*ops(src), states[i % layers], ys[i % layers], **dopt)
+        def time_steps(independent):
+            def one_pass():
+                for i in range(Td):
+                    src = {n: toks[n][i] for n in names}
+                    lib7.rwkv7_wkv_decode_ext_bf16(*ops(src), states[i % layers], ys[i % layers],
+                                                   independent_state=independent, **dopt)
 
-        sd = torch.cuda.Stream(device=dev)
-        sd.wait_stream(torch.cuda.current_stream())
-        with torch.cuda.stream(sd):
-            one_pass()
-        torch.cuda.current_stream().wait_stream(sd)
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            one_pass()
-        for _ in range(3):
+            sd = torch.cuda.Stream(device=dev)
+            sd.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(sd):
+                one_pass()
+            torch.cuda.current_stream().wait_stream(sd)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                one_pass()
+            for _ in range(3):
+                g.replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
             g.replay()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        g.replay()
-        e1.record()
-        torch.cuda.synchronize()
-        assert lib7.rwkv7_get_last_error() == 0
-        step_s = e0.elapsed_time(e1) / 1e3 / Td
-        dbytes = decode_bytes(Bd, Hd, n_ops=len(names))
-        out["decode"] = {"workload": "decode_l24_d1024_b256", "steps_per_s": 1.0 / step_s,
-                         "us_per_step": step_s * 1e6, "tokens": "fresh token every step",
-                         "roofline": hbm_roofline(dbytes, step_s * 1e3, peaks)}
-        del g, toks, states, ys
+            e1.record()
+            torch.cuda.synchronize()
+            assert lib7.rwkv7_get_last_error() == 0
+            del g
+            step_s = e0.elapsed_time(e1) / 1e3 / Td
+            dbytes = decode_bytes(Bd, Hd, n_ops=len(names))
+            return {"workload": "decode_l24_d1024_b256", "steps_per_s": 1.0 / step_s, "us_per_step": step_s * 1e6,
+                    "tokens": "fresh token every step", "independent_state": independent,
+                    "roofline": hbm_roofline(dbytes, step_s * 1e3, peaks)}
+
+        out["decode"] = time_steps(False)
+        out["decode_independent_state"] = time_steps(True)
+        del toks, states, ys
         free_device()
     out["inputs"] = (("bf16 r, x_w, k, v, x_a [B,T,H,64] + float32 k_k [H,64]; w, a, b formed in-kernel"
                       if native else "bf16 r, w, k, v, a, b [B,T,H,64]")
@@ -743,6 +757,13 @@ def run_ours(args):
             dec["bf16_state"] = bench_decode(lib7, dev, peaks, steps_target=args.decode_steps,
                                              layers=args.decode_layers, bf16_state=True)
             dec["l2_assisted_single_state"] = bench_decode(lib7, dev, peaks, steps_target=args.decode_steps, layers=1)
+            # the same steps with the independent_state option (the 24 layer states are distinct, so a step's
+            # state loads may overlap the last wave of the step before)
+            dec["independent_state"] = bench_decode(lib7, dev, peaks, steps_target=args.decode_steps,
+                                                    layers=args.decode_layers, independent=True)
+            dec["bf16_state_independent_state"] = bench_decode(lib7, dev, peaks, steps_target=args.decode_steps,
+                                                               layers=args.decode_layers, bf16_state=True,
+                                                               independent=True)
             per_workload["decode_l24_d1024_b256_1024steps"] = dec
         per_workload[HEADLINE] = {"B": B, "T": T, "H": H, "launch_ms": per_launch_ms,
                              "tokens_per_s": B * T / (per_launch_ms / 1e3), "status": 0, "roofline": roofline,

@@ -209,6 +209,20 @@ RWKV7_API rwkv7_status rwkv7_wkv_decode_fused_bf16(int B, int H, int N, const ui
  *                         and inverse, state chain on separate warps).  Needs H <= 65535.
  *                     Every schedule is exact for every decay in [0, 1] (see the decay domain
  *                     above).
+ *   independent_state = 1 (decode only, library scheduling with no counterpart on the pages; the
+ *                     prefill ignores it): the caller promises that no decode step queued before
+ *                     this one on `stream`, and possibly still running, writes this step's state.
+ *                     The decode kernels start under programmatic dependent launch: a step's CTAs
+ *                     may start while the step before is finishing, and they read nothing that
+ *                     step writes before it has completed.  With this option they load their
+ *                     state before that wait, so the state loads overlap the previous step's last
+ *                     wave.  Results are the same; only the timing changes.  A model whose layers
+ *                     each keep their own state, stepping them in turn, qualifies when there are
+ *                     at least 3 layer states and B*H exceeds the CTAs the device runs at once
+ *                     (then at most the step before is still running when a step's CTAs start).
+ *                     Consecutive steps of one state do not qualify: with the option set they read
+ *                     a state that is not yet written.  Left 0, every step waits first, which is
+ *                     always correct.
  */
 typedef struct rwkv7_options {
   int model_native;
@@ -217,6 +231,7 @@ typedef struct rwkv7_options {
   const float *ln_w;
   const float *ln_b;
   int chunk_schedule;
+  int independent_state;
 } rwkv7_options;
 
 /* ---- prefill from and to host memory ------------------------------------------------------
@@ -309,6 +324,14 @@ RWKV7_API rwkv7_status rwkv7_wkv_decode_bf16_bf16state(int B, int H, int N, cons
                                                        const uint16_t *k, const uint16_t *v, const uint16_t *a,
                                                        const uint16_t *b, uint16_t *s_inout, uint16_t *y,
                                                        rwkv7_stream_t stream);
+
+/* The same step with options (NULL = none): only independent_state applies (see rwkv7_options);
+ * model_native or group_norm set returns RWKV7_ERR_INVALID.  Other arguments, errors and ownership
+ * as for rwkv7_wkv_decode_bf16_bf16state. */
+RWKV7_API rwkv7_status rwkv7_wkv_decode_ext_bf16state(int B, int H, int N, const uint16_t *r, const uint16_t *w,
+                                                      const uint16_t *k, const uint16_t *v, const uint16_t *a,
+                                                      const uint16_t *b, const rwkv7_options *opt,
+                                                      uint16_t *s_inout, uint16_t *y, rwkv7_stream_t stream);
 
 /* ---- training: forward with checkpoints, and the backward ----------------------------------
  *

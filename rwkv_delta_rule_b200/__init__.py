@@ -29,6 +29,7 @@ __all__ = [
     "rwkv7_wkv_prefill_ext_bf16", "rwkv7_wkv_decode_ext_bf16", "Options",
     "rwkv7_status_string", "rwkv7_get_last_error", "rwkv7_version", "rwkv7_test_set_wait_hooks",
     "rwkv7_wkv_prefill_save_bf16", "rwkv7_wkv_backward_bf16", "rwkv7_wkv_decode_bf16_bf16state",
+    "rwkv7_wkv_decode_ext_bf16state",
     "rwkv7_wkv_prefill_host_bf16", "rwkv7_wkv_prefill_host_noalloc_bf16", "NOALLOC_STAGING_BYTES", "prefill", "decode_", "prefill_model_native", "decode_model_native_", "prefill_ext", "decode_ext_",
     "prefill_save", "backward", "EXPORTED_SYMBOLS",
 ]
@@ -44,7 +45,7 @@ EXPORTED_SYMBOLS = (
     "rwkv7_wkv_prefill_ext_bf16", "rwkv7_wkv_decode_ext_bf16",
     "rwkv7_wkv_prefill_save_bf16", "rwkv7_wkv_backward_bf16", "rwkv7_wkv_decode_bf16_bf16state",
     "rwkv7_wkv_prefill_host_bf16", "rwkv7_status_string", "rwkv7_get_last_error", "rwkv7_version",
-    "rwkv7_wkv_prefill_host_noalloc_bf16", "rwkv7_test_set_wait_hooks",
+    "rwkv7_wkv_prefill_host_noalloc_bf16", "rwkv7_test_set_wait_hooks", "rwkv7_wkv_decode_ext_bf16state",
 )
 # RWKV7_NOALLOC_STAGING_BYTES of include/rwkv7.h: the staging limit of rwkv7_wkv_prefill_host_noalloc_bf16
 NOALLOC_STAGING_BYTES = 32 * 1024 * 1024
@@ -57,7 +58,8 @@ class Options(ctypes.Structure):
     """``rwkv7_options`` of include/rwkv7.h (host struct; the pointers are device addresses)."""
 
     _fields_ = [("model_native", ctypes.c_int), ("k_k", ctypes.c_void_p), ("group_norm", ctypes.c_int),
-                ("ln_w", ctypes.c_void_p), ("ln_b", ctypes.c_void_p), ("chunk_schedule", ctypes.c_int)]
+                ("ln_w", ctypes.c_void_p), ("ln_b", ctypes.c_void_p), ("chunk_schedule", ctypes.c_int),
+                ("independent_state", ctypes.c_int)]
 
 
 class Rwkv7Error(RuntimeError):
@@ -95,6 +97,7 @@ def load_library() -> ctypes.CDLL:
         ("rwkv7_wkv_prefill_save_bf16", [ci, ci, ci, ci, ci] + [vp] * 6 + [vp, vp, vp, vp, vp]),
         ("rwkv7_wkv_backward_bf16", [ci, ci, ci, ci] + [vp] * 6 + [vp, vp, vp] + [vp] * 7 + [vp]),
         ("rwkv7_wkv_decode_bf16_bf16state", [ci, ci, ci] + [vp] * 6 + [vp, vp, vp]),
+        ("rwkv7_wkv_decode_ext_bf16state", [ci, ci, ci] + [vp] * 6 + [ctypes.POINTER(Options), vp, vp, vp]),
         ("rwkv7_wkv_prefill_host_bf16", [ci, ci, ci, ci, ci] + [vp] * 6 + [vp, vp, vp] + [vp] * 6 + [vp, vp, vp]
          + [ci, vp]),
         ("rwkv7_wkv_prefill_host_noalloc_bf16", [ci] + pre),
@@ -279,14 +282,16 @@ def rwkv7_wkv_decode_fused_bf16(r, xw, k, v, xa, k_k, s_inout, y, stream=None) -
           _stream(stream))
 
 
-def _options(model_native: bool, k_k, group_norm: bool, ln_w, ln_b, H: int, N: int, schedule: int = 0) -> Options:
+def _options(model_native: bool, k_k, group_norm: bool, ln_w, ln_b, H: int, N: int, schedule: int = 0,
+             independent_state: bool = False) -> Options:
     if model_native:
         _check(k_k, "k_k", torch.float32, (H, N), allow_none=True)
     if group_norm:
         _check(ln_w, "ln_w", torch.float32, (H, N), allow_none=True)
         _check(ln_b, "ln_b", torch.float32, (H, N), allow_none=True)
     return Options(int(bool(model_native)), _ptr(k_k) if model_native else None, int(bool(group_norm)),
-                   _ptr(ln_w) if group_norm else None, _ptr(ln_b) if group_norm else None, int(schedule))
+                   _ptr(ln_w) if group_norm else None, _ptr(ln_b) if group_norm else None, int(schedule),
+                   int(bool(independent_state)))
 
 
 def rwkv7_wkv_prefill_ext_bf16(path, r, w, k, v, a, b, s_in, y, s_out, *, model_native=False, k_k=None,
@@ -307,14 +312,16 @@ def rwkv7_wkv_prefill_ext_bf16(path, r, w, k, v, a, b, s_in, y, s_out, *, model_
 
 
 def rwkv7_wkv_decode_ext_bf16(r, w, k, v, a, b, s_inout, y, *, model_native=False, k_k=None, group_norm=False,
-                              ln_w=None, ln_b=None, stream=None) -> None:
-    """bf16 decode step with options (see ``rwkv7_wkv_prefill_ext_bf16``)."""
+                              ln_w=None, ln_b=None, independent_state=False, stream=None) -> None:
+    """bf16 decode step with options (see ``rwkv7_wkv_prefill_ext_bf16``); ``independent_state``: no step
+    still running before this one on the stream writes this step's state (``rwkv7_options``), so the
+    state loads may start before the previous step has finished."""
     B, H, N = r.shape
     names = (("r", r), ("w", w), ("k", k), ("v", v), ("a", a), ("y", y)) + (() if model_native else (("b", b),))
     for nm, t in names:
         _check(t, nm, torch.bfloat16, (B, H, N))
     _check(s_inout, "s_inout", torch.float32, (B, H, N, N))
-    opt = _options(model_native, k_k, group_norm, ln_w, ln_b, H, N)
+    opt = _options(model_native, k_k, group_norm, ln_w, ln_b, H, N, independent_state=independent_state)
     _call("rwkv7_wkv_decode_ext_bf16", B, H, N, *[_ptr(t) for t in (r, w, k, v, a, None if model_native else b)],
           ctypes.byref(opt), _ptr(s_inout), _ptr(y), _stream(stream))
 
@@ -327,6 +334,18 @@ def rwkv7_wkv_decode_bf16_bf16state(r, w, k, v, a, b, s_inout, y, stream=None) -
     _check(s_inout, "s_inout", torch.bfloat16, (B, H, N, N))
     _call("rwkv7_wkv_decode_bf16_bf16state", B, H, N, *[_ptr(t) for t in (r, w, k, v, a, b, s_inout, y)],
           _stream(stream))
+
+
+def rwkv7_wkv_decode_ext_bf16state(r, w, k, v, a, b, s_inout, y, *, independent_state=False, stream=None) -> None:
+    """``rwkv7_wkv_decode_bf16_bf16state`` with options: ``independent_state`` as for
+    ``rwkv7_wkv_decode_ext_bf16``."""
+    B, H, N = r.shape
+    for nm, t in (("r", r), ("w", w), ("k", k), ("v", v), ("a", a), ("b", b), ("y", y)):
+        _check(t, nm, torch.bfloat16, (B, H, N))
+    _check(s_inout, "s_inout", torch.bfloat16, (B, H, N, N))
+    opt = Options(0, None, 0, None, None, 0, int(bool(independent_state)))
+    _call("rwkv7_wkv_decode_ext_bf16state", B, H, N, *[_ptr(t) for t in (r, w, k, v, a, b)], ctypes.byref(opt),
+          _ptr(s_inout), _ptr(y), _stream(stream))
 
 
 def n_checkpoints(T: int) -> int:

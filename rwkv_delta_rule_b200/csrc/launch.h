@@ -55,17 +55,19 @@ cudaError_t launch_decode(const TIn *r, const TIn *w, const TIn *k, const TIn *v
 
 // The bf16 step with the state stored as bf16 [B,H,64,64] (widened to float32 for the update, rounded
 // to nearest-even on store).
+// early_state: the state loads go out before the wait for the previous grid on the stream (the caller
+// promises that no step still running before this one writes this step's state).
 cudaError_t launch_decode_bf16state(const uint16_t *r, const uint16_t *w, const uint16_t *k, const uint16_t *v,
-                                    const uint16_t *a, const uint16_t *b, uint16_t *s, uint16_t *y, int B, int H,
-                                    cudaStream_t stream);
+                                    const uint16_t *a, const uint16_t *b, bool early_state, uint16_t *s, uint16_t *y,
+                                    int B, int H, cudaStream_t stream);
 
 // The bf16 step with the optional parts: model-native inputs (w, a slots hold x_w, x_a; b unused;
 // key scale k_k [H,64] float32 or nullptr for ones) and the GroupNorm epilogue on y (ln_w, ln_b
-// [H,64] float32 or nullptr for ones / zeros).
+// [H,64] float32 or nullptr for ones / zeros); early_state as for launch_decode_bf16state.
 cudaError_t launch_decode_ext(const uint16_t *r, const uint16_t *w, const uint16_t *k, const uint16_t *v,
                               const uint16_t *a, const uint16_t *b, bool model_native, const float *k_k,
-                              bool group_norm, const float *ln_w, const float *ln_b, float *s, uint16_t *y, int B,
-                              int H, cudaStream_t stream);
+                              bool group_norm, const float *ln_w, const float *ln_b, bool early_state, float *s,
+                              uint16_t *y, int B, int H, cudaStream_t stream);
 
 // The chunked prefill as a warp-specialised pipeline (one persistent CTA per SM walking its (b, h)
 // pairs' chunks with three chunks in flight); same arguments as launch_chunk_ext without the schedule.

@@ -268,8 +268,8 @@ rwkv7_status rwkv7_wkv_decode_bf16(int B, int H, int N, const uint16_t *r, const
   if (N != kN) return RWKV7_ERR_UNSUPPORTED;
   if (B <= 0 || H <= 0 || !none_null(r, w, k, v, a, b, s_inout, y)) return RWKV7_ERR_INVALID;
   if (!all_aligned(r, w, k, v, a, b, s_inout, y)) return RWKV7_ERR_ALIGN;
-  return from_cuda(launch_decode_ext(r, w, k, v, a, b, false, nullptr, false, nullptr, nullptr, s_inout, y, B, H,
-                                     reinterpret_cast<cudaStream_t>(stream)));
+  return from_cuda(launch_decode_ext(r, w, k, v, a, b, false, nullptr, false, nullptr, nullptr, false, s_inout, y, B,
+                                     H, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 rwkv7_status rwkv7_wkv_prefill_ext_bf16(int path, int B, int T, int H, int N, const uint16_t *r, const uint16_t *w,
@@ -308,7 +308,8 @@ rwkv7_status rwkv7_wkv_decode_ext_bf16(int B, int H, int N, const uint16_t *r, c
   if (B <= 0 || H <= 0 || !none_null(r, w, k, v, a, s_inout, y) || (!native && b == nullptr))
     return RWKV7_ERR_INVALID;
   if (!all_aligned(r, w, k, v, a, b, s_inout, y, k_k, ln_w, ln_b)) return RWKV7_ERR_ALIGN;
-  return from_cuda(launch_decode_ext(r, w, k, v, a, b, native, k_k, ln, ln_w, ln_b, s_inout, y, B, H,
+  const bool early = opt != nullptr && opt->independent_state != 0;
+  return from_cuda(launch_decode_ext(r, w, k, v, a, b, native, k_k, ln, ln_w, ln_b, early, s_inout, y, B, H,
                                      reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -334,7 +335,21 @@ rwkv7_status rwkv7_wkv_decode_bf16_bf16state(int B, int H, int N, const uint16_t
   if (N != kN) return RWKV7_ERR_UNSUPPORTED;
   if (B <= 0 || H <= 0 || !none_null(r, w, k, v, a, b, s_inout, y)) return RWKV7_ERR_INVALID;
   if (!all_aligned(r, w, k, v, a, b, s_inout, y)) return RWKV7_ERR_ALIGN;
-  return from_cuda(launch_decode_bf16state(r, w, k, v, a, b, s_inout, y, B, H, reinterpret_cast<cudaStream_t>(stream)));
+  return from_cuda(
+      launch_decode_bf16state(r, w, k, v, a, b, false, s_inout, y, B, H, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+rwkv7_status rwkv7_wkv_decode_ext_bf16state(int B, int H, int N, const uint16_t *r, const uint16_t *w,
+                                            const uint16_t *k, const uint16_t *v, const uint16_t *a,
+                                            const uint16_t *b, const rwkv7_options *opt, uint16_t *s_inout,
+                                            uint16_t *y, rwkv7_stream_t stream) {
+  if (opt != nullptr && (opt->model_native != 0 || opt->group_norm != 0)) return RWKV7_ERR_INVALID;
+  if (N != kN) return RWKV7_ERR_UNSUPPORTED;
+  if (B <= 0 || H <= 0 || !none_null(r, w, k, v, a, b, s_inout, y)) return RWKV7_ERR_INVALID;
+  if (!all_aligned(r, w, k, v, a, b, s_inout, y)) return RWKV7_ERR_ALIGN;
+  const bool early = opt != nullptr && opt->independent_state != 0;
+  return from_cuda(
+      launch_decode_bf16state(r, w, k, v, a, b, early, s_inout, y, B, H, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 rwkv7_status rwkv7_wkv_prefill_save_bf16(int path, int B, int T, int H, int N, const uint16_t *r,

@@ -51,14 +51,17 @@ __device__ __forceinline__ void st_state(uint16_t *p, float4 x) {
   *reinterpret_cast<uint2 *>(p) = make_uint2(bf16x2_rn(x.x, x.y), bf16x2_rn(x.z, x.w));
 }
 
-template <typename TIn, bool kFused, bool kLN, typename TS = float>
+// kEarly (the caller's promise that no step still running before this one writes this step's state):
+// the state loads go out before the wait for the previous grid, so they overlap its last wave.
+template <typename TIn, bool kFused, bool kLN, bool kEarly, typename TS = float>
 __global__ void __launch_bounds__(256, 5) wkv7_decode_kernel(DecodeArgs<TIn, TS> A) {
   const long long pair = blockIdx.x;  // b * H + h
   const int tid = threadIdx.x;
   // the step before may still be finishing (its launch allowed this grid to start early): every CTA
-  // of this grid has started once all have passed the trigger, and none reads memory before the wait
+  // of this grid has started once all have passed the trigger, and none reads memory the step before
+  // may write (the operands; the state too, without kEarly) before the wait
   pdl_trigger();
-  pdl_wait();
+  if (!kEarly) pdl_wait();
   const int c4 = tid & 15;   // column chunk: columns 4*c4 .. 4*c4+3
   const int rg = tid >> 4;   // rows rg + 16*m
   TS *S = A.s + pair * (kN * kN);
@@ -67,6 +70,7 @@ __global__ void __launch_bounds__(256, 5) wkv7_decode_kernel(DecodeArgs<TIn, TS>
   float4 st[4];
 #pragma unroll
   for (int m = 0; m < 4; ++m) st[m] = ld_state(S + (rg + 16 * m) * kN + 4 * c4);
+  if (kEarly) pdl_wait();
 
   // then every other load, before any arithmetic waits on one: a single memory round trip per CTA
   const long long vb = pair * kN;
@@ -217,21 +221,29 @@ cudaError_t launch_decode(const TIn *r, const TIn *w, const TIn *k, const TIn *v
   DecodeArgs<TIn> A{r, w, k, v, a, b, s, y, nullptr, H, nullptr, nullptr};
   const long long pairs = static_cast<long long>(B) * H;
   if (pairs > 0x7fffffffLL) return cudaErrorInvalidValue;
-  return launch_overlapped(wkv7_decode_kernel<TIn, false, false>, static_cast<unsigned>(pairs), 256, stream, A);
+  return launch_overlapped(wkv7_decode_kernel<TIn, false, false, false>, static_cast<unsigned>(pairs), 256, stream, A);
 }
 
 cudaError_t launch_decode_ext(const uint16_t *r, const uint16_t *w, const uint16_t *k, const uint16_t *v,
                               const uint16_t *a, const uint16_t *b, bool model_native, const float *k_k,
-                              bool group_norm, const float *ln_w, const float *ln_b, float *s, uint16_t *y, int B,
-                              int H, cudaStream_t stream) {
+                              bool group_norm, const float *ln_w, const float *ln_b, bool early_state, float *s,
+                              uint16_t *y, int B, int H, cudaStream_t stream) {
   DecodeArgs<uint16_t> A{r, w, k, v, a, b, s, y, k_k, H, ln_w, ln_b};
   const long long pairs = static_cast<long long>(B) * H;
   if (pairs > 0x7fffffffLL) return cudaErrorInvalidValue;
   const unsigned g = static_cast<unsigned>(pairs);
-  if (model_native && group_norm) return launch_overlapped(wkv7_decode_kernel<uint16_t, true, true>, g, 256, stream, A);
-  if (model_native) return launch_overlapped(wkv7_decode_kernel<uint16_t, true, false>, g, 256, stream, A);
-  if (group_norm) return launch_overlapped(wkv7_decode_kernel<uint16_t, false, true>, g, 256, stream, A);
-  return launch_overlapped(wkv7_decode_kernel<uint16_t, false, false>, g, 256, stream, A);
+  if (early_state) {
+    if (model_native && group_norm)
+      return launch_overlapped(wkv7_decode_kernel<uint16_t, true, true, true>, g, 256, stream, A);
+    if (model_native) return launch_overlapped(wkv7_decode_kernel<uint16_t, true, false, true>, g, 256, stream, A);
+    if (group_norm) return launch_overlapped(wkv7_decode_kernel<uint16_t, false, true, true>, g, 256, stream, A);
+    return launch_overlapped(wkv7_decode_kernel<uint16_t, false, false, true>, g, 256, stream, A);
+  }
+  if (model_native && group_norm)
+    return launch_overlapped(wkv7_decode_kernel<uint16_t, true, true, false>, g, 256, stream, A);
+  if (model_native) return launch_overlapped(wkv7_decode_kernel<uint16_t, true, false, false>, g, 256, stream, A);
+  if (group_norm) return launch_overlapped(wkv7_decode_kernel<uint16_t, false, true, false>, g, 256, stream, A);
+  return launch_overlapped(wkv7_decode_kernel<uint16_t, false, false, false>, g, 256, stream, A);
 }
 
 // The bf16-state step: one CTA of 128 threads per (b, h); thread t holds columns 8*(t%8) .. +7 of
@@ -248,9 +260,10 @@ __device__ __forceinline__ void unpack8(uint4 u, float (&o)[8]) {
   o[7] = __uint_as_float(u.w & 0xffff0000u);
 }
 
+template <bool kEarly>
 __global__ void __launch_bounds__(128) wkv7_decode_bf16state_kernel(DecodeArgs<uint16_t, uint16_t> A) {
   pdl_trigger();
-  pdl_wait();
+  if (!kEarly) pdl_wait();
   const long long pair = blockIdx.x;
   const int tid = threadIdx.x;
   const int c8 = tid & 7, rg = tid >> 3;
@@ -258,6 +271,7 @@ __global__ void __launch_bounds__(128) wkv7_decode_bf16state_kernel(DecodeArgs<u
   uint4 raw[4];
 #pragma unroll
   for (int m = 0; m < 4; ++m) raw[m] = *reinterpret_cast<const uint4 *>(S + (rg + 16 * m) * kN + 8 * c8);
+  if (kEarly) pdl_wait();
   const long long vb = pair * kN;
   float ww[8], kk[8], aa[8], bb[8], rr[8];
   unpack8(*reinterpret_cast<const uint4 *>(A.w + vb + 8 * c8), ww);
@@ -303,12 +317,14 @@ __global__ void __launch_bounds__(128) wkv7_decode_bf16state_kernel(DecodeArgs<u
 }
 
 cudaError_t launch_decode_bf16state(const uint16_t *r, const uint16_t *w, const uint16_t *k, const uint16_t *v,
-                                    const uint16_t *a, const uint16_t *b, uint16_t *s, uint16_t *y, int B, int H,
-                                    cudaStream_t stream) {
+                                    const uint16_t *a, const uint16_t *b, bool early_state, uint16_t *s, uint16_t *y,
+                                    int B, int H, cudaStream_t stream) {
   DecodeArgs<uint16_t, uint16_t> A{r, w, k, v, a, b, s, y, nullptr, H, nullptr, nullptr};
   const long long pairs = static_cast<long long>(B) * H;
   if (pairs > 0x7fffffffLL) return cudaErrorInvalidValue;
-  return launch_overlapped(wkv7_decode_bf16state_kernel, static_cast<unsigned>(pairs), 128, stream, A);
+  const unsigned g = static_cast<unsigned>(pairs);
+  if (early_state) return launch_overlapped(wkv7_decode_bf16state_kernel<true>, g, 128, stream, A);
+  return launch_overlapped(wkv7_decode_bf16state_kernel<false>, g, 128, stream, A);
 }
 
 template cudaError_t launch_decode<float>(const float *, const float *, const float *, const float *, const float *,

@@ -32,6 +32,16 @@ def test_header_declares_binding_names():
     assert declared_symbols() == sorted(lib7.EXPORTED_SYMBOLS)
 
 
+def test_binding_declares_a_signature_for_every_entry_point():
+    """ctypes passes Python ints as 32-bit C ints to a function without argtypes, which truncates
+    pointers: every exported entry point must have its argument types set by load_library."""
+    lib = lib7.load_library()
+    for name in lib7.EXPORTED_SYMBOLS:
+        fn = getattr(lib, name)
+        assert fn.argtypes is not None, name
+        assert fn.restype is not None, name
+
+
 def test_library_exports_every_declared_symbol(cdll):
     out = subprocess.run(["nm", "-D", "--defined-only", lib7.library_path()], capture_output=True, text=True,
                          check=True).stdout
@@ -117,6 +127,15 @@ def test_training_and_bf16_state_entry_points_reject(cdll):
     assert cdll.rwkv7_wkv_decode_bf16_bf16state(1, 1, 64, *ops, None, FAKE, None) == 1
     assert cdll.rwkv7_wkv_decode_bf16_bf16state(1, 1, 64, *ops, MIS, FAKE, None) == 2
     assert cdll.rwkv7_wkv_decode_bf16_bf16state(1, 1, 48, *ops, FAKE, FAKE, None) == 5
+    # rwkv7_wkv_decode_ext_bf16state(B, H, N, ops, opt, s_inout, y, stream): only independent_state applies
+    opt = ctypes.byref(lib7.Options(0, None, 0, None, None, 0, 1))
+    assert cdll.rwkv7_wkv_decode_ext_bf16state(1, 1, 64, *ops, ctypes.byref(lib7.Options(1, None, 0, None, None, 0, 0)),
+                                               FAKE, FAKE, None) == 1  # model-native inputs
+    assert cdll.rwkv7_wkv_decode_ext_bf16state(1, 1, 64, *ops, ctypes.byref(lib7.Options(0, None, 1, None, None, 0, 0)),
+                                               FAKE, FAKE, None) == 1  # group norm
+    assert cdll.rwkv7_wkv_decode_ext_bf16state(1, 1, 64, *ops, opt, None, FAKE, None) == 1
+    assert cdll.rwkv7_wkv_decode_ext_bf16state(1, 1, 64, *ops, opt, MIS, FAKE, None) == 2
+    assert cdll.rwkv7_wkv_decode_ext_bf16state(1, 1, 32, *ops, opt, FAKE, FAKE, None) == 5
 
 
 def test_host_prefill_rejects(cdll):

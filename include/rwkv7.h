@@ -210,18 +210,19 @@ RWKV7_API rwkv7_status rwkv7_wkv_decode_fused_bf16(int B, int H, int N, const ui
  *                     Every schedule is exact for every decay in [0, 1] (see the decay domain
  *                     above).
  *   independent_state = 1 (decode only, library scheduling with no counterpart on the pages; the
- *                     prefill ignores it): the caller promises that no decode step queued before
- *                     this one on `stream`, and possibly still running, writes this step's state.
- *                     The decode kernels start under programmatic dependent launch: a step's CTAs
- *                     may start while the step before is finishing, and they read nothing that
- *                     step writes before it has completed.  With this option they load their
- *                     state before that wait, so the state loads overlap the previous step's last
- *                     wave.  Results are the same; only the timing changes.  A model whose layers
- *                     each keep their own state, stepping them in turn, qualifies when there are
- *                     at least 3 layer states and B*H exceeds the CTAs the device runs at once
- *                     (then at most the step before is still running when a step's CTAs start).
- *                     Consecutive steps of one state do not qualify: with the option set they read
- *                     a state that is not yet written.  Left 0, every step waits first, which is
+ *                     prefill ignores it): the caller promises that the decode step queued just
+ *                     before this one on `stream` does not write this step's state.  The decode
+ *                     kernels start under programmatic dependent launch: a step's CTAs may start
+ *                     while the step before is finishing, and they read nothing that step writes
+ *                     before it has completed.  With this option they load their state before that
+ *                     wait, so the state loads overlap the previous step's last wave.  Results are
+ *                     the same; only the timing changes.  The option takes effect only when B*H
+ *                     exceeds the CTAs the device runs at once (the library checks; smaller steps
+ *                     wait first as without it): with steps of that size queued back to back, no
+ *                     step older than the one before is still running when a step's CTAs start.
+ *                     A model whose layers each keep their own state, stepped in turn, qualifies.
+ *                     Consecutive steps of one state do not: with the option set they could read a
+ *                     state that is not yet written.  Left 0, every step waits first, which is
  *                     always correct.
  */
 typedef struct rwkv7_options {

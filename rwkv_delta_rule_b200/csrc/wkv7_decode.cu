@@ -20,6 +20,8 @@
 // The fused variant takes model-native inputs (decay pre-activation x_w in place of w, the key k,
 // the learning-rate pre-activation x_a in place of a, and the per-channel key scale k_k) and forms
 // w, a = -kk and b = kk * sigmoid(x_a) in-kernel; the key norm is one more 16-lane reduction.
+#include <mutex>
+
 #include "common.cuh"
 #include "launch.h"
 
@@ -215,6 +217,37 @@ static cudaError_t launch_overlapped(void (*kernel)(KArgs...), unsigned grid, un
   return cudaGetLastError();
 }
 
+// Whether a grid of `ctas` CTAs of `kernel` is larger than what the current device runs at once (its
+// SM count times the kernel's resident CTAs per SM; cached per device and kernel).  Only then can no
+// more than one earlier step still be running when a step's CTAs start: the step before cannot place
+// all its CTAs, and so cannot release the next launch, until the one before it has finished.  Smaller
+// grids could chain several waiting steps, so the early state loads are used only above this size.
+// False when the device cannot be queried.
+static bool exceeds_resident(const void *kernel, int threads, long long ctas) {
+  constexpr int kMaxDev = 64, kMaxKernels = 16;
+  static const void *keys[kMaxDev][kMaxKernels] = {};
+  static long long vals[kMaxDev][kMaxKernels] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return false;
+  std::lock_guard<std::mutex> lock(mu);
+  int slot = 0;
+  for (; slot < kMaxKernels && keys[dev][slot] != nullptr; ++slot)
+    if (keys[dev][slot] == kernel) return ctas > vals[dev][slot];
+  int per_sm = 0, sms = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, 0) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || per_sm <= 0 || sms <= 0) {
+    (void)cudaGetLastError();  // clear a failed query; the launch then waits first, which is always correct
+    return false;
+  }
+  const long long resident = static_cast<long long>(per_sm) * sms;
+  if (slot < kMaxKernels) {
+    keys[dev][slot] = kernel;
+    vals[dev][slot] = resident;
+  }
+  return ctas > resident;
+}
+
 template <typename TIn>
 cudaError_t launch_decode(const TIn *r, const TIn *w, const TIn *k, const TIn *v, const TIn *a, const TIn *b,
                           float *s, TIn *y, int B, int H, cudaStream_t stream) {
@@ -232,6 +265,14 @@ cudaError_t launch_decode_ext(const uint16_t *r, const uint16_t *w, const uint16
   const long long pairs = static_cast<long long>(B) * H;
   if (pairs > 0x7fffffffLL) return cudaErrorInvalidValue;
   const unsigned g = static_cast<unsigned>(pairs);
+  if (early_state) {
+    // the residency check takes the variant about to launch
+    const void *kern = model_native && group_norm ? reinterpret_cast<const void *>(wkv7_decode_kernel<uint16_t, true, true, true>)
+                       : model_native             ? reinterpret_cast<const void *>(wkv7_decode_kernel<uint16_t, true, false, true>)
+                       : group_norm               ? reinterpret_cast<const void *>(wkv7_decode_kernel<uint16_t, false, true, true>)
+                                                  : reinterpret_cast<const void *>(wkv7_decode_kernel<uint16_t, false, false, true>);
+    early_state = exceeds_resident(kern, 256, pairs);
+  }
   if (early_state) {
     if (model_native && group_norm)
       return launch_overlapped(wkv7_decode_kernel<uint16_t, true, true, true>, g, 256, stream, A);
@@ -323,7 +364,8 @@ cudaError_t launch_decode_bf16state(const uint16_t *r, const uint16_t *w, const 
   const long long pairs = static_cast<long long>(B) * H;
   if (pairs > 0x7fffffffLL) return cudaErrorInvalidValue;
   const unsigned g = static_cast<unsigned>(pairs);
-  if (early_state) return launch_overlapped(wkv7_decode_bf16state_kernel<true>, g, 128, stream, A);
+  if (early_state && exceeds_resident(reinterpret_cast<const void *>(wkv7_decode_bf16state_kernel<true>), 128, pairs))
+    return launch_overlapped(wkv7_decode_bf16state_kernel<true>, g, 128, stream, A);
   return launch_overlapped(wkv7_decode_bf16state_kernel<false>, g, 128, stream, A);
 }
 

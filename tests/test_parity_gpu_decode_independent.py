@@ -10,7 +10,8 @@ same run without it.  That holds for the float32 state (bf16 operands, model-nat
 GroupNorm epilogue) and for the bf16 state, on a stream and replayed from a CUDA graph.  The run
 without the option is itself checked against the float64 oracle by the other decode tests; its
 first layer's first step is checked here too.  The shape, B256 H16 with three layer states, keeps
-every grid larger than the device runs at once, as the option's contract asks.
+every grid larger than the device runs at once, where the option takes effect; a last test checks
+that smaller steps ignore it.
 """
 
 import pytest
@@ -108,3 +109,30 @@ def test_first_step_matches_the_oracle(mode):
         f32 = {n: first[n].float() for n in OPS}
         yo, _ = oracle.wkv7(*[f32[n][:, None] for n in OPS], s0[0])
     assert rel_err(ys[0], yo[:, 0]) <= TOL_BF16
+
+
+@pytest.mark.parametrize("bf16", [False, True], ids=["f32_state", "bf16_state"])
+def test_small_steps_ignore_the_option(bf16):
+    """Below the device's resident CTA count the library keeps the wait before the state loads, so even
+    steps that violate the promise (every step on one state, B1 H4) stay exact: bit-for-bit the same
+    as without the option."""
+    b, h, steps = 1, 4, 16
+    dev = torch.device("cuda", 0)
+    d = wi.draw(b, steps, h, seed=91, dtype="bf16", device=dev, f32_copies=False)
+    toks = {n: d[n].transpose(0, 1).contiguous() for n in OPS}
+    g = torch.Generator(device="cpu").manual_seed(92)
+    s_init = (torch.randn(b, h, N, N, generator=g) * 0.1).to(dev)
+    out = []
+    for independent in (False, True):
+        state = s_init.to(torch.bfloat16) if bf16 else s_init.clone()
+        ys = torch.empty(steps, b, h, N, dtype=torch.bfloat16, device=dev)
+        for i in range(steps):
+            ops = [toks[n][i] for n in OPS]
+            if bf16:
+                rk.rwkv7_wkv_decode_ext_bf16state(*ops, state, ys[i], independent_state=independent)
+            else:
+                rk.rwkv7_wkv_decode_ext_bf16(*ops, state, ys[i], independent_state=independent)
+        torch.cuda.synchronize()
+        out.append((ys.cpu(), state.float().cpu()))
+    assert torch.equal(out[0][0].view(torch.int16), out[1][0].view(torch.int16))
+    assert torch.equal(out[0][1], out[1][1])
